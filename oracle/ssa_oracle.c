@@ -1,0 +1,461 @@
+/*
+ * ssa_oracle.c -- plain fp64 CPU oracle for the decode step of Simplified
+ * Sparse Attention (gist tokens), single level and two level (gist-of-gist).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library calls, links or
+ * includes this file; only the tests, the package smoke check and the bench's
+ * CPU-baseline leg use it.  It shares no code, header or table with the CUDA
+ * path.
+ *
+ * Source: "Simplified Sparse Attention via Gist Tokens" (Mao, Li, Fox),
+ *   sec. 3.2  gist-based relevance scoring (query . gist key dot products),
+ *   sec. 3.3  top-k chunk selection and hybrid attention over the unfolded
+ *             context,
+ *   sec. 3.5 / App. B.2  coarse-to-fine (gist-of-gist) selection,
+ *   sec. 3.6  split-K partial attention + combination compute the same
+ *             softmax as the single pass written here.
+ * Readings taken where the pages leave a step open (each is also listed in
+ * the design notes):
+ *   - chunk score = max over the GQA group's query heads and the chunk's g
+ *     gist tokens of q.k / sqrt(d); the selection is shared by the group;
+ *   - ties go to the lower chunk index; NaN scores rank as -inf;
+ *   - context = gist K/V of the unselected complete chunks + raw K/V of every
+ *     token of the selected chunks + raw K/V of the incomplete tail chunk
+ *     (the selected chunks' own gists are not in it);
+ *   - two level: meta-gist K/V of unselected complete superchunks + gist K/V
+ *     of unselected candidate chunks (children of selected superchunks plus
+ *     the remainder chunks that belong to no complete superchunk) + raw K/V
+ *     of the selected chunks + tail;
+ *   - seq_lens counts every cached raw token; all of them are visible.
+ *
+ * Inputs are fp32 arrays (bf16 values convert to fp32 exactly); every sum,
+ * product and exponential is fp64.  Layouts (row-major):
+ *   q [B,Hq,d]; k_raw, v_raw [B,Hkv,n_max,d]; k_gist, v_gist [B,Hkv,M_max,g,d]
+ *   (M_max = n_max / C); k_meta, v_meta [B,Hkv,S_max,gm,d] (S_max = M_max / J).
+ *
+ * Mutants: building with -DORACLE_MUTANT=<n> plants one deliberate mistake
+ * (see the MUT() sites) so the tests can show that the pins catch it.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0
+#endif
+#define MUT(n) (ORACLE_MUTANT == (n))
+
+typedef struct {
+    int B, Hq, Hkv, d, n_max, C, g;
+} oshape;
+
+static int ok_shape(const oshape* s) {
+    if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->d < 1 || s->C < 1 || s->g < 1) return 0;
+    if (s->Hq % s->Hkv) return 0;
+    if (s->n_max < 1 || s->n_max % s->C) return 0;
+    return 1;
+}
+
+/* Number of cached raw tokens of sequence b, or -1 if outside [1, n_max]. */
+static int seq_len(const oshape* s, const int32_t* seq_lens, int b) {
+    int n = seq_lens[b];
+    if (n < 1 || n > s->n_max) return -1;
+    return n;
+}
+
+static double dot(const float* a, const float* b, int d) {
+    double acc = 0.0;
+    for (int i = 0; i < d; ++i) acc += (double)a[i] * (double)b[i];
+    return acc;
+}
+
+static double scale_of(int d) {
+    if (MUT(1)) return 1.0;           /* mutant 1: scale dropped from scoring */
+    return 1.0 / sqrt((double)d);
+}
+
+/* Score of one summary slot: max over the group's query heads and the slot's
+ * `ntok` summary tokens (rows[0..ntok)) of q.k * scale (sec. 3.2; aggregation
+ * reading above). */
+static double slot_score(const oshape* s, const float* q, int b, int j, const float* const* rows,
+                         int ntok) {
+    const int G = s->Hq / s->Hkv;
+    const double sc = scale_of(s->d);
+    double best = -INFINITY;
+    for (int gh = 0; gh < G; ++gh) {
+        if (MUT(6) && gh > 0) break;  /* mutant 6: only the group's first head */
+        const int h = MUT(8) ? (j + gh * s->Hkv) : (j * G + gh); /* mutant 8: wrong head map */
+        const float* qh = q + ((size_t)b * s->Hq + h) * s->d;
+        for (int t = 0; t < ntok; ++t) {
+            double v = dot(qh, rows[t], s->d) * sc;
+            if (v > best) best = v;
+        }
+    }
+    return best;
+}
+
+static const float* gist_row(const oshape* s, const float* base, int b, int j, int m, int t) {
+    const int M_max = s->n_max / s->C;
+    if (MUT(10)) /* mutant 10: gist index transposed (t-major instead of chunk-major) */
+        return base + ((((size_t)b * s->Hkv + j) * M_max * s->g) + (size_t)t * M_max + m) * s->d;
+    return base + ((((size_t)b * s->Hkv + j) * M_max + m) * s->g + t) * s->d;
+}
+
+static const float* raw_row(const oshape* s, const float* base, int b, int j, int i) {
+    return base + (((size_t)b * s->Hkv + j) * s->n_max + i) * s->d;
+}
+
+
+static double chunk_score(const oshape* s, const float* q, const float* k_gist, int b, int j,
+                          int m) {
+    const float** r = (const float**)malloc(sizeof(float*) * (size_t)s->g);
+    for (int t = 0; t < s->g; ++t) r[t] = gist_row(s, k_gist, b, j, m, t);
+    double v = slot_score(s, q, b, j, r, s->g);
+    free((void*)r);
+    return v;
+}
+
+static double super_score(const oshape* s, const float* q, const float* k_meta, int S_max,
+                          int gm, int b, int j, int x) {
+    const float** r = (const float**)malloc(sizeof(float*) * (size_t)gm);
+    for (int t = 0; t < gm; ++t)
+        r[t] = k_meta + ((((size_t)b * s->Hkv + j) * S_max + x) * gm + t) * s->d;
+    double v = slot_score(s, q, b, j, r, gm);
+    free((void*)r);
+    return v;
+}
+
+/* ---------------------------------------------------------------- top-k --- */
+
+typedef struct {
+    double v;
+    int i;
+} keyed;
+
+/* Order: larger score first; equal scores -> lower index first (tie reading).
+ * NaN ranks as -inf. */
+static int cmp_desc(const void* pa, const void* pb) {
+    const keyed* a = (const keyed*)pa;
+    const keyed* b = (const keyed*)pb;
+    double va = isnan(a->v) ? -INFINITY : a->v;
+    double vb = isnan(b->v) ? -INFINITY : b->v;
+    if (va > vb) return -1;
+    if (va < vb) return 1;
+    if (MUT(3)) return (a->i > b->i) ? -1 : (a->i < b->i); /* mutant 3: ties to higher index */
+    return (a->i < b->i) ? -1 : (a->i > b->i);
+}
+
+static int cmp_int(const void* pa, const void* pb) {
+    int a = *(const int*)pa, b = *(const int*)pb;
+    return (a > b) - (a < b);
+}
+
+/* The k largest of vals[cand[0..n)] (sec. 3.3 top-k), written ascending by
+ * index into out[0..k), padded with -1 up to `cap`.  Returns k. */
+static int topk_of(const double* vals, const int* cand, int n, int topk, int* out, int cap) {
+    int k = topk < n ? topk : n;
+    if (k < 0) k = 0;
+    keyed* tmp = (keyed*)malloc(sizeof(keyed) * (size_t)(n > 0 ? n : 1));
+    for (int c = 0; c < n; ++c) {
+        tmp[c].v = vals[cand[c]];
+        tmp[c].i = cand[c];
+    }
+    qsort(tmp, (size_t)n, sizeof(keyed), cmp_desc);
+    for (int c = 0; c < k; ++c) out[c] = tmp[c].i;
+    if (!MUT(11)) qsort(out, (size_t)k, sizeof(int), cmp_int); /* mutant 11: not re-sorted */
+    for (int c = k; c < cap; ++c) out[c] = -1;
+    free(tmp);
+    return k;
+}
+
+/* ------------------------------------------------------------- attention --- */
+
+/* Softmax attention of one query head over an explicit list of (key, value)
+ * row pointers: out = sum_x softmax_x(q.k_x * scale) v_x, with the maximum
+ * subtracted before exponentiation.  Writes out[d] and the log-sum-exp. */
+static void attend_list(const float* qh, int d, const float** ks, const float** vs, int n,
+                        double* out, double* lse) {
+    const double sc = MUT(2) ? 1.0 : 1.0 / sqrt((double)d); /* mutant 2: no attention scale */
+    for (int i = 0; i < d; ++i) out[i] = 0.0;
+    if (n == 0) {
+        *lse = -INFINITY;
+        return;
+    }
+    double* logit = (double*)malloc(sizeof(double) * (size_t)n);
+    double mx = -INFINITY;
+    for (int x = 0; x < n; ++x) {
+        logit[x] = dot(qh, ks[x], d) * sc;
+        if (logit[x] > mx) mx = logit[x];
+    }
+    double den = 0.0;
+    for (int x = 0; x < n; ++x) {
+        double p = exp(logit[x] - mx);
+        den += p;
+        for (int i = 0; i < d; ++i) out[i] += p * (double)vs[x][i];
+    }
+    for (int i = 0; i < d; ++i) out[i] /= den;
+    *lse = mx + log(den);
+    free(logit);
+}
+
+/* Append the raw rows [lo, hi) of (b, j) to the context list. */
+static int push_raw(const oshape* s, const float* k_raw, const float* v_raw, int b, int j, int lo,
+                    int hi, const float** ks, const float** vs, int n) {
+    for (int i = lo; i < hi; ++i) {
+        ks[n] = raw_row(s, k_raw, b, j, i);
+        vs[n] = raw_row(s, v_raw, b, j, i);
+        ++n;
+    }
+    return n;
+}
+
+static int is_in(const int* sorted, int k, int m) {
+    for (int c = 0; c < k; ++c)
+        if (sorted[c] == m) return 1;
+    return 0;
+}
+
+/* ----------------------------------------------------- single level path --- */
+
+/*
+ * oracle_decode: the whole single-level decode step.
+ *   scores  [B,Hkv,M_max]  chunk scores (-inf for m >= M_b)         (out)
+ *   sel     [B,Hkv,topk]   selected chunks ascending, -1 padded     (in/out)
+ *   out     [B,Hq,d]       attention output                         (out)
+ *   lse     [B,Hq]         natural log-sum-exp of the logits         (out)
+ *   ctx     [B,Hkv]        context size |X| of each (b, j)           (out)
+ * force_sel != 0: `sel` is an input (a given selection, e.g. the GPU's at a
+ * near tie) and only the attention step runs on it.
+ * Returns 0, or -1 for a bad shape, or 1 + b for a bad seq_lens[b] (that
+ * sequence's outputs are zero, its selections -1).
+ */
+int oracle_decode(int B, int Hq, int Hkv, int d, int n_max, int C, int g, int topk,
+                  const float* q, const float* k_raw, const float* v_raw, const float* k_gist,
+                  const float* v_gist, const int32_t* seq_lens, int force_sel, double* scores,
+                  int32_t* sel, double* out, double* lse, int32_t* ctx) {
+    oshape s = {B, Hq, Hkv, d, n_max, C, g};
+    if (!ok_shape(&s) || topk < 0) return -1;
+    const int G = Hq / Hkv;
+    const int M_max = n_max / C;
+    int bad = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int j = 0; j < Hkv; ++j) {
+            const int n = seq_len(&s, seq_lens, b);
+            const size_t pj = (size_t)b * Hkv + j;
+            double* sc = scores ? scores + pj * M_max : NULL;
+            int32_t* sl = sel + pj * (size_t)topk;
+            if (n < 0) {
+#pragma omp critical
+                if (!bad || b + 1 < bad) bad = b + 1;
+                for (int m = 0; m < M_max && sc; ++m) sc[m] = -INFINITY;
+                if (!force_sel)
+                    for (int c = 0; c < topk; ++c) sl[c] = -1;
+                for (int gh = 0; gh < G; ++gh) {
+                    const size_t h = (size_t)b * Hq + (size_t)j * G + gh;
+                    for (int i = 0; i < d; ++i) out[h * d + i] = 0.0;
+                    if (lse) lse[h] = -INFINITY;
+                }
+                if (ctx) ctx[pj] = 0;
+                continue;
+            }
+            const int M = n / C;       /* complete chunks */
+            const int tail0 = M * C;   /* first tail token */
+            double* own = (double*)malloc(sizeof(double) * (size_t)(M_max > 0 ? M_max : 1));
+            for (int m = 0; m < M_max; ++m) own[m] = -INFINITY;
+            for (int m = 0; m < M; ++m) own[m] = chunk_score(&s, q, k_gist, b, j, m);
+            if (sc)
+                for (int m = 0; m < M_max; ++m) sc[m] = own[m];
+            int* chosen = (int*)malloc(sizeof(int) * (size_t)(topk > 0 ? topk : 1));
+            int k;
+            if (force_sel) {
+                k = 0;
+                for (int c = 0; c < topk; ++c)
+                    if (sl[c] >= 0) chosen[k++] = sl[c];
+            } else {
+                int* all = (int*)malloc(sizeof(int) * (size_t)(M > 0 ? M : 1));
+                for (int m = 0; m < M; ++m) all[m] = m;
+                k = topk_of(own, all, M, topk, chosen, topk);
+                for (int c = 0; c < topk; ++c) sl[c] = chosen[c];
+                free(all);
+            }
+            /* context list (sec. 3.3, reading above) */
+            const int cap = (M * g) + k * C + C + 8;
+            const float** ks = (const float**)malloc(sizeof(float*) * (size_t)cap);
+            const float** vs = (const float**)malloc(sizeof(float*) * (size_t)cap);
+            int nx = 0;
+            for (int m = 0; m < M; ++m) {
+                const int selected = is_in(chosen, k, m);
+                if (!selected || MUT(4)) { /* mutant 4: selected chunks keep their gists */
+                    for (int t = 0; t < g; ++t) {
+                        ks[nx] = gist_row(&s, k_gist, b, j, m, t);
+                        vs[nx] = gist_row(&s, v_gist, b, j, m, t);
+                        ++nx;
+                    }
+                }
+                if (selected) nx = push_raw(&s, k_raw, v_raw, b, j, m * C, m * C + C, ks, vs, nx);
+            }
+            if (!MUT(5)) /* mutant 5: tail dropped; mutant 7: tail starts one late */
+                nx = push_raw(&s, k_raw, v_raw, b, j, tail0 + (MUT(7) ? 1 : 0), n, ks, vs, nx);
+            if (ctx) ctx[pj] = nx;
+            for (int gh = 0; gh < G; ++gh) {
+                const size_t h = (size_t)b * Hq + (size_t)j * G + gh;
+                double l;
+                attend_list(q + h * d, d, ks, vs, nx, out + h * d, &l);
+                if (lse) lse[h] = l;
+            }
+            free(ks);
+            free(vs);
+            free(chosen);
+            free(own);
+        }
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------- two level path --- */
+
+/*
+ * oracle_decode_h2: two-level (gist-of-gist) decode step (sec. 3.5, App. B.2).
+ * Level 2 scores the S_b = floor(M_b / J) complete superchunks with their gm
+ * meta-gist keys and keeps the top topk_super; the candidates are the J
+ * children of each kept superchunk plus the remainder chunks S_b*J .. M_b-1;
+ * level 1 scores the candidates with their gist keys and keeps the top
+ * topk_chunk.  Outputs:
+ *   super_scores [B,Hkv,S_max] (-inf past S_b), chunk_scores [B,Hkv,M_max]
+ *   (-inf for non-candidates), sel_super [B,Hkv,topk_super],
+ *   sel [B,Hkv,topk_chunk], out, lse, ctx as in oracle_decode.
+ * force_sel bit 0: sel_super is given; bit 1: sel is given.
+ */
+int oracle_decode_h2(int B, int Hq, int Hkv, int d, int n_max, int C, int g, int J, int gm,
+                     int topk_super, int topk_chunk, const float* q, const float* k_raw,
+                     const float* v_raw, const float* k_gist, const float* v_gist,
+                     const float* k_meta, const float* v_meta, const int32_t* seq_lens,
+                     int force_sel, double* super_scores, double* chunk_scores,
+                     int32_t* sel_super, int32_t* sel, double* out, double* lse, int32_t* ctx) {
+    oshape s = {B, Hq, Hkv, d, n_max, C, g};
+    if (!ok_shape(&s) || J < 1 || gm < 1 || topk_super < 0 || topk_chunk < 0) return -1;
+    const int G = Hq / Hkv;
+    const int M_max = n_max / C;
+    const int S_max = M_max / J;
+    int bad = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int j = 0; j < Hkv; ++j) {
+            const int n = seq_len(&s, seq_lens, b);
+            const size_t pj = (size_t)b * Hkv + j;
+            int32_t* ss = sel_super + pj * (size_t)topk_super;
+            int32_t* sl = sel + pj * (size_t)topk_chunk;
+            double* s2 = super_scores ? super_scores + pj * (size_t)S_max : NULL;
+            double* s1 = chunk_scores ? chunk_scores + pj * (size_t)M_max : NULL;
+            if (n < 0) {
+#pragma omp critical
+                if (!bad || b + 1 < bad) bad = b + 1;
+                if (!(force_sel & 1))
+                    for (int c = 0; c < topk_super; ++c) ss[c] = -1;
+                if (!(force_sel & 2))
+                    for (int c = 0; c < topk_chunk; ++c) sl[c] = -1;
+                for (int x = 0; x < S_max && s2; ++x) s2[x] = -INFINITY;
+                for (int x = 0; x < M_max && s1; ++x) s1[x] = -INFINITY;
+                for (int gh = 0; gh < G; ++gh) {
+                    const size_t h = (size_t)b * Hq + (size_t)j * G + gh;
+                    for (int i = 0; i < d; ++i) out[h * d + i] = 0.0;
+                    if (lse) lse[h] = -INFINITY;
+                }
+                if (ctx) ctx[pj] = 0;
+                continue;
+            }
+            const int M = n / C;
+            const int S = M / J;   /* complete superchunks */
+            const int tail0 = M * C;
+            /* level 2 */
+            double* sup = (double*)malloc(sizeof(double) * (size_t)(S_max > 0 ? S_max : 1));
+            for (int x = 0; x < S_max; ++x) sup[x] = -INFINITY;
+            for (int x = 0; x < S; ++x)
+                sup[x] = super_score(&s, q, k_meta, S_max, gm, b, j, x);
+            if (s2)
+                for (int x = 0; x < S_max; ++x) s2[x] = sup[x];
+            int* ksel = (int*)malloc(sizeof(int) * (size_t)(topk_super > 0 ? topk_super : 1));
+            int ks_n;
+            if (force_sel & 1) {
+                ks_n = 0;
+                for (int c = 0; c < topk_super; ++c)
+                    if (ss[c] >= 0) ksel[ks_n++] = ss[c];
+            } else {
+                int* all = (int*)malloc(sizeof(int) * (size_t)(S > 0 ? S : 1));
+                for (int x = 0; x < S; ++x) all[x] = x;
+                ks_n = topk_of(sup, all, S, topk_super, ksel, topk_super);
+                for (int c = 0; c < topk_super; ++c) ss[c] = ksel[c];
+                free(all);
+            }
+            /* candidates, ascending */
+            int* cand = (int*)malloc(sizeof(int) * (size_t)(M > 0 ? M : 1));
+            int nc = 0;
+            for (int c = 0; c < ks_n; ++c)
+                for (int i = 0; i < J; ++i) cand[nc++] = ksel[c] * J + i;
+            for (int m = S * J; m < M; ++m) cand[nc++] = m;
+            /* level 1 */
+            double* own = (double*)malloc(sizeof(double) * (size_t)(M_max > 0 ? M_max : 1));
+            for (int m = 0; m < M_max; ++m) own[m] = -INFINITY;
+            for (int c = 0; c < nc; ++c)
+                own[cand[c]] = chunk_score(&s, q, k_gist, b, j, cand[c]);
+            if (s1)
+                for (int m = 0; m < M_max; ++m) s1[m] = own[m];
+            int* csel = (int*)malloc(sizeof(int) * (size_t)(topk_chunk > 0 ? topk_chunk : 1));
+            int kc_n;
+            if (force_sel & 2) {
+                kc_n = 0;
+                for (int c = 0; c < topk_chunk; ++c)
+                    if (sl[c] >= 0) csel[kc_n++] = sl[c];
+            } else {
+                kc_n = topk_of(own, cand, nc, topk_chunk, csel, topk_chunk);
+                for (int c = 0; c < topk_chunk; ++c) sl[c] = csel[c];
+            }
+            /* context */
+            const int cap = S * gm + nc * g + kc_n * C + C + 8;
+            const float** kx = (const float**)malloc(sizeof(float*) * (size_t)cap);
+            const float** vx = (const float**)malloc(sizeof(float*) * (size_t)cap);
+            int nx = 0;
+            for (int x = 0; x < S; ++x) {
+                if (is_in(ksel, ks_n, x)) continue;
+                for (int t = 0; t < gm; ++t) {
+                    const size_t r = ((((size_t)b * Hkv + j) * S_max + x) * gm + t) * d;
+                    kx[nx] = k_meta + r;
+                    vx[nx] = v_meta + r;
+                    ++nx;
+                }
+            }
+            for (int c = 0; c < nc; ++c) {
+                const int m = cand[c];
+                if (is_in(csel, kc_n, m)) {
+                    nx = push_raw(&s, k_raw, v_raw, b, j, m * C, m * C + C, kx, vx, nx);
+                } else {
+                    for (int t = 0; t < g; ++t) {
+                        kx[nx] = gist_row(&s, k_gist, b, j, m, t);
+                        vx[nx] = gist_row(&s, v_gist, b, j, m, t);
+                        ++nx;
+                    }
+                }
+            }
+            nx = push_raw(&s, k_raw, v_raw, b, j, tail0, n, kx, vx, nx);
+            if (ctx) ctx[pj] = nx;
+            for (int gh = 0; gh < G; ++gh) {
+                const size_t h = (size_t)b * Hq + (size_t)j * G + gh;
+                double l;
+                attend_list(q + h * d, d, kx, vx, nx, out + h * d, &l);
+                if (lse) lse[h] = l;
+            }
+            free(kx);
+            free(vx);
+            free(csel);
+            free(own);
+            free(cand);
+            free(ksel);
+            free(sup);
+        }
+    }
+    return bad;
+}
+
+int oracle_mutant_id(void) { return ORACLE_MUTANT; }

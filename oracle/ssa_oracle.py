@@ -1,0 +1,163 @@
+"""ctypes wrapper and build step for the fp64 C oracle (``ssa_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: used by ``tests/``, the package smoke check and the
+bench's CPU-baseline leg.  The product library never imports this module.
+
+The oracle follows "Simplified Sparse Attention via Gist Tokens", sec. 3.2
+(scoring against gist keys), sec. 3.3 (top-k, hybrid attention over the
+unfolded context) and sec. 3.5 / App. B.2 (two-level coarse-to-fine
+selection); the readings it takes where the pages are open are listed in the
+C file's header.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "ssa_oracle.c")
+
+
+def lib_path(mutant: int = 0, out_dir: Optional[str] = None) -> str:
+    out_dir = out_dir or HERE
+    name = "libssa_oracle.so" if mutant == 0 else f"libssa_oracle_mut{mutant}.so"
+    return os.path.join(out_dir, name)
+
+
+def build(mutant: int = 0, out_dir: Optional[str] = None, force: bool = False) -> str:
+    """Compile the oracle (optionally with one planted mutant) with gcc."""
+    out = lib_path(mutant, out_dir)
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(SRC):
+        return out
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", f"-DORACLE_MUTANT={mutant}", SRC,
+           "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+_F = ctypes.POINTER(ctypes.c_float)
+_D = ctypes.POINTER(ctypes.c_double)
+_I = ctypes.POINTER(ctypes.c_int32)
+
+
+def _f32(x) -> np.ndarray:
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu", torch.float32).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def _i32(x) -> np.ndarray:
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu").numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+
+
+def _p(a: np.ndarray, t):
+    return a.ctypes.data_as(t)
+
+
+class Oracle:
+    """Loaded oracle library (default build, or a mutant for the pin tests)."""
+
+    def __init__(self, path: Optional[str] = None, mutant: int = 0):
+        self.path = path or build(mutant)
+        self.lib = ctypes.CDLL(self.path)
+        self.lib.oracle_decode.restype = ctypes.c_int
+        self.lib.oracle_decode_h2.restype = ctypes.c_int
+        self.lib.oracle_mutant_id.restype = ctypes.c_int
+
+    @property
+    def mutant(self) -> int:
+        return int(self.lib.oracle_mutant_id())
+
+    def decode(self, q, k_raw, v_raw, k_gist, v_gist, seq_lens, C: int, g: int, topk: int,
+               sel: Optional[np.ndarray] = None) -> dict:
+        """Single-level decode step.  ``sel`` given => attend on that selection."""
+        q, k_raw, v_raw = _f32(q), _f32(k_raw), _f32(v_raw)
+        k_gist, v_gist = _f32(k_gist), _f32(v_gist)
+        lens = _i32(seq_lens)
+        B, Hq, d = q.shape
+        Hkv, n_max = k_raw.shape[1], k_raw.shape[2]
+        M_max = n_max // C
+        assert k_gist.shape == (B, Hkv, M_max, g, d), (k_gist.shape, (B, Hkv, M_max, g, d))
+        scores = np.empty((B, Hkv, M_max), np.float64)
+        out = np.empty((B, Hq, d), np.float64)
+        lse = np.empty((B, Hq), np.float64)
+        ctx = np.empty((B, Hkv), np.int32)
+        force = sel is not None
+        sel_arr = (_i32(sel).copy() if force else np.empty((B, Hkv, topk), np.int32))
+        assert sel_arr.shape == (B, Hkv, topk)
+        rc = self.lib.oracle_decode(
+            B, Hq, Hkv, d, n_max, C, g, topk, _p(q, _F), _p(k_raw, _F), _p(v_raw, _F),
+            _p(k_gist, _F), _p(v_gist, _F), _p(lens, _I), int(force), _p(scores, _D),
+            _p(sel_arr, _I), _p(out, _D), _p(lse, _D), _p(ctx, _I))
+        if rc < 0:
+            raise ValueError("oracle_decode: bad shape or topk")
+        return {"scores": scores, "sel_idx": sel_arr, "out": out, "lse": lse, "ctx": ctx,
+                "bad_seq": rc}
+
+    def decode_h2(self, q, k_raw, v_raw, k_gist, v_gist, k_meta, v_meta, seq_lens, C: int,
+                  g: int, J: int, gm: int, topk_super: int, topk_chunk: int,
+                  sel_super: Optional[np.ndarray] = None,
+                  sel: Optional[np.ndarray] = None) -> dict:
+        """Two-level decode step; given selections are used instead of top-k."""
+        q, k_raw, v_raw = _f32(q), _f32(k_raw), _f32(v_raw)
+        k_gist, v_gist = _f32(k_gist), _f32(v_gist)
+        k_meta, v_meta = _f32(k_meta), _f32(v_meta)
+        lens = _i32(seq_lens)
+        B, Hq, d = q.shape
+        Hkv, n_max = k_raw.shape[1], k_raw.shape[2]
+        M_max = n_max // C
+        S_max = M_max // J
+        assert k_meta.shape == (B, Hkv, S_max, gm, d)
+        force = 0
+        if sel_super is not None:
+            ss = _i32(sel_super).copy()
+            force |= 1
+        else:
+            ss = np.empty((B, Hkv, topk_super), np.int32)
+        if sel is not None:
+            sl = _i32(sel).copy()
+            force |= 2
+        else:
+            sl = np.empty((B, Hkv, topk_chunk), np.int32)
+        s2 = np.empty((B, Hkv, max(S_max, 1)), np.float64)
+        s1 = np.empty((B, Hkv, M_max), np.float64)
+        out = np.empty((B, Hq, d), np.float64)
+        lse = np.empty((B, Hq), np.float64)
+        ctx = np.empty((B, Hkv), np.int32)
+        rc = self.lib.oracle_decode_h2(
+            B, Hq, Hkv, d, n_max, C, g, J, gm, topk_super, topk_chunk, _p(q, _F),
+            _p(k_raw, _F), _p(v_raw, _F), _p(k_gist, _F), _p(v_gist, _F), _p(k_meta, _F),
+            _p(v_meta, _F), _p(lens, _I), force, _p(s2, _D), _p(s1, _D), _p(ss, _I),
+            _p(sl, _I), _p(out, _D), _p(lse, _D), _p(ctx, _I))
+        if rc < 0:
+            raise ValueError("oracle_decode_h2: bad shape or topk")
+        return {"super_scores": s2[:, :, :S_max], "scores": s1, "sel_super": ss, "sel_idx": sl,
+                "out": out, "lse": lse, "ctx": ctx, "bad_seq": rc}
+
+
+_default: Optional[Oracle] = None
+
+
+def default() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default

@@ -1,0 +1,313 @@
+"""Pins for the fp64 oracle: checks against things other than the oracle itself.
+
+Each ``pin_*`` function takes an ``oracle.ssa_oracle.Oracle`` and raises
+``AssertionError`` when the oracle disagrees with
+  * the independent numpy brute force (dense matmul scoring, k-subset
+    enumeration for top-k, explicit token list + one dense softmax),
+  * textbook attention from ``torch.nn.functional.scaled_dot_product_attention``
+    in fp64 (the k = M and k = 0 invariants of the method),
+  * closed forms (one visible token, all keys equal, a query parallel to one
+    gist key, the context-size identity),
+  * the hand-worked example in ``tests/golden/hand_example.json``.
+The same pins run against every planted mutant of the oracle; each mutant must
+fail at least one of them.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+from oracle import bruteforce
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, lens, J=0, gm=0):
+    M_max = n_max // C
+    case = {
+        "q": rng.standard_normal((B, Hq, d)).astype(np.float32),
+        "k_raw": rng.standard_normal((B, Hkv, n_max, d)).astype(np.float32),
+        "v_raw": rng.standard_normal((B, Hkv, n_max, d)).astype(np.float32),
+        "k_gist": rng.standard_normal((B, Hkv, M_max, g, d)).astype(np.float32),
+        "v_gist": rng.standard_normal((B, Hkv, M_max, g, d)).astype(np.float32),
+        "seq_lens": np.asarray(lens, np.int32),
+    }
+    if J:
+        S_max = M_max // J
+        case["k_meta"] = rng.standard_normal((B, Hkv, S_max, gm, d)).astype(np.float32)
+        case["v_meta"] = rng.standard_normal((B, Hkv, S_max, gm, d)).astype(np.float32)
+    return case
+
+
+def _args(c):
+    return (c["q"], c["k_raw"], c["v_raw"], c["k_gist"], c["v_gist"], c["seq_lens"])
+
+
+def _close(a, b, tol=1e-10, what=""):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    assert a.shape == b.shape, (what, a.shape, b.shape)
+    fin = np.isfinite(b)
+    assert np.array_equal(np.isfinite(a), fin), f"{what}: finiteness differs"
+    assert np.array_equal(a[~fin], b[~fin]), f"{what}: infinities differ"
+    err = np.abs(a[fin] - b[fin]).max() if fin.any() else 0.0
+    assert err <= tol, f"{what}: max abs err {err:g} > {tol:g}"
+
+
+# single-level shapes: (B, Hq, Hkv, d, C, g, n_max, seq_lens, topk)
+SINGLE_CASES = [
+    (1, 1, 1, 8, 4, 2, 32, [27], 3),
+    (2, 4, 2, 8, 4, 2, 40, [40, 33], 4),
+    (2, 8, 2, 16, 8, 2, 64, [61, 9], 2),
+    (1, 6, 3, 8, 5, 3, 50, [49], 5),
+    (2, 4, 1, 8, 4, 1, 24, [23, 3], 0),
+    (1, 2, 2, 8, 3, 2, 30, [30], 20),   # topk > M: select all
+    (2, 4, 2, 8, 4, 2, 16, [2, 16], 2), # M = 0 for one sequence
+]
+
+
+def pin_bruteforce_single(orc):
+    rng = np.random.default_rng(1234)
+    for (B, Hq, Hkv, d, C, g, n_max, lens, topk) in SINGLE_CASES:
+        c = _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, lens)
+        o = orc.decode(*_args(c), C=C, g=g, topk=topk)
+        r = bruteforce.decode(*_args(c), C=C, g=g, topk=topk)
+        _close(o["scores"], r["scores"], 1e-12, "scores")
+        assert np.array_equal(o["sel_idx"], r["sel_idx"]), ("sel", o["sel_idx"], r["sel_idx"])
+        assert np.array_equal(o["ctx"], r["ctx"]), ("ctx", o["ctx"], r["ctx"])
+        _close(o["out"], r["out"], 1e-12, "out")
+        _close(o["lse"], r["lse"], 1e-12, "lse")
+
+
+def pin_given_selection(orc):
+    """Attention on a given (non top-k) selection equals the brute force's."""
+    rng = np.random.default_rng(99)
+    B, Hq, Hkv, d, C, g, n_max, topk = 2, 4, 2, 8, 4, 2, 40, 3
+    c = _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, [38, 21])
+    sel = np.full((B, Hkv, topk), -1, np.int32)
+    sel[0, 0, :3] = [0, 4, 8]
+    sel[0, 1, :1] = [7]
+    sel[1, 0, :2] = [1, 2]
+    o = orc.decode(*_args(c), C=C, g=g, topk=topk, sel=sel)
+    r = bruteforce.decode(*_args(c), C=C, g=g, topk=topk, sel=sel)
+    assert np.array_equal(o["sel_idx"], sel)
+    _close(o["out"], r["out"], 1e-12, "out")
+    assert np.array_equal(o["ctx"], r["ctx"])
+
+
+def pin_ties(orc):
+    """Equal scores go to the lower chunk index."""
+    rng = np.random.default_rng(7)
+    B, Hq, Hkv, d, C, g, n_max = 1, 2, 1, 8, 4, 2, 32
+    c = _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, [32])
+    # chunk 5 is a copy of chunk 2 and both beat every other chunk
+    q = c["q"][0]
+    boost = (q.sum(0) / np.linalg.norm(q.sum(0))).astype(np.float32) * 6.0
+    c["k_gist"][0, 0, 2, 0] = boost
+    c["k_gist"][0, 0, 5] = c["k_gist"][0, 0, 2]
+    o = orc.decode(*_args(c), C=C, g=g, topk=1)
+    assert o["scores"][0, 0, 2] == o["scores"][0, 0, 5]
+    assert list(o["sel_idx"][0, 0]) == [2], o["sel_idx"]
+    o3 = orc.decode(*_args(c), C=C, g=g, topk=2)
+    assert list(o3["sel_idx"][0, 0]) == [2, 5], o3["sel_idx"]
+    # all gist keys equal -> all scores equal -> chunks 0..k-1
+    c["k_gist"][:] = c["k_gist"][0, 0, 0, 0]
+    o = orc.decode(*_args(c), C=C, g=g, topk=3)
+    assert list(o["sel_idx"][0, 0]) == [0, 1, 2], o["sel_idx"]
+    r = bruteforce.decode(*_args(c), C=C, g=g, topk=3)
+    assert np.array_equal(o["sel_idx"], r["sel_idx"])
+
+
+def _sdpa(qh, K, V):
+    """Textbook softmax attention of one query from torch (fp64)."""
+    qt = torch.from_numpy(np.asarray(qh, np.float64))[None, None, None, :]
+    Kt = torch.from_numpy(np.asarray(K, np.float64))[None, None]
+    Vt = torch.from_numpy(np.asarray(V, np.float64))[None, None]
+    out = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt)
+    logits = (Kt[0, 0] @ qt[0, 0, 0]) / math.sqrt(qh.shape[-1])
+    return out[0, 0, 0].numpy(), torch.logsumexp(logits, 0).item()
+
+
+def pin_dense_when_all_selected(orc):
+    """k >= M  =>  dense causal attention over all n raw tokens."""
+    rng = np.random.default_rng(5)
+    B, Hq, Hkv, d, C, g, n_max = 2, 4, 2, 16, 4, 2, 48
+    lens = [45, 17]
+    c = _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, lens)
+    o = orc.decode(*_args(c), C=C, g=g, topk=n_max // C)
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            j = h // G
+            ref, l = _sdpa(c["q"][b, h], c["k_raw"][b, j, :lens[b]], c["v_raw"][b, j, :lens[b]])
+            _close(o["out"][b, h], ref, 1e-12, "dense out")
+            _close(o["lse"][b, h], l, 1e-12, "dense lse")
+
+
+def pin_gists_when_none_selected(orc):
+    """k = 0  =>  attention over all gists of complete chunks plus the tail."""
+    rng = np.random.default_rng(6)
+    B, Hq, Hkv, d, C, g, n_max = 2, 4, 2, 16, 4, 3, 48
+    lens = [47, 12]
+    c = _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, lens)
+    o = orc.decode(*_args(c), C=C, g=g, topk=0)
+    G = Hq // Hkv
+    for b in range(B):
+        M = lens[b] // C
+        for h in range(Hq):
+            j = h // G
+            K = np.concatenate([c["k_gist"][b, j, :M].reshape(M * g, d),
+                                c["k_raw"][b, j, M * C:lens[b]]])
+            V = np.concatenate([c["v_gist"][b, j, :M].reshape(M * g, d),
+                                c["v_raw"][b, j, M * C:lens[b]]])
+            ref, l = _sdpa(c["q"][b, h], K, V)
+            _close(o["out"][b, h], ref, 1e-12, "gist-only out")
+            _close(o["lse"][b, h], l, 1e-12, "gist-only lse")
+
+
+def pin_single_token(orc):
+    """n = 1: the context is the one raw token, so out = its value exactly."""
+    rng = np.random.default_rng(8)
+    c = _rand_case(rng, 1, 2, 1, 8, 4, 2, 8, [1])
+    o = orc.decode(*_args(c), C=4, g=2, topk=2)
+    for h in range(2):
+        assert np.array_equal(o["out"][0, h], c["v_raw"][0, 0, 0].astype(np.float64))
+    assert list(o["sel_idx"][0, 0]) == [-1, -1]
+    assert o["ctx"][0, 0] == 1
+
+
+def pin_equal_keys_mean(orc):
+    """All keys equal => uniform softmax => out = mean of the context's values."""
+    rng = np.random.default_rng(9)
+    B, Hq, Hkv, d, C, g, n_max, n = 1, 2, 1, 8, 4, 2, 28, 26
+    c = _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, [n])
+    key = rng.standard_normal(d).astype(np.float32)
+    c["k_raw"][:] = key
+    c["k_gist"][:] = key
+    sel = np.array([[[1, 4]]], np.int32)
+    o = orc.decode(*_args(c), C=C, g=g, topk=2, sel=sel)
+    M = n // C
+    vals = [c["v_gist"][0, 0, m] for m in range(M) if m not in (1, 4)]
+    vals += [c["v_raw"][0, 0, 4:8], c["v_raw"][0, 0, 16:20], c["v_raw"][0, 0, M * C:n]]
+    mean = np.concatenate(vals).astype(np.float64).mean(0)
+    for h in range(Hq):
+        _close(o["out"][0, h], mean, 1e-12, "equal-keys mean")
+
+
+def pin_context_size(orc):
+    """|X| = (M - k) g + k C + T for every (sequence, KV head)."""
+    rng = np.random.default_rng(10)
+    for (B, Hq, Hkv, d, C, g, n_max, lens, topk) in SINGLE_CASES:
+        c = _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, lens)
+        o = orc.decode(*_args(c), C=C, g=g, topk=topk)
+        for b in range(B):
+            M = lens[b] // C
+            k = min(topk, M)
+            T = lens[b] - M * C
+            assert (o["ctx"][b] == (M - k) * g + k * C + T).all(), (b, o["ctx"][b])
+
+
+def pin_parallel_query(orc):
+    """q = a*e for one head, one nonzero gist key e: that chunk scores a|e|^2/sqrt(d)."""
+    B, Hq, Hkv, d, C, g, n_max = 1, 4, 1, 16, 4, 2, 32
+    z = lambda *s: np.zeros(s, np.float32)
+    c = {"q": z(B, Hq, d), "k_raw": z(B, Hkv, n_max, d), "v_raw": z(B, Hkv, n_max, d),
+         "k_gist": z(B, Hkv, n_max // C, g, d), "v_gist": z(B, Hkv, n_max // C, g, d),
+         "seq_lens": np.array([32], np.int32)}
+    e = np.zeros(d, np.float32)
+    e[3], e[7] = 1.5, -2.0
+    c["k_gist"][0, 0, 6, 1] = e
+    c["q"][0, 2] = 3.0 * e
+    o = orc.decode(*_args(c), C=C, g=g, topk=1)
+    want = 3.0 * float(e @ e) / math.sqrt(d)
+    assert abs(o["scores"][0, 0, 6] - want) <= 1e-12, (o["scores"][0, 0, 6], want)
+    others = np.delete(o["scores"][0, 0], 6)
+    assert (others == 0.0).all()
+    assert list(o["sel_idx"][0, 0]) == [6]
+
+
+def pin_hand_example(orc):
+    """The hand-worked example in tests/golden/hand_example.json."""
+    with open(os.path.join(GOLDEN, "hand_example.json")) as f:
+        ex = json.load(f)
+    s = ex["shape"]
+    arr = lambda k: np.asarray(ex[k], np.float32)
+    o = orc.decode(arr("q"), arr("k_raw"), arr("v_raw"), arr("k_gist"), arr("v_gist"),
+                   np.asarray(ex["seq_lens"], np.int32), C=s["C"], g=s["g"], topk=s["topk"])
+    e = ex["expected"]
+    want_scores = [float(x) for x in e["scores"]]
+    _close(o["scores"][0, 0], want_scores, 1e-15, "hand scores")
+    assert list(o["sel_idx"][0, 0]) == e["sel_idx"]
+    assert int(o["ctx"][0, 0]) == e["ctx"]
+    w = np.exp(np.asarray(e["context_logits"], np.float64))
+    vals = np.asarray(e["context_values"], np.float64)
+    want = (w[:, None] * vals).sum(0) / w.sum()
+    _close(o["out"][0, 0], want, 1e-15, "hand out")
+    _close(o["lse"][0, 0], math.log(w.sum()), 1e-15, "hand lse")
+
+
+H2_CASES = [
+    # (B, Hq, Hkv, d, C, g, n_max, lens, J, gm, topk_super, topk_chunk)
+    (1, 2, 1, 8, 4, 2, 96, [93], 4, 2, 2, 3),      # S=5, R=3 remainder chunks, tail 1
+    (2, 4, 2, 8, 2, 1, 64, [64, 37], 3, 2, 1, 2),  # remainder + tails
+    (1, 4, 1, 8, 4, 2, 64, [64], 4, 3, 0, 2),      # no superchunk kept: remainder only
+]
+
+
+def pin_bruteforce_h2(orc):
+    rng = np.random.default_rng(4321)
+    for (B, Hq, Hkv, d, C, g, n_max, lens, J, gm, ts, tc) in H2_CASES:
+        c = _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, lens, J=J, gm=gm)
+        args = _args(c)[:5] + (c["k_meta"], c["v_meta"], c["seq_lens"])
+        o = orc.decode_h2(*args, C=C, g=g, J=J, gm=gm, topk_super=ts, topk_chunk=tc)
+        r = bruteforce.decode_h2(*args, C=C, g=g, J=J, gm=gm, topk_super=ts, topk_chunk=tc)
+        _close(o["super_scores"], r["super_scores"], 1e-12, "h2 super scores")
+        _close(o["scores"], r["scores"], 1e-12, "h2 chunk scores")
+        assert np.array_equal(o["sel_super"], r["sel_super"]), (o["sel_super"], r["sel_super"])
+        assert np.array_equal(o["sel_idx"], r["sel_idx"]), (o["sel_idx"], r["sel_idx"])
+        assert np.array_equal(o["ctx"], r["ctx"])
+        _close(o["out"], r["out"], 1e-12, "h2 out")
+        _close(o["lse"], r["lse"], 1e-12, "h2 lse")
+
+
+def pin_h2_reduces_to_single(orc):
+    """Keeping every superchunk makes the two-level step the single-level one."""
+    rng = np.random.default_rng(11)
+    B, Hq, Hkv, d, C, g, n_max, J, gm = 2, 4, 2, 8, 4, 2, 96, 3, 2
+    lens = [95, 50]
+    c = _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, lens, J=J, gm=gm)
+    args = _args(c)[:5] + (c["k_meta"], c["v_meta"], c["seq_lens"])
+    o2 = orc.decode_h2(*args, C=C, g=g, J=J, gm=gm, topk_super=100, topk_chunk=4)
+    o1 = orc.decode(*_args(c), C=C, g=g, topk=4)
+    assert np.array_equal(o2["sel_idx"], o1["sel_idx"])
+    _close(o2["out"], o1["out"], 1e-12, "h2->single out")
+    # and with every chunk kept too: dense attention
+    o3 = orc.decode_h2(*args, C=C, g=g, J=J, gm=gm, topk_super=100, topk_chunk=100)
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            ref, _ = _sdpa(c["q"][b, h], c["k_raw"][b, h // G, :lens[b]],
+                           c["v_raw"][b, h // G, :lens[b]])
+            _close(o3["out"][b, h], ref, 1e-12, "h2 dense")
+
+
+def pin_bad_length(orc):
+    """A length outside [1, n_max] is reported and zeroes that sequence."""
+    rng = np.random.default_rng(12)
+    c = _rand_case(rng, 2, 2, 1, 8, 4, 2, 16, [16, 17])
+    o = orc.decode(*_args(c), C=4, g=2, topk=2)
+    assert o["bad_seq"] == 2
+    assert (o["out"][1] == 0).all() and (o["sel_idx"][1] == -1).all()
+    assert np.isfinite(o["out"][0]).all() and (o["sel_idx"][0] >= 0).all()
+
+
+ALL_PINS = [
+    pin_bruteforce_single, pin_given_selection, pin_ties, pin_dense_when_all_selected,
+    pin_gists_when_none_selected, pin_single_token, pin_equal_keys_mean, pin_context_size,
+    pin_parallel_query, pin_hand_example, pin_bruteforce_h2, pin_h2_reduces_to_single,
+    pin_bad_length,
+]
