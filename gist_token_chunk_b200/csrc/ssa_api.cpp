@@ -1,0 +1,482 @@
+// ssa_api.cpp -- the C ABI of libssa (include/ssa.h): argument checks, work
+// planning, workspace handling and dispatch to the kernels.  Never throws
+// across the boundary; never synchronises the host in the hot calls.
+#include "../../include/ssa.h"
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <unordered_map>
+
+#include "ssa_internal.h"
+
+namespace ssa {
+int fused_smem_bytes(const Plan& p);
+}
+
+namespace {
+
+thread_local std::string g_err;
+std::atomic<long long> g_wait_limit{0};
+std::atomic<int> g_debug{0};
+std::atomic<int> g_units_per_item{0};
+std::atomic<int> g_rows_per_score{0};
+
+constexpr long long kDefaultWaitLimitNs = 2000000000ll;  // 2 s
+constexpr int kMaxG = 16;
+constexpr int kMaxTopk = 1024;
+constexpr int kRowsPerScoreItem = 512;
+constexpr int kUnitsPerAttnItem = 6;
+
+int rows_per_score_item() {
+    int v = g_rows_per_score.load();
+    return v > 0 ? v : kRowsPerScoreItem;
+}
+int units_per_attn_item() {
+    int v = g_units_per_item.load();
+    return v > 0 ? v : kUnitsPerAttnItem;
+}
+constexpr int kMaxAttnItems = 1024;
+
+ssa_status fail(ssa_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+ssa_status fail(ssa_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return s;
+}
+
+ssa_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(SSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// Common shape checks.  need_d: check d/dtype (not needed by top-k).
+ssa_status check_shape(const ssa_shape* s, int C, bool need_d) {
+    if (!s) return fail(SSA_ERR_INVALID_ARG, "shape is NULL");
+    if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->n_max < 1)
+        return fail(SSA_ERR_INVALID_ARG, "B, Hq, Hkv, n_max must be >= 1");
+    if (s->Hq % s->Hkv) return fail(SSA_ERR_INVALID_ARG, "Hq (%d) not a multiple of Hkv (%d)",
+                                    s->Hq, s->Hkv);
+    if (s->Hq / s->Hkv > kMaxG)
+        return fail(SSA_ERR_UNSUPPORTED, "group size Hq/Hkv = %d > %d", s->Hq / s->Hkv, kMaxG);
+    if (C < 1) return fail(SSA_ERR_INVALID_ARG, "C must be >= 1");
+    if (s->n_max % C) return fail(SSA_ERR_INVALID_ARG, "n_max (%d) not a multiple of C (%d)",
+                                  s->n_max, C);
+    if (need_d) {
+        if (s->dtype == SSA_BF16) {
+            if (s->d != 64 && s->d != 128)
+                return fail(SSA_ERR_UNSUPPORTED, "bf16 needs d in {64, 128}, got %d", s->d);
+        } else if (s->dtype == SSA_FP32) {
+            if (s->d < 1 || s->d > 256)
+                return fail(SSA_ERR_UNSUPPORTED, "fp32 needs 1 <= d <= 256, got %d", s->d);
+        } else {
+            return fail(SSA_ERR_INVALID_ARG, "unknown dtype %d", s->dtype);
+        }
+    }
+    const long long P = (long long)s->B * s->Hkv;
+    if (P * s->n_max >= (1ll << 31))
+        return fail(SSA_ERR_UNSUPPORTED, "B*Hkv*n_max too large for 32-bit row indices");
+    return SSA_OK;
+}
+
+// Fill shapes of a plan (no pointers).
+void fill_shape(ssa::Plan& p, const ssa_shape* s, int C, int g, int topk) {
+    p.dtype = s->dtype;
+    p.B = s->B;
+    p.Hq = s->Hq;
+    p.Hkv = s->Hkv;
+    p.G = s->Hq / s->Hkv;
+    p.d = s->d;
+    p.n_max = s->n_max;
+    p.C = C;
+    p.g = g;
+    p.M_max = s->n_max / C;
+    p.topk = topk;
+    p.n_pairs = s->B * s->Hkv;
+    long long lim = g_wait_limit.load();
+    p.wait_limit = lim > 0 ? lim : kDefaultWaitLimitNs;
+    p.debug_flags = g_debug.load();
+}
+
+bool fused_path(const ssa::Plan& p) { return p.dtype == SSA_BF16 && (p.d == 64 || p.d == 128); }
+
+ssa_status check_sizes(const ssa::Plan& p) {
+    const long long P = p.n_pairs;
+    if (P * p.M_max * (long long)p.g >= (1ll << 31))
+        return fail(SSA_ERR_UNSUPPORTED, "gist rows too large for 32-bit row indices");
+    if (p.g > 1024) return fail(SSA_ERR_UNSUPPORTED, "g = %d > 1024", p.g);
+    if (p.topk > kMaxTopk) return fail(SSA_ERR_UNSUPPORTED, "topk = %d > %d", p.topk, kMaxTopk);
+    if (p.h2) {
+        if (P * p.S_max * (long long)p.gm >= (1ll << 31))
+            return fail(SSA_ERR_UNSUPPORTED, "meta rows too large for 32-bit row indices");
+        if (p.gm > 1024) return fail(SSA_ERR_UNSUPPORTED, "gm = %d > 1024", p.gm);
+        if ((long long)p.J * p.g > 1024)
+            return fail(SSA_ERR_UNSUPPORTED, "J*g = %lld > 1024", (long long)p.J * p.g);
+        if (p.topk_super > kMaxTopk)
+            return fail(SSA_ERR_UNSUPPORTED, "topk_super = %d > %d", p.topk_super, kMaxTopk);
+    }
+    if (fused_path(p) && ssa::fused_smem_bytes(p) > 227 * 1024)
+        return fail(SSA_ERR_UNSUPPORTED, "shared memory plan too large");
+    return SSA_OK;
+}
+
+}  // namespace
+
+namespace ssa {
+
+void plan_decompose(Plan& p) {
+    const int ntok = p.h2 ? p.gm : p.g;
+    const int slots = p.h2 ? p.S_max : p.M_max;
+    int spi = rows_per_score_item() / (ntok > 0 ? ntok : 1);
+    if (spi < 1) spi = 1;
+    if (spi * ntok > 1024) spi = 1024 / ntok;
+    if (spi < 1) spi = 1;
+    p.score_spi = spi;
+    p.score_items = slots > 0 ? cdiv(slots, spi) : 1;
+    p.cand_items = p.h2 ? p.topk_super + 1 : 0;
+    // attention units of the largest possible sequence
+    const int tpc = cdiv(p.C, 64);
+    const int tail_units = cdiv(p.C - 1, 64);
+    long long U;
+    if (!p.h2) {
+        const int kmax = p.topk < p.M_max ? p.topk : p.M_max;
+        U = cdiv((long long)p.M_max * p.g, 64) + (long long)kmax * tpc + tail_units;
+    } else {
+        const int ks = p.topk_super < p.S_max ? p.topk_super : p.S_max;
+        const long long nc = (long long)ks * p.J + (p.J - 1);
+        const long long kc = p.topk < nc ? p.topk : nc;
+        U = cdiv((long long)p.S_max * p.gm, 64) + (long long)ks * cdiv((long long)p.J * p.g, 64) +
+            cdiv((long long)(p.J - 1) * p.g, 64) + kc * tpc + tail_units;
+    }
+    const int upi = units_per_attn_item();
+    int items = (int)((U + upi - 1) / upi);
+    if (items < 1) items = 1;
+    if (items > kMaxAttnItems) items = kMaxAttnItems;
+    p.attn_items = items;
+    p.mask_words = (cdiv(p.M_max, 32) + 3) / 4 * 4;
+    p.smask_words = p.h2 ? (cdiv(p.S_max, 32) + 3) / 4 * 4 : 0;
+}
+
+int ctrl_words(const Plan& p) { return 2 + 8 * p.n_pairs; }
+
+WsLayout plan_layout(const Plan& p) {
+    WsLayout L;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o += (bytes + 255) / 256 * 256;
+        return at;
+    };
+    const size_t P = (size_t)p.n_pairs;
+    L.ctrl = take((size_t)ctrl_words(p) * 4);
+    L.scores = take(P * p.M_max * 4);
+    L.super_scores = take(p.h2 ? P * p.S_max * 4 : 0);
+    L.cand_scores = take(p.h2 ? P * p.Mc_max * 4 : 0);
+    L.chunk_mask = take(0);
+    L.super_mask = take(0);
+    L.partials = take(fused_path(p) ? P * p.attn_items * p.G * (p.d + 2) * 4 : 0);
+    L.total = o;
+    return L;
+}
+
+}  // namespace ssa
+
+namespace {
+
+void attach_ws(ssa::Plan& p, void* ws) {
+    const ssa::WsLayout L = ssa::plan_layout(p);
+    char* base = static_cast<char*>(ws);
+    p.ctrl = reinterpret_cast<int*>(base + L.ctrl);
+    p.scores = reinterpret_cast<float*>(base + L.scores);
+    p.super_scores = p.h2 ? reinterpret_cast<float*>(base + L.super_scores) : nullptr;
+    p.cand_scores = p.h2 ? reinterpret_cast<float*>(base + L.cand_scores) : nullptr;
+    p.partials = reinterpret_cast<float*>(base + L.partials);
+}
+
+// Control words are left zero by every call, but only the control region of
+// that call's size.  A later call with more (sequence, KV head) pairs has a
+// larger control region that may cover scratch data of earlier calls, so the
+// library remembers the control size each workspace was last used with and
+// zeroes the region (stream-ordered) only when it grows.
+std::mutex g_ws_mu;
+std::unordered_map<const void*, size_t> g_ws_ctrl;
+
+void note_ws_zeroed(const void* ws, size_t bytes) {
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    g_ws_ctrl[ws] = bytes;
+}
+
+cudaError_t prepare_ctrl(void* ws, size_t ctrl_bytes, cudaStream_t stream) {
+    bool zero = false;
+    {
+        std::lock_guard<std::mutex> lk(g_ws_mu);
+        auto it = g_ws_ctrl.find(ws);
+        if (it == g_ws_ctrl.end()) {
+            g_ws_ctrl[ws] = ctrl_bytes;  // first use: the caller zeroed it
+        } else {
+            zero = ctrl_bytes > it->second;
+            it->second = ctrl_bytes;
+        }
+    }
+    return zero ? cudaMemsetAsync(ws, 0, ctrl_bytes, stream) : cudaSuccess;
+}
+
+// Runs a workspace-using plan: caller workspace, or a stream-ordered one.
+ssa_status run_with_ws(ssa::Plan& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    const size_t need = ssa::plan_layout(p).total;
+    void* own = nullptr;
+    if (ws == nullptr) {
+        if (ws_bytes != 0) return fail(SSA_ERR_WORKSPACE, "ws is NULL but ws_bytes != 0");
+        cudaError_t e = cudaMallocAsync(&own, need, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+        e = cudaMemsetAsync(own, 0, need, stream);
+        if (e != cudaSuccess) {
+            cudaFreeAsync(own, stream);
+            return cuda_fail(e, "cudaMemsetAsync(workspace)");
+        }
+        ws = own;
+    } else if (ws_bytes < need) {
+        return fail(SSA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+    } else if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) {
+        return fail(SSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    }
+    attach_ws(p, ws);
+    if (!own) {
+        cudaError_t e = prepare_ctrl(ws, (size_t)ssa::ctrl_words(p) * 4, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(control words)");
+    }
+    cudaError_t e = fused_path(p) ? ssa::launch_fused(p, stream) : ssa::launch_generic(p, stream);
+    if (own) cudaFreeAsync(own, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return SSA_OK;
+}
+
+ssa_status check_tensors(const ssa::Plan& p, std::initializer_list<const void*> ptrs) {
+    for (const void* q : ptrs)
+        if (!q) return fail(SSA_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (fused_path(p))
+        for (const void* q : ptrs)
+            if (!aligned16(q)) return fail(SSA_ERR_UNSUPPORTED, "bf16 tensors must be 16-byte aligned");
+    return SSA_OK;
+}
+
+ssa_status build_single(ssa::Plan& p, const ssa_shape* shape, int C, int g, int topk) {
+    ssa_status st = check_shape(shape, C, true);
+    if (st != SSA_OK) return st;
+    if (g < 1) return fail(SSA_ERR_INVALID_ARG, "g must be >= 1");
+    if (topk < 0) return fail(SSA_ERR_INVALID_ARG, "topk must be >= 0");
+    fill_shape(p, shape, C, g, topk);
+    ssa::plan_decompose(p);
+    return check_sizes(p);
+}
+
+ssa_status build_h2(ssa::Plan& p, const ssa_shape* shape, int C, int g, int J, int gm,
+                    int topk_super, int topk_chunk) {
+    ssa_status st = check_shape(shape, C, true);
+    if (st != SSA_OK) return st;
+    if (g < 1 || J < 1 || gm < 1) return fail(SSA_ERR_INVALID_ARG, "g, J, gm must be >= 1");
+    if (topk_super < 0 || topk_chunk < 0)
+        return fail(SSA_ERR_INVALID_ARG, "topk_super, topk_chunk must be >= 0");
+    fill_shape(p, shape, C, g, topk_chunk);
+    p.h2 = 1;
+    p.J = J;
+    p.gm = gm;
+    p.S_max = p.M_max / J;
+    p.topk_super = topk_super;
+    const int ks = topk_super < p.S_max ? topk_super : p.S_max;
+    long long mc = (long long)ks * J + (J - 1);
+    if (mc > p.M_max) mc = p.M_max;
+    p.Mc_max = (int)(mc > 0 ? mc : 1);
+    ssa::plan_decompose(p);
+    return check_sizes(p);
+}
+
+}  // namespace
+
+extern "C" {
+
+ssa_status ssa_score_gists(const ssa_shape* shape, const void* q, const void* k_gist,
+                           const int32_t* seq_lens, int32_t C, int32_t g, float* scores,
+                           cudaStream_t stream) {
+    ssa::Plan p;
+    ssa_status st = build_single(p, shape, C, g, 0);
+    if (st != SSA_OK) return st;
+    st = check_tensors(p, {q, k_gist, seq_lens, scores});
+    if (st != SSA_OK) return st;
+    p.mode = ssa::kModeScoreOnly;
+    p.q = q;
+    p.k_gist = k_gist;
+    p.k_raw = k_gist;  // unused by scoring; any valid map base
+    p.v_raw = k_gist;
+    p.v_gist = k_gist;
+    p.seq_lens = seq_lens;
+    p.scores = scores;
+    cudaError_t e = fused_path(p) ? ssa::launch_fused(p, stream) : ssa::launch_generic(p, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "ssa_score_gists launch");
+    return SSA_OK;
+}
+
+ssa_status ssa_topk_chunks(const ssa_shape* shape, const float* scores, const int32_t* seq_lens,
+                           int32_t C, int32_t topk, int32_t* sel_idx, cudaStream_t stream) {
+    ssa_status st = check_shape(shape, C, false);
+    if (st != SSA_OK) return st;
+    if (topk < 0) return fail(SSA_ERR_INVALID_ARG, "topk must be >= 0");
+    if (!scores || !seq_lens || !sel_idx) return fail(SSA_ERR_INVALID_ARG, "NULL pointer");
+    if (topk == 0) return SSA_OK;
+    ssa::Plan p;
+    fill_shape(p, shape, C, 1, topk);
+    p.seq_lens = seq_lens;
+    p.sel_idx = sel_idx;
+    cudaError_t e = ssa::launch_topk(p, scores, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "ssa_topk_chunks launch");
+    return SSA_OK;
+}
+
+ssa_status ssa_sparse_decode(const ssa_shape* shape, const void* q, const void* k_raw,
+                             const void* v_raw, const void* k_gist, const void* v_gist,
+                             const int32_t* seq_lens, int32_t C, int32_t g, int32_t topk,
+                             const int32_t* sel_idx, float* out, void* ws, size_t ws_bytes,
+                             cudaStream_t stream) {
+    ssa::Plan p;
+    ssa_status st = build_single(p, shape, C, g, topk);
+    if (st != SSA_OK) return st;
+    st = check_tensors(p, {q, k_raw, v_raw, k_gist, v_gist, seq_lens, out});
+    if (st != SSA_OK) return st;
+    if (topk > 0 && !sel_idx) return fail(SSA_ERR_INVALID_ARG, "sel_idx is NULL");
+    p.mode = ssa::kModeAttnOnly;
+    p.q = q;
+    p.k_raw = k_raw;
+    p.v_raw = v_raw;
+    p.k_gist = k_gist;
+    p.v_gist = v_gist;
+    p.seq_lens = seq_lens;
+    p.sel_idx = const_cast<int32_t*>(sel_idx);
+    p.out = out;
+    return run_with_ws(p, ws, ws_bytes, stream);
+}
+
+ssa_status ssa_decode(const ssa_shape* shape, const void* q, const void* k_raw, const void* v_raw,
+                      const void* k_gist, const void* v_gist, const int32_t* seq_lens, int32_t C,
+                      int32_t g, int32_t topk, float* out, int32_t* sel_idx, void* ws,
+                      size_t ws_bytes, cudaStream_t stream) {
+    ssa::Plan p;
+    ssa_status st = build_single(p, shape, C, g, topk);
+    if (st != SSA_OK) return st;
+    st = check_tensors(p, {q, k_raw, v_raw, k_gist, v_gist, seq_lens, out});
+    if (st != SSA_OK) return st;
+    if (topk > 0 && !sel_idx) return fail(SSA_ERR_INVALID_ARG, "sel_idx is NULL");
+    p.mode = ssa::kModeFull;
+    p.q = q;
+    p.k_raw = k_raw;
+    p.v_raw = v_raw;
+    p.k_gist = k_gist;
+    p.v_gist = v_gist;
+    p.seq_lens = seq_lens;
+    p.sel_idx = sel_idx;
+    p.out = out;
+    return run_with_ws(p, ws, ws_bytes, stream);
+}
+
+ssa_status ssa_decode_h2(const ssa_shape* shape, const void* q, const void* k_raw,
+                         const void* v_raw, const void* k_gist, const void* v_gist,
+                         const void* k_meta, const void* v_meta, const int32_t* seq_lens,
+                         int32_t C, int32_t g, int32_t J, int32_t gm, int32_t topk_super,
+                         int32_t topk_chunk, float* out, int32_t* sel_super, int32_t* sel_idx,
+                         void* ws, size_t ws_bytes, cudaStream_t stream) {
+    ssa::Plan p;
+    ssa_status st = build_h2(p, shape, C, g, J, gm, topk_super, topk_chunk);
+    if (st != SSA_OK) return st;
+    st = check_tensors(p, {q, k_raw, v_raw, k_gist, v_gist, k_meta, v_meta, seq_lens, out});
+    if (st != SSA_OK) return st;
+    if ((topk_super > 0 && !sel_super) || (topk_chunk > 0 && !sel_idx))
+        return fail(SSA_ERR_INVALID_ARG, "selection output is NULL");
+    p.mode = ssa::kModeFull;
+    p.q = q;
+    p.k_raw = k_raw;
+    p.v_raw = v_raw;
+    p.k_gist = k_gist;
+    p.v_gist = v_gist;
+    p.k_meta = k_meta;
+    p.v_meta = v_meta;
+    p.seq_lens = seq_lens;
+    p.sel_idx = sel_idx;
+    p.sel_super = sel_super;
+    p.out = out;
+    return run_with_ws(p, ws, ws_bytes, stream);
+}
+
+ssa_status ssa_workspace_size(const ssa_shape* shape, int32_t C, int32_t g, int32_t topk,
+                              size_t* bytes) {
+    if (!bytes) return fail(SSA_ERR_INVALID_ARG, "bytes is NULL");
+    ssa::Plan p;
+    ssa_status st = build_single(p, shape, C, g, topk);
+    if (st != SSA_OK) return st;
+    *bytes = ssa::plan_layout(p).total;
+    return SSA_OK;
+}
+
+ssa_status ssa_workspace_size_h2(const ssa_shape* shape, int32_t C, int32_t g, int32_t J,
+                                 int32_t gm, int32_t topk_super, int32_t topk_chunk,
+                                 size_t* bytes) {
+    if (!bytes) return fail(SSA_ERR_INVALID_ARG, "bytes is NULL");
+    ssa::Plan p;
+    ssa_status st = build_h2(p, shape, C, g, J, gm, topk_super, topk_chunk);
+    if (st != SSA_OK) return st;
+    *bytes = ssa::plan_layout(p).total;
+    return SSA_OK;
+}
+
+ssa_status ssa_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!ws) return fail(SSA_ERR_INVALID_ARG, "ws is NULL");
+    cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
+    note_ws_zeroed(ws, ws_bytes);
+    return SSA_OK;
+}
+
+ssa_status ssa_get_device_status(int32_t* host_code, cudaStream_t stream) {
+    if (!host_code) return fail(SSA_ERR_INVALID_ARG, "host_code is NULL");
+    int v = 0;
+    cudaError_t e = ssa::read_device_status(&v, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
+    *host_code = v;
+    return SSA_OK;
+}
+
+void ssa_set_wait_limit(int64_t ns) { g_wait_limit.store(ns > 0 ? ns : 0); }
+
+void ssa_set_debug_flags(int32_t flags) { g_debug.store(flags); }
+
+void ssa_set_tuning(int32_t units_per_attn_item, int32_t rows_per_score_item) {
+    g_units_per_item.store(units_per_attn_item > 0 ? units_per_attn_item : 0);
+    g_rows_per_score.store(rows_per_score_item > 0 ? rows_per_score_item : 0);
+}
+
+const char* ssa_status_string(ssa_status s) {
+    switch (s) {
+        case SSA_OK: return "ok";
+        case SSA_ERR_INVALID_ARG: return "invalid argument";
+        case SSA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case SSA_ERR_WORKSPACE: return "workspace missing or too small";
+        case SSA_ERR_CUDA: return "CUDA error";
+        case SSA_ERR_DEVICE_STATUS: return "device reported bad seq_lens or sel_idx";
+        case SSA_ERR_DEVICE_TIMEOUT: return "a bounded device wait timed out";
+    }
+    return "unknown status";
+}
+
+const char* ssa_last_error(void) { return g_err.c_str(); }
+
+int32_t ssa_version(void) { return 1; }
+
+}  // extern "C"

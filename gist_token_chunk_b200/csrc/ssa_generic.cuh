@@ -1,0 +1,278 @@
+// ssa_generic.cuh -- straightforward kernels for every dtype and head dim up
+// to 256 (used for fp32 inputs and for head dims the fused path does not
+// cover).  One warp per dot product, fp32 throughout, one block per query
+// head for the attention.  Same semantics as the fused path; slow by design.
+#pragma once
+
+#include "ssa_device.cuh"
+#include "ssa_internal.h"
+
+namespace ssa {
+namespace gen {
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Sequence length of b, or -1 (and a device status) when outside [1, n_max].
+__device__ __forceinline__ int checked_len(const Plan& p, int b) {
+    int n = p.seq_lens[b];
+    if (n < 1 || n > p.n_max) {
+        report_status(kStatusBadInput);
+        return -1;
+    }
+    return n;
+}
+
+// Number of selected superchunks kept for (p): min(topk_super, S_b).
+__device__ __forceinline__ int kept_super(const Plan& p, int S) {
+    return p.topk_super < S ? p.topk_super : S;
+}
+
+// Candidate position c of pair `pr` -> chunk index (two-level step): the J
+// children of each kept superchunk in ascending order, then the remainder.
+__device__ __forceinline__ int cand_chunk(const Plan& p, int pr, int c, int ks, int S) {
+    if (c < ks * p.J) return p.sel_super[(size_t)pr * p.topk_super + c / p.J] * p.J + c % p.J;
+    return S * p.J + (c - ks * p.J);
+}
+
+// Slot scores: dst[pr*stride + s] = max over the group's heads and the
+// slot's ntok summary rows of q.k/sqrt(d) for s < n_valid, -inf for
+// n_valid <= s < n_slots.  level 0: gist slots of chunks (single level),
+// 1: meta slots of superchunks, 2: candidate chunks (two level).
+template <class T>
+__global__ void score_kernel(Plan p, int level, float* dst, int stride, int n_slots_fixed) {
+    extern __shared__ float qs[];  // [G][d]
+    const int pr = blockIdx.y;
+    const int b = pr / p.Hkv, j = pr % p.Hkv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const T* q = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)j * p.G) * p.d;
+    for (int i = threadIdx.x; i < p.G * p.d; i += blockDim.x) qs[i] = to_f(q[i]);
+    __syncthreads();
+    const int n = checked_len(p, b);
+    const int M = n > 0 ? n / p.C : 0;
+    int n_valid, n_slots, ntok, ks = 0, S = 0;
+    const T* keys;
+    if (level == 0) {
+        n_valid = M;
+        n_slots = n_slots_fixed;
+        ntok = p.g;
+        keys = static_cast<const T*>(p.k_gist) + (size_t)pr * p.M_max * p.g * p.d;
+    } else if (level == 1) {
+        n_valid = M / p.J;
+        n_slots = n_slots_fixed;
+        ntok = p.gm;
+        keys = static_cast<const T*>(p.k_meta) + (size_t)pr * p.S_max * p.gm * p.d;
+    } else {
+        S = M / p.J;
+        ks = kept_super(p, S);
+        n_valid = ks * p.J + (M - S * p.J);
+        n_slots = n_valid;
+        ntok = p.g;
+        keys = static_cast<const T*>(p.k_gist) + (size_t)pr * p.M_max * p.g * p.d;
+    }
+    const float scale = rsqrtf((float)p.d);
+    const int nw = blockDim.x >> 5;
+    for (int s = blockIdx.x * nw + warp; s < n_slots; s += gridDim.x * nw) {
+        float best = -INFINITY;
+        if (s < n_valid) {
+            const int slot = (level == 2) ? cand_chunk(p, pr, s, ks, S) : s;
+            const T* kr = keys + (size_t)slot * ntok * p.d;
+            for (int t = 0; t < ntok; ++t) {
+                for (int h = 0; h < p.G; ++h) {
+                    float acc = 0.f;
+                    for (int i = lane; i < p.d; i += 32)
+                        acc += qs[h * p.d + i] * to_f(kr[(size_t)t * p.d + i]);
+                    acc = warp_sum(acc);
+                    best = fmaxf(best, acc * scale);
+                }
+            }
+        }
+        if (lane == 0) dst[(size_t)pr * stride + s] = best;
+    }
+}
+
+struct BlockSync {
+    __device__ void operator()() const { __syncthreads(); }
+};
+
+// Top-k per pair (block of 128).  level 0: chunks over scores (single level
+// or ssa_topk_chunks); 1: superchunks; 2: candidate chunks (map to chunk ids).
+__global__ void topk_kernel(Plan p, int level, const float* vals, int stride) {
+    __shared__ TopkScratch sc;
+    const int pr = blockIdx.x;
+    const int b = pr / p.Hkv;
+    int n = p.seq_lens[b];
+    if (n < 1 || n > p.n_max) n = 0;  // reported by the scoring kernel
+    const int M = n / p.C;
+    const float* v = vals + (size_t)pr * stride;
+    if (level == 0) {
+        block_topk<128>(v, M, p.topk, p.sel_idx + (size_t)pr * p.topk, nullptr,
+                        [](int i) { return i; }, sc, BlockSync());
+    } else if (level == 1) {
+        block_topk<128>(v, M / p.J, p.topk_super, p.sel_super + (size_t)pr * p.topk_super,
+                        nullptr, [](int i) { return i; }, sc, BlockSync());
+    } else {
+        const int S = M / p.J;
+        const int ks = kept_super(p, S);
+        const int nc = ks * p.J + (M - S * p.J);
+        const Plan* pp = &p;
+        block_topk<128>(v, nc, p.topk, p.sel_idx + (size_t)pr * p.topk, nullptr,
+                        [pp, pr, ks, S](int c) { return cand_chunk(*pp, pr, c, ks, S); }, sc,
+                        BlockSync());
+    }
+}
+
+// Checks a caller-given selection (ssa_sparse_decode): strictly ascending
+// chunk indices in [0, M_b) followed only by -1.  Marks bad pairs in ctrl.
+__global__ void validate_kernel(Plan p, int* bad) {
+    const int pr = blockIdx.x * blockDim.x + threadIdx.x;
+    if (pr >= p.n_pairs) return;
+    const int b = pr / p.Hkv;
+    int n = p.seq_lens[b];
+    const int M = (n >= 1 && n <= p.n_max) ? n / p.C : 0;
+    const int* s = p.sel_idx + (size_t)pr * p.topk;
+    int ok = 1, prev = -1, ended = 0;
+    for (int c = 0; c < p.topk; ++c) {
+        int v = s[c];
+        if (v < 0) {
+            ended = 1;
+            if (v != -1) ok = 0;
+        } else {
+            if (ended || v <= prev || v >= M) ok = 0;
+            prev = v;
+        }
+    }
+    bad[pr] = !ok;
+    if (!ok) report_status(kStatusBadInput);
+}
+
+// One block per (query head, sequence): online softmax over the unfolded
+// context, enumerated chunk by chunk; warps take units round-robin.
+template <class T>
+__global__ void attend_kernel(Plan p, const int* bad) {
+    extern __shared__ float sm[];
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int j = h / p.G;
+    const int pr = b * p.Hkv + j;
+    const int nw = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float* qs = sm;                                   // [d]
+    float* wm = qs + p.d;                             // [nw]
+    float* wl = wm + nw;                              // [nw]
+    float* wacc = wl + nw;                            // [nw][d]
+    uint32_t* cbits = reinterpret_cast<uint32_t*>(wacc + nw * p.d);  // [mask_words]
+    uint32_t* sbits = cbits + p.mask_words;                          // [smask_words]
+    float* outp = p.out + ((size_t)b * p.Hq + h) * p.d;
+
+    int n = p.seq_lens[b];
+    const bool bad_len = (n < 1 || n > p.n_max);
+    const bool bad_sel = bad != nullptr && bad[pr];
+    if (bad_len || bad_sel) {
+        if (bad_len) report_status(kStatusBadInput);
+        for (int i = threadIdx.x; i < p.d; i += blockDim.x) outp[i] = 0.f;
+        return;
+    }
+    const T* qg = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * p.d;
+    for (int i = threadIdx.x; i < p.d; i += blockDim.x) qs[i] = to_f(qg[i]);
+    for (int i = threadIdx.x; i < p.mask_words; i += blockDim.x) cbits[i] = 0;
+    for (int i = threadIdx.x; i < p.smask_words; i += blockDim.x) sbits[i] = 0;
+    __syncthreads();
+    const int M = n / p.C;
+    const int S = p.h2 ? M / p.J : 0;
+    const int ks = p.h2 ? kept_super(p, S) : 0;
+    if (threadIdx.x == 0) {
+        for (int c = 0; c < p.topk; ++c) {
+            int m = p.sel_idx[(size_t)pr * p.topk + c];
+            if (m >= 0) cbits[m >> 5] |= 1u << (m & 31);
+        }
+        for (int c = 0; c < ks; ++c) {
+            int x = p.sel_super[(size_t)pr * p.topk_super + c];
+            sbits[x >> 5] |= 1u << (x & 31);
+        }
+    }
+    __syncthreads();
+    const float scale = rsqrtf((float)p.d) * 1.4426950408889634f;  // log2 domain
+    const T* kr = static_cast<const T*>(p.k_raw) + (size_t)pr * p.n_max * p.d;
+    const T* vr = static_cast<const T*>(p.v_raw) + (size_t)pr * p.n_max * p.d;
+    const T* kg = static_cast<const T*>(p.k_gist) + (size_t)pr * p.M_max * p.g * p.d;
+    const T* vg = static_cast<const T*>(p.v_gist) + (size_t)pr * p.M_max * p.g * p.d;
+    const T* km = p.h2 ? static_cast<const T*>(p.k_meta) + (size_t)pr * p.S_max * p.gm * p.d
+                       : nullptr;
+    const T* vm = p.h2 ? static_cast<const T*>(p.v_meta) + (size_t)pr * p.S_max * p.gm * p.d
+                       : nullptr;
+    float m_run = -INFINITY, l_run = 0.f;
+    float acc[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) acc[r] = 0.f;
+
+    auto visit = [&](const T* kbase, const T* vbase, int rows) {
+        for (int t = 0; t < rows; ++t) {
+            float x = 0.f;
+            for (int i = lane; i < p.d; i += 32) x += qs[i] * to_f(kbase[(size_t)t * p.d + i]);
+            x = warp_sum(x) * scale;
+            float mn = fmaxf(m_run, x);
+            float a = exp2f(m_run - mn);
+            float e = exp2f(x - mn);
+            l_run = l_run * a + e;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                int i = lane + 32 * r;
+                if (i < p.d) acc[r] = acc[r] * a + e * to_f(vbase[(size_t)t * p.d + i]);
+            }
+            m_run = mn;
+        }
+    };
+    auto chunk_unit = [&](int m) {
+        if (cbits[m >> 5] >> (m & 31) & 1u)
+            visit(kr + (size_t)m * p.C * p.d, vr + (size_t)m * p.C * p.d, p.C);
+        else
+            visit(kg + (size_t)m * p.g * p.d, vg + (size_t)m * p.g * p.d, p.g);
+    };
+    // units: single level -> chunks 0..M-1 then the tail;
+    // two level -> superchunks 0..S-1, remainder chunks, then the tail.
+    const int n_units = p.h2 ? S + (M - S * p.J) + 1 : M + 1;
+    for (int u = warp; u < n_units; u += nw) {
+        if (u == n_units - 1) {
+            visit(kr + (size_t)M * p.C * p.d, vr + (size_t)M * p.C * p.d, n - M * p.C);
+        } else if (!p.h2) {
+            chunk_unit(u);
+        } else if (u < S) {
+            if (sbits[u >> 5] >> (u & 31) & 1u) {
+                for (int i = 0; i < p.J; ++i) chunk_unit(u * p.J + i);
+            } else {
+                visit(km + (size_t)u * p.gm * p.d, vm + (size_t)u * p.gm * p.d, p.gm);
+            }
+        } else {
+            chunk_unit(S * p.J + (u - S));
+        }
+    }
+    if (lane == 0) {
+        wm[warp] = m_run;
+        wl[warp] = l_run;
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        int i = lane + 32 * r;
+        if (i < p.d) wacc[warp * p.d + i] = acc[r];
+    }
+    __syncthreads();
+    float mx = -INFINITY;
+    for (int w = 0; w < nw; ++w) mx = fmaxf(mx, wm[w]);
+    float L = 0.f;
+    for (int w = 0; w < nw; ++w) L += (wm[w] == -INFINITY) ? 0.f : wl[w] * exp2f(wm[w] - mx);
+    for (int i = threadIdx.x; i < p.d; i += blockDim.x) {
+        float o = 0.f;
+        for (int w = 0; w < nw; ++w)
+            if (wm[w] != -INFINITY) o += wacc[w * p.d + i] * exp2f(wm[w] - mx);
+        outp[i] = L > 0.f ? o / L : 0.f;
+    }
+}
+
+}  // namespace gen
+}  // namespace ssa

@@ -1,0 +1,77 @@
+// ssa_internal.h -- host-side plan and launcher interface between the C ABI
+// (ssa_api.cpp) and the kernels (ssa_kernels.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime_api.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ssa {
+
+enum Mode : int { kModeFull = 0, kModeScoreOnly = 1, kModeAttnOnly = 2 };
+
+// Everything a launch needs, resolved on the host.  Pointers are device
+// pointers.  Sizes follow the public header's notation.
+struct Plan {
+    int mode = kModeFull;
+    int h2 = 0;            // two-level (gist-of-gist) step
+    int dtype = 0;         // 0 bf16, 1 fp32
+    int B = 0, Hq = 0, Hkv = 0, G = 0, d = 0, n_max = 0, C = 0, g = 0, M_max = 0;
+    int topk = 0;          // single level: topk; two level: topk_chunk
+    int J = 0, gm = 0, S_max = 0, topk_super = 0, Mc_max = 0;
+    int n_pairs = 0;
+
+    // work decomposition of the fused kernel
+    int score_items = 0;   // per pair: gist scoring (single) / meta scoring (two level)
+    int score_spi = 0;     // summary slots per score item
+    int cand_items = 0;    // per pair: candidate-chunk scoring (two level)
+    int attn_items = 0;    // per pair
+    int mask_words = 0, smask_words = 0;
+
+    const void* q = nullptr;
+    const void* k_raw = nullptr;
+    const void* v_raw = nullptr;
+    const void* k_gist = nullptr;
+    const void* v_gist = nullptr;
+    const void* k_meta = nullptr;
+    const void* v_meta = nullptr;
+    const int32_t* seq_lens = nullptr;
+    float* scores = nullptr;        // [P, M_max]
+    float* super_scores = nullptr;  // [P, S_max]
+    float* cand_scores = nullptr;   // [P, Mc_max]
+    int32_t* sel_idx = nullptr;     // [P, topk]
+    int32_t* sel_super = nullptr;   // [P, topk_super]
+    uint32_t* chunk_mask = nullptr; // [P, mask_words]
+    uint32_t* super_mask = nullptr; // [P, smask_words]
+    float* partials = nullptr;      // [P, attn_items, G, d + 2]
+    float* out = nullptr;           // [B, Hq, d]
+    int* ctrl = nullptr;            // control words
+    long long wait_limit = 0;       // ns bound of every device-side wait
+    int debug_flags = 0;
+};
+
+// Workspace layout for a plan (byte offsets from the workspace base).
+struct WsLayout {
+    size_t ctrl = 0, scores = 0, super_scores = 0, cand_scores = 0, chunk_mask = 0,
+           super_mask = 0, partials = 0, total = 0;
+};
+
+// Fills the decomposition fields of `p` (needs shapes) and the layout.
+void plan_decompose(Plan& p);
+WsLayout plan_layout(const Plan& p);
+int ctrl_words(const Plan& p);
+
+// Fast fused path: bf16, d in {64, 128}.  Returns a cudaError_t.
+cudaError_t launch_fused(const Plan& p, cudaStream_t stream);
+// Generic path: any d <= 256, bf16 or fp32, separate simple kernels.
+cudaError_t launch_generic(const Plan& p, cudaStream_t stream);
+// Standalone top-k over user scores (ssa_topk_chunks).
+cudaError_t launch_topk(const Plan& p, const float* scores, cudaStream_t stream);
+
+cudaError_t read_device_status(int* code, cudaStream_t stream);
+
+// Query the SM count of the current device (cached per device).
+int sm_count();
+
+}  // namespace ssa

@@ -1,0 +1,178 @@
+// ssa_kernels.cu -- the one device translation unit of libssa: defines the
+// device status word, instantiates the fused and generic kernels, and holds
+// their host-side launchers (tensor-map encoding, grid sizing).
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "ssa_device.cuh"
+#include "ssa_fused.cuh"
+#include "ssa_generic.cuh"
+#include "ssa_internal.h"
+
+namespace ssa {
+
+int sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    static int cached[64] = {0};
+    if (dev < 64 && cached[dev] > 0) return cached[dev];
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+    if (dev < 64) cached[dev] = n;
+    return n;
+}
+
+cudaError_t read_device_status(int* code, cudaStream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return e;
+    int v = 0;
+    e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
+    if (e != cudaSuccess) return e;
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+    *code = v;
+    return e;
+}
+
+// ------------------------------------------------------------- tensor maps ---
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void* f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// A [rows, d] bf16 row-major tensor as 64 x 64 boxes with 128-byte swizzle.
+static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int d) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)fused::kBoxRows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D>
+static cudaError_t launch_fused_d(const Plan& p, cudaStream_t stream) {
+    CUtensorMap m[6];
+    const uint64_t P = (uint64_t)p.n_pairs;
+    bool ok = make_map(&m[2], p.k_gist, P * p.M_max * p.g, D);
+    if (ok && p.mode == kModeScoreOnly) {
+        m[0] = m[1] = m[3] = m[2];  // scoring reads gist keys only
+    } else if (ok) {
+        ok = make_map(&m[0], p.k_raw, P * p.n_max, D) && make_map(&m[1], p.v_raw, P * p.n_max, D) &&
+             make_map(&m[3], p.v_gist, P * p.M_max * p.g, D);
+    }
+    if (ok && p.h2) {
+        ok = make_map(&m[4], p.k_meta, P * p.S_max * p.gm, D) &&
+             make_map(&m[5], p.v_meta, P * p.S_max * p.gm, D);
+    } else {
+        m[4] = m[2];
+        m[5] = m[3];
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    const fused::SmemLayout L = fused::smem_layout<D>(p.G, p.topk, p.h2 ? p.topk_super : 0);
+    auto kern = fused::fused_kernel<D>;
+    static int attr_done[64][2] = {{0}};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_done[dev][D == 128]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             227 * 1024);
+        if (e != cudaSuccess) return e;
+        attr_done[dev][D == 128] = 1;
+    }
+    int occ = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, fused::kThreads,
+                                                                  (size_t)L.total);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) return cudaErrorInvalidConfiguration;
+    const int per_a = (p.mode == kModeAttnOnly) ? 1 : p.score_items;
+    long long total = (long long)p.n_pairs * per_a;
+    if (p.h2) total += (long long)p.n_pairs * p.cand_items;
+    if (p.mode != kModeScoreOnly) total += (long long)p.n_pairs * p.attn_items;
+    long long grid = (long long)sm_count() * occ;
+    if (grid > total) grid = total;
+    if (grid < 1) grid = 1;
+    kern<<<(unsigned)grid, fused::kThreads, (size_t)L.total, stream>>>(p, m[0], m[1], m[2], m[3],
+                                                                        m[4], m[5]);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fused(const Plan& p, cudaStream_t stream) {
+    if (p.d == 64) return launch_fused_d<64>(p, stream);
+    if (p.d == 128) return launch_fused_d<128>(p, stream);
+    return cudaErrorInvalidValue;
+}
+
+int fused_smem_bytes(const Plan& p) {
+    if (p.d == 64) return fused::smem_layout<64>(p.G, p.topk, p.h2 ? p.topk_super : 0).total;
+    return fused::smem_layout<128>(p.G, p.topk, p.h2 ? p.topk_super : 0).total;
+}
+
+// ----------------------------------------------------------------- generic ---
+
+template <class T>
+static cudaError_t launch_generic_t(const Plan& p, cudaStream_t stream) {
+    const int P = p.n_pairs;
+    // a given selection leaves the score area unused: it holds the flags of
+    // rejected selections (the control words stay untouched, hence zero)
+    int* bad = reinterpret_cast<int*>(p.scores);
+    const size_t qsm = (size_t)p.G * p.d * sizeof(float);
+    auto score = [&](int level, float* dst, int stride, int nslots) {
+        const int per_block = 4;
+        const int gx = (nslots + per_block - 1) / per_block;
+        dim3 grid(gx > 0 ? gx : 1, P);
+        gen::score_kernel<T><<<grid, 128, qsm, stream>>>(p, level, dst, stride, nslots);
+    };
+    if (p.mode == kModeScoreOnly) {
+        score(0, p.scores, p.M_max, p.M_max);
+        return cudaGetLastError();
+    }
+    if (p.mode == kModeAttnOnly) {
+        gen::validate_kernel<<<(P + 127) / 128, 128, 0, stream>>>(p, bad);
+    } else if (!p.h2) {
+        score(0, p.scores, p.M_max, p.M_max);
+        gen::topk_kernel<<<P, 128, 0, stream>>>(p, 0, p.scores, p.M_max);
+    } else {
+        score(1, p.super_scores, p.S_max, p.S_max);
+        gen::topk_kernel<<<P, 128, 0, stream>>>(p, 1, p.super_scores, p.S_max);
+        score(2, p.cand_scores, p.Mc_max, p.Mc_max);
+        gen::topk_kernel<<<P, 128, 0, stream>>>(p, 2, p.cand_scores, p.Mc_max);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int nw = 8;
+    const size_t sm = (size_t)(p.d + 2 * nw + nw * p.d) * sizeof(float) +
+                      (size_t)(p.mask_words + p.smask_words) * sizeof(uint32_t);
+    dim3 grid(p.Hq, p.B);
+    gen::attend_kernel<T><<<grid, 32 * nw, sm, stream>>>(
+        p, p.mode == kModeAttnOnly ? bad : nullptr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_generic(const Plan& p, cudaStream_t stream) {
+    if (p.dtype == 1) return launch_generic_t<float>(p, stream);
+    return launch_generic_t<__nv_bfloat16>(p, stream);
+}
+
+cudaError_t launch_topk(const Plan& p, const float* scores, cudaStream_t stream) {
+    gen::topk_kernel<<<p.n_pairs, 128, 0, stream>>>(p, 0, scores, p.M_max);
+    return cudaGetLastError();
+}
+
+}  // namespace ssa

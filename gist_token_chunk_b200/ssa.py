@@ -1,0 +1,237 @@
+"""Python binding of libssa (argument marshalling only).
+
+Every step of the decode path runs in the library's CUDA kernels; this module
+only turns torch tensors into pointers, allocates outputs with torch (device
+memory is plumbing) and maps status codes to exceptions.  Importing it raises
+``ImportError`` when ``libssa.so`` has not been built -- there is no fallback.
+
+The functions carry the C ABI's names (see ``include/ssa.h``):
+``ssa_score_gists``, ``ssa_topk_chunks``, ``ssa_sparse_decode``, ``ssa_decode``,
+``ssa_decode_h2``, ``ssa_workspace_size``, ``ssa_workspace_size_h2``,
+``ssa_workspace_init``, ``ssa_get_device_status``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libssa.so not found at {LIB_PATH}: build it with gist_token_chunk_b200/build.py "
+        "(or __graft_entry__.build()); there is no non-CUDA fallback")
+lib = ctypes.CDLL(LIB_PATH)
+
+SSA_OK = 0
+SSA_ERR_INVALID_ARG = 1
+SSA_ERR_UNSUPPORTED = 2
+SSA_ERR_WORKSPACE = 3
+SSA_ERR_CUDA = 4
+SSA_ERR_DEVICE_STATUS = 5
+SSA_ERR_DEVICE_TIMEOUT = 6
+SSA_BF16 = 0
+SSA_FP32 = 1
+SSA_DEBUG_SKIP_PUBLISH = 1
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("n_max", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_S = ctypes.c_size_t
+_SH = ctypes.POINTER(Shape)
+
+lib.ssa_score_gists.argtypes = [_SH, _P, _P, _P, _I, _I, _P, _P]
+lib.ssa_topk_chunks.argtypes = [_SH, _P, _P, _I, _I, _P, _P]
+lib.ssa_sparse_decode.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _S, _P]
+lib.ssa_decode.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _S, _P]
+lib.ssa_decode_h2.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P,
+                              _P, _P, _P, _S, _P]
+lib.ssa_workspace_size.argtypes = [_SH, _I, _I, _I, ctypes.POINTER(_S)]
+lib.ssa_workspace_size_h2.argtypes = [_SH, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_S)]
+lib.ssa_workspace_init.argtypes = [_P, _S, _P]
+lib.ssa_get_device_status.argtypes = [ctypes.POINTER(_I), _P]
+lib.ssa_set_wait_limit.argtypes = [ctypes.c_int64]
+lib.ssa_set_wait_limit.restype = None
+lib.ssa_set_debug_flags.argtypes = [_I]
+lib.ssa_set_debug_flags.restype = None
+lib.ssa_set_tuning.argtypes = [_I, _I]
+lib.ssa_set_tuning.restype = None
+lib.ssa_status_string.argtypes = [_I]
+lib.ssa_status_string.restype = ctypes.c_char_p
+lib.ssa_last_error.argtypes = []
+lib.ssa_last_error.restype = ctypes.c_char_p
+lib.ssa_version.restype = _I
+for _f in ("ssa_score_gists", "ssa_topk_chunks", "ssa_sparse_decode", "ssa_decode",
+           "ssa_decode_h2", "ssa_workspace_size", "ssa_workspace_size_h2",
+           "ssa_workspace_init", "ssa_get_device_status"):
+    getattr(lib, _f).restype = _I
+
+
+class SSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.ssa_status_string(status).decode()
+        detail = lib.ssa_last_error().decode()
+        super().__init__(f"{where}: {msg} ({status}){': ' + detail if detail else ''}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != SSA_OK:
+        raise SSAError(status, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SSA_BF16
+    if t.dtype == torch.float32:
+        return SSA_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def make_shape(B, Hq, Hkv, d, n_max, dtype) -> Shape:
+    return Shape(int(B), int(Hq), int(Hkv), int(d), int(n_max), int(dtype))
+
+
+def shape_of(q: torch.Tensor, k_raw: torch.Tensor) -> Shape:
+    B, Hq, d = q.shape
+    Hkv, n_max = k_raw.shape[1], k_raw.shape[2]
+    return make_shape(B, Hq, Hkv, d, n_max, _dtype_code(q))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def ssa_workspace_size(shape: Shape, C: int, g: int, topk: int) -> int:
+    n = _S(0)
+    _check(lib.ssa_workspace_size(ctypes.byref(shape), C, g, topk, ctypes.byref(n)),
+           "ssa_workspace_size")
+    return int(n.value)
+
+
+def ssa_workspace_size_h2(shape: Shape, C, g, J, gm, topk_super, topk_chunk) -> int:
+    n = _S(0)
+    _check(lib.ssa_workspace_size_h2(ctypes.byref(shape), C, g, J, gm, topk_super, topk_chunk,
+                                     ctypes.byref(n)), "ssa_workspace_size_h2")
+    return int(n.value)
+
+
+def ssa_workspace_init(ws: torch.Tensor, stream=None) -> None:
+    _check(lib.ssa_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "ssa_workspace_init")
+
+
+def workspace(nbytes: int, device="cuda", stream=None) -> torch.Tensor:
+    """A caller-owned workspace of ``nbytes``, initialised for first use."""
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    ssa_workspace_init(ws, stream)
+    return ws
+
+
+def ssa_score_gists(q, k_gist, seq_lens, C: int, g: int, n_max: int, scores=None, stream=None):
+    B, Hq, d = q.shape
+    Hkv, M_max = k_gist.shape[1], k_gist.shape[2]
+    shape = make_shape(B, Hq, Hkv, d, n_max, _dtype_code(q))
+    if scores is None:
+        scores = torch.empty((B, Hkv, M_max), dtype=torch.float32, device=q.device)
+    _check(lib.ssa_score_gists(ctypes.byref(shape), _ptr(q), _ptr(k_gist), _ptr(seq_lens), C, g,
+                               _ptr(scores), _stream(stream)), "ssa_score_gists")
+    return scores
+
+
+def ssa_topk_chunks(scores, seq_lens, C: int, topk: int, n_max: int, sel_idx=None, stream=None):
+    B, Hkv, _ = scores.shape
+    shape = make_shape(B, Hkv, Hkv, 64, n_max, SSA_FP32)
+    if sel_idx is None:
+        sel_idx = torch.empty((B, Hkv, topk), dtype=torch.int32, device=scores.device)
+    _check(lib.ssa_topk_chunks(ctypes.byref(shape), _ptr(scores), _ptr(seq_lens), C, topk,
+                               _ptr(sel_idx), _stream(stream)), "ssa_topk_chunks")
+    return sel_idx
+
+
+def ssa_sparse_decode(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C: int, g: int, topk: int,
+                      sel_idx, out=None, ws=None, stream=None):
+    shape = shape_of(q, k_raw)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib.ssa_sparse_decode(ctypes.byref(shape), _ptr(q), _ptr(k_raw), _ptr(v_raw),
+                                 _ptr(k_gist), _ptr(v_gist), _ptr(seq_lens), C, g, topk,
+                                 _ptr(sel_idx), _ptr(out), _ptr(ws), nbytes, _stream(stream)),
+           "ssa_sparse_decode")
+    return out
+
+
+def ssa_decode(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C: int, g: int, topk: int, out=None,
+               sel_idx=None, ws=None, stream=None):
+    shape = shape_of(q, k_raw)
+    B, Hkv = q.shape[0], k_raw.shape[1]
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    if sel_idx is None:
+        sel_idx = torch.empty((B, Hkv, topk), dtype=torch.int32, device=q.device)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib.ssa_decode(ctypes.byref(shape), _ptr(q), _ptr(k_raw), _ptr(v_raw), _ptr(k_gist),
+                          _ptr(v_gist), _ptr(seq_lens), C, g, topk, _ptr(out), _ptr(sel_idx),
+                          _ptr(ws), nbytes, _stream(stream)), "ssa_decode")
+    return out, sel_idx
+
+
+def ssa_decode_h2(q, k_raw, v_raw, k_gist, v_gist, k_meta, v_meta, seq_lens, C: int, g: int,
+                  J: int, gm: int, topk_super: int, topk_chunk: int, out=None, sel_super=None,
+                  sel_idx=None, ws=None, stream=None):
+    shape = shape_of(q, k_raw)
+    B, Hkv = q.shape[0], k_raw.shape[1]
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    if sel_super is None:
+        sel_super = torch.empty((B, Hkv, topk_super), dtype=torch.int32, device=q.device)
+    if sel_idx is None:
+        sel_idx = torch.empty((B, Hkv, topk_chunk), dtype=torch.int32, device=q.device)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib.ssa_decode_h2(ctypes.byref(shape), _ptr(q), _ptr(k_raw), _ptr(v_raw),
+                             _ptr(k_gist), _ptr(v_gist), _ptr(k_meta), _ptr(v_meta),
+                             _ptr(seq_lens), C, g, J, gm, topk_super, topk_chunk, _ptr(out),
+                             _ptr(sel_super), _ptr(sel_idx), _ptr(ws), nbytes, _stream(stream)),
+           "ssa_decode_h2")
+    return out, sel_super, sel_idx
+
+
+def ssa_get_device_status(stream=None) -> int:
+    code = _I(0)
+    _check(lib.ssa_get_device_status(ctypes.byref(code), _stream(stream)),
+           "ssa_get_device_status")
+    return int(code.value)
+
+
+def ssa_set_wait_limit(ns: int) -> None:
+    lib.ssa_set_wait_limit(int(ns))
+
+
+def ssa_set_debug_flags(flags: int) -> None:
+    lib.ssa_set_debug_flags(int(flags))
+
+
+def ssa_set_tuning(units_per_attn_item: int = 0, rows_per_score_item: int = 0) -> None:
+    lib.ssa_set_tuning(int(units_per_attn_item), int(rows_per_score_item))

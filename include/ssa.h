@@ -1,0 +1,230 @@
+/*
+ * ssa.h -- C ABI of libssa: the decode-time hot path of Simplified Sparse
+ * Attention with gist tokens, for NVIDIA B200 (sm_100a).
+ *
+ * Method: "Simplified Sparse Attention via Gist Tokens" (Mao, Li, Fox).
+ *   sec. 3.2  each chunk of C raw tokens carries g gist tokens whose keys
+ *             score the chunk's relevance to the current query;
+ *   sec. 3.3  the top-k chunks are unfolded back to their raw tokens and one
+ *             softmax attention runs over the resulting hybrid context;
+ *   sec. 3.5, App. B.2  gist-of-gist: meta-gists summarise J chunks and the
+ *             selection runs coarse to fine;
+ *   sec. 3.6  decoding touches only the selected keys plus O(n) bytes of
+ *             metadata and splits the attention into partial passes that are
+ *             combined afterwards.
+ * Where the pages leave a step open this library fixes it as follows:
+ *   - chunk score s[b,j,m] = max over the query heads h of KV head j and the
+ *     chunk's g gist tokens t of  q[b,h] . k_gist[b,j,m,t] / sqrt(d);
+ *   - one selection per (sequence, KV head), shared by its query heads;
+ *     ties go to the lower chunk index; NaN scores rank as -inf;
+ *   - the attended context of (b, j) is: the gist K/V of every UNselected
+ *     complete chunk, the raw K/V of every token of the selected chunks, and
+ *     the raw K/V of the tail tokens M_b*C .. n_b-1 (selected chunks' own
+ *     gists are not attended);
+ *   - seq_lens[b] = n_b counts every cached raw token (the current one
+ *     included); M_b = floor(n_b / C) chunks are complete.
+ *
+ * Notation and layouts (row-major, contiguous, all device memory unless said):
+ *   B batch, Hq query heads, Hkv KV heads, G = Hq/Hkv, query head h reads KV
+ *   head h / G; d head dim; n_max cache capacity (a multiple of C);
+ *   M_max = n_max / C.
+ *     q       [B, Hq, d]                 bf16 or fp32 (shape->dtype)
+ *     k_raw   [B, Hkv, n_max, d]         same dtype
+ *     v_raw   [B, Hkv, n_max, d]
+ *     k_gist  [B, Hkv, M_max, g, d]
+ *     v_gist  [B, Hkv, M_max, g, d]
+ *     seq_lens int32 [B]                 (device)
+ *     scores  fp32 [B, Hkv, M_max]
+ *     sel_idx int32 [B, Hkv, topk]       selected chunks ascending, -1 padded
+ *     out     fp32 [B, Hq, d]
+ *   Two-level variant adds J (chunks per superchunk), gm (meta-gists per
+ *   superchunk), S_max = M_max / J and
+ *     k_meta, v_meta [B, Hkv, S_max, gm, d], sel_super int32 [B, Hkv, topk_super].
+ *
+ * Conventions for every call:
+ *   - The caller owns every buffer; the library neither frees nor keeps any
+ *     pointer beyond the call.  Calls are asynchronous on `stream` and never
+ *     synchronise the host (except ssa_get_device_status).
+ *   - Host-checkable errors (null pointer, topk < 0, C < 1, g < 1, n_max not a
+ *     multiple of C, Hq not a multiple of Hkv, Hq/Hkv > 16, d not in
+ *     {64, 128} for bf16 or not in [1, 256] for fp32, unknown dtype, a
+ *     workspace that is too small) return an error code with nothing enqueued.
+ *   - Errors only the device can see (n_b outside [1, n_max]; a sel_idx given
+ *     to ssa_sparse_decode that is out of range, not strictly ascending, or not
+ *     -1 padded) set the library's device status word and zero that
+ *     sequence's outputs; read it with ssa_get_device_status.
+ *   - CUDA launch errors return SSA_ERR_CUDA; ssa_last_error() gives the text.
+ *     No C++ exception crosses this boundary.
+ *   - topk > M_b selects every complete chunk; topk = 0 selects none.
+ *
+ * Workspace: the fused calls need device scratch of ssa_workspace_size()
+ * bytes.  Pass ws = NULL, ws_bytes = 0 to let the library allocate it
+ * stream-ordered (cudaMallocAsync) for that one call.  A caller-owned
+ * workspace must be zeroed once with ssa_workspace_init() (or cudaMemset 0)
+ * before its first use; every call leaves its control words zeroed again, so
+ * it can be reused by later calls on the same stream, for any sizes that fit,
+ * without re-initialising (when a call needs a larger control region than the
+ * workspace's previous call, the library zeroes it stream-ordered first).
+ * After a call that reported SSA_ERR_DEVICE_TIMEOUT, initialise it again.
+ * Two calls that share a workspace must not run concurrently.
+ */
+#ifndef SSA_H_
+#define SSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define SSA_API __attribute__((visibility("default")))
+#else
+#define SSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSA_OK = 0,
+    SSA_ERR_INVALID_ARG = 1,   /* bad pointer, size or parameter            */
+    SSA_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels handle */
+    SSA_ERR_WORKSPACE = 3,     /* workspace missing or too small            */
+    SSA_ERR_CUDA = 4,          /* a CUDA runtime call failed                */
+    SSA_ERR_DEVICE_STATUS = 5, /* device saw bad seq_lens or sel_idx        */
+    SSA_ERR_DEVICE_TIMEOUT = 6 /* a bounded device wait gave up             */
+} ssa_status;
+
+typedef enum { SSA_BF16 = 0, SSA_FP32 = 1 } ssa_dtype;
+
+/* Shapes of one call.  dtype is an ssa_dtype. */
+typedef struct {
+    int32_t B, Hq, Hkv, d, n_max;
+    int32_t dtype;
+} ssa_shape;
+
+/*
+ * ssa_score_gists -- chunk relevance scores (sec. 3.2).
+ *   scores[b,j,m] = max_{h in group j, t < g} q[b,h] . k_gist[b,j,m,t] / sqrt(d)
+ *   for m < M_b, and -inf for M_b <= m < M_max.  Reads gist keys only.
+ * In: q, k_gist, seq_lens.  Out: scores fp32 [B,Hkv,M_max].
+ */
+SSA_API ssa_status ssa_score_gists(const ssa_shape* shape, const void* q, const void* k_gist,
+                           const int32_t* seq_lens, int32_t C, int32_t g, float* scores,
+                           cudaStream_t stream);
+
+/*
+ * ssa_topk_chunks -- top-k chunk selection (sec. 3.3).
+ * Per (b, j): the k_b = min(topk, M_b) chunks with the largest scores among
+ * m < M_b, ties to the lower index, written ascending into sel_idx[b,j,0..k_b)
+ * and -1 in sel_idx[b,j,k_b..topk).  Deterministic.
+ * In: scores fp32 [B,Hkv,M_max], seq_lens.  Out: sel_idx int32 [B,Hkv,topk].
+ * shape->d and shape->dtype are not used.
+ */
+SSA_API ssa_status ssa_topk_chunks(const ssa_shape* shape, const float* scores,
+                           const int32_t* seq_lens, int32_t C, int32_t topk, int32_t* sel_idx,
+                           cudaStream_t stream);
+
+/*
+ * ssa_sparse_decode -- hybrid attention over the unfolded context for a
+ * GIVEN selection (sec. 3.3 attention, sec. 3.6 split partial passes plus
+ * combination).  sel_idx[b,j,:] must hold strictly ascending chunk indices in
+ * [0, M_b) followed only by -1 (at most topk entries); anything else sets the
+ * device status and zeroes out[b,...].
+ * Out: out fp32 [B,Hq,d].  Needs ssa_workspace_size() bytes of workspace.
+ */
+SSA_API ssa_status ssa_sparse_decode(const ssa_shape* shape, const void* q, const void* k_raw,
+                             const void* v_raw, const void* k_gist, const void* v_gist,
+                             const int32_t* seq_lens, int32_t C, int32_t g, int32_t topk,
+                             const int32_t* sel_idx, float* out, void* ws, size_t ws_bytes,
+                             cudaStream_t stream);
+
+/*
+ * ssa_decode -- the whole decode step: score, top-k, hybrid attention,
+ * combination, in one stream-ordered call (sec. 3.2, 3.3, 3.6).
+ * Out: out fp32 [B,Hq,d] and the selection sel_idx int32 [B,Hkv,topk].
+ * Needs ssa_workspace_size() bytes of workspace.
+ */
+SSA_API ssa_status ssa_decode(const ssa_shape* shape, const void* q, const void* k_raw,
+                      const void* v_raw, const void* k_gist, const void* v_gist,
+                      const int32_t* seq_lens, int32_t C, int32_t g, int32_t topk, float* out,
+                      int32_t* sel_idx, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * ssa_decode_h2 -- two-level (gist-of-gist) decode step (sec. 3.5, App. B.2).
+ * Level 2 scores the S_b = floor(M_b / J) complete superchunks with their gm
+ * meta-gist keys (same max-over-heads-and-tokens score) and keeps the top
+ * topk_super (ties to the lower index) -> sel_super.  The candidates are the J
+ * chunks of each kept superchunk plus the remainder chunks S_b*J .. M_b-1;
+ * level 1 scores the candidates with their gist keys and keeps the top
+ * topk_chunk -> sel_idx.  The attended context is: meta-gist K/V of every
+ * unselected complete superchunk, gist K/V of every unselected candidate
+ * chunk, raw K/V of the selected chunks, and the raw tail.
+ * Out: out, sel_super [B,Hkv,topk_super], sel_idx [B,Hkv,topk_chunk].
+ * Needs ssa_workspace_size_h2() bytes of workspace.
+ */
+SSA_API ssa_status ssa_decode_h2(const ssa_shape* shape, const void* q, const void* k_raw,
+                         const void* v_raw, const void* k_gist, const void* v_gist,
+                         const void* k_meta, const void* v_meta, const int32_t* seq_lens,
+                         int32_t C, int32_t g, int32_t J, int32_t gm, int32_t topk_super,
+                         int32_t topk_chunk, float* out, int32_t* sel_super, int32_t* sel_idx,
+                         void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes needed by ssa_decode / ssa_sparse_decode for these sizes. */
+SSA_API ssa_status ssa_workspace_size(const ssa_shape* shape, int32_t C, int32_t g, int32_t topk,
+                              size_t* bytes);
+
+/* Workspace bytes needed by ssa_decode_h2. */
+SSA_API ssa_status ssa_workspace_size_h2(const ssa_shape* shape, int32_t C, int32_t g, int32_t J,
+                                 int32_t gm, int32_t topk_super, int32_t topk_chunk,
+                                 size_t* bytes);
+
+/* Zero a caller-owned workspace (stream-ordered cudaMemsetAsync). */
+SSA_API ssa_status ssa_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * Synchronise `stream`, then return in *host_code the library's device status
+ * word for the current device (SSA_OK, SSA_ERR_DEVICE_STATUS or
+ * SSA_ERR_DEVICE_TIMEOUT; the first error since the last read wins) and clear
+ * it.  For tests and diagnostics; the hot calls never read it.
+ */
+SSA_API ssa_status ssa_get_device_status(int32_t* host_code, cudaStream_t stream);
+
+/*
+ * Upper bound, in nanoseconds of GPU time, on every device-side wait (a flag
+ * set by another block of the same launch, or a shared-memory barrier).  A
+ * wait that runs out records SSA_ERR_DEVICE_TIMEOUT and the kernel carries on
+ * without blocking.  The default (2 s) is far above any legal wait.  Values
+ * < 1 restore the default.  Process-wide; affects later launches.
+ */
+SSA_API void ssa_set_wait_limit(int64_t ns);
+
+/*
+ * Work-splitting knobs of the fused kernel (process-wide, later launches):
+ * units_per_attn_item = 64-row context tiles per attention work item (the
+ * split-K granularity), rows_per_score_item = summary rows per scoring work
+ * item.  Values < 1 restore the defaults (6 and 512).  Results do not depend
+ * on them beyond fp32 summation order.
+ */
+SSA_API void ssa_set_tuning(int32_t units_per_attn_item, int32_t rows_per_score_item);
+
+/*
+ * Test hook: with SSA_DEBUG_SKIP_PUBLISH set, the selection step of
+ * ssa_sparse_decode never publishes its "selection ready" flag, so every
+ * attention block waits until its wait limit and the call reports
+ * SSA_ERR_DEVICE_TIMEOUT through ssa_get_device_status.  0 disables.
+ */
+#define SSA_DEBUG_SKIP_PUBLISH 1
+SSA_API void ssa_set_debug_flags(int32_t flags);
+
+SSA_API const char* ssa_status_string(ssa_status status);
+/* Detail of the last error returned on this host thread ("" if none). */
+SSA_API const char* ssa_last_error(void);
+SSA_API int32_t ssa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSA_H_ */

@@ -1,0 +1,135 @@
+"""Device-side behaviour of the C ABI: status words for bad inputs, bounded
+waits that time out with a status instead of hanging, determinism, workspace
+reuse, and invariance to the split-K decomposition."""
+import numpy as np
+import pytest
+import torch
+
+from gist_token_chunk_b200.inputs import Workload, make_inputs
+from parity import host
+
+pytestmark = pytest.mark.gpu
+
+W1 = Workload("abi", B=2, Hq=32, Hkv=8, d=64, n_max=4096, C=64, g=8, topk=16,
+              seq_lens=(4096, 2500), planted=16)
+
+
+@pytest.fixture(scope="module")
+def ssa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from gist_token_chunk_b200 import ssa as mod
+
+    yield mod
+    mod.ssa_set_tuning(0, 0)
+    mod.ssa_set_debug_flags(0)
+    mod.ssa_set_wait_limit(0)
+
+
+@pytest.fixture(scope="module")
+def inp():
+    i = make_inputs(W1, seed=31)
+    return {k: v.cuda() if k != "planted_idx" else v for k, v in i.items()}
+
+
+def run(ssa, inp, ws=None, w=W1):
+    return ssa.ssa_decode(inp["q"], inp["k_raw"], inp["v_raw"], inp["k_gist"], inp["v_gist"],
+                          inp["seq_lens"], w.C, w.g, w.topk, ws=ws)
+
+
+def test_bitwise_deterministic(ssa, inp):
+    o1, s1 = run(ssa, inp)
+    o2, s2 = run(ssa, inp)
+    assert torch.equal(s1, s2) and torch.equal(o1, o2)
+
+
+def test_workspace_reuse_stays_clean(ssa, inp):
+    sh = ssa.shape_of(inp["q"], inp["k_raw"])
+    ws = ssa.workspace(ssa.ssa_workspace_size(sh, W1.C, W1.g, W1.topk))
+    o0, s0 = run(ssa, inp)  # library-allocated workspace
+    for _ in range(3):
+        o, s = run(ssa, inp, ws=ws)
+        assert torch.equal(s, s0) and torch.equal(o, o0)
+    # the same workspace serves another problem size, then the first again
+    other = Workload("abi2", B=1, Hq=32, Hkv=8, d=64, n_max=2048, C=64, g=8, topk=4,
+                     seq_lens=(1500,))
+    oi = {k: v.cuda() if k != "planted_idx" else v for k, v in make_inputs(other, 3).items()}
+    run(ssa, oi, ws=ws, w=other)
+    o, s = run(ssa, inp, ws=ws)
+    assert torch.equal(s, s0) and torch.equal(o, o0)
+    assert ssa.ssa_get_device_status() == 0
+
+
+@pytest.mark.parametrize("units", [1, 3, 64])
+def test_split_invariance(ssa, inp, units):
+    o0, s0 = run(ssa, inp)
+    ssa.ssa_set_tuning(units, 128)
+    try:
+        o, s = run(ssa, inp)
+    finally:
+        ssa.ssa_set_tuning(0, 0)
+    assert torch.equal(s, s0)
+    assert (o - o0).abs().max().item() <= 1e-6
+
+
+def test_bad_length_sets_status_and_zeroes(ssa, inp):
+    bad = dict(inp)
+    bad["seq_lens"] = torch.tensor([4096, 5000], dtype=torch.int32, device="cuda")  # > n_max
+    out, sel = run(ssa, bad)
+    assert ssa.ssa_get_device_status() == ssa.SSA_ERR_DEVICE_STATUS
+    assert (out[1] == 0).all() and (sel[1] == -1).all()
+    good, _ = run(ssa, inp)
+    assert torch.equal(out[0], good[0])
+    assert ssa.ssa_get_device_status() == 0
+
+
+def test_bad_selection_sets_status_and_zeroes(ssa, inp):
+    _, sel = run(ssa, inp)
+    bad = sel.clone()
+    bad[0, 3, 0], bad[0, 3, 1] = bad[0, 3, 1], bad[0, 3, 0]  # not ascending
+    bad[1, 5, 0] = 10_000                                     # out of range
+    out = ssa.ssa_sparse_decode(inp["q"], inp["k_raw"], inp["v_raw"], inp["k_gist"],
+                                inp["v_gist"], inp["seq_lens"], W1.C, W1.g, W1.topk, bad)
+    assert ssa.ssa_get_device_status() == ssa.SSA_ERR_DEVICE_STATUS
+    G = W1.Hq // W1.Hkv
+    assert (out[0, 3 * G:4 * G] == 0).all() and (out[1, 5 * G:6 * G] == 0).all()
+    ref = ssa.ssa_sparse_decode(inp["q"], inp["k_raw"], inp["v_raw"], inp["k_gist"],
+                                inp["v_gist"], inp["seq_lens"], W1.C, W1.g, W1.topk, sel)
+    keep = torch.ones(W1.B, W1.Hq, dtype=torch.bool, device="cuda")
+    keep[0, 3 * G:4 * G] = False
+    keep[1, 5 * G:6 * G] = False
+    assert torch.equal(out[keep], ref[keep])
+    assert ssa.ssa_get_device_status() == 0
+
+
+def test_wait_that_never_ends_times_out_with_status(ssa, inp):
+    """A selection flag that nothing sets: the bounded waits run out, the
+    call reports SSA_ERR_DEVICE_TIMEOUT, and the context stays usable."""
+    _, sel = run(ssa, inp)
+    sh = ssa.shape_of(inp["q"], inp["k_raw"])
+    ws = ssa.workspace(ssa.ssa_workspace_size(sh, W1.C, W1.g, W1.topk))
+    ssa.ssa_set_wait_limit(2_000_000)  # 2 ms
+    ssa.ssa_set_debug_flags(ssa.SSA_DEBUG_SKIP_PUBLISH)
+    try:
+        ssa.ssa_sparse_decode(inp["q"], inp["k_raw"], inp["v_raw"], inp["k_gist"],
+                              inp["v_gist"], inp["seq_lens"], W1.C, W1.g, W1.topk, sel, ws=ws)
+        assert ssa.ssa_get_device_status() == ssa.SSA_ERR_DEVICE_TIMEOUT
+    finally:
+        ssa.ssa_set_debug_flags(0)
+        ssa.ssa_set_wait_limit(0)
+    ssa.ssa_workspace_init(ws)
+    out = ssa.ssa_sparse_decode(inp["q"], inp["k_raw"], inp["v_raw"], inp["k_gist"],
+                                inp["v_gist"], inp["seq_lens"], W1.C, W1.g, W1.topk, sel, ws=ws)
+    ref, _ = run(ssa, inp)
+    assert ssa.ssa_get_device_status() == 0
+    assert (out - ref).abs().max().item() <= 1e-6
+
+
+def test_fused_equals_components(ssa, inp):
+    out, sel = run(ssa, inp)
+    scores = ssa.ssa_score_gists(inp["q"], inp["k_gist"], inp["seq_lens"], W1.C, W1.g, W1.n_max)
+    sel2 = ssa.ssa_topk_chunks(scores, inp["seq_lens"], W1.C, W1.topk, W1.n_max)
+    assert torch.equal(sel, sel2)
+    out2 = ssa.ssa_sparse_decode(inp["q"], inp["k_raw"], inp["v_raw"], inp["k_gist"],
+                                 inp["v_gist"], inp["seq_lens"], W1.C, W1.g, W1.topk, sel2)
+    assert (out - out2).abs().max().item() <= 1e-6
