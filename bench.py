@@ -1,0 +1,516 @@
+#!/usr/bin/env python3
+"""Decode-step throughput of the SSA (gist token) hot path on B200.
+
+One step = one fused ``ssa_decode`` call over a batch of B sequences (all
+query heads of one layer): gist scoring, top-k chunk selection, hybrid
+attention over the unfolded context and the combination of split partials.
+The default workload is the 128K-context one (B=4, 32/8 heads, d=64, bf16,
+lengths uniform in [64K, 128K], C=128, g=8, top-32).
+
+Prints ONE JSON line (rank 0):
+  value        decode queries/s over all GPUs, inputs resident in HBM; steps
+               are CUDA-graph replays of the fused kernel, timed with CUDA
+               events on the launching stream, max over ranks; 4 input sets
+               rotate so every step starts with the previous steps' >= 3x83 MB
+               of other data in L2 (L2 is 126 MB)
+  e2e          the same metric through the public call per step, with the
+               query and lengths copied host->device (pinned) and the output
+               and selection copied back inside the timed region
+  roofline     HBM roofline of the fused kernel: algorithmic bytes per launch
+               (gist K + unselected gist V + selected raw K/V + tail + q, out,
+               selection, lengths) / average launch time, vs the measured
+               copy bandwidth in MEASURED_PEAKS.json
+  cpu_baseline the fp64 CPU oracle on the host, on a bounded sample
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm) instead.
+Multi-GPU: one process per GPU (torchrun); each rank decodes its own batch
+(weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gist_token_chunk_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "decode queries/s and achieved HBM GB/s (% of B200 peak) at 32K–512K context"
+UNIT = "queries/s"
+DEFAULT_CONFIG = "llama1b_128k_var"
+NSETS = 4
+FALLBACK_HBM_GBS = 6650.0
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ------------------------------------------------------------ bytes model ---
+
+def algorithmic_bytes(w, seq_lens) -> int:
+    """Bytes one decode step must move, each read once: per (sequence, KV
+    head) the gist keys of all complete chunks, the gist values of the
+    unselected ones, the raw K/V of the selected chunks and of the tail
+    (two-level: meta keys, unselected meta values, candidate gist keys,
+    unselected candidate gist values, selected raw K/V, tail), plus q, the
+    output, the selection and the lengths."""
+    e = 2 if w.dtype == "bf16" else 4
+    tot = 0
+    for n in seq_lens:
+        n = int(n)
+        M = n // w.C
+        T = n - M * w.C
+        if not w.two_level:
+            k = min(w.topk, M)
+            rows = M * w.g + (M - k) * w.g + 2 * k * w.C + 2 * T
+        else:
+            S = M // w.J
+            R = M - S * w.J
+            ks = min(w.topk_super, S)
+            Mc = ks * w.J + R
+            kc = min(w.topk, Mc)
+            rows = (S * w.gm + (S - ks) * w.gm + Mc * w.g + (Mc - kc) * w.g + 2 * kc * w.C
+                    + 2 * T)
+        tot += w.Hkv * rows * w.d * e
+    sel_k = w.topk + (w.topk_super if w.two_level else 0)
+    tot += w.B * w.Hq * w.d * e + w.B * w.Hq * w.d * 4 + w.B * w.Hkv * sel_k * 4 + w.B * 4
+    return tot
+
+
+# ----------------------------------------------------------------- peaks ---
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gist_token_chunk_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(config: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(config)
+    except Exception:
+        return None
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML during a region."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.ok = False
+        self.samples = []
+        self.reasons = 0
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            # NVML numbers GPUs without CUDA_VISIBLE_DEVICES: find ours by
+            # UUID (a string -- pynvml passes its argument as a C pointer)
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover
+            log("clock sampling unavailable:", e)
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except AttributeError:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.reasons |= int(r) & ~0x1
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            self._stop.wait(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": [n for bit, n in self.REASONS.items() if self.reasons & bit],
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------- cpu oracle ---
+
+def oracle_time(inp, w, min_seconds: float, max_reps: int = 1000):
+    """Time the fp64 oracle on whole decode steps of `inp` (host tensors)."""
+    from oracle import ssa_oracle
+
+    orc = ssa_oracle.default()
+    args = [inp["q"], inp["k_raw"], inp["v_raw"], inp["k_gist"], inp["v_gist"]]
+    if w.two_level:
+        args += [inp["k_meta"], inp["v_meta"]]
+    import numpy as _np
+
+    args = [_np.ascontiguousarray(a.float().numpy()) for a in args]
+    lens = inp["seq_lens"].numpy()
+
+    def one():
+        if w.two_level:
+            orc.decode_h2(*args, lens, C=w.C, g=w.g, J=w.J, gm=w.gm, topk_super=w.topk_super,
+                          topk_chunk=w.topk)
+        else:
+            orc.decode(*args, lens, C=w.C, g=w.g, topk=w.topk)
+
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        one()
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or reps >= max_reps:
+            return reps, el
+
+
+def oracle_cores(pairs: int) -> int:
+    n = os.environ.get("OMP_NUM_THREADS")
+    avail = int(n) if n else (len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity")
+                              else os.cpu_count())
+    return max(1, min(avail, pairs))
+
+
+def config_of(w) -> dict:
+    cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "n_max": w.n_max,
+           "C": w.C, "g": w.g, "topk": w.topk}
+    if w.seq_range:
+        cfg["seq_lens"] = f"uniform[{w.seq_range[0]},{w.seq_range[1]}]"
+    else:
+        cfg["seq_lens"] = list(w.seq_lens)
+    if w.two_level:
+        cfg.update({"J": w.J, "gm": w.gm, "topk_super": w.topk_super})
+    return cfg
+
+
+# -------------------------------------------------------- reference arm ---
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.config]
+    inp = make_inputs(w, seed=args.seed, device="cpu")
+    from oracle import ssa_oracle
+
+    orc = ssa_oracle.default()
+    host = {k: np.ascontiguousarray(v.float().numpy()) for k, v in inp.items()
+            if k not in ("seq_lens", "planted_idx")}
+    lens = inp["seq_lens"].numpy()
+
+    def step(i):
+        b = i % w.B
+        sl = {k: v[b:b + 1] for k, v in host.items()}
+        if w.two_level:
+            orc.decode_h2(sl["q"], sl["k_raw"], sl["v_raw"], sl["k_gist"], sl["v_gist"],
+                          sl["k_meta"], sl["v_meta"], lens[b:b + 1], C=w.C, g=w.g, J=w.J, gm=w.gm,
+                          topk_super=w.topk_super, topk_chunk=w.topk)
+        else:
+            orc.decode(sl["q"], sl["k_raw"], sl["v_raw"], sl["k_gist"], sl["v_gist"],
+                       lens[b:b + 1], C=w.C, g=w.g, topk=w.topk)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    el = time.perf_counter() - t0
+    value = args.steps / el
+    cores = oracle_cores(w.Hkv)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(config_of(w), parallelism="host cores (OpenMP over KV heads)"),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": "each step = one sequence (all KV heads) of the workload, "
+                                       "cycling through the batch"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------- GPU arm ---
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
+    ap.add_argument("--seed", type=int, default=1003)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=1000)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    from gist_token_chunk_b200 import ssa
+
+    w = WORKLOADS[args.config]
+    # each rank decodes its own batch (independent sequences)
+    sets = [make_inputs(w, seed=args.seed + 7919 * s + 100003 * rank, device=dev)
+            for s in range(NSETS)]
+    for s in sets:
+        s.pop("planted_idx", None)
+    shape = ssa.shape_of(sets[0]["q"], sets[0]["k_raw"])
+    if w.two_level:
+        nbytes = ssa.ssa_workspace_size_h2(shape, w.C, w.g, w.J, w.gm, w.topk_super, w.topk)
+    else:
+        nbytes = ssa.ssa_workspace_size(shape, w.C, w.g, w.topk)
+    ws = ssa.workspace(nbytes, device=dev)
+    outs = [torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev) for _ in range(NSETS)]
+    sels = [torch.empty(w.B, w.Hkv, w.topk, dtype=torch.int32, device=dev) for _ in range(NSETS)]
+    sups = [torch.empty(w.B, w.Hkv, max(w.topk_super, 1), dtype=torch.int32, device=dev)
+            for _ in range(NSETS)]
+
+    def step(i, stream=None):
+        s = i % NSETS
+        x = sets[s]
+        if w.two_level:
+            ssa.ssa_decode_h2(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
+                              x["k_meta"], x["v_meta"], x["seq_lens"], w.C, w.g, w.J, w.gm,
+                              w.topk_super, w.topk, out=outs[s], sel_super=sups[s],
+                              sel_idx=sels[s], ws=ws, stream=stream)
+        else:
+            ssa.ssa_decode(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
+                           x["seq_lens"], w.C, w.g, w.topk, out=outs[s], sel_idx=sels[s], ws=ws,
+                           stream=stream)
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for i in range(NSETS):
+            step(i)  # eager first use (workspace control region, attributes)
+    stream.synchronize()
+    # graphs: a chunk of REP*NSETS steps and single steps for the remainder
+    REP = 8
+    g_chunk = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_chunk, stream=stream):
+        for i in range(REP * NSETS):
+            step(i, stream=stream)
+    g_one = []
+    for s in range(NSETS):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(s, stream=stream)
+        g_one.append(g)
+    assert ssa.ssa_get_device_status(stream) == 0
+
+    def run_steps(k):
+        done = 0
+        while k - done >= REP * NSETS:
+            g_chunk.replay()
+            done += REP * NSETS
+        while done < k:
+            g_one[done % NSETS].replay()
+            done += 1
+
+    with torch.cuda.stream(stream):
+        run_steps(args.warmup)
+    stream.synchronize()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            run_steps(args.steps)
+            ev1.record(stream)
+        ev1.synchronize()
+    torch.cuda.synchronize(dev)
+    ms = ev0.elapsed_time(ev1)
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    status = ssa.ssa_get_device_status(stream)
+    if status != 0:
+        raise SystemExit(f"device status {status} after the timed region")
+
+    queries = args.steps * w.B * world
+    value = queries / (ms / 1e3)
+    ms_step = ms / args.steps
+    # bytes model, averaged over the rotating sets
+    bytes_per_launch = statistics.mean(
+        algorithmic_bytes(w, s["seq_lens"].cpu().tolist()) for s in sets)
+    per_launch_s = (ms / 1e3) / args.steps
+    achieved = bytes_per_launch / per_launch_s / 1e9
+    peak, peak_src = hbm_peak()
+
+    # ---- end to end through the public call, host buffers
+    ek = max(NSETS, min(args.steps, args.e2e_steps))
+    q_host = [x["q"].cpu().pin_memory() for x in sets]
+    len_host = [x["seq_lens"].cpu().pin_memory() for x in sets]
+    q_dev = [torch.empty_like(x["q"]) for x in sets]
+    len_dev = [torch.empty_like(x["seq_lens"]) for x in sets]
+    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    sel_host = [torch.empty(s.shape, dtype=s.dtype).pin_memory() for s in sels]
+
+    def e2e_step(i):
+        s = i % NSETS
+        q_dev[s].copy_(q_host[s], non_blocking=True)
+        len_dev[s].copy_(len_host[s], non_blocking=True)
+        x = dict(sets[s], q=q_dev[s], seq_lens=len_dev[s])
+        if w.two_level:
+            ssa.ssa_decode_h2(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
+                              x["k_meta"], x["v_meta"], x["seq_lens"], w.C, w.g, w.J, w.gm,
+                              w.topk_super, w.topk, out=outs[s], sel_super=sups[s],
+                              sel_idx=sels[s], ws=ws, stream=stream)
+        else:
+            ssa.ssa_decode(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
+                           x["seq_lens"], w.C, w.g, w.topk, out=outs[s], sel_idx=sels[s], ws=ws,
+                           stream=stream)
+        out_host[s].copy_(outs[s], non_blocking=True)
+        sel_host[s].copy_(sels[s], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(NSETS):
+            e2e_step(i)
+    stream.synchronize()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for i in range(ek):
+            e2e_step(i)
+        ev1.record(stream)
+    ev1.synchronize()
+    e2e_ms = ev0.elapsed_time(ev1)
+    if pg:
+        t = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = ek * w.B * world / (e2e_ms / 1e3)
+    h2d = sets[0]["q"].numel() * sets[0]["q"].element_size() + sets[0]["seq_lens"].numel() * 4
+    d2h = outs[0].numel() * 4 + sels[0].numel() * 4
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": dict(config_of(w), global_batch=w.B * world,
+                       l2=f"{NSETS} input sets rotate (each step follows >= 3 steps over other "
+                          "sets; inputs larger than L2)",
+                       timing="CUDA-graph replays of the fused kernel, CUDA events, max over ranks",
+                       parallelism=f"dp{world} (independent sequences per GPU, no collective)"),
+        "hbm_gbs": achieved, "hbm_frac_of_peak": achieved / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"{peak_src} copy bandwidth",
+                     "algorithmic_bytes_per_launch": int(bytes_per_launch),
+                     "traffic": profiled_traffic(args.config),
+                     "kernel": "ssa::fused::fused_kernel<64>"},
+        "gpu_launches": args.steps,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": ek,
+                "path": "ssa_decode per step (Python binding -> C ABI) with pinned host copies"},
+    }
+    clk = sampler.summary()
+    if clk is not None:
+        line["clocks"] = clk
+
+    # ---- CPU baseline: the oracle on the host (rank 0, N = 1 only)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = {k: v.cpu() for k, v in sets[0].items()}
+        reps, el = oracle_time(host, w, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": reps * w.B / el, "unit": UNIT, "cores": oracle_cores(w.B * w.Hkv),
+            "kind": "oracle",
+            "sample": f"{reps} whole decode step(s) (B={w.B} sequences) of input set 0, "
+                      f"{el:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        del g_chunk, g_one
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -33,18 +33,20 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, extra=(), out: str = LIB) -> str:
+    """Compile libssa.so; ``extra`` nvcc flags (e.g. -DSSA_TRACE) and another
+    ``out`` path give instrumented variants without touching the product."""
+    if out == LIB and not force and not _stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = out + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC,-O3,-fvisibility=hidden", "-I", os.path.join(ROOT, "include"),
            "-o", tmp, *[os.path.join(CSRC, f) for f in SOURCES], *extra]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

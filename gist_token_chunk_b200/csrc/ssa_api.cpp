@@ -23,13 +23,17 @@ thread_local std::string g_err;
 std::atomic<long long> g_wait_limit{0};
 std::atomic<int> g_debug{0};
 std::atomic<int> g_units_per_item{0};
+#ifdef SSA_TRACE
+std::atomic<void*> g_trace{nullptr};
+std::atomic<int> g_trace_cap{0};
+#endif
 std::atomic<int> g_rows_per_score{0};
 
 constexpr long long kDefaultWaitLimitNs = 2000000000ll;  // 2 s
 constexpr int kMaxG = 16;
 constexpr int kMaxTopk = 1024;
 constexpr int kRowsPerScoreItem = 512;
-constexpr int kUnitsPerAttnItem = 6;
+constexpr int kUnitsPerAttnItem = 12;
 
 int rows_per_score_item() {
     int v = g_rows_per_score.load();
@@ -106,6 +110,10 @@ void fill_shape(ssa::Plan& p, const ssa_shape* s, int C, int g, int topk) {
     long long lim = g_wait_limit.load();
     p.wait_limit = lim > 0 ? lim : kDefaultWaitLimitNs;
     p.debug_flags = g_debug.load();
+#ifdef SSA_TRACE
+    p.trace = static_cast<uint4*>(g_trace.load());
+    p.trace_cap = g_trace_cap.load();
+#endif
 }
 
 bool fused_path(const ssa::Plan& p) { return p.dtype == SSA_BF16 && (p.d == 64 || p.d == 128); }
@@ -162,12 +170,17 @@ void plan_decompose(Plan& p) {
     int items = (int)((U + upi - 1) / upi);
     if (items < 1) items = 1;
     if (items > kMaxAttnItems) items = kMaxAttnItems;
+    // the combination stages 3 floats per (query head, item) in shared memory
+    const int cap = 16384 / (48 * (p.G > 0 ? p.G : 1));
+    if (items > cap) items = cap;
     p.attn_items = items;
+    // counters line, published-count line, then the published selection(s)
+    p.pair_ints = 64 + (p.topk + (p.h2 ? p.topk_super : 0) + 31) / 32 * 32;
     p.mask_words = (cdiv(p.M_max, 32) + 3) / 4 * 4;
     p.smask_words = p.h2 ? (cdiv(p.S_max, 32) + 3) / 4 * 4 : 0;
 }
 
-int ctrl_words(const Plan& p) { return 2 + 8 * p.n_pairs; }
+int ctrl_words(const Plan& p) { return 64 + p.pair_ints * p.n_pairs; }  // see ssa_fused.cuh
 
 WsLayout plan_layout(const Plan& p) {
     WsLayout L;
@@ -184,7 +197,8 @@ WsLayout plan_layout(const Plan& p) {
     L.cand_scores = take(p.h2 ? P * p.Mc_max * 4 : 0);
     L.chunk_mask = take(0);
     L.super_mask = take(0);
-    L.partials = take(fused_path(p) ? P * p.attn_items * p.G * (p.d + 2) * 4 : 0);
+    // one partial per (pair, attention item, consumer warp, query head)
+    L.partials = take(fused_path(p) ? P * p.attn_items * 4 * p.G * (p.d + 2) * 4 : 0);
     L.total = o;
     return L;
 }
@@ -478,5 +492,13 @@ const char* ssa_status_string(ssa_status s) {
 const char* ssa_last_error(void) { return g_err.c_str(); }
 
 int32_t ssa_version(void) { return 1; }
+
+#ifdef SSA_TRACE
+// Trace builds only: device buffer of blocks x cap x 16-byte events.
+__attribute__((visibility("default"))) void ssa_set_trace(void* buf, int32_t cap) {
+    g_trace.store(buf);
+    g_trace_cap.store(cap);
+}
+#endif
 
 }  // extern "C"

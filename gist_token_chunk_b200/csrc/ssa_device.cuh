@@ -39,10 +39,25 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+__device__ __forceinline__ int ld_relaxed(const int* p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void fence_acquire_gpu() {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 __device__ __forceinline__ int ld_acquire(const int* p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+// Release increment without a returned value (fire and forget).
+__device__ __forceinline__ void red_release_add(int* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ void st_release(int* p, int v) {
@@ -55,15 +70,31 @@ __device__ __forceinline__ uint64_t now_ns() {
     return t;
 }
 
-// Poll *p until it is >= target, for at most `limit_ns` nanoseconds.  On
+// Wait bounds count SM clock cycles (clock64 is a cheap per-SM counter; the
+// global timer is not polled in hot loops).  2 cycles per ns covers SM clocks
+// up to 2 GHz, so a bound of N ns never ends a wait earlier than N ns.
+__device__ __forceinline__ long long wait_cycles(long long limit_ns) { return 2 * limit_ns; }
+
+// Poll *p until it is >= target, for at most `limit_ns` nanoseconds, then
+// acquire.  Relaxed polls with a capped exponential back-off keep many
+// waiting blocks from saturating the L2 slice that holds the word.  On
 // running out it records a timeout in the status word and returns false
 // (never blocks for longer).
 __device__ __forceinline__ bool wait_geq(const int* p, int target, long long limit_ns) {
-    const uint64_t t0 = now_ns();
+    if (ld_relaxed(p) >= target) {
+        fence_acquire_gpu();
+        return true;
+    }
+    const long long c0 = clock64(), lim = wait_cycles(limit_ns);
+    unsigned sleep_ns = 32;
     for (;;) {
-        if (ld_acquire(p) >= target) return true;
-        if ((long long)(now_ns() - t0) > limit_ns) break;
-        __nanosleep(128);
+        __nanosleep(sleep_ns);
+        if (sleep_ns < 512) sleep_ns *= 2;
+        if (ld_relaxed(p) >= target) {
+            fence_acquire_gpu();
+            return true;
+        }
+        if (clock64() - c0 > lim) break;
     }
     report_status(kStatusTimeout);
     return false;
@@ -101,14 +132,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the warp sleeps in hardware until the
+// phase completes or `hint_ns` passes, instead of re-polling shared memory
+// (polling warps would compete with the neighbour block for the SM's
+// shared-memory pipe).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking test of phase completion (never suspends the warp).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete, for at most
-// `limit_ns` nanoseconds (plus one hardware suspend interval).
+// `limit_ns` nanoseconds (plus one suspend interval).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = now_ns();
+    const long long c0 = clock64(), lim = wait_cycles(limit_ns);
     for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((long long)(now_ns() - t0) > limit_ns) break;
+        if (mbar_test_wait(bar, parity)) return true;
+        __nanosleep(20);
+        if (clock64() - c0 > lim) break;
     }
     report_status(kStatusTimeout);
     return false;
@@ -213,25 +275,40 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sm, int& total, 
 }
 
 // ---------------------------------------------------- block top-k ---
+struct NoProbe {
+    __device__ void operator()(int) const {}
+};
+
+constexpr int kTopkCandCap = 512;  // candidates the filtered selection ranks directly
+
 struct TopkScratch {
     int hist[256];
     int bcast[4];
     int scan[8];
+    alignas(16) uint32_t tmax[128];           // per-thread key maxima (NT <= 128)
+    alignas(16) uint32_t ckey[kTopkCandCap];  // candidate keys, in index order
+    int cidx[kTopkCandCap];                   // candidate positions
 };
 
 // Deterministic top-k over vals[0..n) (sec. 3.3 "top-k chunks"): selects the
-// k = min(topk, n) largest values, ties to the lower position, and writes
-// map(i) for the selected positions i in ascending order of i to
-// out[0..k), then -1 to out[k..topk).  If `mask` is not null, bit map(i) of
-// `mask` is set for each selected i (the caller zeroes it beforehand).
-// Runs on the NT threads that call it together; vals is read with
-// L2-coherent loads so it may have been written by other blocks of the same
-// launch.  Method: 4-pass MSB-first radix select on the order-preserving
-// 32-bit key finds the k-th largest key tau and how many keys equal to tau
-// are taken; a prefix count in index order then picks the lowest-index ties.
-template <int NT, class Map, class Sync>
-__device__ void block_topk(const float* vals, int n, int topk, int* out, uint32_t* mask, Map map,
-                           TopkScratch& sc, Sync sync) {
+// k = min(topk, n) largest values, ties to the lower position, and writes the
+// selected positions in ascending order to out[0..k), then -1 to
+// out[k..topk).  Runs on the NT (<= 128) threads that call it together.
+// vals is read with L2-coherent loads (it may have been written by other
+// blocks of the same launch), in batches so that many loads are in flight.
+//
+// Filtered path (k <= NT): each thread takes the maximum key of its strided
+// share; the k-th largest of those NT maxima is a lower bound tau on the k-th
+// largest key (k distinct keys reach it), so every selected key -- ties at
+// the boundary included -- is >= tau.  The keys >= tau are compacted in index
+// order and ranked exactly by counting (larger key first, then lower index).
+// Fallback (k > NT, or more than kTopkCandCap keys >= tau): MSB-first radix
+// select on the order-preserving 32-bit key, reading vals from L2 per pass.
+// If `pub` is not null, each selected position i is also written there as
+// pub[rank] = i + 1 (a published copy that is never 0 once written).
+template <int NT, class Sync, class Probe = NoProbe>
+__device__ void block_topk(const float* vals, int n, int topk, int* out, TopkScratch& sc,
+                           Sync sync, Probe probe = Probe(), int* pub = nullptr) {
     const int tid = threadIdx.x & (NT - 1);
     const int k = topk < n ? topk : n;
     if (k <= 0) {
@@ -239,13 +316,111 @@ __device__ void block_topk(const float* vals, int n, int topk, int* out, uint32_
         return;
     }
     if (k == n) {
-        for (int c = tid; c < topk; c += NT) out[c] = c < n ? map(c) : -1;
-        if (mask)
-            for (int c = tid; c < n; c += NT) {
-                int m = map(c);
-                atomicOr(&mask[m >> 5], 1u << (m & 31));
-            }
+        for (int c = tid; c < topk; c += NT) {
+            out[c] = c < n ? c : -1;
+            if (pub && c < n) pub[c] = c + 1;
+        }
         return;
+    }
+    constexpr int U = 8;
+    if (k <= NT) {
+        uint32_t mx = 0u;
+        for (int base = 0; base < n; base += NT * U) {
+            float v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = base + u * NT + tid;
+                v[u] = i < n ? __ldcg(vals + i) : -INFINITY;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) mx = max(mx, score_key(v[u]));
+        }
+        sc.tmax[tid] = mx;
+        probe(1);
+        sync();
+        int rank = 0;
+        const uint4* tm4 = reinterpret_cast<const uint4*>(sc.tmax);
+#pragma unroll
+        for (int j4 = 0; j4 < NT / 4; ++j4) {
+            const uint4 o = tm4[j4];
+            const int j = 4 * j4;
+            rank += (o.x > mx) || (o.x == mx && j < tid);
+            rank += (o.y > mx) || (o.y == mx && j + 1 < tid);
+            rank += (o.z > mx) || (o.z == mx && j + 2 < tid);
+            rank += (o.w > mx) || (o.w == mx && j + 3 < tid);
+        }
+        if (rank == k - 1) sc.bcast[3] = (int)mx;
+        probe(4);
+        sync();
+        const uint32_t tau = (uint32_t)sc.bcast[3];
+        // contiguous share [lo, hi) per thread, loaded in batches of U
+        const int per = (n + NT - 1) / NT;
+        const int lo = min(tid * per, n), hi = min(lo + per, n);
+        int nc = 0;
+        for (int b0 = lo; b0 < hi; b0 += U) {
+            float v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) v[u] = b0 + u < hi ? __ldcg(vals + b0 + u) : -INFINITY;
+#pragma unroll
+            for (int u = 0; u < U; ++u) nc += (b0 + u < hi) && score_key(v[u]) >= tau;
+        }
+        int total;
+        probe(5);
+        int at = block_exclusive_scan<NT>(nc, sc.scan, total, sync);
+        probe(6);
+        if (total <= kTopkCandCap) {
+            for (int b0 = lo; b0 < hi; b0 += U) {
+                float v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) v[u] = b0 + u < hi ? __ldcg(vals + b0 + u) : -INFINITY;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const uint32_t key = score_key(v[u]);
+                    if (b0 + u < hi && key >= tau) {
+                        sc.ckey[at] = key;
+                        sc.cidx[at] = b0 + u;
+                        ++at;
+                    }
+                }
+            }
+            // pad to a multiple of 4 with key 0, below every real key
+            const int total4 = (total + 3) & ~3;
+            if (tid < total4 - total) sc.ckey[total + tid] = 0u;
+            sync();
+            probe(2);
+            const int cper = (total + NT - 1) / NT;  // <= kTopkCandCap / NT <= 32
+            const int clo = min(tid * cper, total), chi = min(clo + cper, total);
+            uint32_t taken = 0u;  // bit c - clo: candidate c is selected
+            int ntaken = 0;
+            const uint4* ck4 = reinterpret_cast<const uint4*>(sc.ckey);
+            for (int c = clo; c < chi; ++c) {
+                const uint32_t kc = sc.ckey[c];
+                int r = 0;
+#pragma unroll 8
+                for (int o4 = 0; o4 < total4 / 4; ++o4) {
+                    const uint4 ko = ck4[o4];
+                    const int o = 4 * o4;
+                    r += (ko.x > kc) || (ko.x == kc && o < c);
+                    r += (ko.y > kc) || (ko.y == kc && o + 1 < c);
+                    r += (ko.z > kc) || (ko.z == kc && o + 2 < c);
+                    r += (ko.w > kc) || (ko.w == kc && o + 3 < c);
+                }
+                if (r < k) {
+                    taken |= 1u << (c - clo);
+                    ++ntaken;
+                }
+            }
+            int pos = block_exclusive_scan<NT>(ntaken, sc.scan, total, sync);
+            for (int c = clo; c < chi; ++c)
+                if (taken >> (c - clo) & 1u) {
+                    if (pub) pub[pos] = sc.cidx[c] + 1;
+                    out[pos++] = sc.cidx[c];
+                }
+            for (int c = k + tid; c < topk; c += NT) out[c] = -1;
+            probe(3);
+            return;
+        }
+        // too many keys >= tau (e.g. many equal scores): exact radix path
     }
     uint32_t prefix = 0, pmask = 0;
     int remaining = k;
@@ -254,7 +429,7 @@ __device__ void block_topk(const float* vals, int n, int topk, int* out, uint32_
         for (int i = tid; i < 256; i += NT) sc.hist[i] = 0;
         sync();
         for (int i = tid; i < n; i += NT) {
-            uint32_t key = score_key(__ldcg(vals + i));
+            const uint32_t key = score_key(__ldcg(vals + i));
             if ((key & pmask) == prefix) atomicAdd(&sc.hist[(key >> shift) & 255u], 1);
         }
         sync();
@@ -281,29 +456,26 @@ __device__ void block_topk(const float* vals, int n, int topk, int* out, uint32_
             }
         }
         sync();
-        const uint32_t digit = (uint32_t)sc.bcast[0];
         remaining -= sc.bcast[1];
-        prefix |= digit << shift;
+        prefix |= (uint32_t)sc.bcast[0] << shift;
         pmask |= 0xffu << shift;
     }
-    const uint32_t tau = prefix;
-    const int need_eq = remaining;  // keys equal to tau that are taken
-
+    // prefix is now the k-th largest key; `remaining` keys equal to it are taken
+    const int need_eq = remaining;
     const int per = (n + NT - 1) / NT;
-    const int lo = tid * per;
-    const int hi = min(lo + per, n);
+    const int lo = min(tid * per, n), hi = min(lo + per, n);
     int n_eq = 0;
-    for (int i = lo; i < hi; ++i) n_eq += (score_key(__ldcg(vals + i)) == tau);
+    for (int i = lo; i < hi; ++i) n_eq += (score_key(__ldcg(vals + i)) == prefix);
     int tot;
-    int eq_rank = block_exclusive_scan<NT>(n_eq, sc.scan, tot, sync);
+    const int eq_rank = block_exclusive_scan<NT>(n_eq, sc.scan, tot, sync);
     int n_sel = 0;
     {
         int r = eq_rank;
         for (int i = lo; i < hi; ++i) {
-            uint32_t key = score_key(__ldcg(vals + i));
-            if (key > tau) {
+            const uint32_t key = score_key(__ldcg(vals + i));
+            if (key > prefix) {
                 ++n_sel;
-            } else if (key == tau) {
+            } else if (key == prefix) {
                 n_sel += (r < need_eq);
                 ++r;
             }
@@ -313,22 +485,22 @@ __device__ void block_topk(const float* vals, int n, int topk, int* out, uint32_
     {
         int r = eq_rank;
         for (int i = lo; i < hi; ++i) {
-            uint32_t key = score_key(__ldcg(vals + i));
+            const uint32_t key = score_key(__ldcg(vals + i));
             bool take = false;
-            if (key > tau) {
+            if (key > prefix) {
                 take = true;
-            } else if (key == tau) {
+            } else if (key == prefix) {
                 take = (r < need_eq);
                 ++r;
             }
             if (take) {
-                int m = map(i);
-                out[pos++] = m;
-                if (mask) atomicOr(&mask[m >> 5], 1u << (m & 31));
+                if (pub) pub[pos] = i + 1;
+                out[pos++] = i;
             }
         }
     }
     for (int c = k + tid; c < topk; c += NT) out[c] = -1;
+    probe(3);
 }
 
 }  // namespace ssa

@@ -4,17 +4,21 @@
 // Gist Tokens", sec. 3.2 scoring, sec. 3.3 top-k + hybrid attention, sec. 3.5
 // coarse-to-fine selection, sec. 3.6 split partial attention + combination):
 //
-//   phase A  score items   -- gist keys (or meta-gist keys) of a slot range
-//   phase B  cand items    -- two-level only: gist keys of candidate chunks
-//   phase C  attention     -- a range of 64-row tiles of the unfolded context
+//   score items    -- gist keys (two level: meta-gist keys) of a slot range
+//   select items   -- one per (sequence, KV head) pair: top-k over its
+//                     scores (or: check a caller-given selection)
+//   cand items     -- two level only: gist keys of the candidate chunks
+//   select items   -- two level only: top-k over the candidates
+//   attention      -- a range of 64-row tiles of the unfolded context
+//   combine items  -- one per pair: merge its split partials into `out`
 //
 // Work is handed out by a global ticket counter in that order.  An item only
-// ever waits for items with smaller tickets (a selection published by the
-// last score item of its pair), and a ticket is only taken by a running
-// block, so the waits always end; each is bounded anyway.  The last score
-// item of a (sequence, KV head) pair runs that pair's top-k in-kernel; the
-// last attention item of a pair merges the pair's partial results (the
-// "combination" step) and resets the pair's control words for the next call.
+// ever waits for items with smaller tickets (a count of finished items, or a
+// published selection), and a ticket is only taken by a running block, so
+// the waits always end; each is bounded anyway.  Items signal completion with
+// a release increment and never wait on it themselves, so no item's tail
+// holds a block.  A combine item resets its pair's control words for the
+// next call.
 //
 // Block layout: 4 consumer warps + 1 producer warp.  The producer streams
 // 64-row tiles with 2-D TMA (128-byte swizzle) into a ring of stages (slot A:
@@ -39,25 +43,31 @@ constexpr int kBoxRows = 64;          // rows per TMA box and per attention tile
 constexpr int kRowmaxCap = 1024;      // summary rows per score item
 constexpr int kBarConsumers = 1;      // named barrier id of the consumer warps
 
-enum : int { K_END = 0, K_SCORE = 1, K_ATTN = 2, K_SELECT = 3 };
+enum : int { K_END = 0, K_SCORE = 1, K_ATTN = 2, K_SELECT = 3, K_COMBINE = 4 };
 enum : int { F_FIRST = 1, F_LAST = 2, F_QLOAD = 4 };
-enum : int { L_GIST = 0, L_META = 1, L_CAND = 2 };
+enum : int { L_GIST = 0, L_META = 1, L_CAND = 2, L_VALIDATE = 3 };
 
-// per-pair control arrays (ints), after [ticket, exit]
+// Control words.  The ticket and exit counters sit in their own 128-byte
+// lines, then one record of Plan::pair_ints words per (sequence, KV head):
+//   line 0   completion counters (score, candidate and attention items);
+//   line 1   published counts: count + 1 (0: not published yet; kBadBit:
+//            the caller's selection was rejected);
+//   then     the published selection itself, entry + 1 (0: not written yet):
+//            topk chunk entries, then topk_super superchunk entries.
+// Every word is written once per call and cleared by the pair's combine item,
+// so a reader needs no separate ready flag: one round of relaxed loads tells
+// whether the count and every entry it needs are there.
+constexpr int kLineInts = 32;
+constexpr int C_TICKET = 0, C_EXIT = kLineInts, C_ARR = 2 * kLineInts;
 enum : int {
-    A_DONE_A = 0,  // phase-A score items finished
-    A_DONE_B,      // phase-B candidate items finished
-    A_READY_S,     // superchunk selection published
-    A_READY,       // chunk selection published
-    A_ATTN,        // attention items finished
-    A_KSEL,        // number of selected chunks
-    A_KSUP,        // number of selected superchunks
-    A_BAD,         // caller's selection rejected
-    A_COUNT
+    A_DONE_A = 0,             // score items (first level) finished
+    A_DONE_B = 1,             // candidate score items finished
+    A_ATTN = 2,               // attention partials written (4 per item)
+    A_COUNT = kLineInts,      // published chunk selection count
+    A_SCOUNT = kLineInts + 1, // published superchunk selection count
+    A_ENTRIES = 2 * kLineInts // chunk entries, then superchunk entries
 };
-constexpr int C_TICKET = 0, C_EXIT = 1, C_ARR = 2;
-
-__host__ __device__ inline int ctrl_words_for(int n_pairs) { return C_ARR + A_COUNT * n_pairs; }
+constexpr int kBadBit = 1 << 30;
 
 struct StageMeta {
     int kind, pair, nvalid, flags;
@@ -79,9 +89,11 @@ struct SmemLayout {
 };
 
 template <int D>
-__host__ __device__ inline SmemLayout smem_layout(int G, int topk, int topk_super) {
+__host__ __device__ inline SmemLayout smem_layout(const Plan& p) {
     SmemLayout L;
     const int NS = Cfg<D>::kStages;
+    const int G = p.G;
+    const int topk_super = p.h2 ? p.topk_super : 0;
     int o = 0;
     L.ring = o;
     o += NS * Cfg<D>::kStageBytes;
@@ -94,22 +106,56 @@ __host__ __device__ inline SmemLayout smem_layout(int G, int topk, int topk_supe
     L.bars = o;
     o += 2 * NS * 8;
     L.psel = o;
-    o += ((topk + 3) / 4 * 4) * 4;
+    o += ((p.topk + 3) / 4 * 4) * 4;
     L.psup = o;
     o += ((topk_super + 3) / 4 * 4) * 4;
     o = (o + 15) / 16 * 16;
     L.uni = o;
-    int merge = kConsumerWarps * G * (D + 2) * 4;
-    int rowmax = kRowmaxCap * 4;
-    int topk_sc = (int)sizeof(TopkScratch);
-    int u = merge > rowmax ? merge : rowmax;
-    u = u > topk_sc ? u : topk_sc;
+    // the consumers use this area for one thing at a time
+    int u = kRowmaxCap * 4;                                      // score rows
+    const int tk = (int)sizeof(TopkScratch);                     // top-k
+    u = u > tk ? u : tk;
+    const int cmb = 3 * G * p.attn_items * kConsumerWarps * 4;   // combination
+    u = u > cmb ? u : cmb;
     o += (u + 15) / 16 * 16;
     L.misc = o;
     o += 64;
     L.total = o + 1024;  // slack to align the ring to 1024 bytes
     return L;
 }
+
+// Timeline trace: builds compiled with SSA_TRACE record (time, event, a, b)
+// per block into Plan::trace; the product build compiles these to nothing.
+enum : int { TR_KSTART = 1, TR_TICKET, TR_P_READY, TR_P_ISSUED, TR_C_FIRST, TR_C_LAST,
+             TR_C_DONE, TR_C_TOPK0, TR_C_TOPK1, TR_C_COMB0, TR_C_COMB1, TR_KEND };
+#ifdef SSA_TRACE
+// Events carry the per-SM cycle counter (cheap); KSTART and KEND also record
+// the global timer in a second event (ev | 0x80) so blocks can be aligned.
+__device__ __forceinline__ void trace_event(const Plan& p, int* counter, int ev, int a, int b) {
+    if (!p.trace) return;
+    const int i = atomicAdd(counter, 1);
+    if (i >= p.trace_cap) return;
+    const uint64_t t = (ev & 0x80) ? now_ns() : (uint64_t)clock64();
+    p.trace[(size_t)blockIdx.x * p.trace_cap + i] =
+        make_uint4((uint32_t)t, (uint32_t)(t >> 32), (uint32_t)ev | ((uint32_t)a << 8), (uint32_t)b);
+}
+#define SSA_TR(ev, a, b) trace_event(p, &misc[15], (ev), (a), (b))
+struct TraceProbe {
+    const Plan& p;
+    int* counter;
+    int pair;
+    __device__ void operator()(int stage) const {
+        if ((threadIdx.x & 31) == 0 && threadIdx.x < 128)
+            trace_event(p, counter, 13, stage + 16 * (threadIdx.x >> 5), pair);
+    }
+};
+#define SSA_PROBE(pair) TraceProbe{p, &misc[15], (pair)}
+#else
+#define SSA_PROBE(pair) NoProbe()
+#define SSA_TR(ev, a, b) ((void)0)
+#endif
+
+__device__ __forceinline__ int pair_of(const StageMeta& m) { return m.pair; }
 
 struct ConsumerSync {
     __device__ void operator()() const { named_sync(kBarConsumers, kConsumers); }
@@ -276,6 +322,53 @@ struct Producer {
         }
     }
 
+    // Reads a published selection (count word, `cap` entries at `ent`) into
+    // shared `dst` as plain indices.  One round of relaxed loads per attempt;
+    // polls with back-off until the count and its entries are all written.
+    // Returns the count and sets `bad` for a rejected caller selection; a
+    // wait that runs out records a timeout and returns 0.
+    __device__ int fetch_selection(const int* cnt_word, const int* ent, int cap, int* dst,
+                                   bool& bad) {
+        const long long c0 = clock64(), lim = wait_cycles(p.wait_limit);
+        unsigned sleep_ns = 32;
+        for (;;) {
+            int cw = lane == 0 ? ld_relaxed(cnt_word) : 0;
+            int e[4];
+            for (int base = 0; base < max(cap, 1); base += 128) {
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int c = base + 32 * r + lane;
+                    e[r] = c < cap ? ld_relaxed(ent + c) : 1;
+                }
+                cw = __shfl_sync(0xffffffffu, cw, 0);
+                // not published yet: write nothing, retry (dst holds `cap` words)
+                const int k = cw == 0 ? 0 : min((cw & (kBadBit - 1)) - 1, cap);
+                bool ok = cw != 0;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int c = base + 32 * r + lane;
+                    if (c < k) {
+                        ok = ok && e[r] != 0;
+                        dst[c] = e[r] - 1;
+                    }
+                }
+                if (!__all_sync(0xffffffffu, ok)) break;
+                if (base + 128 >= min(k, cap)) {
+                    __syncwarp();
+                    bad = (cw & kBadBit) != 0;
+                    return k;
+                }
+            }
+            if (clock64() - c0 > lim) {
+                if (lane == 0) report_status(kStatusTimeout);
+                bad = false;
+                return 0;
+            }
+            __nanosleep(sleep_ns);
+            if (sleep_ns < 512) sleep_ns *= 2;
+        }
+    }
+
     // Rows of [r0, r0+cnt) (in units where slot x covers rows [x*ntok, x*ntok+ntok))
     // that belong to one of the n sorted slots in list[]: bit r set.
     __device__ uint64_t excluded_rows(const int* list, int n, int r0, int cnt, int ntok) {
@@ -312,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const SmemLayout L = smem_layout<D>(p.G, p.topk, p.h2 ? p.topk_super : 0);
+    const SmemLayout L = smem_layout<D>(p);
     constexpr int NS = Cfg<D>::kStages;
     uint8_t* ring = smem + L.ring;
     uint8_t* qbuf = smem + L.qbuf;
@@ -326,6 +419,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
+        misc[15] = 0;
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
@@ -333,15 +427,24 @@ __global__ void __launch_bounds__(kThreads, 2)
         fence_barrier_init();
     }
     __syncthreads();
+    if (threadIdx.x == 0) {
+        SSA_TR(TR_KSTART | 0x80, 0, 0);
+        SSA_TR(TR_KSTART, 0, 0);
+    }
 
+    // ticket phases, in hand-out order
     const int P = p.n_pairs;
-    const int per_a = (p.mode == kModeAttnOnly) ? 1 : p.score_items;
-    const int tot_a = P * per_a;
-    const int tot_b = p.h2 ? P * p.cand_items : 0;
-    const int tot_c = (p.mode == kModeScoreOnly) ? 0 : P * p.attn_items;
-    const int total = tot_a + tot_b + tot_c;
+    const bool so = p.mode == kModeScoreOnly;
+    const int nA = (p.mode == kModeAttnOnly) ? 0 : P * p.score_items;  // score items
+    const int nS1 = so ? 0 : P;                                         // first selection
+    const int nB = p.h2 ? P * p.cand_items : 0;                         // candidate scoring
+    const int nS2 = p.h2 ? P : 0;                                       // second selection
+    const int nC = so ? 0 : P * p.attn_items;                           // attention
+    const int nD = so ? 0 : P;                                          // combination
+    const int oS1 = nA, oB = oS1 + nS1, oS2 = oB + nB, oC = oS2 + nS2, oD = oC + nC;
+    const int total = oD + nD;
     int* ctrl = p.ctrl;
-    auto arr = [&](int a, int pair) -> int* { return ctrl + C_ARR + a * P + pair; };
+    auto arr = [&](int a, int pair) -> int* { return ctrl + C_ARR + pair * p.pair_ints + a; };
 
     // ================================================================ producer
     if (warp == kConsumerWarps) {
@@ -365,9 +468,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                 break;
             }
             if (lane == 0) next_t = dyn ? atomicAdd(ctrl + C_TICKET, 1) : t + (int)gridDim.x;
+            if (lane == 0) SSA_TR(TR_TICKET, t < oS1 ? 0 : t < oC ? 1 : t < oD ? 2 : 3, t);
 
-            if (t < tot_a) {
-                const int pair = t / per_a, i = t % per_a;
+            if (t < oS1) {
+                const int pair = t / p.score_items, i = t % p.score_items;
                 const int b = pair / p.Hkv;
                 int n = seq_len_checked(p, b);
                 if (n < 0) {
@@ -375,9 +479,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     n = 0;
                 }
                 const int M = n / p.C;
-                if (p.mode == kModeAttnOnly) {
-                    pr.push_plain(K_SELECT, pair, F_FIRST | F_LAST, 0);
-                } else if (!p.h2) {
+                if (!p.h2) {
                     const int s0 = i * p.score_spi;
                     const int s1 = min(s0 + p.score_spi, p.M_max);
                     const int vs = max(0, min(M, s1) - s0);
@@ -392,22 +494,51 @@ __global__ void __launch_bounds__(kThreads, 2)
                     pr.score_item(pair, L_META, &tm_kmeta, (pair * p.S_max + s0) * p.gm,
                                   vs * p.gm, vs, 0, pair * p.S_max + s0, p.gm);
                 }
+                if (lane == 0) SSA_TR(TR_P_ISSUED, 0, t);
                 continue;
             }
-            if (t < tot_a + tot_b) {
-                const int u = t - tot_a;
+            if (t < oB || (t >= oS2 && t < oC)) {
+                // selection item: after every score item of the pair is done
+                const bool first = t < oB;
+                const int pair = first ? t - oS1 : t - oS2;
+                int level;
+                if (!first) {
+                    level = L_CAND;
+                    if (lane == 0) wait_geq(arr(A_DONE_B, pair), p.cand_items, p.wait_limit);
+                } else if (p.mode == kModeAttnOnly) {
+                    level = L_VALIDATE;
+                } else {
+                    level = p.h2 ? L_META : L_GIST;
+                    if (lane == 0) wait_geq(arr(A_DONE_A, pair), p.score_items, p.wait_limit);
+                }
+                __syncwarp();
+                pr.push_plain(K_SELECT, pair, F_FIRST | F_LAST, level);
+                continue;
+            }
+            if (t >= oD) {
+                // combination item: after every attention item of the pair
+                const int pair = t - oD;
+                if (lane == 0)
+                    wait_geq(arr(A_ATTN, pair), p.attn_items * kConsumerWarps, p.wait_limit);
+                __syncwarp();
+                pr.push_plain(K_COMBINE, pair, F_FIRST | F_LAST, 0);
+                continue;
+            }
+            if (t < oS2) {
+                const int u = t - oB;
                 const int pair = u / p.cand_items, i = u % p.cand_items;
                 const int b = pair / p.Hkv;
                 int n = seq_len_checked(p, b);
                 if (n < 0) n = 0;
                 const int M = n / p.C, S = M / p.J, R = M - S * p.J;
-                if (lane == 0) wait_geq(arr(A_READY_S, pair), 1, p.wait_limit);
-                __syncwarp();
-                const int ks = __ldcg(arr(A_KSUP, pair));
+                bool bad_s;
+                const int ks = pr.fetch_selection(arr(A_SCOUNT, pair),
+                                                  arr(A_ENTRIES + p.topk, pair), p.topk_super,
+                                                  psup, bad_s);
                 int chunk0 = 0, nch = 0, c0 = 0;
                 if (i < p.topk_super) {
                     if (i < ks) {
-                        chunk0 = __ldcg(p.sel_super + (size_t)pair * p.topk_super + i) * p.J;
+                        chunk0 = psup[i] * p.J;
                         nch = p.J;
                         c0 = i * p.J;
                     }
@@ -418,10 +549,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
                 pr.score_item(pair, L_CAND, &tm_kgist, (pair * p.M_max + chunk0) * p.g, nch * p.g,
                               nch, 0, pair * p.Mc_max + c0, p.g);
+                if (lane == 0) SSA_TR(TR_P_ISSUED, 1, t);
                 continue;
             }
             // ------------------------------------------------ attention item
-            const int u = t - tot_a - tot_b;
+            const int u = t - oC;
             const int pair = u / p.attn_items, item = u % p.attn_items;
             const int b = pair / p.Hkv, j = pair % p.Hkv;
             int n = seq_len_checked(p, b);
@@ -449,20 +581,23 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int u0 = (int)((U * item) / p.attn_items);
             const int u1 = (int)((U * (item + 1)) / p.attn_items);
 
-            bool have_sel = false;
+            bool have_sel = false, bad_sel = false;
             int ksel = 0, ksup = 0;
             auto need_selection = [&]() {
                 if (have_sel) return;
                 have_sel = true;
-                if (lane == 0) wait_geq(arr(A_READY, pair), 1, p.wait_limit);
-                __syncwarp();
-                ksel = min(__ldcg(arr(A_KSEL, pair)), p.topk);
-                ksup = p.h2 ? min(__ldcg(arr(A_KSUP, pair)), p.topk_super) : 0;
-                for (int c = lane; c < ksel; c += 32)
-                    psel[c] = __ldcg(p.sel_idx + (size_t)pair * p.topk + c);
-                for (int c = lane; c < ksup; c += 32)
-                    psup[c] = __ldcg(p.sel_super + (size_t)pair * p.topk_super + c);
-                __syncwarp();
+                ksel = pr.fetch_selection(arr(A_COUNT, pair), arr(A_ENTRIES, pair), p.topk, psel,
+                                          bad_sel);
+                if (p.h2) {
+                    bool b2;
+                    ksup = pr.fetch_selection(arr(A_SCOUNT, pair), arr(A_ENTRIES + p.topk, pair),
+                                              p.topk_super, psup, b2);
+                }
+                if (lane == 0) SSA_TR(TR_P_READY, pair, item);
+                if (bad_sel) {  // rejected caller selection: this pair attends to nothing
+                    ksel = 0;
+                    ksup = 0;
+                }
             };
 
             Tile pending{};
@@ -555,11 +690,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                     tl.y = pair * p.n_max + r0;
                     tl.excl = 0;
                 }
+                if (bad_sel) ok = false;
                 if (!ok) continue;
                 if (has_pending) emit(pending, false);
                 pending = tl;
                 has_pending = true;
             }
+            if (lane == 0) SSA_TR(TR_P_ISSUED, 2, t);
             if (has_pending) {
                 emit(pending, true);
             } else {
@@ -588,8 +725,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float scale = rsqrtf((float)D);
     const float scale_log2 = scale * 1.4426950408889634f;
     float* rowmax = reinterpret_cast<float*>(uni);
-    float* merge = reinterpret_cast<float*>(uni);
     TopkScratch& tsc = *reinterpret_cast<TopkScratch*>(uni);
+    float* cmb = reinterpret_cast<float*>(uni);
     ConsumerSync csync;
 
     uint32_t qa[D / 16][4];
@@ -605,6 +742,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!mbar_wait(&full[stage], (uint32_t)(round & 1), p.wait_limit)) break;
         const StageMeta mt = meta[stage];
         if (mt.kind == K_END) break;
+        if (tid == 0 && (mt.flags & F_FIRST)) SSA_TR(TR_C_FIRST, mt.kind, pair_of(mt));
         const uint32_t slotA = smem_u32(ring + (size_t)stage * Cfg<D>::kStageBytes);
         const uint32_t slotB = slotA + Cfg<D>::kSlotBytes;
         if (mt.flags & F_QLOAD) {
@@ -647,6 +785,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
             if (mt.flags & F_LAST) {
+                if (tid == 0) SSA_TR(TR_C_LAST, K_SCORE, pair);
                 csync();
                 float* dst = mt.item == L_GIST ? p.scores
                              : mt.item == L_META ? p.super_scores
@@ -658,104 +797,193 @@ __global__ void __launch_bounds__(kThreads, 2)
                     dst[mt.dst + i] = v;
                 }
                 csync();
-                if (p.mode != kModeScoreOnly) {
-                    const bool cand = mt.item == L_CAND;
-                    if (tid == 0) {
-                        __threadfence();
-                        const int target = cand ? p.cand_items : p.score_items;
-                        const int old = atomicAdd(arr(cand ? A_DONE_B : A_DONE_A, pair), 1);
-                        misc[0] = (old == target - 1);
-                    }
-                    csync();
-                    if (misc[0]) {
-                        __threadfence();
-                        // ---- selection for this pair (sec. 3.3 top-k; sec. 3.5 levels)
-                        const int b = pair / p.Hkv;
-                        int n = seq_len_checked(p, b);
-                        if (n < 0) n = 0;
-                        const int M = n / p.C;
-                        if (mt.item == L_META) {
-                            const int S = M / p.J;
-                            block_topk<kConsumers>(p.super_scores + (size_t)pair * p.S_max, S,
-                                                   p.topk_super,
-                                                   p.sel_super + (size_t)pair * p.topk_super,
-                                                   nullptr, [](int i) { return i; }, tsc, csync);
-                            csync();
-                            if (tid == 0) {
-                                __threadfence();
-                                *arr(A_KSUP, pair) = min(p.topk_super, S);
-                                st_release(arr(A_READY_S, pair), 1);
-                            }
-                        } else {
-                            int k;
-                            if (mt.item == L_GIST) {
-                                block_topk<kConsumers>(p.scores + (size_t)pair * p.M_max, M, p.topk,
-                                                       p.sel_idx + (size_t)pair * p.topk, nullptr,
-                                                       [](int i) { return i; }, tsc, csync);
-                                k = min(p.topk, M);
-                            } else {
-                                const int S = M / p.J, R = M - S * p.J;
-                                const int ks = min(__ldcg(arr(A_KSUP, pair)), p.topk_super);
-                                const int nc = ks * p.J + R;
-                                const int* ss = p.sel_super + (size_t)pair * p.topk_super;
-                                const int J = p.J;
-                                block_topk<kConsumers>(
-                                    p.cand_scores + (size_t)pair * p.Mc_max, nc, p.topk,
-                                    p.sel_idx + (size_t)pair * p.topk, nullptr,
-                                    [ss, ks, J, S](int c) {
-                                        return c < ks * J ? __ldcg(ss + c / J) * J + c % J
-                                                          : S * J + (c - ks * J);
-                                    },
-                                    tsc, csync);
-                                k = min(p.topk, nc);
-                            }
-                            csync();
-                            if (tid == 0) {
-                                __threadfence();
-                                *arr(A_KSEL, pair) = k;
-                                st_release(arr(A_READY, pair), 1);
+                if (p.mode != kModeScoreOnly && tid == 0)
+                    red_release_add(arr(mt.item == L_CAND ? A_DONE_B : A_DONE_A, pair), 1);
+                if (tid == 0) SSA_TR(TR_C_DONE, K_SCORE, pair);
+            }
+        } else if (mt.kind == K_SELECT) {
+#ifdef SSA_TRACE
+            if (lane == 0) trace_event(p, &misc[15], 13, 15 + 16 * warp, pair);
+#endif
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (tid == 0) SSA_TR(TR_C_TOPK0, mt.item, pair);
+            if (mt.item != L_VALIDATE) {
+                // ---- selection for this pair (sec. 3.3 top-k; sec. 3.5 levels)
+                const int b = pair / p.Hkv;
+                int n = seq_len_checked(p, b);
+                if (n < 0) n = 0;
+                const int M = n / p.C;
+                if (mt.item == L_META) {
+                    const int S = M / p.J;
+                    block_topk<kConsumers>(p.super_scores + (size_t)pair * p.S_max, S,
+                                           p.topk_super,
+                                           p.sel_super + (size_t)pair * p.topk_super,
+                                           tsc, csync, NoProbe(), arr(A_ENTRIES + p.topk, pair));
+                    if (tid == 0) *arr(A_SCOUNT, pair) = min(p.topk_super, S) + 1;
+                } else {
+                    int k;
+                    if (mt.item == L_GIST) {
+                        block_topk<kConsumers>(p.scores + (size_t)pair * p.M_max, M, p.topk,
+                                               p.sel_idx + (size_t)pair * p.topk, tsc, csync,
+                                               SSA_PROBE(pair), arr(A_ENTRIES, pair));
+                        k = min(p.topk, M);
+                    } else {
+                        const int S = M / p.J, R = M - S * p.J;
+                        const int ks = min(p.topk_super, S);
+                        const int nc = ks * p.J + R;
+                        int* out = p.sel_idx + (size_t)pair * p.topk;
+                        block_topk<kConsumers>(p.cand_scores + (size_t)pair * p.Mc_max, nc,
+                                               p.topk, out, tsc, csync);
+                        csync();
+                        // candidate position -> chunk id (increasing map); the
+                        // superchunks come from their published copy (entry + 1)
+                        const int* sup = arr(A_ENTRIES + p.topk, pair);
+                        int* pub = arr(A_ENTRIES, pair);
+                        for (int c = tid; c < p.topk; c += kConsumers) {
+                            const int pos = out[c];
+                            if (pos >= 0) {
+                                int m;
+                                if (pos < ks * p.J) {
+                                    int e = ld_relaxed(sup + pos / p.J);
+                                    for (int tries = 0; e == 0 && tries < (1 << 20); ++tries) {
+                                        __nanosleep(64);
+                                        e = ld_relaxed(sup + pos / p.J);
+                                    }
+                                    if (e == 0) report_status(kStatusTimeout);
+                                    m = (e - 1) * p.J + pos % p.J;
+                                } else {
+                                    m = S * p.J + (pos - ks * p.J);
+                                }
+                                out[c] = m;
+                                pub[c] = m + 1;
                             }
                         }
+                        k = min(p.topk, nc);
                     }
+                    if (tid == 0) *arr(A_COUNT, pair) = k + 1;
+                }
+                csync();  // the shared union area is free again for the next item
+            } else {
+                // ---- validate a caller-given selection and publish it
+                const int b = pair / p.Hkv;
+                int n = seq_len_checked(p, b);
+                if (n < 0) n = 0;
+                const int M = n / p.C;
+                const int* sl = p.sel_idx + (size_t)pair * p.topk;
+                if (tid == 0) {
+                    misc[2] = 1;
+                    misc[3] = 0;
+                }
+                csync();
+                for (int c = tid; c < p.topk; c += kConsumers) {
+                    const int v = sl[c];
+                    const int prev = c > 0 ? sl[c - 1] : -1;
+                    bool ok;
+                    if (v < 0) {
+                        ok = (v == -1);
+                    } else {
+                        ok = (v < M) && (c == 0 || (prev >= 0 && prev < v));
+                        atomicAdd(&misc[3], 1);
+                    }
+                    if (!ok) misc[2] = 0;
+                }
+                csync();
+                const bool good = misc[2] != 0;
+                if (good) {
+                    int* pub = arr(A_ENTRIES, pair);
+                    for (int c = tid; c < misc[3]; c += kConsumers) pub[c] = sl[c] + 1;
+                }
+                if (tid == 0) {
+                    if (!good) report_status(kStatusBadInput);
+                    if (!(p.debug_flags & 1))
+                        st_release(arr(A_COUNT, pair), good ? misc[3] + 1 : (kBadBit | 1));
                 }
                 csync();
             }
-        } else if (mt.kind == K_SELECT) {
+            if (tid == 0) SSA_TR(TR_C_TOPK1, mt.item, pair);
+        } else if (mt.kind == K_COMBINE) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
-            // ---- validate a caller-given selection and publish it
-            const int b = pair / p.Hkv;
-            int n = seq_len_checked(p, b);
-            if (n < 0) n = 0;
-            const int M = n / p.C;
-            const int* sl = p.sel_idx + (size_t)pair * p.topk;
-            if (tid == 0) {
-                misc[2] = 1;
-                misc[3] = 0;
-            }
-            csync();
-            for (int c = tid; c < p.topk; c += kConsumers) {
-                const int v = sl[c];
-                const int prev = c > 0 ? sl[c - 1] : -1;
-                bool ok;
-                if (v < 0) {
-                    ok = (v == -1);
-                } else {
-                    ok = (v < M) && (c == 0 || (prev >= 0 && prev < v));
-                    atomicAdd(&misc[3], 1);
+            if (tid == 0) SSA_TR(TR_C_COMB0, 0, pair);
+            const int G = p.G;
+            // ---- combination of the pair's partial passes (sec. 3.6)
+            const int b = pair / p.Hkv, j = pair % p.Hkv;
+            bool bad = false;
+            if (p.mode == kModeAttnOnly) {
+                if (tid == 0) {
+                    wait_geq(arr(A_COUNT, pair), 1, p.wait_limit);
+                    misc[4] = (ld_acquire(arr(A_COUNT, pair)) & kBadBit) != 0;
                 }
-                if (!ok) misc[2] = 0;
+                csync();
+                bad = misc[4] != 0;
+            }
+            const int NP = p.attn_items * kConsumerWarps;  // one partial per item and warp
+            const size_t stride = (size_t)G * (D + 2);
+            const float* pbase = p.partials + (size_t)pair * NP * stride;
+            float* mS = cmb;               // [G][NP] maxima
+            float* lS = cmb + G * NP;      // [G][NP] sums
+            float* fS = cmb + 2 * G * NP;  // [G][NP] weights
+            for (int base = 0; base < G * NP; base += kConsumers * 4) {
+                float mv[4], lv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int idx = base + u * kConsumers + tid;
+                    const int h = idx / NP, sp = idx - (idx / NP) * NP;
+                    const float* pp = pbase + sp * stride + (size_t)h * (D + 2);
+                    mv[u] = idx < G * NP ? __ldcg(pp) : -INFINITY;
+                    lv[u] = idx < G * NP ? __ldcg(pp + 1) : 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int idx = base + u * kConsumers + tid;
+                    if (idx < G * NP) {
+                        mS[idx] = mv[u];
+                        lS[idx] = lv[u];
+                    }
+                }
             }
             csync();
-            const bool good = misc[2] != 0;
-            if (tid == 0) {
-                if (!good) report_status(kStatusBadInput);
-                __threadfence();
-                *arr(A_KSEL, pair) = good ? misc[3] : 0;
-                *arr(A_BAD, pair) = good ? 0 : 1;
-                if (!(p.debug_flags & 1)) st_release(arr(A_READY, pair), 1);
+            for (int h = warp; h < G; h += kConsumerWarps) {
+                float mx = -INFINITY;
+                for (int sp = lane; sp < NP; sp += 32) mx = fmaxf(mx, mS[h * NP + sp]);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                float Lsum = 0.f;
+                for (int sp = lane; sp < NP; sp += 32) {
+                    const float ms = mS[h * NP + sp];
+                    const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - mx);
+                    fS[h * NP + sp] = f;
+                    Lsum += f * lS[h * NP + sp];
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+                __syncwarp();
+                float* op = p.out + ((size_t)b * p.Hq + (size_t)j * G + h) * D;
+                const float inv = (!bad && Lsum > 0.f) ? 1.f / Lsum : 0.f;
+#pragma unroll
+                for (int d0 = 2 * lane; d0 < D; d0 += 64) {
+                    float ox = 0.f, oy = 0.f;
+                    const float* col = pbase + (size_t)h * (D + 2) + 2 + d0;
+#pragma unroll 8
+                    for (int sp = 0; sp < NP; ++sp) {
+                        const float2 a = __ldcg(reinterpret_cast<const float2*>(col + sp * stride));
+                        const float f = fS[h * NP + sp];
+                        ox += f * a.x;
+                        oy += f * a.y;
+                    }
+                    *reinterpret_cast<float2*>(op + d0) = make_float2(ox * inv, oy * inv);
+                }
             }
             csync();
+            {
+                // clear this pair's record for the next call
+                int* rec = arr(0, pair);
+                const int used = A_ENTRIES + p.topk + (p.h2 ? p.topk_super : 0);
+                for (int a = tid; a < used; a += kConsumers) rec[a] = 0;
+            }
+            if (tid == 0) SSA_TR(TR_C_COMB1, 0, pair);
         } else {  // K_ATTN
             if (mt.flags & F_FIRST) {
                 mrow[0] = mrow[1] = -INFINITY;
@@ -806,7 +1034,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (lane == 0) mbar_arrive(&empty[stage]);
 
             if (mt.flags & F_LAST) {
-                // ---- merge the 4 warps' states, write this item's partial
+                if (tid == 0) SSA_TR(TR_C_LAST, K_ATTN, pair);
+                // ---- write this warp's partial (m, l, acc) for its heads; the
+                // combination merges the warps' partials, so items end without
+                // a block-wide barrier
                 const int G = p.G;
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
@@ -815,92 +1046,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                     l += __shfl_xor_sync(0xffffffffu, l, 2);
                     const int h = g8 + 8 * r;
                     if (h < G) {
-                        float* mg = merge + ((size_t)warp * G + h) * (D + 2);
-                        if (tig == 0) {
-                            mg[0] = mrow[r];
-                            mg[1] = l;
-                        }
+                        float* dstp = p.partials +
+                                      ((((size_t)pair * p.attn_items + mt.item) * kConsumerWarps +
+                                        warp) * G + h) * (D + 2);
+                        if (tig == 0) *reinterpret_cast<float2*>(dstp) = make_float2(mrow[r], l);
 #pragma unroll
-                        for (int nt = 0; nt < D / 8; ++nt) {
-                            mg[2 + nt * 8 + 2 * tig] = acc[nt][2 * r];
-                            mg[2 + nt * 8 + 2 * tig + 1] = acc[nt][2 * r + 1];
-                        }
+                        for (int nt = 0; nt < D / 8; ++nt)
+                            *reinterpret_cast<float2*>(dstp + 2 + nt * 8 + 2 * tig) =
+                                make_float2(acc[nt][2 * r], acc[nt][2 * r + 1]);
                     }
                 }
-                csync();
-                for (int h = warp; h < G; h += kConsumerWarps) {
-                    float mx = -INFINITY;
-#pragma unroll
-                    for (int w = 0; w < kConsumerWarps; ++w)
-                        mx = fmaxf(mx, merge[((size_t)w * G + h) * (D + 2)]);
-                    float f[kConsumerWarps];
-                    float Lsum = 0.f;
-#pragma unroll
-                    for (int w = 0; w < kConsumerWarps; ++w) {
-                        const float mw = merge[((size_t)w * G + h) * (D + 2)];
-                        f[w] = (mw == -INFINITY) ? 0.f : exp2f(mw - mx);
-                        Lsum += f[w] * merge[((size_t)w * G + h) * (D + 2) + 1];
-                    }
-                    float* dstp = p.partials +
-                                  (((size_t)pair * p.attn_items + mt.item) * G + h) * (D + 2);
-                    if (lane == 0) {
-                        dstp[0] = mx;
-                        dstp[1] = Lsum;
-                    }
-                    for (int dd = lane; dd < D; dd += 32) {
-                        float o = 0.f;
-#pragma unroll
-                        for (int w = 0; w < kConsumerWarps; ++w)
-                            o += f[w] * merge[((size_t)w * G + h) * (D + 2) + 2 + dd];
-                        dstp[2 + dd] = o;
-                    }
-                }
-                csync();
-                if (tid == 0) {
-                    __threadfence();
-                    const int old = atomicAdd(arr(A_ATTN, pair), 1);
-                    misc[1] = (old == p.attn_items - 1);
-                }
-                csync();
-                if (misc[1]) {
-                    __threadfence();
-                    // ---- combination of the pair's partial passes (sec. 3.6)
-                    const int b = pair / p.Hkv, j = pair % p.Hkv;
-                    const bool bad = __ldcg(arr(A_BAD, pair)) != 0;
-                    const size_t stride = (size_t)G * (D + 2);
-                    for (int h = warp; h < G; h += kConsumerWarps) {
-                        const float* base =
-                            p.partials + ((size_t)pair * p.attn_items * G + h) * (D + 2);
-                        float mx = -INFINITY;
-                        for (int s = lane; s < p.attn_items; s += 32)
-                            mx = fmaxf(mx, __ldcg(base + s * stride));
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1)
-                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                        float Lsum = 0.f;
-                        for (int s = lane; s < p.attn_items; s += 32) {
-                            const float ms = __ldcg(base + s * stride);
-                            if (ms != -INFINITY) Lsum += exp2f(ms - mx) * __ldcg(base + s * stride + 1);
-                        }
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
-                        float* op = p.out + ((size_t)b * p.Hq + (size_t)j * G + h) * D;
-                        for (int dd = lane; dd < D; dd += 32) {
-                            float o = 0.f;
-                            for (int s = 0; s < p.attn_items; ++s) {
-                                const float ms = __ldcg(base + s * stride);
-                                if (ms != -INFINITY)
-                                    o += exp2f(ms - mx) * __ldcg(base + s * stride + 2 + dd);
-                            }
-                            op[dd] = (!bad && Lsum > 0.f) ? o / Lsum : 0.f;
-                        }
-                    }
-                    csync();
-                    if (tid == 0) {
-                        for (int a = 0; a < A_COUNT; ++a) *arr(a, pair) = 0;
-                    }
-                }
-                csync();
+                __syncwarp();
+                if (lane == 0) red_release_add(arr(A_ATTN, pair), 1);
+                if (tid == 0) SSA_TR(TR_C_DONE, K_ATTN, pair);
             }
         }
         if (++stage == NS) {
@@ -910,6 +1068,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     // ---- last block out resets the ticket for the next launch
     csync();
+    if (tid == 0) {
+        SSA_TR(TR_KEND, 0, 0);
+        SSA_TR(TR_KEND | 0x80, 0, 0);
+    }
     if (p.mode != kModeScoreOnly && tid == 0) {
         __threadfence();
         const int old = atomicAdd(ctrl + C_EXIT, 1);

@@ -102,7 +102,8 @@ struct BlockSync {
 };
 
 // Top-k per pair (block of 128).  level 0: chunks over scores (single level
-// or ssa_topk_chunks); 1: superchunks; 2: candidate chunks (map to chunk ids).
+// or ssa_topk_chunks); 1: superchunks; 2: candidate chunks (positions are
+// mapped to chunk ids afterwards; the map is increasing, so the order holds).
 __global__ void topk_kernel(Plan p, int level, const float* vals, int stride) {
     __shared__ TopkScratch sc;
     const int pr = blockIdx.x;
@@ -112,19 +113,21 @@ __global__ void topk_kernel(Plan p, int level, const float* vals, int stride) {
     const int M = n / p.C;
     const float* v = vals + (size_t)pr * stride;
     if (level == 0) {
-        block_topk<128>(v, M, p.topk, p.sel_idx + (size_t)pr * p.topk, nullptr,
-                        [](int i) { return i; }, sc, BlockSync());
+        block_topk<128>(v, M, p.topk, p.sel_idx + (size_t)pr * p.topk, sc, BlockSync());
     } else if (level == 1) {
-        block_topk<128>(v, M / p.J, p.topk_super, p.sel_super + (size_t)pr * p.topk_super,
-                        nullptr, [](int i) { return i; }, sc, BlockSync());
+        block_topk<128>(v, M / p.J, p.topk_super, p.sel_super + (size_t)pr * p.topk_super, sc,
+                        BlockSync());
     } else {
         const int S = M / p.J;
         const int ks = kept_super(p, S);
         const int nc = ks * p.J + (M - S * p.J);
-        const Plan* pp = &p;
-        block_topk<128>(v, nc, p.topk, p.sel_idx + (size_t)pr * p.topk, nullptr,
-                        [pp, pr, ks, S](int c) { return cand_chunk(*pp, pr, c, ks, S); }, sc,
-                        BlockSync());
+        int* out = p.sel_idx + (size_t)pr * p.topk;
+        block_topk<128>(v, nc, p.topk, out, sc, BlockSync());
+        __syncthreads();
+        for (int c = threadIdx.x; c < p.topk; c += blockDim.x) {
+            const int pos = out[c];
+            if (pos >= 0) out[c] = cand_chunk(p, pr, pos, ks, S);
+        }
     }
 }
 

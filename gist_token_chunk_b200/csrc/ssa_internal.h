@@ -27,6 +27,7 @@ struct Plan {
     int score_spi = 0;     // summary slots per score item
     int cand_items = 0;    // per pair: candidate-chunk scoring (two level)
     int attn_items = 0;    // per pair
+    int pair_ints = 0;     // control words per pair (counters + published selection)
     int mask_words = 0, smask_words = 0;
 
     const void* q = nullptr;
@@ -49,6 +50,9 @@ struct Plan {
     int* ctrl = nullptr;            // control words
     long long wait_limit = 0;       // ns bound of every device-side wait
     int debug_flags = 0;
+    // timeline trace (only written by builds compiled with SSA_TRACE)
+    uint4* trace = nullptr;         // [gridDim.x][trace_cap] events
+    int trace_cap = 0;
 };
 
 // Workspace layout for a plan (byte offsets from the workspace base).

@@ -85,7 +85,7 @@ static cudaError_t launch_fused_d(const Plan& p, cudaStream_t stream) {
         m[5] = m[3];
     }
     if (!ok) return cudaErrorInvalidValue;
-    const fused::SmemLayout L = fused::smem_layout<D>(p.G, p.topk, p.h2 ? p.topk_super : 0);
+    const fused::SmemLayout L = fused::smem_layout<D>(p);
     auto kern = fused::fused_kernel<D>;
     static int attr_done[64][2] = {{0}};
     int dev = 0;
@@ -120,8 +120,8 @@ cudaError_t launch_fused(const Plan& p, cudaStream_t stream) {
 }
 
 int fused_smem_bytes(const Plan& p) {
-    if (p.d == 64) return fused::smem_layout<64>(p.G, p.topk, p.h2 ? p.topk_super : 0).total;
-    return fused::smem_layout<128>(p.G, p.topk, p.h2 ? p.topk_super : 0).total;
+    if (p.d == 64) return fused::smem_layout<64>(p).total;
+    return fused::smem_layout<128>(p).total;
 }
 
 // ----------------------------------------------------------------- generic ---

@@ -21,7 +21,8 @@ Recipe (stated once, used everywhere):
   orthogonal to ``u`` -- a key with cosine 0.3 to the group's query direction.
   For the two-level variant the meta-gist keys of the superchunks holding a
   planted chunk get the same treatment.
-* ``seq_lens`` is either fixed or uniform on an integer interval.
+* ``seq_lens`` is either fixed or uniform on an integer interval (drawn from a
+  CPU generator with the same seed, so it does not depend on the device).
 
 Layouts (row-major, contiguous): q [B,Hq,d]; k_raw, v_raw [B,Hkv,n_max,d];
 k_gist, v_gist [B,Hkv,M_max,g,d] with M_max = n_max // C;
@@ -135,8 +136,12 @@ def make_inputs(w: Workload, seed: int, device="cpu", planted_scale: float = 0.3
         lens = torch.tensor(list(w.seq_lens), dtype=torch.int64)
         assert lens.numel() == B
     elif w.seq_range is not None:
+        # drawn on a CPU generator so the lengths (hence the work per query)
+        # are the same whichever device the tensors are made on
         lo, hi = w.seq_range
-        lens = torch.randint(lo, hi + 1, (B,), generator=gen, device=device).cpu()
+        cpu_gen = torch.Generator()
+        cpu_gen.manual_seed(int(seed))
+        lens = torch.randint(lo, hi + 1, (B,), generator=cpu_gen)
     else:
         lens = torch.full((B,), w.n_max, dtype=torch.int64)
     seq_lens = lens.to(torch.int32)

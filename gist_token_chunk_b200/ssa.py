@@ -19,7 +19,9 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libssa.so")
+# SSA_LIB_PATH selects another build of the same library (e.g. one compiled
+# with the SSA_TRACE timeline instrumentation); default: the in-tree build.
+LIB_PATH = os.environ.get("SSA_LIB_PATH") or os.path.join(_HERE, "libssa.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(

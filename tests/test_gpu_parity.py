@@ -185,3 +185,35 @@ def test_full_size_h2_sampled(ssa, orc):
         stats = check_h2(orc, one, w.C, w.g, w.J, w.gm, w.topk_super, w.topk, out[b:b + 1],
                          sup[b:b + 1], sel[b:b + 1])
         print("hssa_128k", b, stats)
+
+
+@pytest.mark.parametrize("M,topk,levels", [
+    (1024, 32, 0),      # continuous scores: filtered path
+    (2048, 64, 4),      # 4 distinct values: many ties at the boundary
+    (2048, 200, 0),     # k > 128: radix path
+    (2048, 64, 1),      # all equal: more candidates than the filter keeps
+    (777, 100, 9),      # ragged length, ties
+    (4096, 1, 0),
+])
+def test_topk_ties_and_paths(ssa, M, topk, levels):
+    """ssa_topk_chunks on given scores equals the top-k definition on those
+    same fp32 values: largest first, ties to the lower index, ascending."""
+    B, Hkv, C = 2, 3, 16
+    g = torch.Generator().manual_seed(M + topk)
+    sc = torch.randn(B, Hkv, M, generator=g)
+    if levels:
+        sc = torch.randint(0, levels, (B, Hkv, M), generator=g).float()
+    sc[:, 1, 5] = float("nan")          # NaN ranks as -inf
+    sc[:, 2, 7] = -0.0                  # -0 and +0 compare equal
+    lens = torch.tensor([M * C, (M - 3) * C + 5], dtype=torch.int32)
+    sel = ssa.ssa_topk_chunks(sc.cuda(), lens.cuda(), C, topk, M * C)
+    got = sel.cpu().numpy()
+    for b in range(B):
+        Mb = int(lens[b]) // C
+        k = min(topk, Mb)
+        for j in range(Hkv):
+            v = sc[b, j, :Mb].double().numpy()
+            v = np.where(np.isnan(v), -np.inf, v)
+            order = sorted(range(Mb), key=lambda m: (-v[m], m))[:k]
+            want = sorted(order) + [-1] * (topk - k)
+            assert list(got[b, j]) == want, (b, j)
