@@ -22,7 +22,7 @@ namespace {
 thread_local std::string g_err;
 std::atomic<long long> g_wait_limit{0};
 std::atomic<int> g_debug{0};
-std::atomic<int> g_units_per_item{0};
+std::atomic<int> g_max_blocks{0};
 #ifdef SSA_TRACE
 std::atomic<void*> g_trace{nullptr};
 std::atomic<int> g_trace_cap{0};
@@ -32,18 +32,13 @@ std::atomic<int> g_rows_per_score{0};
 constexpr long long kDefaultWaitLimitNs = 2000000000ll;  // 2 s
 constexpr int kMaxG = 16;
 constexpr int kMaxTopk = 1024;
-constexpr int kRowsPerScoreItem = 512;
-constexpr int kUnitsPerAttnItem = 12;
+constexpr int kRowsPerScoreItem = 1024;
 
 int rows_per_score_item() {
     int v = g_rows_per_score.load();
     return v > 0 ? v : kRowsPerScoreItem;
 }
-int units_per_attn_item() {
-    int v = g_units_per_item.load();
-    return v > 0 ? v : kUnitsPerAttnItem;
-}
-constexpr int kMaxAttnItems = 1024;
+int max_blocks() { return g_max_blocks.load(); }
 
 ssa_status fail(ssa_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 ssa_status fail(ssa_status s, const char* fmt, ...) {
@@ -116,7 +111,9 @@ void fill_shape(ssa::Plan& p, const ssa_shape* s, int C, int g, int topk) {
 #endif
 }
 
-bool fused_path(const ssa::Plan& p) { return p.dtype == SSA_BF16 && (p.d == 64 || p.d == 128); }
+bool fused_path(const ssa::Plan& p) {
+    return p.dtype == SSA_BF16 && (p.d == 64 || p.d == 128) && p.B <= ssa::kFusedMaxB;
+}
 
 ssa_status check_sizes(const ssa::Plan& p) {
     const long long P = p.n_pairs;
@@ -143,37 +140,8 @@ ssa_status check_sizes(const ssa::Plan& p) {
 namespace ssa {
 
 void plan_decompose(Plan& p) {
-    const int ntok = p.h2 ? p.gm : p.g;
-    const int slots = p.h2 ? p.S_max : p.M_max;
-    int spi = rows_per_score_item() / (ntok > 0 ? ntok : 1);
-    if (spi < 1) spi = 1;
-    if (spi * ntok > 1024) spi = 1024 / ntok;
-    if (spi < 1) spi = 1;
-    p.score_spi = spi;
-    p.score_items = slots > 0 ? cdiv(slots, spi) : 1;
-    p.cand_items = p.h2 ? p.topk_super + 1 : 0;
-    // attention units of the largest possible sequence
-    const int tpc = cdiv(p.C, 64);
-    const int tail_units = cdiv(p.C - 1, 64);
-    long long U;
-    if (!p.h2) {
-        const int kmax = p.topk < p.M_max ? p.topk : p.M_max;
-        U = cdiv((long long)p.M_max * p.g, 64) + (long long)kmax * tpc + tail_units;
-    } else {
-        const int ks = p.topk_super < p.S_max ? p.topk_super : p.S_max;
-        const long long nc = (long long)ks * p.J + (p.J - 1);
-        const long long kc = p.topk < nc ? p.topk : nc;
-        U = cdiv((long long)p.S_max * p.gm, 64) + (long long)ks * cdiv((long long)p.J * p.g, 64) +
-            cdiv((long long)(p.J - 1) * p.g, 64) + kc * tpc + tail_units;
-    }
-    const int upi = units_per_attn_item();
-    int items = (int)((U + upi - 1) / upi);
-    if (items < 1) items = 1;
-    if (items > kMaxAttnItems) items = kMaxAttnItems;
-    // the combination stages 3 floats per (query head, item) in shared memory
-    const int cap = 16384 / (48 * (p.G > 0 ? p.G : 1));
-    if (items > cap) items = cap;
-    p.attn_items = items;
+    p.grid_cap = max_blocks();
+    p.score_rows = rows_per_score_item();
     // counters line, published-count line, then the published selection(s)
     p.pair_ints = 64 + (p.topk + (p.h2 ? p.topk_super : 0) + 31) / 32 * 32;
     p.mask_words = (cdiv(p.M_max, 32) + 3) / 4 * 4;
@@ -197,8 +165,9 @@ WsLayout plan_layout(const Plan& p) {
     L.cand_scores = take(p.h2 ? P * p.Mc_max * 4 : 0);
     L.chunk_mask = take(0);
     L.super_mask = take(0);
-    // one partial per (pair, attention item, consumer warp, query head)
-    L.partials = take(fused_path(p) ? P * p.attn_items * 4 * p.G * (p.d + 2) * 4 : 0);
+    // one partial per (attention list, segment slot, query head)
+    L.partials =
+        take(fused_path(p) ? 3 * (ssa::kFusedMaxGrid + P) * p.G * (size_t)(p.d + 2) * 4 : 0);
     L.total = o;
     return L;
 }
@@ -217,32 +186,53 @@ void attach_ws(ssa::Plan& p, void* ws) {
     p.partials = reinterpret_cast<float*>(base + L.partials);
 }
 
-// Control words are left zero by every call, but only the control region of
-// that call's size.  A later call with more (sequence, KV head) pairs has a
-// larger control region that may cover scratch data of earlier calls, so the
-// library remembers the control size each workspace was last used with and
-// zeroes the region (stream-ordered) only when it grows.
+// A fused call leaves its control words and its score areas zero (the
+// kernel clears what it used), but only for its own layout.  The library
+// remembers, per workspace, what the last call left: all zero (after
+// ssa_workspace_init, up to a size), a fused layout (control + score bytes
+// that are zero), or unknown (a generic-path call).  Before a fused call whose
+// layout is not already known to be zero, it zeroes that prefix
+// (stream-ordered).
+struct WsState {
+    int kind = 0;      // 0: zero up to `bytes`; 1: fused layout; 2: unknown
+    size_t bytes = 0;  // kind 0: zeroed bytes; kind 1: zero prefix of the layout
+    size_t ctrl = 0;   // kind 1: control bytes of the layout
+};
 std::mutex g_ws_mu;
-std::unordered_map<const void*, size_t> g_ws_ctrl;
+std::unordered_map<const void*, WsState> g_ws;
 
 void note_ws_zeroed(const void* ws, size_t bytes) {
     std::lock_guard<std::mutex> lk(g_ws_mu);
-    g_ws_ctrl[ws] = bytes;
+    WsState st;
+    st.kind = 0;
+    st.bytes = bytes;
+    g_ws[ws] = st;
 }
 
-cudaError_t prepare_ctrl(void* ws, size_t ctrl_bytes, cudaStream_t stream) {
+cudaError_t prepare_ws(void* ws, bool fused, size_t ctrl_bytes, size_t clean_bytes,
+                       cudaStream_t stream) {
     bool zero = false;
     {
         std::lock_guard<std::mutex> lk(g_ws_mu);
-        auto it = g_ws_ctrl.find(ws);
-        if (it == g_ws_ctrl.end()) {
-            g_ws_ctrl[ws] = ctrl_bytes;  // first use: the caller zeroed it
-        } else {
-            zero = ctrl_bytes > it->second;
-            it->second = ctrl_bytes;
+        auto it = g_ws.find(ws);
+        WsState next;
+        next.kind = fused ? 1 : 2;
+        next.bytes = clean_bytes;
+        next.ctrl = ctrl_bytes;
+        if (fused) {
+            if (it == g_ws.end()) {
+                zero = false;  // first use: the caller zeroed it
+            } else if (it->second.kind == 0) {
+                zero = it->second.bytes < clean_bytes;
+            } else if (it->second.kind == 1) {
+                zero = !(it->second.bytes == clean_bytes && it->second.ctrl == ctrl_bytes);
+            } else {
+                zero = true;
+            }
         }
+        g_ws[ws] = next;
     }
-    return zero ? cudaMemsetAsync(ws, 0, ctrl_bytes, stream) : cudaSuccess;
+    return zero ? cudaMemsetAsync(ws, 0, clean_bytes, stream) : cudaSuccess;
 }
 
 // Runs a workspace-using plan: caller workspace, or a stream-ordered one.
@@ -266,7 +256,9 @@ ssa_status run_with_ws(ssa::Plan& p, void* ws, size_t ws_bytes, cudaStream_t str
     }
     attach_ws(p, ws);
     if (!own) {
-        cudaError_t e = prepare_ctrl(ws, (size_t)ssa::ctrl_words(p) * 4, stream);
+        const ssa::WsLayout L = ssa::plan_layout(p);
+        cudaError_t e = prepare_ws(ws, fused_path(p), (size_t)ssa::ctrl_words(p) * 4, L.partials,
+                                   stream);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(control words)");
     }
     cudaError_t e = fused_path(p) ? ssa::launch_fused(p, stream) : ssa::launch_generic(p, stream);
@@ -471,8 +463,8 @@ void ssa_set_wait_limit(int64_t ns) { g_wait_limit.store(ns > 0 ? ns : 0); }
 
 void ssa_set_debug_flags(int32_t flags) { g_debug.store(flags); }
 
-void ssa_set_tuning(int32_t units_per_attn_item, int32_t rows_per_score_item) {
-    g_units_per_item.store(units_per_attn_item > 0 ? units_per_attn_item : 0);
+void ssa_set_tuning(int32_t max_blocks, int32_t rows_per_score_item) {
+    g_max_blocks.store(max_blocks > 0 ? max_blocks : 0);
     g_rows_per_score.store(rows_per_score_item > 0 ? rows_per_score_item : 0);
 }
 

@@ -188,6 +188,36 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+// The same with an L2 eviction-priority policy (from l2_policy_*).
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, int x, int y,
+                                                 uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+// Prefetch one 2-D box of a tensor map into L2 (no shared memory involved).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+
+// L2 policies: keep lines that are read again soon; drop single-use lines first.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 // 1-D bulk copy global -> shared (16-byte aligned addresses, size % 16 == 0).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
                                           uint64_t* bar) {
@@ -247,6 +277,20 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Barrier over `nthreads` threads that also ORs a predicate across them.
+__device__ __forceinline__ bool named_sync_or(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
 // ------------------------------------------------------ block scan ---
 // Exclusive prefix sum over the NT threads that call it together; `sync`
 // synchronises exactly those threads; `sm` holds NT/32 + 1 ints.
@@ -280,14 +324,15 @@ struct NoProbe {
 };
 
 constexpr int kTopkCandCap = 512;  // candidates the filtered selection ranks directly
+constexpr int kTopkRegPer = 16;    // values per thread the filtered selection holds
 
 struct TopkScratch {
     int hist[256];
     int bcast[4];
     int scan[8];
     alignas(16) uint32_t tmax[128];           // per-thread key maxima (NT <= 128)
-    alignas(16) uint32_t ckey[kTopkCandCap];  // candidate keys, in index order
-    int cidx[kTopkCandCap];                   // candidate positions
+    // candidates: key << 32 | ~position (a larger value ranks first)
+    alignas(16) unsigned long long ccomp[kTopkCandCap];
 };
 
 // Deterministic top-k over vals[0..n) (sec. 3.3 "top-k chunks"): selects the
@@ -297,20 +342,47 @@ struct TopkScratch {
 // vals is read with L2-coherent loads (it may have been written by other
 // blocks of the same launch), in batches so that many loads are in flight.
 //
-// Filtered path (k <= NT): each thread takes the maximum key of its strided
-// share; the k-th largest of those NT maxima is a lower bound tau on the k-th
-// largest key (k distinct keys reach it), so every selected key -- ties at
-// the boundary included -- is >= tau.  The keys >= tau are compacted in index
-// order and ranked exactly by counting (larger key first, then lower index).
-// Fallback (k > NT, or more than kTopkCandCap keys >= tau): MSB-first radix
-// select on the order-preserving 32-bit key, reading vals from L2 per pass.
+// Filtered path (k <= NT, n <= NT * kTopkRegPer): one round of loads puts
+// every value in registers (strided, coalesced); each thread takes its
+// maximum key; the k-th largest of those NT maxima is a lower bound tau on
+// the k-th largest key (k distinct keys reach it), so every selected key --
+// ties at the boundary included -- is >= tau.  The keys >= tau go to shared
+// memory as (key, position) pairs and are ranked exactly by counting (larger
+// key first, then lower position); the k best are then ordered by position.
+// Fallback (k > NT, larger n, or more than kTopkCandCap keys >= tau):
+// MSB-first radix select on the order-preserving 32-bit key, reading vals
+// from L2 per pass.
 // If `pub` is not null, each selected position i is also written there as
 // pub[rank] = i + 1 (a published copy that is never 0 once written).
+// With poll_ns > 0, vals may still be being written by other blocks: a value
+// whose bits are all zero is not written yet (writers store +0 as -0), and
+// the loads repeat (for at most poll_ns) until every value is present.
+// Sync must provide or_(bool): a barrier that ORs a predicate.
 template <int NT, class Sync, class Probe = NoProbe>
 __device__ void block_topk(const float* vals, int n, int topk, int* out, TopkScratch& sc,
-                           Sync sync, Probe probe = Probe(), int* pub = nullptr) {
+                           Sync sync, Probe probe = Probe(), int* pub = nullptr,
+                           long long poll_ns = 0) {
     const int tid = threadIdx.x & (NT - 1);
     const int k = topk < n ? topk : n;
+    // polling: wait until every value is present (the filtered path below
+    // does this in its own loads)
+    auto poll_all = [&]() {
+        const int* iv = reinterpret_cast<const int*>(vals);
+        const long long c0 = clock64(), lim = wait_cycles(poll_ns);
+        for (;;) {
+            bool missing = false;
+            for (int i = tid; i < n; i += NT) missing |= ld_relaxed(iv + i) == 0;
+            // every thread takes the same branch: the vote decides
+            const bool expired = clock64() - c0 > lim;
+            if (!sync.or_(missing && !expired)) {
+                if (missing) report_status(kStatusTimeout);
+                break;
+            }
+            __nanosleep(128);
+        }
+    };
+    const bool filtered = k > 0 && k < n && k <= NT && n <= NT * kTopkRegPer;
+    if (poll_ns > 0 && !filtered && n > 0) poll_all();
     if (k <= 0) {
         for (int c = tid; c < topk; c += NT) out[c] = -1;
         return;
@@ -322,102 +394,135 @@ __device__ void block_topk(const float* vals, int n, int topk, int* out, TopkScr
         }
         return;
     }
-    constexpr int U = 8;
-    if (k <= NT) {
-        uint32_t mx = 0u;
-        for (int base = 0; base < n; base += NT * U) {
-            float v[U];
+    if (filtered) {
+        // one round of loads: every value of the range, held in registers
+        uint32_t key[kTopkRegPer];
+        if (poll_ns <= 0) {
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int i = base + u * NT + tid;
-                v[u] = i < n ? __ldcg(vals + i) : -INFINITY;
+            for (int u = 0; u < kTopkRegPer; ++u) {
+                const int i = u * NT + tid;
+                key[u] = i < n ? score_key(__ldcg(vals + i)) : 0u;  // 0: below every real key
             }
+        } else {
+            const int* iv = reinterpret_cast<const int*>(vals);
+            const long long c0 = clock64(), lim = wait_cycles(poll_ns);
+            unsigned sleep_ns = 32;
+            for (;;) {
+                bool missing = false;
 #pragma unroll
-            for (int u = 0; u < U; ++u) mx = max(mx, score_key(v[u]));
+                for (int u = 0; u < kTopkRegPer; ++u) {
+                    const int i = u * NT + tid;
+                    const int b = i < n ? ld_relaxed(iv + i) : 1;
+                    missing |= (b == 0);
+                    key[u] = i < n ? score_key(__int_as_float(b)) : 0u;
+                }
+                // every thread takes the same branch: the vote decides
+                const bool expired = clock64() - c0 > lim;
+                if (!sync.or_(missing && !expired)) {
+                    if (missing) report_status(kStatusTimeout);
+                    break;
+                }
+                __nanosleep(sleep_ns);
+                if (sleep_ns < 256) sleep_ns *= 2;
+            }
         }
+        uint32_t mx = 0u;
+#pragma unroll
+        for (int u = 0; u < kTopkRegPer; ++u) mx = max(mx, key[u]);
         sc.tmax[tid] = mx;
+        if (tid == 0) sc.bcast[2] = 0;
         probe(1);
         sync();
-        int rank = 0;
+        // tau: the k-th largest of the NT maxima (ties by thread), reached by
+        // at least k distinct values, so every selected value is >= tau
+        int r0 = 0, r1 = 0, r2 = 0, r3 = 0;  // independent partial counts
         const uint4* tm4 = reinterpret_cast<const uint4*>(sc.tmax);
 #pragma unroll
         for (int j4 = 0; j4 < NT / 4; ++j4) {
             const uint4 o = tm4[j4];
             const int j = 4 * j4;
-            rank += (o.x > mx) || (o.x == mx && j < tid);
-            rank += (o.y > mx) || (o.y == mx && j + 1 < tid);
-            rank += (o.z > mx) || (o.z == mx && j + 2 < tid);
-            rank += (o.w > mx) || (o.w == mx && j + 3 < tid);
+            r0 += int(o.x > mx) | (int(o.x == mx) & int(j < tid));
+            r1 += int(o.y > mx) | (int(o.y == mx) & int(j + 1 < tid));
+            r2 += int(o.z > mx) | (int(o.z == mx) & int(j + 2 < tid));
+            r3 += int(o.w > mx) | (int(o.w == mx) & int(j + 3 < tid));
         }
+        const int rank = (r0 + r1) + (r2 + r3);
+        probe(7);
         if (rank == k - 1) sc.bcast[3] = (int)mx;
-        probe(4);
         sync();
+        probe(8);
         const uint32_t tau = (uint32_t)sc.bcast[3];
-        // contiguous share [lo, hi) per thread, loaded in batches of U
-        const int per = (n + NT - 1) / NT;
-        const int lo = min(tid * per, n), hi = min(lo + per, n);
-        int nc = 0;
-        for (int b0 = lo; b0 < hi; b0 += U) {
-            float v[U];
+        // candidates (key >= tau) into shared memory, in any order: the
+        // ranking below compares (key, position) pairs, never slots.  Each
+        // warp reserves room for its candidates with one shared atomic.
+        int mine = 0;
 #pragma unroll
-            for (int u = 0; u < U; ++u) v[u] = b0 + u < hi ? __ldcg(vals + b0 + u) : -INFINITY;
+        for (int u = 0; u < kTopkRegPer; ++u) mine += (key[u] >= tau && key[u] != 0u);
+        const int lane = threadIdx.x & 31;
+        int incl = mine;
 #pragma unroll
-            for (int u = 0; u < U; ++u) nc += (b0 + u < hi) && score_key(v[u]) >= tau;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
         }
-        int total;
+        int base = 0;
+        if (lane == 31 && incl > 0) base = atomicAdd(&sc.bcast[2], incl);
+        base = __shfl_sync(0xffffffffu, base, 31) + incl - mine;
+#pragma unroll
+        for (int u = 0; u < kTopkRegPer; ++u) {
+            if (key[u] >= tau && key[u] != 0u) {
+                if (base < kTopkCandCap)
+                    sc.ccomp[base] = ((unsigned long long)key[u] << 32) |
+                                     (uint32_t)~(uint32_t)(u * NT + tid);
+                ++base;
+            }
+        }
         probe(5);
-        int at = block_exclusive_scan<NT>(nc, sc.scan, total, sync);
-        probe(6);
-        if (total <= kTopkCandCap) {
-            for (int b0 = lo; b0 < hi; b0 += U) {
-                float v[U];
-#pragma unroll
-                for (int u = 0; u < U; ++u) v[u] = b0 + u < hi ? __ldcg(vals + b0 + u) : -INFINITY;
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const uint32_t key = score_key(v[u]);
-                    if (b0 + u < hi && key >= tau) {
-                        sc.ckey[at] = key;
-                        sc.cidx[at] = b0 + u;
-                        ++at;
-                    }
-                }
-            }
-            // pad to a multiple of 4 with key 0, below every real key
-            const int total4 = (total + 3) & ~3;
-            if (tid < total4 - total) sc.ckey[total + tid] = 0u;
+        sync();
+        probe(9);
+        const int total = sc.bcast[2];
+        if (total <= kTopkCandCap - 1) {
+            // exact rank of each candidate (pairs of entries per load; an
+            // odd count is padded with 0, below every candidate); the k best
+            // land in sel[rank]
+            int* sel = sc.hist;
+            const int total2 = (total + 1) >> 1;
+            if (tid == 0 && (total & 1)) sc.ccomp[total] = 0ull;
+            if (tid < 4 - (k & 3) && (k & 3)) sel[k + tid] = 0x7fffffff;  // pad for the placement
             sync();
-            probe(2);
-            const int cper = (total + NT - 1) / NT;  // <= kTopkCandCap / NT <= 32
-            const int clo = min(tid * cper, total), chi = min(clo + cper, total);
-            uint32_t taken = 0u;  // bit c - clo: candidate c is selected
-            int ntaken = 0;
-            const uint4* ck4 = reinterpret_cast<const uint4*>(sc.ckey);
-            for (int c = clo; c < chi; ++c) {
-                const uint32_t kc = sc.ckey[c];
-                int r = 0;
-#pragma unroll 8
-                for (int o4 = 0; o4 < total4 / 4; ++o4) {
-                    const uint4 ko = ck4[o4];
-                    const int o = 4 * o4;
-                    r += (ko.x > kc) || (ko.x == kc && o < c);
-                    r += (ko.y > kc) || (ko.y == kc && o + 1 < c);
-                    r += (ko.z > kc) || (ko.z == kc && o + 2 < c);
-                    r += (ko.w > kc) || (ko.w == kc && o + 3 < c);
+            const ulonglong2* cc2 = reinterpret_cast<const ulonglong2*>(sc.ccomp);
+            for (int c = tid; c < total; c += NT) {
+                const unsigned long long mine = sc.ccomp[c];
+                int ra = 0, rb = 0;
+#pragma unroll 4
+                for (int o = 0; o < total2; ++o) {
+                    const ulonglong2 v = cc2[o];
+                    ra += v.x > mine;
+                    rb += v.y > mine;
                 }
-                if (r < k) {
-                    taken |= 1u << (c - clo);
-                    ++ntaken;
-                }
+                const int r = ra + rb;
+                if (r < k) sel[r] = (int)~(uint32_t)mine;
             }
-            int pos = block_exclusive_scan<NT>(ntaken, sc.scan, total, sync);
-            for (int c = clo; c < chi; ++c)
-                if (taken >> (c - clo) & 1u) {
-                    if (pub) pub[pos] = sc.cidx[c] + 1;
-                    out[pos++] = sc.cidx[c];
+            sync();
+            // ascending positions: place each selected one by counting smaller ones
+            if (tid < k) {
+                const int mine = sel[tid];
+                int pa = 0, pb = 0, pc = 0, pd = 0;
+                const int4* s4 = reinterpret_cast<const int4*>(sel);
+                for (int j = 0; j < (k + 3) >> 2; ++j) {
+                    const int4 v = s4[j];
+                    pa += v.x < mine;
+                    pb += v.y < mine;
+                    pc += v.z < mine;
+                    pd += v.w < mine;
                 }
+                const int pos = (pa + pb) + (pc + pd);
+                out[pos] = mine;
+                if (pub) pub[pos] = mine + 1;
+            }
             for (int c = k + tid; c < topk; c += NT) out[c] = -1;
             probe(3);
+            sync();  // sel (the histogram area) is free again
             return;
         }
         // too many keys >= tau (e.g. many equal scores): exact radix path

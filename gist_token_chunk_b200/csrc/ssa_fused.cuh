@@ -1,33 +1,40 @@
 // ssa_fused.cuh -- the fused, persistent decode kernel for bf16, d in {64,128}.
 //
-// One launch runs the whole decode step ("Simplified Sparse Attention via
-// Gist Tokens", sec. 3.2 scoring, sec. 3.3 top-k + hybrid attention, sec. 3.5
-// coarse-to-fine selection, sec. 3.6 split partial attention + combination):
+// One cooperative launch runs the whole decode step ("Simplified Sparse
+// Attention via Gist Tokens": sec. 3.2 gist scoring, sec. 3.3 top-k and hybrid
+// attention over the unfolded context, sec. 3.5 coarse-to-fine selection,
+// sec. 3.6 split partial attention plus combination).
 //
-//   score items    -- gist keys (two level: meta-gist keys) of a slot range
-//   select items   -- one per (sequence, KV head) pair: top-k over its
-//                     scores (or: check a caller-given selection)
-//   cand items     -- two level only: gist keys of the candidate chunks
-//   select items   -- two level only: top-k over the candidates
-//   attention      -- a range of 64-row tiles of the unfolded context
-//   combine items  -- one per pair: merge its split partials into `out`
+// Static, byte-balanced schedule.  The work of a call is laid out as global
+// lists; each is the concatenation over (sequence, KV head) pairs of that
+// pair's elements:
+//   SCORE  summary slots to score: chunks (single level) or superchunks
+//   META   64-row tiles of meta-gist K/V                       (two level)
+//   CAND   candidate chunks to score                           (two level)
+//   GIST   64-row tiles of gist K/V: every complete chunk (single level) or
+//          the candidate chunks (two level)
+//   RAW    64-row tiles of raw K/V: the selected chunks, then the tail
+// Every block takes an equal contiguous share of every list.  A share may
+// cross pair boundaries; a (block, pair) intersection is a segment and yields
+// one partial (m, l, o) per query head.  Each block runs, in this order: its
+// SCORE share; the top-k of the pairs it owns; [its META share; its CAND
+// share; the second top-k of its pairs;] its GIST share; its RAW share; the
+// combination of the pairs it owns.  A wait (a pair's scores complete, a
+// selection published, a pair's partials complete) is always on work of an
+// earlier phase, which never waits on a later one, and all blocks are
+// co-resident (cooperative launch), so every wait ends; each is also bounded.
 //
-// Work is handed out by a global ticket counter in that order.  An item only
-// ever waits for items with smaller tickets (a count of finished items, or a
-// published selection), and a ticket is only taken by a running block, so
-// the waits always end; each is bounded anyway.  Items signal completion with
-// a release increment and never wait on it themselves, so no item's tail
-// holds a block.  A combine item resets its pair's control words for the
-// next call.
+// GIST and META tiles need the selection only to mask excluded rows, so the
+// producer issues them before the selection exists and the consumers apply
+// the mask once it is published: the selection latency hides behind loads.
 //
 // Block layout: 4 consumer warps + 1 producer warp.  The producer streams
 // 64-row tiles with 2-D TMA (128-byte swizzle) into a ring of stages (slot A:
-// keys, slot B: values; score stages use both slots for keys) and never
-// stalls the consumers on control flow.  Each consumer warp takes 16 rows of
-// every stage: Q.K^T and P.V run on tensor cores (mma.sync m16n8k16, bf16 in,
-// fp32 accumulate; the GQA group's query heads are the M rows), the softmax
-// is an fp32 online softmax in the log2 domain, and P is fed to the P.V
-// product as bf16 hi + lo parts so it keeps ~16 significant bits.
+// keys, slot B: values; score stages use both slots for keys).  Each consumer
+// warp takes 16 rows of every stage: Q.K^T and P.V run on tensor cores
+// (mma.sync m16n8k16, bf16 in, fp32 accumulate; the GQA group's query heads
+// are the M rows), the softmax is an fp32 online softmax in the log2 domain,
+// and P enters the P.V product as bf16 hi + lo parts (~16 significant bits).
 #pragma once
 
 #include "ssa_device.cuh"
@@ -40,29 +47,32 @@ constexpr int kConsumerWarps = 4;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;
 constexpr int kBoxRows = 64;          // rows per TMA box and per attention tile
-constexpr int kRowmaxCap = 1024;      // summary rows per score item
+constexpr int kRowmaxCap = 1024;      // summary rows per score sub-item
 constexpr int kBarConsumers = 1;      // named barrier id of the consumer warps
+constexpr int kMaxGrid = kFusedMaxGrid;
+constexpr int kMaxTopkEntries = 1024;  // largest topk / topk_super the library accepts
 
 enum : int { K_END = 0, K_SCORE = 1, K_ATTN = 2, K_SELECT = 3, K_COMBINE = 4 };
 enum : int { F_FIRST = 1, F_LAST = 2, F_QLOAD = 4 };
-enum : int { L_GIST = 0, L_META = 1, L_CAND = 2, L_VALIDATE = 3 };
+enum : int { L_SCORE = 0, L_CAND = 1, L_META = 2, L_GIST = 3, L_RAW = 4, kNumLists = 5 };
+// what a K_SELECT stage does
+enum : int { SEL_CHUNKS = 0, SEL_SUPER = 1, SEL_CAND = 2, SEL_VALIDATE = 3 };
+// which published selection masks the rows of an attention segment
+enum : int { MASK_NONE = 0, MASK_CHUNK = 1, MASK_SUPER = 2 };
 
-// Control words.  The ticket and exit counters sit in their own 128-byte
-// lines, then one record of Plan::pair_ints words per (sequence, KV head):
-//   line 0   completion counters (score, candidate and attention items);
+// Control words: after a 64-word header (unused), one record of
+// Plan::pair_ints words per pair:
+//   line 0   completion counter: attention segments written;
 //   line 1   published counts: count + 1 (0: not published yet; kBadBit:
 //            the caller's selection was rejected);
-//   then     the published selection itself, entry + 1 (0: not written yet):
-//            topk chunk entries, then topk_super superchunk entries.
-// Every word is written once per call and cleared by the pair's combine item,
-// so a reader needs no separate ready flag: one round of relaxed loads tells
-// whether the count and every entry it needs are there.
+//   then     the published selection, entry + 1 (0: not written yet): topk
+//            chunk entries, then topk_super superchunk entries.
+// Every word is written at most once per call and cleared by the pair's
+// combination, so a reader needs no separate ready flag.
 constexpr int kLineInts = 32;
-constexpr int C_TICKET = 0, C_EXIT = kLineInts, C_ARR = 2 * kLineInts;
+constexpr int C_ARR = 2 * kLineInts;
 enum : int {
-    A_DONE_A = 0,             // score items (first level) finished
-    A_DONE_B = 1,             // candidate score items finished
-    A_ATTN = 2,               // attention partials written (4 per item)
+    A_ATTN = 2,               // attention segments written
     A_COUNT = kLineInts,      // published chunk selection count
     A_SCOUNT = kLineInts + 1, // published superchunk selection count
     A_ENTRIES = 2 * kLineInts // chunk entries, then superchunk entries
@@ -71,9 +81,16 @@ constexpr int kBadBit = 1 << 30;
 
 struct StageMeta {
     int kind, pair, nvalid, flags;
-    int row_off, item, nslot, npad;
-    int dst, ntok;
-    uint32_t rmask_lo, rmask_hi;  // attention: excluded rows of the tile
+    // K_SCORE: a0 row offset in the sub-item, a1 slots, a2 -inf pad slots,
+    //          a3 destination index, a4 rows per slot, a5 level (1: candidates)
+    // K_ATTN:  a0 first summary row of the tile, a1 mask kind, a2 rows per
+    //          masked slot, a3 attention list (0 META, 1 GIST, 2 RAW)
+    // K_SELECT: a0 what to do (SEL_*)
+    // Data stages go to the consumer warps in turn (one warp per stage);
+    // every warp still visits every stage (release, segment start and end).
+    int a0, a1, a2, a3, a4, a5;
+    int owner;  // K_SCORE, K_ATTN: the consumer warp that processes the stage
+    int pad1;
 };
 
 template <int D>
@@ -85,15 +102,16 @@ struct Cfg {
 };
 
 struct SmemLayout {
-    int ring, qbuf, qbytes, meta, bars, psel, psup, uni, misc, total;
+    int ring, qbuf, qbytes, meta, bars, psel, psup, plan, bits, uni, misc, total;
 };
+
+__host__ __device__ inline int mask_words_for(const Plan& p) { return (p.M_max + 31) / 32; }
 
 template <int D>
 __host__ __device__ inline SmemLayout smem_layout(const Plan& p) {
     SmemLayout L;
     const int NS = Cfg<D>::kStages;
     const int G = p.G;
-    const int topk_super = p.h2 ? p.topk_super : 0;
     int o = 0;
     L.ring = o;
     o += NS * Cfg<D>::kStageBytes;
@@ -108,15 +126,19 @@ __host__ __device__ inline SmemLayout smem_layout(const Plan& p) {
     L.psel = o;
     o += ((p.topk + 3) / 4 * 4) * 4;
     L.psup = o;
-    o += ((topk_super + 3) / 4 * 4) * 4;
+    o += (((p.h2 ? p.topk_super : 0) + 3) / 4 * 4) * 4;
+    L.plan = o;  // lengths [B], then per list prefixes [B + 1]
+    o += (p.B + kNumLists * (p.B + 1)) * 4;
     o = (o + 15) / 16 * 16;
+    L.bits = o;  // selection bitmap of the current segment's pair
+    o += ((mask_words_for(p) + 3) / 4 * 4) * 4;
     L.uni = o;
     // the consumers use this area for one thing at a time
     int u = kRowmaxCap * 4;                                      // score rows
     const int tk = (int)sizeof(TopkScratch);                     // top-k
     u = u > tk ? u : tk;
-    const int cmb = 3 * G * p.attn_items * kConsumerWarps * 4;   // combination
-    u = u > cmb ? u : cmb;
+    const int mg = kConsumerWarps * G * (D + 2) * 4;             // warp merge
+    u = u > mg ? u : mg;
     o += (u + 15) / 16 * 16;
     L.misc = o;
     o += 64;
@@ -124,13 +146,11 @@ __host__ __device__ inline SmemLayout smem_layout(const Plan& p) {
     return L;
 }
 
-// Timeline trace: builds compiled with SSA_TRACE record (time, event, a, b)
+// Timeline trace: builds compiled with SSA_TRACE record (cycles, event, a, b)
 // per block into Plan::trace; the product build compiles these to nothing.
-enum : int { TR_KSTART = 1, TR_TICKET, TR_P_READY, TR_P_ISSUED, TR_C_FIRST, TR_C_LAST,
-             TR_C_DONE, TR_C_TOPK0, TR_C_TOPK1, TR_C_COMB0, TR_C_COMB1, TR_KEND };
+enum : int { TR_KSTART = 1, TR_SEG, TR_P_SEL, TR_C_SEG0, TR_C_SEG1, TR_C_SEL0, TR_C_SEL1,
+             TR_C_COMB0, TR_C_COMB1, TR_KEND, TR_C_SELW, TR_C_SCD };
 #ifdef SSA_TRACE
-// Events carry the per-SM cycle counter (cheap); KSTART and KEND also record
-// the global timer in a second event (ev | 0x80) so blocks can be aligned.
 __device__ __forceinline__ void trace_event(const Plan& p, int* counter, int ev, int a, int b) {
     if (!p.trace) return;
     const int i = atomicAdd(counter, 1);
@@ -140,13 +160,13 @@ __device__ __forceinline__ void trace_event(const Plan& p, int* counter, int ev,
         make_uint4((uint32_t)t, (uint32_t)(t >> 32), (uint32_t)ev | ((uint32_t)a << 8), (uint32_t)b);
 }
 #define SSA_TR(ev, a, b) trace_event(p, &misc[15], (ev), (a), (b))
+// probe points inside the block top-k (thread 0 only): event 13, a = point
 struct TraceProbe {
     const Plan& p;
     int* counter;
     int pair;
-    __device__ void operator()(int stage) const {
-        if ((threadIdx.x & 31) == 0 && threadIdx.x < 128)
-            trace_event(p, counter, 13, stage + 16 * (threadIdx.x >> 5), pair);
+    __device__ void operator()(int point) const {
+        if (threadIdx.x == 0) trace_event(p, counter, 13, point, pair);
     }
 };
 #define SSA_PROBE(pair) TraceProbe{p, &misc[15], (pair)}
@@ -155,17 +175,10 @@ struct TraceProbe {
 #define SSA_TR(ev, a, b) ((void)0)
 #endif
 
-__device__ __forceinline__ int pair_of(const StageMeta& m) { return m.pair; }
-
 struct ConsumerSync {
     __device__ void operator()() const { named_sync(kBarConsumers, kConsumers); }
+    __device__ bool or_(bool pred) const { return named_sync_or(kBarConsumers, kConsumers, pred); }
 };
-
-__device__ __forceinline__ int seq_len_checked(const Plan& p, int b) {
-    int n = __ldg(p.seq_lens + b);
-    if (n < 1 || n > p.n_max) return -1;
-    return n;
-}
 
 // swizzled (128B) address of 16-byte unit `chunk` of row `row` in a slot
 template <int D>
@@ -193,6 +206,59 @@ __device__ __forceinline__ void qk16(uint32_t slot, int r0, const uint32_t (&qa)
     }
 }
 
+// S^T[token][head] for 16 rows starting at r0 of a key slot, with the keys as
+// the M operand: the A fragments are the key rows (the same ldmatrix loads as
+// qk16, reordered) and the B fragments are the query registers.  st[nt] holds
+// heads 8 nt .. 8 nt + 7: st[nt][0..1] token g8, heads 2 tig, 2 tig + 1;
+// st[nt][2..3] token g8 + 8.
+template <int D, int NT>
+__device__ __forceinline__ void qkT16(uint32_t slot, int r0, const uint32_t (&qa)[D / 16][4],
+                                      float (&st)[NT][4], int lane) {
+#pragma unroll
+    for (int i = 0; i < NT; ++i)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) st[i][c] = 0.f;
+    const int row = r0 + ((lane >> 4) << 3) + (lane & 7);
+    const int csel = (lane >> 3) & 1;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(tile_addr<D>(slot, row, 2 * kk + csel), b0, b1, b2, b3);
+        const uint32_t a[4] = {b0, b2, b1, b3};
+        mma_bf16_16816(st[0], a, qa[kk][0], qa[kk][2]);
+        if (NT == 2) mma_bf16_16816(st[NT - 1], a, qa[kk][1], qa[kk][3]);
+    }
+}
+
+// Scores of up to 128 summary rows (two 64-row boxes) by one warp: per row,
+// the maximum over the group's query heads of q.k / sqrt(d), into rowmax.
+template <int D, int NT>
+__device__ __forceinline__ void score_tile(uint32_t slotA, uint32_t slotB, int nvalid, int G,
+                                           const uint32_t (&qa)[D / 16][4], float scale,
+                                           float* rowmax, int lane) {
+    const int g8 = lane >> 2, tig = lane & 3;
+#pragma unroll 4
+    for (int sb = 0; sb < 8; ++sb) {
+        if (16 * sb >= nvalid) break;
+        float st[NT][4];
+        qkT16<D, NT>(sb < 4 ? slotA : slotB, 16 * (sb & 3), qa, st, lane);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float v = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int h = nt * 8 + 2 * tig;
+                if (h < G) v = fmaxf(v, st[nt][2 * half]);
+                if (h + 1 < G) v = fmaxf(v, st[nt][2 * half + 1]);
+            }
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+            const int lr = 16 * sb + 8 * half + g8;
+            if (tig == 0 && lr < nvalid) rowmax[lr] = v * scale;
+        }
+    }
+}
+
 // acc[dim n-tile] += P(hi+lo) * V for 16 rows starting at r0 of a value slot.
 template <int D>
 __device__ __forceinline__ void pv16(uint32_t slot, int r0, const uint32_t (&phi)[4],
@@ -210,6 +276,199 @@ __device__ __forceinline__ void pv16(uint32_t slot, int r0, const uint32_t (&phi
     }
 }
 
+// One consumer warp's pass over a whole 64-row attention tile: S = Q.K^T for
+// the tile's rows (excluded rows -inf), online-softmax update of (m, l) per
+// query head, acc += P.V with P split into bf16 hi + lo parts.
+template <int D>
+__device__ __forceinline__ void attn_tile(uint32_t slotA, uint32_t slotB, int nvalid,
+                                          uint32_t ex_lo, uint32_t ex_hi,
+                                          const uint32_t (&qa)[D / 16][4], float (&mrow)[2],
+                                          float (&lrow)[2], float (&acc)[D / 8][4],
+                                          bool two_rows, float scale_log2, int lane) {
+    const int tig = lane & 3;
+    // 16-row sub-blocks per pass: independent Q.K products, one
+    // softmax update per pass
+    constexpr int SB = (D == 64) ? 4 : 2;
+#pragma unroll
+    for (int pass = 0; pass < 4 / SB; ++pass) {
+        if (16 * SB * pass >= nvalid) break;
+        float sc4[SB][2][4];
+#pragma unroll
+        for (int sb = 0; sb < SB; ++sb) qk16<D>(slotA, 16 * (SB * pass + sb), qa, sc4[sb], lane);
+#pragma unroll
+        for (int sb = 0; sb < SB; ++sb)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int t = 16 * (SB * pass + sb) + nt * 8 + 2 * tig + (c & 1);
+                    const uint32_t ex = t < 32 ? (ex_lo >> t) : (ex_hi >> (t - 32));
+                    sc4[sb][nt][c] = (ex & 1u) ? -INFINITY : sc4[sb][nt][c] * scale_log2;
+                }
+        uint32_t phi[SB][4], plo[SB][4];
+#pragma unroll
+        for (int sb = 0; sb < SB; ++sb)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) phi[sb][c] = plo[sb][c] = 0u;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            if (r == 1 && !two_rows) break;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int sb = 0; sb < SB; ++sb)
+                mx = fmaxf(mx, fmaxf(fmaxf(sc4[sb][0][2 * r], sc4[sb][0][2 * r + 1]),
+                                     fmaxf(sc4[sb][1][2 * r], sc4[sb][1][2 * r + 1])));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float mnew = fmaxf(mrow[r], mx);
+            const float ref = (mnew == -INFINITY) ? 0.f : mnew;
+            const float alpha = exp2f(mrow[r] - ref);
+            float lsum = 0.f;
+#pragma unroll
+            for (int sb = 0; sb < SB; ++sb) {
+                const float p00 = exp2f(sc4[sb][0][2 * r] - ref);
+                const float p01 = exp2f(sc4[sb][0][2 * r + 1] - ref);
+                const float p10 = exp2f(sc4[sb][1][2 * r] - ref);
+                const float p11 = exp2f(sc4[sb][1][2 * r + 1] - ref);
+                lsum += (p00 + p01) + (p10 + p11);
+                split_bf16(p00, p01, phi[sb][r], plo[sb][r]);          // tokens 0..7
+                split_bf16(p10, p11, phi[sb][2 + r], plo[sb][2 + r]);  // tokens 8..15
+            }
+            lrow[r] = lrow[r] * alpha + lsum;
+            mrow[r] = mnew;
+            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                for (int nt = 0; nt < D / 8; ++nt) {
+                    acc[nt][2 * r] *= alpha;
+                    acc[nt][2 * r + 1] *= alpha;
+                }
+            }
+        }
+#pragma unroll
+        for (int sb = 0; sb < SB; ++sb)
+            if (16 * (SB * pass + sb) < nvalid)
+                pv16<D>(slotB, 16 * (SB * pass + sb), phi[sb], plo[sb], acc, lane);
+    }
+}
+
+// ---------------------------------------------------------------- plan ---
+
+// Derived sizes of one pair from its raw length n (0 for an invalid length).
+struct PairSizes {
+    int n, M, T;            // raw length, complete chunks, tail tokens
+    int S, R, ks, Mc, kc;   // superchunks, remainder chunks, kept superchunks,
+                            // candidates (single level: M), kept chunks
+};
+
+__device__ __forceinline__ PairSizes pair_sizes(const Plan& p, int n) {
+    PairSizes z;
+    z.n = n;
+    z.M = n / p.C;
+    z.T = n - z.M * p.C;
+    if (p.h2) {
+        z.S = z.M / p.J;
+        z.R = z.M - z.S * p.J;
+        z.ks = min(p.topk_super, z.S);
+        z.Mc = z.ks * p.J + z.R;
+    } else {
+        z.S = z.R = z.ks = 0;
+        z.Mc = z.M;
+    }
+    z.kc = min(p.topk, z.Mc);
+    return z;
+}
+
+// Elements of list `L` for one pair of raw length n.
+__device__ __forceinline__ int list_count(const Plan& p, int L, int n) {
+    const PairSizes z = pair_sizes(p, n);
+    const int tpc = (p.C + kBoxRows - 1) / kBoxRows;
+    switch (L) {
+        case L_SCORE:
+            if (p.mode == kModeAttnOnly) return 0;
+            if (p.mode == kModeScoreOnly) return p.M_max;
+            return p.h2 ? z.S : z.M;
+        case L_CAND:
+            return p.h2 ? z.Mc : 0;
+        case L_META:
+            return p.h2 ? (z.S * p.gm + kBoxRows - 1) / kBoxRows : 0;
+        case L_GIST:
+            if (p.mode == kModeScoreOnly) return 0;
+            if (!p.h2) return (z.M * p.g + kBoxRows - 1) / kBoxRows;
+            return z.ks * ((p.J * p.g + kBoxRows - 1) / kBoxRows) +
+                   (z.R * p.g + kBoxRows - 1) / kBoxRows;
+        case L_RAW:
+            if (p.mode == kModeScoreOnly) return 0;
+            return z.kc * tpc + (z.T + kBoxRows - 1) / kBoxRows;
+    }
+    return 0;
+}
+
+// The block-local plan: lengths per sequence and prefix sums per list.
+struct PlanView {
+    const Plan& p;
+    const int* nb;   // [B] raw lengths (0: invalid)
+    const int* ps;   // [kNumLists][B + 1] prefix over sequences of Hkv * count
+    int nblocks;
+
+    __device__ int total(int L) const { return ps[L * (p.B + 1) + p.B]; }
+    __device__ int parts(int L) const { return min(nblocks, total(L)); }
+    // share of block c in list L: [lo, hi)
+    __device__ void share(int L, int c, int& lo, int& hi) const {
+        const long long t = total(L), n = parts(L);
+        if (c >= n) {
+            lo = hi = 0;
+            return;
+        }
+        lo = (int)((t * c) / n);
+        hi = (int)((t * (c + 1)) / n);
+    }
+    // block holding element x of list L
+    __device__ int block_of(int L, int x) const {
+        const long long t = total(L), n = parts(L);
+        return (int)(((long long)(x + 1) * n - 1) / t);
+    }
+    // pair holding element x of list L, its first element and element count
+    __device__ void locate(int L, int x, int& pair, int& first, int& count) const {
+        const int* q = ps + L * (p.B + 1);
+        int lo = 0, hi = p.B;  // q[lo] <= x < q[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (q[mid] <= x) lo = mid; else hi = mid;
+        }
+        count = list_count(p, L, nb[lo]);
+        const int j = (x - q[lo]) / count;
+        pair = lo * p.Hkv + j;
+        first = q[lo] + j * count;
+    }
+    // blocks holding the segments of pair `pair` in list L: [c0, c0 + n)
+    __device__ void pair_blocks(int L, int pair, int& c0, int& n) const {
+        const int b = pair / p.Hkv, j = pair % p.Hkv;
+        const int count = list_count(p, L, nb[b]);
+        if (count == 0) {
+            c0 = n = 0;
+            return;
+        }
+        const int first = ps[L * (p.B + 1) + b] + j * count;
+        c0 = block_of(L, first);
+        n = block_of(L, first + count - 1) - c0 + 1;
+    }
+};
+
+// Pairs whose top-k block c runs: those with floor(pair * N / P) == c.  Their
+// combination runs on the mirrored block N - 1 - c.
+__device__ __forceinline__ void owned_pairs(int c, int N, int P, int& lo, int& hi) {
+    lo = (int)(((long long)c * P + N - 1) / N);
+    hi = (int)(((long long)(c + 1) * P + N - 1) / N);
+}
+
+// Partial of segment (attention list a, block c, pair), query head h.  Along
+// a list, the segments' (block + pair) strictly increase, so the slots differ.
+__device__ __forceinline__ size_t partial_offset(const Plan& p, int a, int c, int pair, int h,
+                                                 int D) {
+    const size_t slot = (size_t)a * (kMaxGrid + p.n_pairs) + c + pair;
+    return (slot * p.G + h) * (size_t)(D + 2);
+}
+
 // ------------------------------------------------------------ producer ---
 
 template <int D>
@@ -222,18 +481,31 @@ struct Producer {
     StageMeta* meta;
     uint64_t* full;
     uint64_t* empty;
-    int* psel;
-    int* psup;
+    int* ctrl;
     int lane;
+    long long long_limit;  // bound of ring waits (several device-side waits)
     int stage = 0, round = 0;
+    bool dead = false;     // a ring wait ran out: issue nothing more
+    int* trace_ctr = nullptr;
+    uint64_t pol_keep = 0, pol_once = 0;
+    int rr = 0;            // consumer warp for the next data stage
 
-    __device__ int acquire() {
-        const int s = stage;
+    __device__ int* rec(int a, int pair) const { return ctrl + C_ARR + pair * p.pair_ints + a; }
+
+    // Next free stage; false once the ring is given up.
+    __device__ bool acquire(int& s) {
+        s = stage;
+        if (dead) return false;
         if (round > 0) {
-            if (lane == 0) mbar_wait(&empty[s], (uint32_t)((round - 1) & 1), p.wait_limit);
-            __syncwarp();
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(&empty[s], (uint32_t)((round - 1) & 1), long_limit);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) {
+                dead = true;
+                return false;
+            }
         }
-        return s;
+        return true;
     }
     __device__ void advance() {
         if (++stage == Cfg<D>::kStages) {
@@ -244,82 +516,104 @@ struct Producer {
     __device__ uint8_t* slot(int s, int which) {
         return ring + (size_t)s * Cfg<D>::kStageBytes + which * Cfg<D>::kSlotBytes;
     }
-    // one 64-row box (all D columns) of map `m` at global row y into slot
-    __device__ void box(int s, int which, const CUtensorMap* m, int y) {
+    // one 64-row box (all D columns) of map `m` at global row y into slot,
+    // with an L2 policy: summary keys are read twice (scoring, attention) and
+    // kept in L2 in between; everything else is read once
+    __device__ void box(int s, int which, const CUtensorMap* m, int y, uint64_t pol) {
 #pragma unroll
         for (int sub = 0; sub < D / 64; ++sub)
-            tma_load_2d(slot(s, which) + sub * (kBoxRows * 128), m, sub * 64, y, &full[s]);
+            tma_load_2d_hint(slot(s, which) + sub * (kBoxRows * 128), m, sub * 64, y, &full[s],
+                             pol);
     }
-    __device__ void load_q(int s, int b, int j) {
+    __device__ void load_q(int s, int pair) {
+        const int b = pair / p.Hkv, j = pair % p.Hkv;
         const __nv_bfloat16* src =
             static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + (size_t)j * p.G) * D;
         bulk_load(qbuf + (size_t)s * qbytes, src, (uint32_t)(p.G * D * 2), &full[s]);
     }
-    __device__ void push_plain(int kind, int pair, int flags, int item) {
-        const int s = acquire();
+    // a stage without data (select, combine, end, empty segment)
+    __device__ void push_plain(const StageMeta& m) {
+        int s;
+        if (!acquire(s)) return;
         if (lane == 0) {
-            StageMeta m = {};
-            m.kind = kind;
-            m.pair = pair;
-            m.flags = flags;
-            m.item = item;
             meta[s] = m;
             mbar_arrive(&full[s]);
         }
         __syncwarp();
         advance();
     }
+    // Waits until every stage this warp issued has landed (bounded), so no
+    // copy is in flight when the block exits, whatever the consumers did.
+    __device__ void drain() {
+        constexpr int NS = Cfg<D>::kStages;
+        const int issued = round * NS + stage;
+        if (lane == 0)
+            for (int i = 0; i < NS && i < issued; ++i) {
+                const int idx = issued - 1 - i;
+                mbar_wait(&full[idx % NS], (uint32_t)((idx / NS) & 1), long_limit);
+            }
+        __syncwarp();
+    }
 
-    // Score item: rows [0, rows) of a summary tensor starting at global row y0.
-    __device__ void score_item(int pair, int level, const CUtensorMap* m, int y0, int rows,
-                               int nslot, int npad, int dst, int ntok) {
-        const int b = pair / p.Hkv, j = pair % p.Hkv;
-        if (rows <= 0) {
-            const int s = acquire();
-            if (lane == 0) {
+    // Scores `nslot` consecutive summary slots of `ntok` rows each, starting
+    // at global row y0 of map m, into dst[0..nslot), then writes `npad` slots
+    // of -inf.  Split into sub-items of at most `per_rows` rows.
+    __device__ void score_run(int pair, int level, const CUtensorMap* m, int y0, int nslot,
+                              int npad, int dst, int ntok, int per_rows) {
+        const int per = max(1, per_rows / ntok);  // slots per sub-item
+        int s0 = 0;
+        do {
+            const int ns = min(per, nslot - s0);
+            const int np = (s0 + ns >= nslot) ? npad : 0;
+            const int rows = ns * ntok;
+            if (rows <= 0) {
                 StageMeta mt = {};
                 mt.kind = K_SCORE;
                 mt.pair = pair;
                 mt.flags = F_FIRST | F_LAST;
-                mt.item = level;
-                mt.nslot = 0;
-                mt.npad = npad;
-                mt.dst = dst;
-                mt.ntok = ntok;
-                meta[s] = mt;
-                mbar_arrive(&full[s]);
+                mt.a2 = np;
+                mt.a3 = dst + s0;
+                mt.a4 = ntok;
+                mt.a5 = level;
+                push_plain(mt);
             }
-            __syncwarp();
-            advance();
-            return;
-        }
-        for (int off = 0; off < rows; off += 2 * kBoxRows) {
-            const int s = acquire();
-            const int nv = min(2 * kBoxRows, rows - off);
-            const int nbox = (nv + kBoxRows - 1) / kBoxRows;
-            const bool first = off == 0;
-            if (lane == 0) {
-                StageMeta mt = {};
-                mt.kind = K_SCORE;
-                mt.pair = pair;
-                mt.nvalid = nv;
-                mt.flags = (first ? (F_FIRST | F_QLOAD) : 0) |
-                           (off + 2 * kBoxRows >= rows ? F_LAST : 0);
-                mt.row_off = off;
-                mt.item = level;
-                mt.nslot = nslot;
-                mt.npad = npad;
-                mt.dst = dst;
-                mt.ntok = ntok;
-                meta[s] = mt;
-                uint32_t bytes = nbox * Cfg<D>::kBoxBytes + (first ? p.G * D * 2 : 0);
-                mbar_arrive_expect_tx(&full[s], bytes);
-                if (first) load_q(s, b, j);
-                for (int bx = 0; bx < nbox; ++bx) box(s, bx, m, y0 + off + bx * kBoxRows);
+            for (int off = 0; off < rows; off += 2 * kBoxRows) {
+                int s;
+                if (!acquire(s)) return;
+                const int nv = min(2 * kBoxRows, rows - off);
+                const int nbox = (nv + kBoxRows - 1) / kBoxRows;
+                const bool first = off == 0;
+                const int own = rr;
+                rr = (rr + 1) % kConsumerWarps;
+                if (lane == 0) {
+                    StageMeta mt = {};
+                    mt.kind = K_SCORE;
+                    mt.owner = own;
+                    mt.pair = pair;
+                    mt.nvalid = nv;
+                    mt.flags = (first ? (F_FIRST | F_QLOAD) : 0) |
+                               (off + 2 * kBoxRows >= rows ? F_LAST : 0);
+                    mt.a0 = off;
+                    mt.a1 = ns;
+                    mt.a2 = np;
+                    mt.a3 = dst + s0;
+                    mt.a4 = ntok;
+                    mt.a5 = level;
+                    meta[s] = mt;
+                    const uint32_t bytes = nbox * Cfg<D>::kBoxBytes + (first ? p.G * D * 2 : 0);
+                    mbar_arrive_expect_tx(&full[s], bytes);
+#ifdef SSA_TRACE
+                    trace_event(p, trace_ctr, 14, 1, round * Cfg<D>::kStages + s);
+#endif
+                    if (first) load_q(s, pair);
+                    for (int bx = 0; bx < nbox; ++bx)
+                        box(s, bx, m, y0 + s0 * ntok + off + bx * kBoxRows, pol_keep);
+                }
+                __syncwarp();
+                advance();
             }
-            __syncwarp();
-            advance();
-        }
+            s0 += ns;
+        } while (s0 < nslot);
     }
 
     // Reads a published selection (count word, `cap` entries at `ent`) into
@@ -329,6 +623,8 @@ struct Producer {
     // wait that runs out records a timeout and returns 0.
     __device__ int fetch_selection(const int* cnt_word, const int* ent, int cap, int* dst,
                                    bool& bad) {
+        bad = false;
+        if (dead) return 0;
         const long long c0 = clock64(), lim = wait_cycles(p.wait_limit);
         unsigned sleep_ns = 32;
         for (;;) {
@@ -361,35 +657,12 @@ struct Producer {
             }
             if (clock64() - c0 > lim) {
                 if (lane == 0) report_status(kStatusTimeout);
-                bad = false;
                 return 0;
             }
             __nanosleep(sleep_ns);
             if (sleep_ns < 512) sleep_ns *= 2;
         }
     }
-
-    // Rows of [r0, r0+cnt) (in units where slot x covers rows [x*ntok, x*ntok+ntok))
-    // that belong to one of the n sorted slots in list[]: bit r set.
-    __device__ uint64_t excluded_rows(const int* list, int n, int r0, int cnt, int ntok) {
-        uint64_t bits = 0;
-        for (int c = lane; c < n; c += 32) {
-            const int x = list[c];
-            const int lo = max(x * ntok, r0), hi = min(x * ntok + ntok, r0 + cnt);
-            for (int r = lo; r < hi; ++r) bits |= 1ull << (r - r0);
-        }
-        uint32_t lo32 = __reduce_or_sync(0xffffffffu, (uint32_t)bits);
-        uint32_t hi32 = __reduce_or_sync(0xffffffffu, (uint32_t)(bits >> 32));
-        return ((uint64_t)hi32 << 32) | lo32;
-    }
-};
-
-// Tile descriptor of one attention unit.
-struct Tile {
-    int src;      // 0 raw, 1 gist, 2 meta
-    int y;        // global row of the TMA box
-    int nvalid;   // rows of the tile in the context (before exclusions)
-    uint64_t excl;
 };
 
 // ------------------------------------------------------------ the kernel ---
@@ -414,10 +687,20 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t* empty = full + NS;
     int* psel = reinterpret_cast<int*>(smem + L.psel);
     int* psup = reinterpret_cast<int*>(smem + L.psup);
+    int* nbv = reinterpret_cast<int*>(smem + L.plan);
+    int* psv = nbv + p.B;
+    uint32_t* bits = reinterpret_cast<uint32_t*>(smem + L.bits);
     uint8_t* uni = smem + L.uni;
     int* misc = reinterpret_cast<int*>(smem + L.misc);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int P = p.n_pairs, N = gridDim.x, cta = blockIdx.x;
+    int* ctrl = p.ctrl;
+    auto rec = [&](int a, int pair) -> int* { return ctrl + C_ARR + pair * p.pair_ints + a; };
+    // ring waits span at most a few bounded device-side waits of the other side
+    const long long long_limit = 8 * p.wait_limit;
+
+    // ---- prologue: barriers and the block-local plan (the same in every block)
     if (threadIdx.x == 0) {
         misc[15] = 0;
         for (int s = 0; s < NS; ++s) {
@@ -426,296 +709,310 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         fence_barrier_init();
     }
+    for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+        const int n = __ldg(p.seq_lens + b);
+        const bool ok = n >= 1 && n <= p.n_max;
+        if (!ok && cta == 0) report_status(kStatusBadInput);
+        nbv[b] = ok ? n : 0;
+    }
+    __syncthreads();
+    if (warp < kNumLists) {  // warp w: exclusive prefix over sequences of list w
+        int carry = 0;
+        for (int b0 = 0; b0 < p.B; b0 += 32) {
+            const int b = b0 + lane;
+            const int v = b < p.B ? p.Hkv * list_count(p, warp, nbv[b]) : 0;
+            int x = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (b < p.B) psv[warp * (p.B + 1) + b] = carry + x - v;
+            carry += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (lane == 0) psv[warp * (p.B + 1) + p.B] = carry;
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
         SSA_TR(TR_KSTART | 0x80, 0, 0);
         SSA_TR(TR_KSTART, 0, 0);
     }
-
-    // ticket phases, in hand-out order
-    const int P = p.n_pairs;
+    const PlanView pv{p, nbv, psv, N};
     const bool so = p.mode == kModeScoreOnly;
-    const int nA = (p.mode == kModeAttnOnly) ? 0 : P * p.score_items;  // score items
-    const int nS1 = so ? 0 : P;                                         // first selection
-    const int nB = p.h2 ? P * p.cand_items : 0;                         // candidate scoring
-    const int nS2 = p.h2 ? P : 0;                                       // second selection
-    const int nC = so ? 0 : P * p.attn_items;                           // attention
-    const int nD = so ? 0 : P;                                          // combination
-    const int oS1 = nA, oB = oS1 + nS1, oS2 = oB + nB, oC = oS2 + nS2, oD = oC + nC;
-    const int total = oD + nD;
-    int* ctrl = p.ctrl;
-    auto arr = [&](int a, int pair) -> int* { return ctrl + C_ARR + pair * p.pair_ints + a; };
+    const int score_rows = min(kRowmaxCap, max(p.score_rows, 1));
 
     // ================================================================ producer
     if (warp == kConsumerWarps) {
-        Producer<D> pr{p, {&tm_kraw, &tm_vraw, &tm_kgist, &tm_vgist, &tm_kmeta, &tm_vmeta},
-                       ring, qbuf, L.qbytes, meta, full, empty, psel, psup, lane};
-        if (lane == 0) {
+        Producer<D> pr{p,    {&tm_kraw, &tm_vraw, &tm_kgist, &tm_vgist, &tm_kmeta, &tm_vmeta},
+                       ring, qbuf, L.qbytes, meta, full, empty, ctrl, lane, long_limit};
+        if (lane == 0)
             for (int i = 0; i < 6; ++i) prefetch_tensormap(pr.tm[i]);
-        }
-        // lane 0 keeps one ticket in hand: the atomic for the next item is
-        // issued as soon as the current one is known, so its latency overlaps
-        // the current item's issue work.
-        // Scoring alone never waits, so it strides over items statically and
-        // needs no control words.
-        const bool dyn = p.mode != kModeScoreOnly;
-        int next_t = 0;
-        if (lane == 0) next_t = dyn ? atomicAdd(ctrl + C_TICKET, 1) : (int)blockIdx.x;
-        for (;;) {
-            const int t = __shfl_sync(0xffffffffu, next_t, 0);
-            if (t >= total) {
-                pr.push_plain(K_END, 0, 0, 0);
-                break;
-            }
-            if (lane == 0) next_t = dyn ? atomicAdd(ctrl + C_TICKET, 1) : t + (int)gridDim.x;
-            if (lane == 0) SSA_TR(TR_TICKET, t < oS1 ? 0 : t < oC ? 1 : t < oD ? 2 : 3, t);
+        pr.pol_once = l2_policy_evict_first();
+        pr.trace_ctr = &misc[15];
+        pr.pol_keep = so ? pr.pol_once : l2_policy_evict_last();
+        int sel_lo, sel_hi, cmb_lo, cmb_hi;
+        owned_pairs(cta, N, P, sel_lo, sel_hi);
+        owned_pairs(N - 1 - cta, N, P, cmb_lo, cmb_hi);
 
-            if (t < oS1) {
-                const int pair = t / p.score_items, i = t % p.score_items;
-                const int b = pair / p.Hkv;
-                int n = seq_len_checked(p, b);
-                if (n < 0) {
-                    if (lane == 0 && i == 0 && pair % p.Hkv == 0) report_status(kStatusBadInput);
-                    n = 0;
-                }
-                const int M = n / p.C;
-                if (!p.h2) {
-                    const int s0 = i * p.score_spi;
-                    const int s1 = min(s0 + p.score_spi, p.M_max);
-                    const int vs = max(0, min(M, s1) - s0);
-                    const int npad = (p.mode == kModeScoreOnly) ? (s1 - s0 - vs) : 0;
-                    pr.score_item(pair, L_GIST, &tm_kgist, (pair * p.M_max + s0) * p.g, vs * p.g,
-                                  vs, npad, pair * p.M_max + s0, p.g);
+        // -------- this block's share of a scoring list (first level or candidates)
+        auto score_list = [&](int Ls) {
+            int lo, hi;
+            pv.share(Ls, cta, lo, hi);
+            for (int x = lo; x < hi;) {
+                int pair, first, count;
+                pv.locate(Ls, x, pair, first, count);
+                const int i0 = x - first, i1 = min(hi, first + count) - first;
+                const PairSizes z = pair_sizes(p, nbv[pair / p.Hkv]);
+                if (lane == 0) SSA_TR(TR_SEG, Ls, pair);
+                if (Ls == L_SCORE && !p.h2) {
+                    // score-only calls also cover the slots past M (as -inf)
+                    const int nv = max(0, min(i1, z.M) - i0);
+                    const int npad = (i1 - i0) - nv;
+                    pr.score_run(pair, 0, &tm_kgist, (pair * p.M_max + i0) * p.g, nv, npad,
+                                 pair * p.M_max + i0, p.g, score_rows);
+                } else if (Ls == L_SCORE) {
+                    pr.score_run(pair, 0, &tm_kmeta, (pair * p.S_max + i0) * p.gm, i1 - i0, 0,
+                                 pair * p.S_max + i0, p.gm, score_rows);
                 } else {
-                    const int S = M / p.J;
-                    const int s0 = i * p.score_spi;
-                    const int s1 = min(s0 + p.score_spi, p.S_max);
-                    const int vs = max(0, min(S, s1) - s0);
-                    pr.score_item(pair, L_META, &tm_kmeta, (pair * p.S_max + s0) * p.gm,
-                                  vs * p.gm, vs, 0, pair * p.S_max + s0, p.gm);
-                }
-                if (lane == 0) SSA_TR(TR_P_ISSUED, 0, t);
-                continue;
-            }
-            if (t < oB || (t >= oS2 && t < oC)) {
-                // selection item: after every score item of the pair is done
-                const bool first = t < oB;
-                const int pair = first ? t - oS1 : t - oS2;
-                int level;
-                if (!first) {
-                    level = L_CAND;
-                    if (lane == 0) wait_geq(arr(A_DONE_B, pair), p.cand_items, p.wait_limit);
-                } else if (p.mode == kModeAttnOnly) {
-                    level = L_VALIDATE;
-                } else {
-                    level = p.h2 ? L_META : L_GIST;
-                    if (lane == 0) wait_geq(arr(A_DONE_A, pair), p.score_items, p.wait_limit);
-                }
-                __syncwarp();
-                pr.push_plain(K_SELECT, pair, F_FIRST | F_LAST, level);
-                continue;
-            }
-            if (t >= oD) {
-                // combination item: after every attention item of the pair
-                const int pair = t - oD;
-                if (lane == 0)
-                    wait_geq(arr(A_ATTN, pair), p.attn_items * kConsumerWarps, p.wait_limit);
-                __syncwarp();
-                pr.push_plain(K_COMBINE, pair, F_FIRST | F_LAST, 0);
-                continue;
-            }
-            if (t < oS2) {
-                const int u = t - oB;
-                const int pair = u / p.cand_items, i = u % p.cand_items;
-                const int b = pair / p.Hkv;
-                int n = seq_len_checked(p, b);
-                if (n < 0) n = 0;
-                const int M = n / p.C, S = M / p.J, R = M - S * p.J;
-                bool bad_s;
-                const int ks = pr.fetch_selection(arr(A_SCOUNT, pair),
-                                                  arr(A_ENTRIES + p.topk, pair), p.topk_super,
-                                                  psup, bad_s);
-                int chunk0 = 0, nch = 0, c0 = 0;
-                if (i < p.topk_super) {
-                    if (i < ks) {
-                        chunk0 = psup[i] * p.J;
-                        nch = p.J;
-                        c0 = i * p.J;
-                    }
-                } else {
-                    chunk0 = S * p.J;
-                    nch = R;
-                    c0 = ks * p.J;
-                }
-                pr.score_item(pair, L_CAND, &tm_kgist, (pair * p.M_max + chunk0) * p.g, nch * p.g,
-                              nch, 0, pair * p.Mc_max + c0, p.g);
-                if (lane == 0) SSA_TR(TR_P_ISSUED, 1, t);
-                continue;
-            }
-            // ------------------------------------------------ attention item
-            const int u = t - oC;
-            const int pair = u / p.attn_items, item = u % p.attn_items;
-            const int b = pair / p.Hkv, j = pair % p.Hkv;
-            int n = seq_len_checked(p, b);
-            if (n < 0) n = 0;
-            const int M = n / p.C, T = n - M * p.C;
-            const int tpc = (p.C + kBoxRows - 1) / kBoxRows;
-            int Ug = 0, Um = 0, Ucs = 0, Urem = 0, tsc = 0, S = 0, R = 0, kmax_s = 0, kmax_c;
-            if (!p.h2) {
-                Ug = (M * p.g + kBoxRows - 1) / kBoxRows;
-                kmax_c = min(p.topk, M);
-            } else {
-                S = M / p.J;
-                R = M - S * p.J;
-                kmax_s = min(p.topk_super, S);
-                Um = (S * p.gm + kBoxRows - 1) / kBoxRows;
-                tsc = (p.J * p.g + kBoxRows - 1) / kBoxRows;
-                Ucs = kmax_s * tsc;
-                Urem = (R * p.g + kBoxRows - 1) / kBoxRows;
-                kmax_c = min(p.topk, kmax_s * p.J + R);
-            }
-            const int Usum = Ug + Um + Ucs + Urem;  // summary tiles
-            const int Ur = kmax_c * tpc;
-            const int Ut = (T + kBoxRows - 1) / kBoxRows;
-            const long long U = (long long)Usum + Ur + Ut;
-            const int u0 = (int)((U * item) / p.attn_items);
-            const int u1 = (int)((U * (item + 1)) / p.attn_items);
-
-            bool have_sel = false, bad_sel = false;
-            int ksel = 0, ksup = 0;
-            auto need_selection = [&]() {
-                if (have_sel) return;
-                have_sel = true;
-                ksel = pr.fetch_selection(arr(A_COUNT, pair), arr(A_ENTRIES, pair), p.topk, psel,
-                                          bad_sel);
-                if (p.h2) {
-                    bool b2;
-                    ksup = pr.fetch_selection(arr(A_SCOUNT, pair), arr(A_ENTRIES + p.topk, pair),
-                                              p.topk_super, psup, b2);
-                }
-                if (lane == 0) SSA_TR(TR_P_READY, pair, item);
-                if (bad_sel) {  // rejected caller selection: this pair attends to nothing
-                    ksel = 0;
-                    ksup = 0;
-                }
-            };
-
-            Tile pending{};
-            bool has_pending = false, emitted = false;
-            auto emit = [&](const Tile& tl, bool last) {
-                const int s = pr.acquire();
-                if (lane == 0) {
-                    StageMeta mt = {};
-                    mt.kind = K_ATTN;
-                    mt.pair = pair;
-                    mt.nvalid = tl.nvalid;
-                    mt.flags = (emitted ? 0 : (F_FIRST | F_QLOAD)) | (last ? F_LAST : 0);
-                    mt.item = item;
-                    mt.rmask_lo = (uint32_t)tl.excl;
-                    mt.rmask_hi = (uint32_t)(tl.excl >> 32);
-                    meta[s] = mt;
-                    uint32_t bytes = 2 * Cfg<D>::kBoxBytes + (emitted ? 0 : p.G * D * 2);
-                    mbar_arrive_expect_tx(&full[s], bytes);
-                    if (!emitted) pr.load_q(s, b, j);
-                    const CUtensorMap* km = tl.src == 0 ? &tm_kraw : tl.src == 1 ? &tm_kgist : &tm_kmeta;
-                    const CUtensorMap* vm = tl.src == 0 ? &tm_vraw : tl.src == 1 ? &tm_vgist : &tm_vmeta;
-                    pr.box(s, 0, km, tl.y);
-                    pr.box(s, 1, vm, tl.y);
-                }
-                __syncwarp();
-                pr.advance();
-                emitted = true;
-            };
-
-            for (int v = u0; v < u1; ++v) {
-                Tile tl{};
-                bool ok = true;
-                if (v < Usum) {
-                    need_selection();
-                    if (!p.h2) {
-                        const int r0 = v * kBoxRows;
-                        tl.src = 1;
-                        tl.nvalid = min(kBoxRows, M * p.g - r0);
-                        tl.y = pair * p.M_max * p.g + r0;
-                        tl.excl = pr.excluded_rows(psel, ksel, r0, tl.nvalid, p.g);
-                    } else if (v < Um) {
-                        const int r0 = v * kBoxRows;
-                        tl.src = 2;
-                        tl.nvalid = min(kBoxRows, S * p.gm - r0);
-                        tl.y = pair * p.S_max * p.gm + r0;
-                        tl.excl = pr.excluded_rows(psup, ksup, r0, tl.nvalid, p.gm);
-                    } else {
-                        const int w = v - Um;
-                        int r0, cnt;
-                        if (w < Ucs) {
-                            const int slot = w / tsc, part = w % tsc;
-                            if (slot >= ksup) {
-                                ok = false;
-                            } else {
-                                r0 = psup[slot] * p.J * p.g + part * kBoxRows;
-                                cnt = min(kBoxRows, p.J * p.g - part * kBoxRows);
-                            }
+                    // candidates: runs of consecutive chunks (J per kept
+                    // superchunk, in superchunk order, then the remainder),
+                    // addressed through the published superchunk selection
+                    bool bad;
+                    const int ks = pr.fetch_selection(rec(A_SCOUNT, pair),
+                                                      rec(A_ENTRIES + p.topk, pair),
+                                                      p.topk_super, psup, bad);
+                    for (int c = i0; c < i1;) {
+                        int chunk0, run;
+                        if (c < ks * p.J) {
+                            chunk0 = psup[c / p.J] * p.J + c % p.J;
+                            run = min(i1, (c / p.J + 1) * p.J) - c;
                         } else {
-                            r0 = S * p.J * p.g + (w - Ucs) * kBoxRows;
-                            cnt = min(kBoxRows, M * p.g - r0);
+                            chunk0 = z.S * p.J + (c - ks * p.J);
+                            run = i1 - c;
                         }
-                        if (ok) {
-                            tl.src = 1;
-                            tl.nvalid = cnt;
-                            tl.y = pair * p.M_max * p.g + r0;
-                            tl.excl = pr.excluded_rows(psel, ksel, r0, cnt, p.g);
-                        }
+                        pr.score_run(pair, 1, &tm_kgist, (pair * p.M_max + chunk0) * p.g, run, 0,
+                                     pair * p.Mc_max + c, p.g, score_rows);
+                        c += run;
                     }
-                    if (ok) {
-                        const uint64_t valid =
-                            tl.nvalid >= 64 ? ~0ull : ((1ull << tl.nvalid) - 1ull);
-                        if ((tl.excl & valid) == valid) ok = false;  // every row excluded
-                    }
-                } else if (v < Usum + Ur) {
-                    need_selection();
-                    const int c = (v - Usum) / tpc, part = (v - Usum) % tpc;
-                    if (c >= ksel) {
-                        ok = false;
-                    } else {
-                        const int m = psel[c];
-                        tl.src = 0;
-                        tl.nvalid = min(kBoxRows, p.C - part * kBoxRows);
-                        tl.y = pair * p.n_max + m * p.C + part * kBoxRows;
-                        tl.excl = 0;
-                    }
-                } else {
-                    const int r0 = M * p.C + (v - Usum - Ur) * kBoxRows;
-                    tl.src = 0;
-                    tl.nvalid = min(kBoxRows, n - r0);
-                    tl.y = pair * p.n_max + r0;
-                    tl.excl = 0;
                 }
-                if (bad_sel) ok = false;
-                if (!ok) continue;
-                if (has_pending) emit(pending, false);
-                pending = tl;
-                has_pending = true;
+                x = first + i1;
             }
-            if (lane == 0) SSA_TR(TR_P_ISSUED, 2, t);
-            if (has_pending) {
-                emit(pending, true);
-            } else {
-                // nothing of the context falls in this item: neutral partial
-                const int s = pr.acquire();
-                if (lane == 0) {
+        };
+
+        // -------- this block's share of an attention list (META, GIST or RAW)
+        auto attn_list = [&](int La) {
+            const int alist = La == L_META ? 0 : La == L_GIST ? 1 : 2;
+            const int tpc = (p.C + kBoxRows - 1) / kBoxRows;
+            const int tsc = (p.J * p.g + kBoxRows - 1) / kBoxRows;
+            int lo, hi;
+            pv.share(La, cta, lo, hi);
+            for (int x = lo; x < hi;) {
+                int pair, first, count;
+                pv.locate(La, x, pair, first, count);
+                const int u0 = x - first, u1 = min(hi, first + count) - first;
+                const PairSizes z = pair_sizes(p, nbv[pair / p.Hkv]);
+                if (lane == 0) SSA_TR(TR_SEG, La, pair);
+                int ks = 0, ksel = 0;
+                bool bad = false;
+                if (La == L_GIST && p.h2) {
+                    bool b2;
+                    ks = pr.fetch_selection(rec(A_SCOUNT, pair), rec(A_ENTRIES + p.topk, pair),
+                                            p.topk_super, psup, b2);
+                }
+                if (La == L_RAW) {
+                    ksel = pr.fetch_selection(rec(A_COUNT, pair), rec(A_ENTRIES, pair), p.topk,
+                                              psel, bad);
+                    if (lane == 0) SSA_TR(TR_P_SEL, pair, ksel);
+                }
+                bool emitted = false;
+                // each tile is issued once the next is known, so the last
+                // tile of the segment carries F_LAST
+                int pend_src = -1, pend_y = 0, pend_nv = 0, pend_r0 = 0;
+                auto emit = [&](bool last) {
+                    int s;
+                    if (!pr.acquire(s)) return;
+                    const int own = pr.rr;
+                    pr.rr = (pr.rr + 1) % kConsumerWarps;
+                    if (lane == 0) {
+                        StageMeta mt = {};
+                        mt.kind = K_ATTN;
+                        mt.owner = own;
+                        mt.pair = pair;
+                        mt.nvalid = pend_nv;
+                        mt.flags = (emitted ? 0 : (F_FIRST | F_QLOAD)) | (last ? F_LAST : 0);
+                        mt.a0 = pend_r0;
+                        mt.a1 = La == L_META ? MASK_SUPER : La == L_GIST ? MASK_CHUNK : MASK_NONE;
+                        mt.a2 = La == L_META ? p.gm : p.g;
+                        mt.a3 = alist;
+                        meta[s] = mt;
+                        const uint32_t bytes = 2 * Cfg<D>::kBoxBytes + (emitted ? 0 : p.G * D * 2);
+                        mbar_arrive_expect_tx(&full[s], bytes);
+#ifdef SSA_TRACE
+                        trace_event(p, &misc[15], 14, 2, pr.round * NS + s);
+#endif
+                        if (!emitted) pr.load_q(s, pair);
+                        const CUtensorMap* km =
+                            pend_src == 0 ? &tm_kraw : pend_src == 1 ? &tm_kgist : &tm_kmeta;
+                        const CUtensorMap* vm =
+                            pend_src == 0 ? &tm_vraw : pend_src == 1 ? &tm_vgist : &tm_vmeta;
+                        pr.box(s, 0, km, pend_y, pr.pol_once);
+                        pr.box(s, 1, vm, pend_y, pr.pol_once);
+                    }
+                    __syncwarp();
+                    pr.advance();
+                    emitted = true;
+                };
+                for (int u = u0; u < u1; ++u) {
+                    int src, y, nv, r0;
+                    if (La == L_META) {
+                        r0 = u * kBoxRows;
+                        nv = min(kBoxRows, z.S * p.gm - r0);
+                        src = 2;
+                        y = pair * p.S_max * p.gm + r0;
+                    } else if (La == L_GIST && !p.h2) {
+                        r0 = u * kBoxRows;
+                        nv = min(kBoxRows, z.M * p.g - r0);
+                        src = 1;
+                        y = pair * p.M_max * p.g + r0;
+                    } else if (La == L_GIST) {
+                        if (u < z.ks * tsc) {
+                            const int sl = u / tsc, part = u % tsc;
+                            if (sl >= ks) continue;
+                            r0 = psup[sl] * p.J * p.g + part * kBoxRows;
+                            nv = min(kBoxRows, p.J * p.g - part * kBoxRows);
+                        } else {
+                            r0 = z.S * p.J * p.g + (u - z.ks * tsc) * kBoxRows;
+                            nv = min(kBoxRows, z.M * p.g - r0);
+                        }
+                        src = 1;
+                        y = pair * p.M_max * p.g + r0;
+                    } else {
+                        // a rejected caller selection: the pair attends to nothing
+                        if (bad) continue;
+                        if (u < z.kc * tpc) {
+                            const int c = u / tpc, part = u % tpc;
+                            if (c >= ksel) continue;
+                            r0 = psel[c] * p.C + part * kBoxRows;
+                            nv = min(kBoxRows, p.C - part * kBoxRows);
+                        } else {
+                            r0 = z.M * p.C + (u - z.kc * tpc) * kBoxRows;
+                            nv = min(kBoxRows, z.n - r0);
+                        }
+                        src = 0;
+                        y = pair * p.n_max + r0;
+                    }
+                    if (pend_src >= 0) emit(false);
+                    pend_src = src;
+                    pend_y = y;
+                    pend_nv = nv;
+                    pend_r0 = r0;
+                }
+                if (pend_src >= 0) {
+                    emit(true);
+                } else {
+                    // nothing of the context falls in this segment: neutral partial
                     StageMeta mt = {};
                     mt.kind = K_ATTN;
                     mt.pair = pair;
-                    mt.nvalid = 0;
                     mt.flags = F_FIRST | F_LAST;
-                    mt.item = item;
-                    meta[s] = mt;
-                    mbar_arrive(&full[s]);
+                    mt.a1 = MASK_NONE;
+                    mt.a3 = alist;
+                    pr.push_plain(mt);
                 }
-                __syncwarp();
-                pr.advance();
+                x = first + u1;
             }
+        };
+
+        // -------- L2 prefetch of the tiles of this block's share of list La
+        // whose address needs no selection (single-level gist tiles, meta
+        // tiles, the raw tail): issued while the selection is computed, so
+        // the memory system stays busy through that wait
+        auto prefetch_share = [&](int La) {
+            const int tpc = (p.C + kBoxRows - 1) / kBoxRows;
+            const int tsc = (p.J * p.g + kBoxRows - 1) / kBoxRows;
+            int lo, hi;
+            pv.share(La, cta, lo, hi);
+            for (int x = lo; x < hi;) {
+                int pair, first, count;
+                pv.locate(La, x, pair, first, count);
+                const int u0 = x - first, u1 = min(hi, first + count) - first;
+                const PairSizes z = pair_sizes(p, nbv[pair / p.Hkv]);
+                for (int u = u0 + lane; u < u1; u += 32) {
+                    const CUtensorMap *km, *vm;
+                    int y;
+                    if (La == L_META) {
+                        km = &tm_kmeta;
+                        vm = &tm_vmeta;
+                        y = pair * p.S_max * p.gm + u * kBoxRows;
+                    } else if (La == L_GIST) {
+                        if (p.h2 && u < z.ks * tsc) continue;
+                        km = &tm_kgist;
+                        vm = &tm_vgist;
+                        y = pair * p.M_max * p.g +
+                            (p.h2 ? z.S * p.J * p.g + (u - z.ks * tsc) * kBoxRows : u * kBoxRows);
+                    } else {
+                        if (u < z.kc * tpc) continue;
+                        km = &tm_kraw;
+                        vm = &tm_vraw;
+                        y = pair * p.n_max + z.M * p.C + (u - z.kc * tpc) * kBoxRows;
+                    }
+#pragma unroll
+                    for (int sub = 0; sub < D / 64; ++sub) {
+                        tma_prefetch_2d(km, sub * 64, y);
+                        tma_prefetch_2d(vm, sub * 64, y);
+                    }
+                }
+                x = first + u1;
+            }
+            __syncwarp();
+        };
+
+        auto selects = [&](int what) {
+            for (int pair = sel_lo; pair < sel_hi; ++pair) {
+                StageMeta mt = {};
+                mt.kind = K_SELECT;
+                mt.pair = pair;
+                mt.flags = F_FIRST | F_LAST;
+                mt.a0 = what;
+                pr.push_plain(mt);
+            }
+        };
+
+        if (so) {
+            score_list(L_SCORE);
+        } else if (!p.h2) {
+            if (p.mode == kModeAttnOnly) {
+                selects(SEL_VALIDATE);
+            } else {
+                score_list(L_SCORE);
+                prefetch_share(L_GIST);
+                prefetch_share(L_RAW);
+                selects(SEL_CHUNKS);
+            }
+            attn_list(L_GIST);
+            attn_list(L_RAW);
+        } else {
+            score_list(L_SCORE);
+            prefetch_share(L_META);
+            selects(SEL_SUPER);
+            attn_list(L_META);
+            score_list(L_CAND);
+            selects(SEL_CAND);
+            attn_list(L_GIST);
+            attn_list(L_RAW);
         }
+        if (!so)
+            for (int pair = cmb_lo; pair < cmb_hi; ++pair) {
+                StageMeta mt = {};
+                mt.kind = K_COMBINE;
+                mt.pair = pair;
+                mt.flags = F_FIRST | F_LAST;
+                pr.push_plain(mt);
+            }
+        StageMeta end = {};
+        end.kind = K_END;
+        pr.push_plain(end);
+        pr.drain();
         return;
     }
 
@@ -725,24 +1022,80 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float scale = rsqrtf((float)D);
     const float scale_log2 = scale * 1.4426950408889634f;
     float* rowmax = reinterpret_cast<float*>(uni);
+    float* merge = reinterpret_cast<float*>(uni);
     TopkScratch& tsc = *reinterpret_cast<TopkScratch*>(uni);
-    float* cmb = reinterpret_cast<float*>(uni);
     ConsumerSync csync;
+    const bool two_rows = p.G > 8;  // query heads 8..15 of the group present
+    const int mask_words = mask_words_for(p);
 
     uint32_t qa[D / 16][4];
     float acc[D / 8][4];
-    float mrow[2], lrow[2];
+    float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk)
 #pragma unroll
         for (int c = 0; c < 4; ++c) qa[kk][c] = 0u;
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
+
+    // Loads the published selection (chunks or superchunks) of `pair` into
+    // the shared bitmap.  One round of loads reads the count and every entry
+    // (self-validating: 0 = not written yet); rounds repeat until complete.
+    auto load_bitmap = [&](int pair, int level) {
+        for (int w = tid; w < mask_words; w += kConsumers) bits[w] = 0u;
+        const int* cnt_word = rec(level == MASK_SUPER ? A_SCOUNT : A_COUNT, pair);
+        const int* ent = rec(level == MASK_SUPER ? A_ENTRIES + p.topk : A_ENTRIES, pair);
+        const int cap = level == MASK_SUPER ? p.topk_super : p.topk;
+        constexpr int kPer = (kMaxTopkEntries + kConsumers - 1) / kConsumers;
+        int e[kPer];
+        int cw = 0;
+        const long long c0 = clock64(), lim = wait_cycles(p.wait_limit);
+        bool missing;
+        for (;;) {
+            cw = ld_relaxed(cnt_word);
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int c = tid + kConsumers * j;
+                e[j] = c < cap ? ld_relaxed(ent + c) : 1;
+            }
+            const int k = (cw == 0 || (cw & kBadBit)) ? 0 : min((cw & (kBadBit - 1)) - 1, cap);
+            missing = cw == 0;
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) missing |= (tid + kConsumers * j < k) && e[j] == 0;
+            // every thread takes the same branch: the vote decides (the first
+            // vote also orders the clearing of the bitmap before the updates)
+            const bool expired = clock64() - c0 > lim;
+            if (!csync.or_(missing && !expired)) break;
+            __nanosleep(64);
+        }
+        if (missing) report_status(kStatusTimeout);
+        const int k = (cw == 0 || (cw & kBadBit)) ? 0 : min((cw & (kBadBit - 1)) - 1, cap);
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int c = tid + kConsumers * j;
+            if (c < k && e[j] != 0) atomicOr(&bits[(e[j] - 1) >> 5], 1u << ((e[j] - 1) & 31));
+        }
+        // a rejected caller selection excludes every summary row of the pair
+        if (cw & kBadBit)
+            for (int w = tid; w < mask_words; w += kConsumers) bits[w] = ~0u;
+        csync();
+    };
 
     int stage = 0, round = 0;
+    int seg_mask = MASK_NONE;
     for (;;) {
-        if (!mbar_wait(&full[stage], (uint32_t)(round & 1), p.wait_limit)) break;
+        // The producer's own waits are bounded and it always closes the ring
+        // with an END stage; this bound only ends the loop if it is gone, in
+        // which case no consumer warp receives another stage.
+        if (!mbar_wait(&full[stage], (uint32_t)(round & 1), long_limit)) break;
         const StageMeta mt = meta[stage];
+#ifdef SSA_TRACE
+        const int tr_warp = (mt.kind == K_ATTN || mt.kind == K_SCORE) ? mt.owner : 0;
+        if (lane == 0 && warp == tr_warp) trace_event(p, &misc[15], 15, mt.kind, round * NS + stage);
+#endif
         if (mt.kind == K_END) break;
-        if (tid == 0 && (mt.flags & F_FIRST)) SSA_TR(TR_C_FIRST, mt.kind, pair_of(mt));
         const uint32_t slotA = smem_u32(ring + (size_t)stage * Cfg<D>::kStageBytes);
         const uint32_t slotB = slotA + Cfg<D>::kSlotBytes;
         if (mt.flags & F_QLOAD) {
@@ -761,115 +1114,196 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         const int pair = mt.pair;
 
-        if (mt.kind == K_SCORE) {
+        if (mt.kind == K_ATTN) {
+            if (mt.flags & F_FIRST) {
+                if (tid == 0) SSA_TR(TR_C_SEG0, mt.a3, pair);
+                mrow[0] = mrow[1] = -INFINITY;
+                lrow[0] = lrow[1] = 0.f;
 #pragma unroll
-            for (int sl = 0; sl < 2; ++sl) {
-                const int rbase = sl * kBoxRows + 16 * warp;
-                if (rbase < mt.nvalid) {
-                    float s[2][4];
-                    qk16<D>(sl ? slotB : slotA, 16 * warp, qa, s, lane);
+                for (int nt = 0; nt < D / 8; ++nt)
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
+                    for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
+                seg_mask = mt.a1;
+                if (seg_mask != MASK_NONE) load_bitmap(pair, seg_mask);
+            }
+            if (warp == mt.owner && mt.nvalid > 0) {
+                // ---- this warp takes the whole 64-row tile: excluded rows (past
+                // the tile's valid rows, or in a selected chunk / superchunk),
+                // lane l tests rows l and l + 32
+                uint32_t ex_lo, ex_hi;
+                {
+                    bool e[2];
 #pragma unroll
-                        for (int c = 0; c < 2; ++c) {
-                            float v = g8 < p.G ? s[nt][c] : -INFINITY;
-                            if (g8 + 8 < p.G) v = fmaxf(v, s[nt][2 + c]);
-                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-                            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-                            const int lr = rbase + nt * 8 + 2 * tig + c;
-                            if (g8 == 0 && lr < mt.nvalid) rowmax[mt.row_off + lr] = v * scale;
+                    for (int hlf = 0; hlf < 2; ++hlf) {
+                        const int lr = lane + 32 * hlf;
+                        e[hlf] = lr >= mt.nvalid;
+                        if (!e[hlf] && seg_mask != MASK_NONE) {
+                            const int sid = (mt.a0 + lr) / mt.a2;
+                            e[hlf] = (bits[sid >> 5] >> (sid & 31)) & 1u;
                         }
+                    }
+                    ex_lo = __ballot_sync(0xffffffffu, e[0]);
+                    ex_hi = __ballot_sync(0xffffffffu, e[1]);
                 }
+                attn_tile<D>(slotA, slotB, mt.nvalid, ex_lo, ex_hi, qa, mrow, lrow, acc, two_rows,
+                             scale_log2, lane);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
+#ifdef SSA_TRACE
+            if (lane == 0 && warp == tr_warp) trace_event(p, &misc[15], 16, mt.kind, round * NS + stage);
+#endif
+
             if (mt.flags & F_LAST) {
-                if (tid == 0) SSA_TR(TR_C_LAST, K_SCORE, pair);
-                csync();
-                float* dst = mt.item == L_GIST ? p.scores
-                             : mt.item == L_META ? p.super_scores
-                                                 : p.cand_scores;
-                for (int i = tid; i < mt.nslot + mt.npad; i += kConsumers) {
-                    float v = -INFINITY;
-                    if (i < mt.nslot)
-                        for (int t = 0; t < mt.ntok; ++t) v = fmaxf(v, rowmax[i * mt.ntok + t]);
-                    dst[mt.dst + i] = v;
+                // ---- merge the 4 warps' states: one partial per head and segment
+                const int G = p.G;
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    float l = lrow[r];
+                    l += __shfl_xor_sync(0xffffffffu, l, 1);
+                    l += __shfl_xor_sync(0xffffffffu, l, 2);
+                    const int h = g8 + 8 * r;
+                    if (h < G) {
+                        float* mg = merge + ((size_t)warp * G + h) * (D + 2);
+                        if (tig == 0) {
+                            mg[0] = mrow[r];
+                            mg[1] = l;
+                        }
+#pragma unroll
+                        for (int nt = 0; nt < D / 8; ++nt)
+                            *reinterpret_cast<float2*>(mg + 2 + nt * 8 + 2 * tig) =
+                                make_float2(acc[nt][2 * r], acc[nt][2 * r + 1]);
+                    }
                 }
                 csync();
-                if (p.mode != kModeScoreOnly && tid == 0)
-                    red_release_add(arr(mt.item == L_CAND ? A_DONE_B : A_DONE_A, pair), 1);
-                if (tid == 0) SSA_TR(TR_C_DONE, K_SCORE, pair);
+                for (int h = warp; h < G; h += kConsumerWarps) {
+                    float mw[kConsumerWarps], f[kConsumerWarps];
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w) {
+                        mw[w] = merge[((size_t)w * G + h) * (D + 2)];
+                        mx = fmaxf(mx, mw[w]);
+                    }
+                    float lsum = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w) {
+                        f[w] = (mw[w] == -INFINITY) ? 0.f : exp2f(mw[w] - mx);
+                        lsum += f[w] * merge[((size_t)w * G + h) * (D + 2) + 1];
+                    }
+                    float* dstp = p.partials + partial_offset(p, mt.a3, cta, pair, h, D);
+                    if (lane == 0) *reinterpret_cast<float2*>(dstp) = make_float2(mx, lsum);
+                    for (int d0 = 2 * lane; d0 < D; d0 += 64) {
+                        float ox = 0.f, oy = 0.f;
+#pragma unroll
+                        for (int w = 0; w < kConsumerWarps; ++w) {
+                            const float2 a = *reinterpret_cast<const float2*>(
+                                merge + ((size_t)w * G + h) * (D + 2) + 2 + d0);
+                            ox += f[w] * a.x;
+                            oy += f[w] * a.y;
+                        }
+                        *reinterpret_cast<float2*>(dstp + 2 + d0) = make_float2(ox, oy);
+                    }
+                }
+                csync();
+                if (tid == 0) red_release_add(rec(A_ATTN, pair), 1);
+                if (tid == 0) SSA_TR(TR_C_SEG1, mt.a3, pair);
+            }
+        } else if (mt.kind == K_SCORE) {
+            if (warp == mt.owner) {
+                // ---- this warp scores all rows of the stage (two 64-row boxes)
+                if (two_rows)
+                    score_tile<D, 2>(slotA, slotB, mt.nvalid, p.G, qa, scale, rowmax + mt.a0, lane);
+                else
+                    score_tile<D, 1>(slotA, slotB, mt.nvalid, p.G, qa, scale, rowmax + mt.a0, lane);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+#ifdef SSA_TRACE
+            if (lane == 0 && warp == tr_warp) trace_event(p, &misc[15], 16, mt.kind, round * NS + stage);
+#endif
+            if (mt.flags & F_LAST) {
+                csync();
+                // slot score = max over its summary rows (sec. 3.2)
+                float* dst = mt.a5 == 1 ? p.cand_scores : p.h2 ? p.super_scores : p.scores;
+                for (int i = tid; i < mt.a1 + mt.a2; i += kConsumers) {
+                    float v = -INFINITY;
+                    if (i < mt.a1)
+                        for (int t = 0; t < mt.a4; ++t) v = fmaxf(v, rowmax[i * mt.a4 + t]);
+                    // for the selection, +0 is stored as -0 (same rank): an
+                    // all-zero word means "not written yet"
+                    dst[mt.a3 + i] = (so || v != 0.f) ? v : -0.f;
+                }
+                csync();
+                if (tid == 0) SSA_TR(TR_C_SCD, mt.a5, pair);
             }
         } else if (mt.kind == K_SELECT) {
-#ifdef SSA_TRACE
-            if (lane == 0) trace_event(p, &misc[15], 13, 15 + 16 * warp, pair);
-#endif
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
-            if (tid == 0) SSA_TR(TR_C_TOPK0, mt.item, pair);
-            if (mt.item != L_VALIDATE) {
-                // ---- selection for this pair (sec. 3.3 top-k; sec. 3.5 levels)
-                const int b = pair / p.Hkv;
-                int n = seq_len_checked(p, b);
-                if (n < 0) n = 0;
-                const int M = n / p.C;
-                if (mt.item == L_META) {
-                    const int S = M / p.J;
-                    block_topk<kConsumers>(p.super_scores + (size_t)pair * p.S_max, S,
-                                           p.topk_super,
-                                           p.sel_super + (size_t)pair * p.topk_super,
-                                           tsc, csync, NoProbe(), arr(A_ENTRIES + p.topk, pair));
-                    if (tid == 0) *arr(A_SCOUNT, pair) = min(p.topk_super, S) + 1;
+#ifdef SSA_TRACE
+            if (lane == 0 && warp == tr_warp) trace_event(p, &misc[15], 16, mt.kind, round * NS + stage);
+#endif
+            if (tid == 0) SSA_TR(TR_C_SEL0, mt.a0, pair);
+            const PairSizes z = pair_sizes(p, nbv[pair / p.Hkv]);
+            const int what = mt.a0;
+            if (what != SEL_VALIDATE) {
+                // ---- selection for this pair (sec. 3.3 top-k; sec. 3.5 levels).
+                // The scores are self-validating (a written score is never all
+                // zero bits): the top-k polls until every one is present, and
+                // afterwards this block clears them for the next call.
+                float* vals;
+                int nv;
+                if (what == SEL_SUPER) {
+                    vals = p.super_scores + (size_t)pair * p.S_max;
+                    nv = z.S;
+                    block_topk<kConsumers>(vals, nv, p.topk_super,
+                                           p.sel_super + (size_t)pair * p.topk_super, tsc, csync,
+                                           NoProbe(), rec(A_ENTRIES + p.topk, pair), p.wait_limit);
+                    if (tid == 0) *rec(A_SCOUNT, pair) = z.ks + 1;
+                } else if (what == SEL_CHUNKS) {
+                    vals = p.scores + (size_t)pair * p.M_max;
+                    nv = z.M;
+                    block_topk<kConsumers>(vals, nv, p.topk, p.sel_idx + (size_t)pair * p.topk, tsc,
+                                           csync, SSA_PROBE(pair), rec(A_ENTRIES, pair),
+                                           p.wait_limit);
+                    if (tid == 0) *rec(A_COUNT, pair) = z.kc + 1;
                 } else {
-                    int k;
-                    if (mt.item == L_GIST) {
-                        block_topk<kConsumers>(p.scores + (size_t)pair * p.M_max, M, p.topk,
-                                               p.sel_idx + (size_t)pair * p.topk, tsc, csync,
-                                               SSA_PROBE(pair), arr(A_ENTRIES, pair));
-                        k = min(p.topk, M);
-                    } else {
-                        const int S = M / p.J, R = M - S * p.J;
-                        const int ks = min(p.topk_super, S);
-                        const int nc = ks * p.J + R;
-                        int* out = p.sel_idx + (size_t)pair * p.topk;
-                        block_topk<kConsumers>(p.cand_scores + (size_t)pair * p.Mc_max, nc,
-                                               p.topk, out, tsc, csync);
-                        csync();
-                        // candidate position -> chunk id (increasing map); the
-                        // superchunks come from their published copy (entry + 1)
-                        const int* sup = arr(A_ENTRIES + p.topk, pair);
-                        int* pub = arr(A_ENTRIES, pair);
-                        for (int c = tid; c < p.topk; c += kConsumers) {
-                            const int pos = out[c];
-                            if (pos >= 0) {
-                                int m;
-                                if (pos < ks * p.J) {
-                                    int e = ld_relaxed(sup + pos / p.J);
-                                    for (int tries = 0; e == 0 && tries < (1 << 20); ++tries) {
-                                        __nanosleep(64);
-                                        e = ld_relaxed(sup + pos / p.J);
-                                    }
-                                    if (e == 0) report_status(kStatusTimeout);
-                                    m = (e - 1) * p.J + pos % p.J;
-                                } else {
-                                    m = S * p.J + (pos - ks * p.J);
+                    vals = p.cand_scores + (size_t)pair * p.Mc_max;
+                    nv = z.Mc;
+                    int* out = p.sel_idx + (size_t)pair * p.topk;
+                    block_topk<kConsumers>(vals, nv, p.topk, out, tsc, csync, NoProbe(), nullptr,
+                                           p.wait_limit);
+                    csync();
+                    // candidate position -> chunk id (an increasing map); the
+                    // superchunks come from their published copy (entry + 1)
+                    const int* sup = rec(A_ENTRIES + p.topk, pair);
+                    int* pub = rec(A_ENTRIES, pair);
+                    for (int c = tid; c < p.topk; c += kConsumers) {
+                        const int pos = out[c];
+                        if (pos >= 0) {
+                            int m;
+                            if (pos < z.ks * p.J) {
+                                int e = ld_relaxed(sup + pos / p.J);
+                                const long long c0 = clock64(), lim = wait_cycles(p.wait_limit);
+                                while (e == 0 && clock64() - c0 < lim) {
+                                    __nanosleep(64);
+                                    e = ld_relaxed(sup + pos / p.J);
                                 }
-                                out[c] = m;
-                                pub[c] = m + 1;
+                                if (e == 0) report_status(kStatusTimeout);
+                                m = (e - 1) * p.J + pos % p.J;
+                            } else {
+                                m = z.S * p.J + (pos - z.ks * p.J);
                             }
+                            out[c] = m;
+                            pub[c] = m + 1;
                         }
-                        k = min(p.topk, nc);
                     }
-                    if (tid == 0) *arr(A_COUNT, pair) = k + 1;
+                    if (tid == 0) *rec(A_COUNT, pair) = z.kc + 1;
                 }
-                csync();  // the shared union area is free again for the next item
+                csync();
+                for (int i = tid; i < nv; i += kConsumers) vals[i] = 0.f;
+                csync();  // the shared union area is free again
             } else {
-                // ---- validate a caller-given selection and publish it
-                const int b = pair / p.Hkv;
-                int n = seq_len_checked(p, b);
-                if (n < 0) n = 0;
-                const int M = n / p.C;
+                // ---- check a caller-given selection and publish it
                 const int* sl = p.sel_idx + (size_t)pair * p.topk;
                 if (tid == 0) {
                     misc[2] = 1;
@@ -883,7 +1317,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                     if (v < 0) {
                         ok = (v == -1);
                     } else {
-                        ok = (v < M) && (c == 0 || (prev >= 0 && prev < v));
+                        // ascending chunk ids, entries before any -1
+                        ok = (v < z.M) && (c == 0 || (prev >= 0 && prev < v));
                         atomicAdd(&misc[3], 1);
                     }
                     if (!ok) misc[2] = 0;
@@ -891,195 +1326,139 @@ __global__ void __launch_bounds__(kThreads, 2)
                 csync();
                 const bool good = misc[2] != 0;
                 if (good) {
-                    int* pub = arr(A_ENTRIES, pair);
+                    int* pub = rec(A_ENTRIES, pair);
                     for (int c = tid; c < misc[3]; c += kConsumers) pub[c] = sl[c] + 1;
                 }
                 if (tid == 0) {
                     if (!good) report_status(kStatusBadInput);
                     if (!(p.debug_flags & 1))
-                        st_release(arr(A_COUNT, pair), good ? misc[3] + 1 : (kBadBit | 1));
+                        st_release(rec(A_COUNT, pair), good ? misc[3] + 1 : (kBadBit | 1));
                 }
                 csync();
             }
-            if (tid == 0) SSA_TR(TR_C_TOPK1, mt.item, pair);
-        } else if (mt.kind == K_COMBINE) {
+            if (tid == 0) SSA_TR(TR_C_SEL1, what, pair);
+        } else {  // K_COMBINE
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
+#ifdef SSA_TRACE
+            if (lane == 0 && warp == tr_warp) trace_event(p, &misc[15], 16, mt.kind, round * NS + stage);
+#endif
             if (tid == 0) SSA_TR(TR_C_COMB0, 0, pair);
-            const int G = p.G;
             // ---- combination of the pair's partial passes (sec. 3.6)
+            const int G = p.G;
             const int b = pair / p.Hkv, j = pair % p.Hkv;
-            bool bad = false;
-            if (p.mode == kModeAttnOnly) {
-                if (tid == 0) {
-                    wait_geq(arr(A_COUNT, pair), 1, p.wait_limit);
-                    misc[4] = (ld_acquire(arr(A_COUNT, pair)) & kBadBit) != 0;
+            int c0[3], nseg[3];
+            pv.pair_blocks(L_META, pair, c0[0], nseg[0]);
+            pv.pair_blocks(L_GIST, pair, c0[1], nseg[1]);
+            pv.pair_blocks(L_RAW, pair, c0[2], nseg[2]);
+            const int NP = nseg[0] + nseg[1] + nseg[2];
+            if (tid == 0) {
+                wait_geq(rec(A_ATTN, pair), NP, p.wait_limit);
+                bool bad = false;
+                if (p.mode == kModeAttnOnly) {
+                    wait_geq(rec(A_COUNT, pair), 1, p.wait_limit);
+                    bad = (ld_acquire(rec(A_COUNT, pair)) & kBadBit) != 0;
                 }
-                csync();
-                bad = misc[4] != 0;
-            }
-            const int NP = p.attn_items * kConsumerWarps;  // one partial per item and warp
-            const size_t stride = (size_t)G * (D + 2);
-            const float* pbase = p.partials + (size_t)pair * NP * stride;
-            float* mS = cmb;               // [G][NP] maxima
-            float* lS = cmb + G * NP;      // [G][NP] sums
-            float* fS = cmb + 2 * G * NP;  // [G][NP] weights
-            for (int base = 0; base < G * NP; base += kConsumers * 4) {
-                float mv[4], lv[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int idx = base + u * kConsumers + tid;
-                    const int h = idx / NP, sp = idx - (idx / NP) * NP;
-                    const float* pp = pbase + sp * stride + (size_t)h * (D + 2);
-                    mv[u] = idx < G * NP ? __ldcg(pp) : -INFINITY;
-                    lv[u] = idx < G * NP ? __ldcg(pp + 1) : 0.f;
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int idx = base + u * kConsumers + tid;
-                    if (idx < G * NP) {
-                        mS[idx] = mv[u];
-                        lS[idx] = lv[u];
-                    }
-                }
+                misc[5] = bad;
             }
             csync();
+            const bool bad = misc[5] != 0;
+            // lane i of a warp handles segments i, i + 32, ...: its partial's
+            // address (for head 0) and, per head, its weight
+            auto seg_base = [&](int s) -> const float* {
+                int a = 0;
+                while (a < 2 && s >= nseg[a]) s -= nseg[a++];
+                return p.partials + partial_offset(p, a, c0[a] + s, pair, 0, D);
+            };
             for (int h = warp; h < G; h += kConsumerWarps) {
-                float mx = -INFINITY;
-                for (int sp = lane; sp < NP; sp += 32) mx = fmaxf(mx, mS[h * NP + sp]);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                float Lsum = 0.f;
-                for (int sp = lane; sp < NP; sp += 32) {
-                    const float ms = mS[h * NP + sp];
-                    const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - mx);
-                    fS[h * NP + sp] = f;
-                    Lsum += f * lS[h * NP + sp];
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
-                __syncwarp();
                 float* op = p.out + ((size_t)b * p.Hq + (size_t)j * G + h) * D;
-                const float inv = (!bad && Lsum > 0.f) ? 1.f / Lsum : 0.f;
+                float ox[D / 64][2];
 #pragma unroll
-                for (int d0 = 2 * lane; d0 < D; d0 += 64) {
-                    float ox = 0.f, oy = 0.f;
-                    const float* col = pbase + (size_t)h * (D + 2) + 2 + d0;
-#pragma unroll 8
-                    for (int sp = 0; sp < NP; ++sp) {
-                        const float2 a = __ldcg(reinterpret_cast<const float2*>(col + sp * stride));
-                        const float f = fS[h * NP + sp];
-                        ox += f * a.x;
-                        oy += f * a.y;
+                for (int t = 0; t < D / 64; ++t) ox[t][0] = ox[t][1] = 0.f;
+                float mx = -INFINITY, lsum = 0.f;
+                // pass 1: maxima and normaliser (one load per lane and 32 segments)
+                for (int sb = 0; sb < NP; sb += 32) {
+                    float2 ml = make_float2(-INFINITY, 0.f);
+                    if (sb + lane < NP)
+                        ml = __ldcg(reinterpret_cast<const float2*>(seg_base(sb + lane) +
+                                                                    (size_t)h * (D + 2)));
+                    float m32 = ml.x;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1)
+                        m32 = fmaxf(m32, __shfl_xor_sync(0xffffffffu, m32, o));
+                    const float mnew = fmaxf(mx, m32);
+                    const float ref = (mnew == -INFINITY) ? 0.f : mnew;
+                    const float alpha = exp2f(mx - ref);
+                    const float fl = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - ref);
+                    float l32 = fl * ml.y;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) l32 += __shfl_xor_sync(0xffffffffu, l32, o);
+                    lsum = lsum * alpha + l32;
+#pragma unroll
+                    for (int t = 0; t < D / 64; ++t) {
+                        ox[t][0] *= alpha;
+                        ox[t][1] *= alpha;
                     }
-                    *reinterpret_cast<float2*>(op + d0) = make_float2(ox * inv, oy * inv);
+                    mx = mnew;
+                    // pass 2 for these 32 segments: weighted sum of their outputs,
+                    // kCB independent loads in flight per lane
+                    const float* mine = (sb + lane < NP)
+                                            ? seg_base(sb + lane) + (size_t)h * (D + 2) + 2
+                                            : p.partials;
+                    const int cnt = min(32, NP - sb);
+                    constexpr int kCB = D == 64 ? 16 : 4;
+                    for (int i0 = 0; i0 < cnt; i0 += kCB) {
+                        float2 a[kCB][D / 64];
+                        float f[kCB];
+#pragma unroll
+                        for (int u = 0; u < kCB; ++u) {
+                            const int i = (i0 + u) & 31;
+                            const float* q = reinterpret_cast<const float*>(__shfl_sync(
+                                0xffffffffu, reinterpret_cast<uintptr_t>(mine), i));
+                            f[u] = __shfl_sync(0xffffffffu, fl, i);
+                            if (i0 + u < cnt) {
+#pragma unroll
+                                for (int t = 0; t < D / 64; ++t)
+                                    a[u][t] = __ldcg(reinterpret_cast<const float2*>(
+                                        q + 64 * t + 2 * lane));
+                            } else {
+                                f[u] = 0.f;
+#pragma unroll
+                                for (int t = 0; t < D / 64; ++t) a[u][t] = make_float2(0.f, 0.f);
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < kCB; ++u)
+#pragma unroll
+                            for (int t = 0; t < D / 64; ++t) {
+                                ox[t][0] += f[u] * a[u][t].x;
+                                ox[t][1] += f[u] * a[u][t].y;
+                            }
+                    }
                 }
+                const float inv = (!bad && lsum > 0.f) ? 1.f / lsum : 0.f;
+#pragma unroll
+                for (int t = 0; t < D / 64; ++t)
+                    *reinterpret_cast<float2*>(op + 64 * t + 2 * lane) =
+                        make_float2(ox[t][0] * inv, ox[t][1] * inv);
             }
             csync();
             {
                 // clear this pair's record for the next call
-                int* rec = arr(0, pair);
+                int* r = rec(0, pair);
                 const int used = A_ENTRIES + p.topk + (p.h2 ? p.topk_super : 0);
-                for (int a = tid; a < used; a += kConsumers) rec[a] = 0;
+                for (int a = tid; a < used; a += kConsumers) r[a] = 0;
             }
             if (tid == 0) SSA_TR(TR_C_COMB1, 0, pair);
-        } else {  // K_ATTN
-            if (mt.flags & F_FIRST) {
-                mrow[0] = mrow[1] = -INFINITY;
-                lrow[0] = lrow[1] = 0.f;
-#pragma unroll
-                for (int nt = 0; nt < D / 8; ++nt)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
-            }
-            const int rbase = 16 * warp;
-            if (rbase < mt.nvalid) {
-                float s[2][4];
-                qk16<D>(slotA, rbase, qa, s, lane);
-                const uint64_t excl = ((uint64_t)mt.rmask_hi << 32) | mt.rmask_lo;
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int lr = rbase + nt * 8 + 2 * tig + (c & 1);
-                        const bool out = lr >= mt.nvalid || ((excl >> lr) & 1ull);
-                        s[nt][c] = out ? -INFINITY : s[nt][c] * scale_log2;
-                    }
-                uint32_t phi[4], plo[4];
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    float mx = fmaxf(fmaxf(s[0][2 * r], s[0][2 * r + 1]),
-                                     fmaxf(s[1][2 * r], s[1][2 * r + 1]));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                    const float mnew = fmaxf(mrow[r], mx);
-                    const float ref = (mnew == -INFINITY) ? 0.f : mnew;
-                    const float alpha = exp2f(mrow[r] - ref);
-                    const float p00 = exp2f(s[0][2 * r] - ref), p01 = exp2f(s[0][2 * r + 1] - ref);
-                    const float p10 = exp2f(s[1][2 * r] - ref), p11 = exp2f(s[1][2 * r + 1] - ref);
-                    lrow[r] = lrow[r] * alpha + (p00 + p01 + p10 + p11);
-                    mrow[r] = mnew;
-#pragma unroll
-                    for (int nt = 0; nt < D / 8; ++nt) {
-                        acc[nt][2 * r] *= alpha;
-                        acc[nt][2 * r + 1] *= alpha;
-                    }
-                    split_bf16(p00, p01, phi[r], plo[r]);          // tokens 0..7
-                    split_bf16(p10, p11, phi[2 + r], plo[2 + r]);  // tokens 8..15
-                }
-                pv16<D>(slotB, rbase, phi, plo, acc, lane);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
-
-            if (mt.flags & F_LAST) {
-                if (tid == 0) SSA_TR(TR_C_LAST, K_ATTN, pair);
-                // ---- write this warp's partial (m, l, acc) for its heads; the
-                // combination merges the warps' partials, so items end without
-                // a block-wide barrier
-                const int G = p.G;
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    float l = lrow[r];
-                    l += __shfl_xor_sync(0xffffffffu, l, 1);
-                    l += __shfl_xor_sync(0xffffffffu, l, 2);
-                    const int h = g8 + 8 * r;
-                    if (h < G) {
-                        float* dstp = p.partials +
-                                      ((((size_t)pair * p.attn_items + mt.item) * kConsumerWarps +
-                                        warp) * G + h) * (D + 2);
-                        if (tig == 0) *reinterpret_cast<float2*>(dstp) = make_float2(mrow[r], l);
-#pragma unroll
-                        for (int nt = 0; nt < D / 8; ++nt)
-                            *reinterpret_cast<float2*>(dstp + 2 + nt * 8 + 2 * tig) =
-                                make_float2(acc[nt][2 * r], acc[nt][2 * r + 1]);
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) red_release_add(arr(A_ATTN, pair), 1);
-                if (tid == 0) SSA_TR(TR_C_DONE, K_ATTN, pair);
-            }
         }
         if (++stage == NS) {
             stage = 0;
             ++round;
         }
     }
-    // ---- last block out resets the ticket for the next launch
-    csync();
     if (tid == 0) {
         SSA_TR(TR_KEND, 0, 0);
         SSA_TR(TR_KEND | 0x80, 0, 0);
-    }
-    if (p.mode != kModeScoreOnly && tid == 0) {
-        __threadfence();
-        const int old = atomicAdd(ctrl + C_EXIT, 1);
-        if (old == (int)gridDim.x - 1) {
-            ctrl[C_TICKET] = 0;
-            ctrl[C_EXIT] = 0;
-            __threadfence();
-        }
     }
 }
 

@@ -99,6 +99,7 @@ __global__ void score_kernel(Plan p, int level, float* dst, int stride, int n_sl
 
 struct BlockSync {
     __device__ void operator()() const { __syncthreads(); }
+    __device__ bool or_(bool pred) const { return __syncthreads_or(pred) != 0; }
 };
 
 // Top-k per pair (block of 128).  level 0: chunks over scores (single level

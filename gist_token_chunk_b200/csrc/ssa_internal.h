@@ -11,6 +11,11 @@ namespace ssa {
 
 enum Mode : int { kModeFull = 0, kModeScoreOnly = 1, kModeAttnOnly = 2 };
 
+// Upper bound on the fused kernel's grid (sizes the partials area).
+constexpr int kFusedMaxGrid = 1024;
+// Sequences the fused kernel's in-block plan holds.
+constexpr int kFusedMaxB = 128;
+
 // Everything a launch needs, resolved on the host.  Pointers are device
 // pointers.  Sizes follow the public header's notation.
 struct Plan {
@@ -22,12 +27,11 @@ struct Plan {
     int J = 0, gm = 0, S_max = 0, topk_super = 0, Mc_max = 0;
     int n_pairs = 0;
 
-    // work decomposition of the fused kernel
-    int score_items = 0;   // per pair: gist scoring (single) / meta scoring (two level)
-    int score_spi = 0;     // summary slots per score item
-    int cand_items = 0;    // per pair: candidate-chunk scoring (two level)
-    int attn_items = 0;    // per pair
-    int pair_ints = 0;     // control words per pair (counters + published selection)
+    // fused kernel: blocks (0: every co-resident block), summary rows per
+    // scoring sub-item, control words per pair (counters + published selection)
+    int grid_cap = 0;
+    int score_rows = 1024;
+    int pair_ints = 0;
     int mask_words = 0, smask_words = 0;
 
     const void* q = nullptr;
@@ -45,7 +49,7 @@ struct Plan {
     int32_t* sel_super = nullptr;   // [P, topk_super]
     uint32_t* chunk_mask = nullptr; // [P, mask_words]
     uint32_t* super_mask = nullptr; // [P, smask_words]
-    float* partials = nullptr;      // [P, attn_items, G, d + 2]
+    float* partials = nullptr;      // [3, kFusedMaxGrid + P, G, d + 2]
     float* out = nullptr;           // [B, Hq, d]
     int* ctrl = nullptr;            // control words
     long long wait_limit = 0;       // ns bound of every device-side wait

@@ -101,16 +101,37 @@ static cudaError_t launch_fused_d(const Plan& p, cudaStream_t stream) {
                                                                   (size_t)L.total);
     if (e != cudaSuccess) return e;
     if (occ < 1) return cudaErrorInvalidConfiguration;
-    const int per_a = (p.mode == kModeAttnOnly) ? 1 : p.score_items;
-    long long total = (long long)p.n_pairs * per_a;
-    if (p.h2) total += (long long)p.n_pairs * p.cand_items;
-    if (p.mode != kModeScoreOnly) total += (long long)p.n_pairs * p.attn_items;
+    // One block per co-resident slot: the static schedule waits across blocks,
+    // so the launch is cooperative (all blocks resident at once).  Fewer
+    // blocks when the call has little work (upper bound from n_max).
+    const long long NP = p.n_pairs;
+    const long long tpc = (p.C + fused::kBoxRows - 1) / fused::kBoxRows;
+    long long work;
+    if (p.mode == kModeScoreOnly) {
+        work = NP * p.M_max;
+    } else if (!p.h2) {
+        const long long kc = p.topk < p.M_max ? p.topk : p.M_max;
+        work = NP * (p.M_max + ((long long)p.M_max * p.g + 63) / 64 + kc * tpc + tpc + 1);
+    } else {
+        work = NP * (p.S_max + p.Mc_max + ((long long)p.S_max * p.gm + 63) / 64 +
+                    ((long long)p.Mc_max * p.g + 63) / 64 + (long long)p.topk * tpc + tpc + 2);
+    }
     long long grid = (long long)sm_count() * occ;
-    if (grid > total) grid = total;
+    if (p.grid_cap > 0 && grid > p.grid_cap) grid = p.grid_cap;
+    if (grid > kFusedMaxGrid) grid = kFusedMaxGrid;
+    if (grid > work) grid = work;
     if (grid < 1) grid = 1;
-    kern<<<(unsigned)grid, fused::kThreads, (size_t)L.total, stream>>>(p, m[0], m[1], m[2], m[3],
-                                                                        m[4], m[5]);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(fused::kThreads);
+    cfg.dynamicSmemBytes = (size_t)L.total;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p, m[0], m[1], m[2], m[3], m[4], m[5]);
 }
 
 cudaError_t launch_fused(const Plan& p, cudaStream_t stream) {

@@ -235,5 +235,5 @@ def ssa_set_debug_flags(flags: int) -> None:
     lib.ssa_set_debug_flags(int(flags))
 
 
-def ssa_set_tuning(units_per_attn_item: int = 0, rows_per_score_item: int = 0) -> None:
-    lib.ssa_set_tuning(int(units_per_attn_item), int(rows_per_score_item))
+def ssa_set_tuning(max_blocks: int = 0, rows_per_score_item: int = 0) -> None:
+    lib.ssa_set_tuning(int(max_blocks), int(rows_per_score_item))

@@ -61,10 +61,11 @@
  * bytes.  Pass ws = NULL, ws_bytes = 0 to let the library allocate it
  * stream-ordered (cudaMallocAsync) for that one call.  A caller-owned
  * workspace must be zeroed once with ssa_workspace_init() (or cudaMemset 0)
- * before its first use; every call leaves its control words zeroed again, so
- * it can be reused by later calls on the same stream, for any sizes that fit,
- * without re-initialising (when a call needs a larger control region than the
- * workspace's previous call, the library zeroes it stream-ordered first).
+ * before its first use; every call leaves the state it used (control words
+ * and score scratch) zeroed again, so it can be reused by later calls on the
+ * same stream, for any sizes that fit, without re-initialising (when a call
+ * lays the workspace out differently from the workspace's previous call, the
+ * library zeroes the part it needs stream-ordered first).
  * After a call that reported SSA_ERR_DEVICE_TIMEOUT, initialise it again.
  * Two calls that share a workspace must not run concurrently.
  */
@@ -202,12 +203,13 @@ SSA_API void ssa_set_wait_limit(int64_t ns);
 
 /*
  * Work-splitting knobs of the fused kernel (process-wide, later launches):
- * units_per_attn_item = 64-row context tiles per attention work item (the
- * split-K granularity), rows_per_score_item = summary rows per scoring work
- * item.  Values < 1 restore the defaults (6 and 512).  Results do not depend
- * on them beyond fp32 summation order.
+ * max_blocks caps the blocks of the launch (every list of work is split into
+ * that many equal shares; default: every block the device holds at once),
+ * rows_per_score_item caps the summary rows a block scores before writing
+ * chunk scores (at most 1024, the default).  Values < 1 restore the
+ * defaults.  Results do not depend on them beyond fp32 summation order.
  */
-SSA_API void ssa_set_tuning(int32_t units_per_attn_item, int32_t rows_per_score_item);
+SSA_API void ssa_set_tuning(int32_t max_blocks, int32_t rows_per_score_item);
 
 /*
  * Test hook: with SSA_DEBUG_SKIP_PUBLISH set, the selection step of

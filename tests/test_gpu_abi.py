@@ -60,10 +60,10 @@ def test_workspace_reuse_stays_clean(ssa, inp):
     assert ssa.ssa_get_device_status() == 0
 
 
-@pytest.mark.parametrize("units", [1, 3, 64])
-def test_split_invariance(ssa, inp, units):
+@pytest.mark.parametrize("blocks", [1, 3, 37])
+def test_split_invariance(ssa, inp, blocks):
     o0, s0 = run(ssa, inp)
-    ssa.ssa_set_tuning(units, 128)
+    ssa.ssa_set_tuning(blocks, 128)
     try:
         o, s = run(ssa, inp)
     finally:
