@@ -89,6 +89,23 @@ def algorithmic_bytes(w, seq_lens) -> int:
     return tot
 
 
+# --------------------------------------------------------- multi-rank ---
+
+def rank_seed(seed: int, s: int, rank: int) -> int:
+    """Seed of input set `s` on rank `rank`: every rank decodes its own batch
+    of independent sequences (weak scaling, no exchange between ranks)."""
+    return seed + 7919 * s + 100003 * rank
+
+
+def max_over_ranks(x: float, pg, device) -> float:
+    """The maximum of `x` over all ranks (the slowest rank's time)."""
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------- peaks ---
 
 def hbm_peak():
@@ -304,7 +321,10 @@ def main():
     ap.add_argument("--seed", type=int, default=1003)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=1000)
+    ap.add_argument("--e2e-steps", type=int, default=1000,
+                    help="steps of the end-to-end measurement (0: skip it)")
+    ap.add_argument("--sets", type=int, default=NSETS,
+                    help="rotating input sets (fewer only for profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -330,8 +350,9 @@ def main():
 
     w = WORKLOADS[args.config]
     # each rank decodes its own batch (independent sequences)
-    sets = [make_inputs(w, seed=args.seed + 7919 * s + 100003 * rank, device=dev)
-            for s in range(NSETS)]
+    NS = max(1, args.sets)
+    sets = [make_inputs(w, seed=rank_seed(args.seed, s, rank), device=dev)
+            for s in range(NS)]
     for s in sets:
         s.pop("planted_idx", None)
     shape = ssa.shape_of(sets[0]["q"], sets[0]["k_raw"])
@@ -340,13 +361,13 @@ def main():
     else:
         nbytes = ssa.ssa_workspace_size(shape, w.C, w.g, w.topk)
     ws = ssa.workspace(nbytes, device=dev)
-    outs = [torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev) for _ in range(NSETS)]
-    sels = [torch.empty(w.B, w.Hkv, w.topk, dtype=torch.int32, device=dev) for _ in range(NSETS)]
+    outs = [torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev) for _ in range(NS)]
+    sels = [torch.empty(w.B, w.Hkv, w.topk, dtype=torch.int32, device=dev) for _ in range(NS)]
     sups = [torch.empty(w.B, w.Hkv, max(w.topk_super, 1), dtype=torch.int32, device=dev)
-            for _ in range(NSETS)]
+            for _ in range(NS)]
 
     def step(i, stream=None):
-        s = i % NSETS
+        s = i % NS
         x = sets[s]
         if w.two_level:
             ssa.ssa_decode_h2(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
@@ -361,17 +382,17 @@ def main():
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize(dev)
     with torch.cuda.stream(stream):
-        for i in range(NSETS):
+        for i in range(NS):
             step(i)  # eager first use (workspace control region, attributes)
     stream.synchronize()
-    # graphs: a chunk of REP*NSETS steps and single steps for the remainder
+    # graphs: a chunk of REP*NS steps and single steps for the remainder
     REP = 8
     g_chunk = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_chunk, stream=stream):
-        for i in range(REP * NSETS):
+        for i in range(REP * NS):
             step(i, stream=stream)
     g_one = []
-    for s in range(NSETS):
+    for s in range(NS):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             step(s, stream=stream)
@@ -380,11 +401,11 @@ def main():
 
     def run_steps(k):
         done = 0
-        while k - done >= REP * NSETS:
+        while k - done >= REP * NS:
             g_chunk.replay()
-            done += REP * NSETS
+            done += REP * NS
         while done < k:
-            g_one[done % NSETS].replay()
+            g_one[done % NS].replay()
             done += 1
 
     with torch.cuda.stream(stream):
@@ -403,11 +424,7 @@ def main():
             ev1.record(stream)
         ev1.synchronize()
     torch.cuda.synchronize(dev)
-    ms = ev0.elapsed_time(ev1)
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), pg, dev)
     status = ssa.ssa_get_device_status(stream)
     if status != 0:
         raise SystemExit(f"device status {status} after the timed region")
@@ -423,7 +440,7 @@ def main():
     peak, peak_src = hbm_peak()
 
     # ---- end to end through the public call, host buffers
-    ek = max(NSETS, min(args.steps, args.e2e_steps))
+    ek = max(NS, min(args.steps, args.e2e_steps)) if args.e2e_steps > 0 else 0
     q_host = [x["q"].cpu().pin_memory() for x in sets]
     len_host = [x["seq_lens"].cpu().pin_memory() for x in sets]
     q_dev = [torch.empty_like(x["q"]) for x in sets]
@@ -432,7 +449,7 @@ def main():
     sel_host = [torch.empty(s.shape, dtype=s.dtype).pin_memory() for s in sels]
 
     def e2e_step(i):
-        s = i % NSETS
+        s = i % NS
         q_dev[s].copy_(q_host[s], non_blocking=True)
         len_dev[s].copy_(len_host[s], non_blocking=True)
         x = dict(sets[s], q=q_dev[s], seq_lens=len_dev[s])
@@ -448,25 +465,23 @@ def main():
         out_host[s].copy_(outs[s], non_blocking=True)
         sel_host[s].copy_(sels[s], non_blocking=True)
 
-    with torch.cuda.stream(stream):
-        for i in range(NSETS):
-            e2e_step(i)
-    stream.synchronize()
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize(dev)
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        for i in range(ek):
-            e2e_step(i)
-        ev1.record(stream)
-    ev1.synchronize()
-    e2e_ms = ev0.elapsed_time(ev1)
-    if pg:
-        t = torch.tensor([e2e_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = ek * w.B * world / (e2e_ms / 1e3)
+    e2e_value = None
+    if ek > 0:
+        with torch.cuda.stream(stream):
+            for i in range(NS):
+                e2e_step(i)
+        stream.synchronize()
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for i in range(ek):
+                e2e_step(i)
+            ev1.record(stream)
+        ev1.synchronize()
+        e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), pg, dev)
+        e2e_value = ek * w.B * world / (e2e_ms / 1e3)
     h2d = sets[0]["q"].numel() * sets[0]["q"].element_size() + sets[0]["seq_lens"].numel() * 4
     d2h = outs[0].numel() * 4 + sels[0].numel() * 4
 
@@ -476,8 +491,8 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
         "config": dict(config_of(w), global_batch=w.B * world,
-                       l2=f"{NSETS} input sets rotate (each step follows >= 3 steps over other "
-                          "sets; inputs larger than L2)",
+                       l2=f"{NS} input sets rotate (each step follows {NS - 1} steps over "
+                          "other sets; inputs larger than L2)",
                        timing="CUDA-graph replays of the fused kernel, CUDA events, max over ranks",
                        parallelism=f"dp{world} (independent sequences per GPU, no collective)"),
         "hbm_gbs": achieved, "hbm_frac_of_peak": achieved / peak,
