@@ -393,6 +393,44 @@ ssa_status ssa_decode(const ssa_shape* shape, const void* q, const void* k_raw, 
     return run_with_ws(p, ws, ws_bytes, stream);
 }
 
+ssa_status ssa_decode_noalloc(const ssa_shape* shape, const void* q, const void* k_raw,
+                              const void* v_raw, const void* k_gist, const void* v_gist,
+                              const int32_t* seq_lens, int32_t C, int32_t g, int32_t topk,
+                              float* out, int32_t* sel_idx, cudaStream_t stream) {
+    ssa::Plan p;
+    ssa_status st = build_single(p, shape, C, g, topk);
+    if (st != SSA_OK) return st;
+    st = check_tensors(p, {q, k_raw, v_raw, k_gist, v_gist, seq_lens, out});
+    if (st != SSA_OK) return st;
+    if (topk > 0 && !sel_idx) return fail(SSA_ERR_INVALID_ARG, "sel_idx is NULL");
+    const ssa::WsLayout L = ssa::plan_layout(p);
+    if (L.total > ssa::kBuiltinWsBytes)
+        return fail(SSA_ERR_WORKSPACE,
+                    "ssa_decode_noalloc: these sizes need %zu bytes of scratch, the built-in "
+                    "area holds %zu; use ssa_decode with a workspace",
+                    L.total, ssa::kBuiltinWsBytes);
+    void* ws = nullptr;
+    cudaError_t e = ssa::builtin_workspace(&ws);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(built-in scratch)");
+    p.mode = ssa::kModeFull;
+    p.q = q;
+    p.k_raw = k_raw;
+    p.v_raw = v_raw;
+    p.k_gist = k_gist;
+    p.v_gist = v_gist;
+    p.seq_lens = seq_lens;
+    p.sel_idx = sel_idx;
+    p.out = out;
+    attach_ws(p, ws);
+    // the area keeps whatever the previous call left: clear the part that
+    // must start at zero (control words and scores), stream-ordered
+    e = cudaMemsetAsync(ws, 0, L.partials, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(built-in scratch)");
+    e = fused_path(p) ? ssa::launch_fused(p, stream) : ssa::launch_generic(p, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return SSA_OK;
+}
+
 ssa_status ssa_decode_h2(const ssa_shape* shape, const void* q, const void* k_raw,
                          const void* v_raw, const void* k_gist, const void* v_gist,
                          const void* k_meta, const void* v_meta, const int32_t* seq_lens,

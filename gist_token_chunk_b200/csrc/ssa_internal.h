@@ -79,6 +79,12 @@ cudaError_t launch_topk(const Plan& p, const float* scores, cudaStream_t stream)
 
 cudaError_t read_device_status(int* code, cudaStream_t stream);
 
+// Built-in scratch of ssa_decode_noalloc: a fixed device array in the
+// library's device code (no allocation).  Its device address for the current
+// device, looked up once per device.
+constexpr size_t kBuiltinWsBytes = size_t(8) << 20;
+cudaError_t builtin_workspace(void** ptr);
+
 // Query the SM count of the current device (cached per device).
 int sm_count();
 

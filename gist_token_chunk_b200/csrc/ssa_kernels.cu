@@ -36,6 +36,30 @@ cudaError_t read_device_status(int* code, cudaStream_t stream) {
     return e;
 }
 
+// ------------------------------------------------------- built-in scratch ---
+// The scratch of ssa_decode_noalloc lives in the library's own device code, so
+// that entry point never allocates.  Every call shares it.
+static __device__ __align__(256) unsigned char g_builtin_ws[kBuiltinWsBytes];
+
+cudaError_t builtin_workspace(void** ptr) {
+    static std::mutex mu;
+    static void* addr[64] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!addr[dev]) {
+        // first use on this device (which is current): look up the address
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_builtin_ws);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return cudaSuccess;
+}
+
 // ------------------------------------------------------------- tensor maps ---
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {

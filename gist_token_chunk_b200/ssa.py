@@ -55,6 +55,7 @@ lib.ssa_score_gists.argtypes = [_SH, _P, _P, _P, _I, _I, _P, _P]
 lib.ssa_topk_chunks.argtypes = [_SH, _P, _P, _I, _I, _P, _P]
 lib.ssa_sparse_decode.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _S, _P]
 lib.ssa_decode.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _S, _P]
+lib.ssa_decode_noalloc.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P]
 lib.ssa_decode_h2.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P,
                               _P, _P, _P, _S, _P]
 lib.ssa_workspace_size.argtypes = [_SH, _I, _I, _I, ctypes.POINTER(_S)]
@@ -73,7 +74,7 @@ lib.ssa_last_error.argtypes = []
 lib.ssa_last_error.restype = ctypes.c_char_p
 lib.ssa_version.restype = _I
 for _f in ("ssa_score_gists", "ssa_topk_chunks", "ssa_sparse_decode", "ssa_decode",
-           "ssa_decode_h2", "ssa_workspace_size", "ssa_workspace_size_h2",
+           "ssa_decode_noalloc", "ssa_decode_h2", "ssa_workspace_size", "ssa_workspace_size_h2",
            "ssa_workspace_init", "ssa_get_device_status"):
     getattr(lib, _f).restype = _I
 
@@ -197,6 +198,19 @@ def ssa_decode(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C: int, g: int, topk: 
     _check(lib.ssa_decode(ctypes.byref(shape), _ptr(q), _ptr(k_raw), _ptr(v_raw), _ptr(k_gist),
                           _ptr(v_gist), _ptr(seq_lens), C, g, topk, _ptr(out), _ptr(sel_idx),
                           _ptr(ws), nbytes, _stream(stream)), "ssa_decode")
+    return out, sel_idx
+
+
+def ssa_decode_noalloc(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C: int, g: int, topk: int,
+                       out, sel_idx, stream=None):
+    """ssa_decode without a workspace, for callers that cannot allocate:
+    the library's built-in scratch is used (see include/ssa.h).  The caller
+    passes the outputs; nothing is allocated here either."""
+    shape = shape_of(q, k_raw)
+    _check(lib.ssa_decode_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k_raw), _ptr(v_raw),
+                                  _ptr(k_gist), _ptr(v_gist), _ptr(seq_lens), C, g, topk,
+                                  _ptr(out), _ptr(sel_idx), _stream(stream)),
+           "ssa_decode_noalloc")
     return out, sel_idx
 
 

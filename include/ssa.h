@@ -153,6 +153,30 @@ SSA_API ssa_status ssa_decode(const ssa_shape* shape, const void* q, const void*
                       int32_t* sel_idx, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * ssa_decode_noalloc -- ssa_decode for callers that cannot allocate device
+ * memory and cannot pass a workspace: for example an engine that reserves all
+ * device memory for itself before serving, or a plugin interface that hands
+ * over only the tensors.  The pages have no counterpart; this is a library
+ * convenience, not a step of the method.
+ * Same arguments and results as ssa_decode without ws / ws_bytes.  It
+ * allocates nothing: its scratch is a fixed 8 MiB area inside the library's
+ * device code (enough for the 32K, 128K and 512K batch workloads of this
+ * library's tests; larger sizes return SSA_ERR_WORKSPACE with the byte count
+ * in ssa_last_error(); use ssa_decode with a workspace then).
+ * The first call on each device, with that device current, looks up the
+ * area's device address (a CUDA runtime query); make that first call before
+ * any stream capture.  Every call clears the part of the area that must start
+ * at zero (a stream-ordered memset) before the kernel runs.  All calls share
+ * the one area and it keeps the last call's contents, so two calls whose work
+ * overlaps on the GPU (different streams without ordering, several host
+ * threads) race on it: order them on one stream.
+ */
+SSA_API ssa_status ssa_decode_noalloc(const ssa_shape* shape, const void* q, const void* k_raw,
+                              const void* v_raw, const void* k_gist, const void* v_gist,
+                              const int32_t* seq_lens, int32_t C, int32_t g, int32_t topk,
+                              float* out, int32_t* sel_idx, cudaStream_t stream);
+
+/*
  * ssa_decode_h2 -- two-level (gist-of-gist) decode step (sec. 3.5, App. B.2).
  * Level 2 scores the S_b = floor(M_b / J) complete superchunks with their gm
  * meta-gist keys (same max-over-heads-and-tokens score) and keeps the top
