@@ -198,14 +198,6 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
         : "memory");
 }
 
-// Prefetch one 2-D box of a tensor map into L2 (no shared memory involved).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(x), "r"(y)
-                 : "memory");
-}
-
 // L2 policies: keep lines that are read again soon; drop single-use lines first.
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
     uint64_t pol;
@@ -359,7 +351,7 @@ struct TopkScratch {
 // the loads repeat (for at most poll_ns) until every value is present.
 // Sync must provide or_(bool): a barrier that ORs a predicate.
 template <int NT, class Sync, class Probe = NoProbe>
-__device__ void block_topk(const float* vals, int n, int topk, int* out, TopkScratch& sc,
+__device__ __noinline__ void block_topk(const float* vals, int n, int topk, int* out, TopkScratch& sc,
                            Sync sync, Probe probe = Probe(), int* pub = nullptr,
                            long long poll_ns = 0) {
     const int tid = threadIdx.x & (NT - 1);

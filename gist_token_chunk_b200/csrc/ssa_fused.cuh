@@ -19,22 +19,31 @@
 // one partial (m, l, o) per query head.  Each block runs, in this order: its
 // SCORE share; the top-k of the pairs it owns; [its META share; its CAND
 // share; the second top-k of its pairs;] its GIST share; its RAW share; the
-// combination of the pairs it owns.  A wait (a pair's scores complete, a
-// selection published, a pair's partials complete) is always on work of an
-// earlier phase, which never waits on a later one, and all blocks are
-// co-resident (cooperative launch), so every wait ends; each is also bounded.
+// combination of the pairs whose last attention element it holds.  A wait (a
+// pair's scores complete, a selection published, a pair's partials complete)
+// is always on work of an earlier phase, which never waits on a later one,
+// and all blocks are co-resident (cooperative launch), so every wait ends;
+// each is also bounded.
 //
-// GIST and META tiles need the selection only to mask excluded rows, so the
+// Logits mode (single level, whole step): the scoring phase keeps every
+// head's logit of its gist rows in shared memory, and the gist phase streams
+// only the values of the same rows (the block's gist share is its score
+// share), so half the bytes go through the ring and most of them arrive
+// while the top-k runs.
+//
+// Gist and meta tiles need the selection only to mask excluded rows, so the
 // producer issues them before the selection exists and the consumers apply
 // the mask once it is published: the selection latency hides behind loads.
 //
 // Block layout: 4 consumer warps + 1 producer warp.  The producer streams
 // 64-row tiles with 2-D TMA (128-byte swizzle) into a ring of stages (slot A:
-// keys, slot B: values; score stages use both slots for keys).  Each consumer
-// warp takes 16 rows of every stage: Q.K^T and P.V run on tensor cores
-// (mma.sync m16n8k16, bf16 in, fp32 accumulate; the GQA group's query heads
-// are the M rows), the softmax is an fp32 online softmax in the log2 domain,
-// and P enters the P.V product as bf16 hi + lo parts (~16 significant bits).
+// keys, slot B: values; score and value-only stages use both slots for one
+// kind of row).  Each consumer warp takes 16 rows of every 64-row box:
+// Q.K^T and P.V run on tensor cores (mma.sync m16n8k16, bf16 in, fp32
+// accumulate; the GQA group's query heads are the M rows; scoring uses the
+// keys as M rows, 16 keys x 8 heads per MMA), the softmax is an fp32 online
+// softmax in the log2 domain, and P enters the P.V product as bf16 hi + lo
+// parts (~16 significant bits).
 #pragma once
 
 #include "ssa_device.cuh"
@@ -51,8 +60,24 @@ constexpr int kRowmaxCap = 1024;      // summary rows per score sub-item
 constexpr int kBarConsumers = 1;      // named barrier id of the consumer warps
 constexpr int kMaxGrid = kFusedMaxGrid;
 constexpr int kMaxTopkEntries = 1024;  // largest topk / topk_super the library accepts
+constexpr int kLogitBytes = 16 * 1024; // shared memory for the kept logits (logits mode)
+// Selection bitmaps a block keeps.  One: loading the selections of several
+// pairs in one round makes the first segment wait for the latest of them.
+constexpr int kMaxBitmaps = 1;
+// P.V formulation: heads as the M rows of the MMA (false: heads as N, dims as M)
+#ifndef SSA_PV_HEADS_M
+#define SSA_PV_HEADS_M 1
+#endif
+constexpr bool kPvHeadsM = SSA_PV_HEADS_M != 0;
 
-enum : int { K_END = 0, K_SCORE = 1, K_ATTN = 2, K_SELECT = 3, K_COMBINE = 4 };
+// Rows of kept logits a block can hold for G query heads, and the row stride
+// of one head's logits (a multiple of 32 plus 8: conflict-free reads).
+__host__ __device__ inline int logit_rows_cap(int G) {
+    const int r = (kLogitBytes / (4 * G) - 8) / 32 * 32;
+    return r > 0 ? r : 0;
+}
+
+enum : int { K_END = 0, K_SCORE = 1, K_ATTN = 2, K_SELECT = 3, K_COMBINE = 4, K_GISTV = 5 };
 enum : int { F_FIRST = 1, F_LAST = 2, F_QLOAD = 4 };
 enum : int { L_SCORE = 0, L_CAND = 1, L_META = 2, L_GIST = 3, L_RAW = 4, kNumLists = 5 };
 // what a K_SELECT stage does
@@ -86,11 +111,11 @@ struct StageMeta {
     // K_ATTN:  a0 first summary row of the tile, a1 mask kind, a2 rows per
     //          masked slot, a3 attention list (0 META, 1 GIST, 2 RAW)
     // K_SELECT: a0 what to do (SEL_*)
-    // Data stages go to the consumer warps in turn (one warp per stage);
-    // every warp still visits every stage (release, segment start and end).
+    // K_GISTV: a0 first gist row of the stage (in the pair), a2 rows per chunk;
+    //          slot A / slot B hold the values of rows 0..63 / 64..127
     int a0, a1, a2, a3, a4, a5;
-    int owner;  // K_SCORE, K_ATTN: the consumer warp that processes the stage
-    int pad1;
+    int pad0;
+    int lrow;   // logits mode: row of the stage's first row in the block's kept logits
 };
 
 template <int D>
@@ -102,7 +127,7 @@ struct Cfg {
 };
 
 struct SmemLayout {
-    int ring, qbuf, qbytes, meta, bars, psel, psup, plan, bits, uni, misc, total;
+    int ring, qbuf, qbytes, meta, bars, psel, psup, plan, bits, uni, logit, misc, total;
 };
 
 __host__ __device__ inline int mask_words_for(const Plan& p) { return (p.M_max + 31) / 32; }
@@ -110,7 +135,7 @@ __host__ __device__ inline int mask_words_for(const Plan& p) { return (p.M_max +
 template <int D>
 __host__ __device__ inline SmemLayout smem_layout(const Plan& p) {
     SmemLayout L;
-    const int NS = Cfg<D>::kStages;
+    const int NS = p.stages > 0 ? p.stages : Cfg<D>::kStages;
     const int G = p.G;
     int o = 0;
     L.ring = o;
@@ -130,8 +155,8 @@ __host__ __device__ inline SmemLayout smem_layout(const Plan& p) {
     L.plan = o;  // lengths [B], then per list prefixes [B + 1]
     o += (p.B + kNumLists * (p.B + 1)) * 4;
     o = (o + 15) / 16 * 16;
-    L.bits = o;  // selection bitmap of the current segment's pair
-    o += ((mask_words_for(p) + 3) / 4 * 4) * 4;
+    L.bits = o;  // selection bitmaps of the pairs of the block's masked segments
+    o += kMaxBitmaps * ((mask_words_for(p) + 3) / 4 * 4) * 4;
     L.uni = o;
     // the consumers use this area for one thing at a time
     int u = kRowmaxCap * 4;                                      // score rows
@@ -140,6 +165,10 @@ __host__ __device__ inline SmemLayout smem_layout(const Plan& p) {
     const int mg = kConsumerWarps * G * (D + 2) * 4;             // warp merge
     u = u > mg ? u : mg;
     o += (u + 15) / 16 * 16;
+    L.logit = o;
+    // + 128 rows of padding: a 128-row tile's reads may run past the last
+    // head's kept rows (those rows are masked, but stay inside the area)
+    if (p.logits) o += (G * p.logit_stride + 128) * 4;
     L.misc = o;
     o += 64;
     L.total = o + 1024;  // slack to align the ring to 1024 bytes
@@ -230,18 +259,33 @@ __device__ __forceinline__ void qkT16(uint32_t slot, int r0, const uint32_t (&qa
     }
 }
 
-// Scores of up to 128 summary rows (two 64-row boxes) by one warp: per row,
-// the maximum over the group's query heads of q.k / sqrt(d), into rowmax.
+// Scores of the 16-row blocks `w` of the two 64-row boxes of a score stage
+// (rows 16 w.. of slot A, and 64 + 16 w.. of slot B) by warp w: per row, the
+// maximum over the group's query heads of q.k / sqrt(d), into rowmax.  With
+// lg != nullptr, also keeps every head's logit in the log2 domain
+// (q.k / sqrt(d) * log2 e) at lg[head * lstride + row].
 template <int D, int NT>
-__device__ __forceinline__ void score_tile(uint32_t slotA, uint32_t slotB, int nvalid, int G,
-                                           const uint32_t (&qa)[D / 16][4], float scale,
-                                           float* rowmax, int lane) {
+__device__ __forceinline__ void score_rows2(uint32_t slotA, uint32_t slotB, int w, int nvalid,
+                                            int G, const uint32_t (&qa)[D / 16][4], float scale,
+                                            float* rowmax, float* lg, int lstride,
+                                            float scale_log2, int lane) {
     const int g8 = lane >> 2, tig = lane & 3;
-#pragma unroll 4
-    for (int sb = 0; sb < 8; ++sb) {
-        if (16 * sb >= nvalid) break;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int r0 = 64 * j + 16 * w;
+        if (r0 >= nvalid) break;
         float st[NT][4];
-        qkT16<D, NT>(sb < 4 ? slotA : slotB, 16 * (sb & 3), qa, st, lane);
+        qkT16<D, NT>(j ? slotB : slotA, 16 * w, qa, st, lane);
+        if (lg) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int h = nt * 8 + 2 * tig + (c & 1);
+                    const int row = r0 + 8 * (c >> 1) + g8;
+                    if (h < G && row < nvalid) lg[h * lstride + row] = st[nt][c] * scale_log2;
+                }
+        }
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             float v = -INFINITY;
@@ -253,102 +297,138 @@ __device__ __forceinline__ void score_tile(uint32_t slotA, uint32_t slotB, int n
             }
             v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
             v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
-            const int lr = 16 * sb + 8 * half + g8;
+            const int lr = r0 + 8 * half + g8;
             if (tig == 0 && lr < nvalid) rowmax[lr] = v * scale;
         }
     }
 }
 
-// acc[dim n-tile] += P(hi+lo) * V for 16 rows starting at r0 of a value slot.
+// O^T += V^T . P^T for 16 rows starting at r0 of a value slot, with the
+// head dimension as the M operand (so a GQA group of <= 8 heads fills one
+// 8-wide N tile): the A fragments are the value rows (ldmatrix.trans, the
+// same loads as a P.V product, reordered); the B fragments are P in the
+// layout a Q.K^T accumulator already has (p[nt] tokens 0..7, p[2 + nt]
+// tokens 8..15 of head 8 nt + g8), as bf16 hi and lo parts.
+// acc[nt][mm][c]: heads 8 nt + 2 tig + (c & 1), dims 16 mm + g8 + 8 (c >> 1).
 template <int D>
-__device__ __forceinline__ void pv16(uint32_t slot, int r0, const uint32_t (&phi)[4],
-                                     const uint32_t (&plo)[4], float (&acc)[D / 8][4], int lane) {
+__device__ __forceinline__ void pvT16(uint32_t slot, int r0, const uint32_t (&phi)[4],
+                                      const uint32_t (&plo)[4], float (&acc)[2][D / 16][4],
+                                      bool two, int lane) {
+    const int row = r0 + (lane & 15);
+    const int csel = lane >> 4;
+#pragma unroll
+    for (int mm = 0; mm < D / 16; ++mm) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_trans(tile_addr<D>(slot, row, 2 * mm + csel), b0, b1, b2, b3);
+        const uint32_t a[4] = {b0, b2, b1, b3};
+        mma_bf16_16816(acc[0][mm], a, phi[0], phi[2]);
+        mma_bf16_16816(acc[0][mm], a, plo[0], plo[2]);
+        if (two) {
+            mma_bf16_16816(acc[1][mm], a, phi[1], phi[3]);
+            mma_bf16_16816(acc[1][mm], a, plo[1], plo[3]);
+        }
+    }
+}
+
+// acc += P(hi + lo) . V for 16 rows at r0 of a value slot with the heads as
+// the M rows (P straight from a Q.K^T accumulator; rows 8..15 are heads
+// 8..15).  The same accumulator storage read as acc8(x) = x-th 8-dim tile:
+// lane holds heads g8 (c < 2) / g8 + 8, dims 8 x + 2 tig + (c & 1).
+template <int D>
+__device__ __forceinline__ float (&acc8(float (&acc)[2][D / 16][4], int x))[4] {
+    return acc[x / (D / 16)][x % (D / 16)];
+}
+template <int D>
+__device__ __forceinline__ void pvM16(uint32_t slot, int r0, const uint32_t (&phi)[4],
+                                      const uint32_t (&plo)[4], float (&acc)[2][D / 16][4],
+                                      int lane) {
     const int row = r0 + (lane & 15);
     const int csel = lane >> 4;
 #pragma unroll
     for (int nn = 0; nn < D / 16; ++nn) {
         uint32_t b0, b1, b2, b3;
         ldsm_x4_trans(tile_addr<D>(slot, row, 2 * nn + csel), b0, b1, b2, b3);
-        mma_bf16_16816(acc[2 * nn], phi, b0, b1);
-        mma_bf16_16816(acc[2 * nn], plo, b0, b1);
-        mma_bf16_16816(acc[2 * nn + 1], phi, b2, b3);
-        mma_bf16_16816(acc[2 * nn + 1], plo, b2, b3);
+        mma_bf16_16816(acc8<D>(acc, 2 * nn), phi, b0, b1);
+        mma_bf16_16816(acc8<D>(acc, 2 * nn), plo, b0, b1);
+        mma_bf16_16816(acc8<D>(acc, 2 * nn + 1), phi, b2, b3);
+        mma_bf16_16816(acc8<D>(acc, 2 * nn + 1), plo, b2, b3);
     }
 }
 
-// One consumer warp's pass over a whole 64-row attention tile: S = Q.K^T for
-// the tile's rows (excluded rows -inf), online-softmax update of (m, l) per
-// query head, acc += P.V with P split into bf16 hi + lo parts.
+// Multiplies the accumulator columns of the heads of n tile r by alpha (held,
+// S-layout, by the lanes of group g8 = head): each lane fetches the factors of
+// its two heads 8 r + 2 tig and 8 r + 2 tig + 1.
 template <int D>
-__device__ __forceinline__ void attn_tile(uint32_t slotA, uint32_t slotB, int nvalid,
-                                          uint32_t ex_lo, uint32_t ex_hi,
-                                          const uint32_t (&qa)[D / 16][4], float (&mrow)[2],
-                                          float (&lrow)[2], float (&acc)[D / 8][4],
-                                          bool two_rows, float scale_log2, int lane) {
-    const int tig = lane & 3;
-    // 16-row sub-blocks per pass: independent Q.K products, one
-    // softmax update per pass
-    constexpr int SB = (D == 64) ? 4 : 2;
+__device__ __forceinline__ void rescale_acc(float (&acc)[2][D / 16][4], int r, float alpha,
+                                            int tig) {
+    if (kPvHeadsM) {
 #pragma unroll
-    for (int pass = 0; pass < 4 / SB; ++pass) {
-        if (16 * SB * pass >= nvalid) break;
-        float sc4[SB][2][4];
-#pragma unroll
-        for (int sb = 0; sb < SB; ++sb) qk16<D>(slotA, 16 * (SB * pass + sb), qa, sc4[sb], lane);
-#pragma unroll
-        for (int sb = 0; sb < SB; ++sb)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int t = 16 * (SB * pass + sb) + nt * 8 + 2 * tig + (c & 1);
-                    const uint32_t ex = t < 32 ? (ex_lo >> t) : (ex_hi >> (t - 32));
-                    sc4[sb][nt][c] = (ex & 1u) ? -INFINITY : sc4[sb][nt][c] * scale_log2;
-                }
-        uint32_t phi[SB][4], plo[SB][4];
-#pragma unroll
-        for (int sb = 0; sb < SB; ++sb)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) phi[sb][c] = plo[sb][c] = 0u;
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            if (r == 1 && !two_rows) break;
-            float mx = -INFINITY;
-#pragma unroll
-            for (int sb = 0; sb < SB; ++sb)
-                mx = fmaxf(mx, fmaxf(fmaxf(sc4[sb][0][2 * r], sc4[sb][0][2 * r + 1]),
-                                     fmaxf(sc4[sb][1][2 * r], sc4[sb][1][2 * r + 1])));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float mnew = fmaxf(mrow[r], mx);
-            const float ref = (mnew == -INFINITY) ? 0.f : mnew;
-            const float alpha = exp2f(mrow[r] - ref);
-            float lsum = 0.f;
-#pragma unroll
-            for (int sb = 0; sb < SB; ++sb) {
-                const float p00 = exp2f(sc4[sb][0][2 * r] - ref);
-                const float p01 = exp2f(sc4[sb][0][2 * r + 1] - ref);
-                const float p10 = exp2f(sc4[sb][1][2 * r] - ref);
-                const float p11 = exp2f(sc4[sb][1][2 * r + 1] - ref);
-                lsum += (p00 + p01) + (p10 + p11);
-                split_bf16(p00, p01, phi[sb][r], plo[sb][r]);          // tokens 0..7
-                split_bf16(p10, p11, phi[sb][2 + r], plo[sb][2 + r]);  // tokens 8..15
-            }
-            lrow[r] = lrow[r] * alpha + lsum;
-            mrow[r] = mnew;
-            if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-                for (int nt = 0; nt < D / 8; ++nt) {
-                    acc[nt][2 * r] *= alpha;
-                    acc[nt][2 * r + 1] *= alpha;
-                }
-            }
+        for (int x = 0; x < D / 8; ++x) {
+            acc8<D>(acc, x)[2 * r] *= alpha;
+            acc8<D>(acc, x)[2 * r + 1] *= alpha;
         }
-#pragma unroll
-        for (int sb = 0; sb < SB; ++sb)
-            if (16 * (SB * pass + sb) < nvalid)
-                pv16<D>(slotB, 16 * (SB * pass + sb), phi[sb], plo[sb], acc, lane);
+        return;
     }
+    const float a0 = __shfl_sync(0xffffffffu, alpha, (2 * tig) << 2);
+    const float a1 = __shfl_sync(0xffffffffu, alpha, (2 * tig + 1) << 2);
+#pragma unroll
+    for (int mm = 0; mm < D / 16; ++mm) {
+        acc[r][mm][0] *= a0;
+        acc[r][mm][1] *= a1;
+        acc[r][mm][2] *= a0;
+        acc[r][mm][3] *= a1;
+    }
+}
+
+// Online-softmax update and P.V for NSB 16-row blocks of one warp.  sc holds
+// the blocks' logits in the log2 domain in the layout of a Q.K^T accumulator
+// with the heads as M rows (sc[i][nt][c]: head g8 (c < 2) or g8 + 8, token
+// nt * 8 + 2 tig + (c & 1)); excluded tokens are -inf.  One max / rescale per
+// call; block i's values are the 16 rows at vrow[i] of slot vslot[i] (blocks
+// with valid[i] false are skipped).
+template <int D, int NSB>
+__device__ __forceinline__ void softmax_pv(float (&sc)[NSB][2][4], const uint32_t (&vslot)[NSB],
+                                           const int (&vrow)[NSB], const bool (&valid)[NSB],
+                                           float (&mrow)[2], float (&lrow)[2],
+                                           float (&acc)[2][D / 16][4], bool two_rows, int lane) {
+    const int tig = lane & 3;
+    uint32_t phi[NSB][4], plo[NSB][4];
+#pragma unroll
+    for (int i = 0; i < NSB; ++i)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) phi[i][c] = plo[i][c] = 0u;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        if (r == 1 && !two_rows) break;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < NSB; ++i)
+            mx = fmaxf(mx, fmaxf(fmaxf(sc[i][0][2 * r], sc[i][0][2 * r + 1]),
+                                 fmaxf(sc[i][1][2 * r], sc[i][1][2 * r + 1])));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float mnew = fmaxf(mrow[r], mx);
+        const float ref = (mnew == -INFINITY) ? 0.f : mnew;
+        const float alpha = exp2f(mrow[r] - ref);
+        float lsum = 0.f;
+#pragma unroll
+        for (int i = 0; i < NSB; ++i) {
+            const float p00 = exp2f(sc[i][0][2 * r] - ref), p01 = exp2f(sc[i][0][2 * r + 1] - ref);
+            const float p10 = exp2f(sc[i][1][2 * r] - ref), p11 = exp2f(sc[i][1][2 * r + 1] - ref);
+            lsum += (p00 + p01) + (p10 + p11);
+            split_bf16(p00, p01, phi[i][r], plo[i][r]);          // tokens 0..7
+            split_bf16(p10, p11, phi[i][2 + r], plo[i][2 + r]);  // tokens 8..15
+        }
+        lrow[r] = lrow[r] * alpha + lsum;
+        mrow[r] = mnew;
+        if (__any_sync(0xffffffffu, alpha != 1.f)) rescale_acc<D>(acc, r, alpha, tig);
+    }
+#pragma unroll
+    for (int i = 0; i < NSB; ++i)
+        if (valid[i]) {
+            if (kPvHeadsM) pvM16<D>(vslot[i], vrow[i], phi[i], plo[i], acc, lane);
+            else pvT16<D>(vslot[i], vrow[i], phi[i], plo[i], acc, two_rows, lane);
+        }
 }
 
 // ---------------------------------------------------------------- plan ---
@@ -488,7 +568,6 @@ struct Producer {
     bool dead = false;     // a ring wait ran out: issue nothing more
     int* trace_ctr = nullptr;
     uint64_t pol_keep = 0, pol_once = 0;
-    int rr = 0;            // consumer warp for the next data stage
 
     __device__ int* rec(int a, int pair) const { return ctrl + C_ARR + pair * p.pair_ints + a; }
 
@@ -508,7 +587,7 @@ struct Producer {
         return true;
     }
     __device__ void advance() {
-        if (++stage == Cfg<D>::kStages) {
+        if (++stage == p.stages) {
             stage = 0;
             ++round;
         }
@@ -545,7 +624,7 @@ struct Producer {
     // Waits until every stage this warp issued has landed (bounded), so no
     // copy is in flight when the block exits, whatever the consumers did.
     __device__ void drain() {
-        constexpr int NS = Cfg<D>::kStages;
+        const int NS = p.stages;
         const int issued = round * NS + stage;
         if (lane == 0)
             for (int i = 0; i < NS && i < issued; ++i) {
@@ -559,7 +638,7 @@ struct Producer {
     // at global row y0 of map m, into dst[0..nslot), then writes `npad` slots
     // of -inf.  Split into sub-items of at most `per_rows` rows.
     __device__ void score_run(int pair, int level, const CUtensorMap* m, int y0, int nslot,
-                              int npad, int dst, int ntok, int per_rows) {
+                              int npad, int dst, int ntok, int per_rows, int lrow0) {
         const int per = max(1, per_rows / ntok);  // slots per sub-item
         int s0 = 0;
         do {
@@ -583,12 +662,9 @@ struct Producer {
                 const int nv = min(2 * kBoxRows, rows - off);
                 const int nbox = (nv + kBoxRows - 1) / kBoxRows;
                 const bool first = off == 0;
-                const int own = rr;
-                rr = (rr + 1) % kConsumerWarps;
                 if (lane == 0) {
                     StageMeta mt = {};
                     mt.kind = K_SCORE;
-                    mt.owner = own;
                     mt.pair = pair;
                     mt.nvalid = nv;
                     mt.flags = (first ? (F_FIRST | F_QLOAD) : 0) |
@@ -599,11 +675,12 @@ struct Producer {
                     mt.a3 = dst + s0;
                     mt.a4 = ntok;
                     mt.a5 = level;
+                    mt.lrow = lrow0 + s0 * ntok + off;
                     meta[s] = mt;
                     const uint32_t bytes = nbox * Cfg<D>::kBoxBytes + (first ? p.G * D * 2 : 0);
                     mbar_arrive_expect_tx(&full[s], bytes);
 #ifdef SSA_TRACE
-                    trace_event(p, trace_ctr, 14, 1, round * Cfg<D>::kStages + s);
+                    trace_event(p, trace_ctr, 14, 1, round * p.stages + s);
 #endif
                     if (first) load_q(s, pair);
                     for (int bx = 0; bx < nbox; ++bx)
@@ -679,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const SmemLayout L = smem_layout<D>(p);
-    constexpr int NS = Cfg<D>::kStages;
+    const int NS = p.stages;
     uint8_t* ring = smem + L.ring;
     uint8_t* qbuf = smem + L.qbuf;
     StageMeta* meta = reinterpret_cast<StageMeta*>(smem + L.meta);
@@ -691,6 +768,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     int* psv = nbv + p.B;
     uint32_t* bits = reinterpret_cast<uint32_t*>(smem + L.bits);
     uint8_t* uni = smem + L.uni;
+    float* logits = reinterpret_cast<float*>(smem + L.logit);
     int* misc = reinterpret_cast<int*>(smem + L.misc);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -750,14 +828,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         pr.pol_once = l2_policy_evict_first();
         pr.trace_ctr = &misc[15];
         pr.pol_keep = so ? pr.pol_once : l2_policy_evict_last();
-        int sel_lo, sel_hi, cmb_lo, cmb_hi;
+        int sel_lo, sel_hi;
         owned_pairs(cta, N, P, sel_lo, sel_hi);
-        owned_pairs(N - 1 - cta, N, P, cmb_lo, cmb_hi);
 
         // -------- this block's share of a scoring list (first level or candidates)
         auto score_list = [&](int Ls) {
             int lo, hi;
             pv.share(Ls, cta, lo, hi);
+            int seg_base = 0;  // rows of this share scored so far (kept-logit rows)
             for (int x = lo; x < hi;) {
                 int pair, first, count;
                 pv.locate(Ls, x, pair, first, count);
@@ -769,10 +847,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                     const int nv = max(0, min(i1, z.M) - i0);
                     const int npad = (i1 - i0) - nv;
                     pr.score_run(pair, 0, &tm_kgist, (pair * p.M_max + i0) * p.g, nv, npad,
-                                 pair * p.M_max + i0, p.g, score_rows);
+                                 pair * p.M_max + i0, p.g, score_rows, seg_base);
+                    seg_base += nv * p.g;
                 } else if (Ls == L_SCORE) {
                     pr.score_run(pair, 0, &tm_kmeta, (pair * p.S_max + i0) * p.gm, i1 - i0, 0,
-                                 pair * p.S_max + i0, p.gm, score_rows);
+                                 pair * p.S_max + i0, p.gm, score_rows, 0);
                 } else {
                     // candidates: runs of consecutive chunks (J per kept
                     // superchunk, in superchunk order, then the remainder),
@@ -791,7 +870,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                             run = i1 - c;
                         }
                         pr.score_run(pair, 1, &tm_kgist, (pair * p.M_max + chunk0) * p.g, run, 0,
-                                     pair * p.Mc_max + c, p.g, score_rows);
+                                     pair * p.Mc_max + c, p.g, score_rows, 0);
                         c += run;
                     }
                 }
@@ -831,13 +910,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                 auto emit = [&](bool last) {
                     int s;
                     if (!pr.acquire(s)) return;
-                    const int own = pr.rr;
-                    pr.rr = (pr.rr + 1) % kConsumerWarps;
                     if (lane == 0) {
                         StageMeta mt = {};
                         mt.kind = K_ATTN;
-                        mt.owner = own;
-                        mt.pair = pair;
+                            mt.pair = pair;
                         mt.nvalid = pend_nv;
                         mt.flags = (emitted ? 0 : (F_FIRST | F_QLOAD)) | (last ? F_LAST : 0);
                         mt.a0 = pend_r0;
@@ -923,48 +999,45 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         };
 
-        // -------- L2 prefetch of the tiles of this block's share of list La
-        // whose address needs no selection (single-level gist tiles, meta
-        // tiles, the raw tail): issued while the selection is computed, so
-        // the memory system stays busy through that wait
-        auto prefetch_share = [&](int La) {
-            const int tpc = (p.C + kBoxRows - 1) / kBoxRows;
-            const int tsc = (p.J * p.g + kBoxRows - 1) / kBoxRows;
+        // -------- logits mode: the values of this block's scored gist rows, in
+        // the same order as its score share (issued before the selection)
+        auto gistv_list = [&]() {
             int lo, hi;
-            pv.share(La, cta, lo, hi);
+            pv.share(L_SCORE, cta, lo, hi);
+            int seg_base = 0;
             for (int x = lo; x < hi;) {
                 int pair, first, count;
-                pv.locate(La, x, pair, first, count);
-                const int u0 = x - first, u1 = min(hi, first + count) - first;
-                const PairSizes z = pair_sizes(p, nbv[pair / p.Hkv]);
-                for (int u = u0 + lane; u < u1; u += 32) {
-                    const CUtensorMap *km, *vm;
-                    int y;
-                    if (La == L_META) {
-                        km = &tm_kmeta;
-                        vm = &tm_vmeta;
-                        y = pair * p.S_max * p.gm + u * kBoxRows;
-                    } else if (La == L_GIST) {
-                        if (p.h2 && u < z.ks * tsc) continue;
-                        km = &tm_kgist;
-                        vm = &tm_vgist;
-                        y = pair * p.M_max * p.g +
-                            (p.h2 ? z.S * p.J * p.g + (u - z.ks * tsc) * kBoxRows : u * kBoxRows);
-                    } else {
-                        if (u < z.kc * tpc) continue;
-                        km = &tm_kraw;
-                        vm = &tm_vraw;
-                        y = pair * p.n_max + z.M * p.C + (u - z.kc * tpc) * kBoxRows;
+                pv.locate(L_SCORE, x, pair, first, count);
+                const int i0 = x - first, i1 = min(hi, first + count) - first;
+                const int rows = (i1 - i0) * p.g, row0 = i0 * p.g;
+                if (lane == 0) SSA_TR(TR_SEG, L_GIST, pair);
+                for (int off = 0; off < rows; off += 2 * kBoxRows) {
+                    int s;
+                    if (!pr.acquire(s)) return;
+                    const int nv = min(2 * kBoxRows, rows - off);
+                    if (lane == 0) {
+                        StageMeta mt = {};
+                        mt.kind = K_GISTV;
+                        mt.pair = pair;
+                        mt.nvalid = nv;
+                        mt.flags = (off == 0 ? F_FIRST : 0) | (off + 2 * kBoxRows >= rows ? F_LAST : 0);
+                        mt.a0 = row0 + off;
+                        mt.a2 = p.g;
+                        mt.a3 = 1;
+                            mt.lrow = seg_base + off;
+                        meta[s] = mt;
+                        const int nbox = (nv + kBoxRows - 1) / kBoxRows;
+                        mbar_arrive_expect_tx(&full[s], nbox * Cfg<D>::kBoxBytes);
+                        for (int bx = 0; bx < nbox; ++bx)
+                            pr.box(s, bx, &tm_vgist, pair * p.M_max * p.g + row0 + off + bx * kBoxRows,
+                                   pr.pol_once);
                     }
-#pragma unroll
-                    for (int sub = 0; sub < D / 64; ++sub) {
-                        tma_prefetch_2d(km, sub * 64, y);
-                        tma_prefetch_2d(vm, sub * 64, y);
-                    }
+                    __syncwarp();
+                    pr.advance();
                 }
-                x = first + u1;
+                seg_base += rows;
+                x = first + i1;
             }
-            __syncwarp();
         };
 
         auto selects = [&](int what) {
@@ -978,37 +1051,81 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         };
 
+        // The phases of this mode, run by one loop so that each phase's code
+        // exists once in the kernel (instruction cache).
+        enum : int { OP_SCORE = 1, OP_SELECT, OP_GISTV, OP_ATTN };
+        int prog[8], np = 0;
         if (so) {
-            score_list(L_SCORE);
+            prog[np++] = OP_SCORE << 8 | L_SCORE;
         } else if (!p.h2) {
             if (p.mode == kModeAttnOnly) {
-                selects(SEL_VALIDATE);
+                prog[np++] = OP_SELECT << 8 | SEL_VALIDATE;
             } else {
-                score_list(L_SCORE);
-                prefetch_share(L_GIST);
-                prefetch_share(L_RAW);
-                selects(SEL_CHUNKS);
+                prog[np++] = OP_SCORE << 8 | L_SCORE;
+                prog[np++] = OP_SELECT << 8 | SEL_CHUNKS;
             }
-            attn_list(L_GIST);
-            attn_list(L_RAW);
+            prog[np++] = p.logits ? OP_GISTV << 8 : (OP_ATTN << 8 | L_GIST);
+            prog[np++] = OP_ATTN << 8 | L_RAW;
         } else {
-            score_list(L_SCORE);
-            prefetch_share(L_META);
-            selects(SEL_SUPER);
-            attn_list(L_META);
-            score_list(L_CAND);
-            selects(SEL_CAND);
-            attn_list(L_GIST);
-            attn_list(L_RAW);
+            prog[np++] = OP_SCORE << 8 | L_SCORE;
+            prog[np++] = OP_SELECT << 8 | SEL_SUPER;
+            prog[np++] = OP_ATTN << 8 | L_META;
+            prog[np++] = OP_SCORE << 8 | L_CAND;
+            prog[np++] = OP_SELECT << 8 | SEL_CAND;
+            prog[np++] = OP_ATTN << 8 | L_GIST;
+            prog[np++] = OP_ATTN << 8 | L_RAW;
         }
-        if (!so)
-            for (int pair = cmb_lo; pair < cmb_hi; ++pair) {
-                StageMeta mt = {};
-                mt.kind = K_COMBINE;
-                mt.pair = pair;
-                mt.flags = F_FIRST | F_LAST;
-                pr.push_plain(mt);
+#pragma unroll 1
+        for (int i = 0; i < np; ++i) {
+            const int op = prog[i] >> 8, arg = prog[i] & 255;
+            if (op == OP_SCORE) score_list(arg);
+            else if (op == OP_SELECT) selects(arg);
+            else if (op == OP_GISTV) gistv_list();
+            else attn_list(arg);
+        }
+        if (!so) {
+            // The combination of pair p runs on the block that holds p's last
+            // attention element (its last raw tile; else its last gist / meta
+            // tile), right after that block's own share, so it waits only for
+            // the other segments of p, which finish at about the same time.
+            // Pairs without any attention element go to block p mod N.
+            const int Lg = p.logits ? L_SCORE : L_GIST;
+            const int order[3] = {L_RAW, Lg, L_META};
+            auto cnt = [&](int L, int pair) { return list_count(p, L, nbv[pair / p.Hkv]); };
+            for (int oi = 0; oi < 3; ++oi) {
+                const int La = order[oi];
+                if (La == L_META && !p.h2) continue;
+                int lo, hi;
+                pv.share(La, cta, lo, hi);
+                for (int x = lo; x < hi;) {
+                    int pair, first, count;
+                    pv.locate(La, x, pair, first, count);
+                    const int i1 = min(hi, first + count) - first;
+                    bool mine = i1 == count;  // this block holds the pair's last element
+                    for (int oj = 0; oj < oi && mine; ++oj)
+                        if (!(order[oj] == L_META && !p.h2)) mine = cnt(order[oj], pair) == 0;
+                    if (mine) {
+                        StageMeta mt = {};
+                        mt.kind = K_COMBINE;
+                        mt.pair = pair;
+                        mt.flags = F_FIRST | F_LAST;
+                        pr.push_plain(mt);
+                    }
+                    x = first + i1;
+                }
             }
+            for (int pair = cta; pair < P; pair += N) {
+                bool none = cnt(L_RAW, pair) == 0 && cnt(Lg, pair) == 0;
+                if (p.h2) none = none && cnt(L_META, pair) == 0;
+                if (none) {
+                    StageMeta mt = {};
+                    mt.kind = K_COMBINE;
+                    mt.pair = pair;
+                    mt.flags = F_FIRST | F_LAST;
+                    pr.push_plain(mt);
+                }
+            }
+        }
         StageMeta end = {};
         end.kind = K_END;
         pr.push_plain(end);
@@ -1029,58 +1146,111 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int mask_words = mask_words_for(p);
 
     uint32_t qa[D / 16][4];
-    float acc[D / 8][4];
+    float acc[2][D / 16][4];  // O^T: [head n tile][dim m tile][fragment]
     float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk)
 #pragma unroll
         for (int c = 0; c < 4; ++c) qa[kk][c] = 0u;
+    auto zero_acc = [&]() {
 #pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt)
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
+            for (int mm = 0; mm < D / 16; ++mm)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[nt][mm][c] = 0.f;
+    };
+    zero_acc();
 
-    // Loads the published selection (chunks or superchunks) of `pair` into
-    // the shared bitmap.  One round of loads reads the count and every entry
-    // (self-validating: 0 = not written yet); rounds repeat until complete.
-    auto load_bitmap = [&](int pair, int level) {
-        for (int w = tid; w < mask_words; w += kConsumers) bits[w] = 0u;
-        const int* cnt_word = rec(level == MASK_SUPER ? A_SCOUNT : A_COUNT, pair);
-        const int* ent = rec(level == MASK_SUPER ? A_ENTRIES + p.topk : A_ENTRIES, pair);
+    // Loads the published selections (chunks or superchunks) of pairs[0..n)
+    // into bitmap slots 0..n-1.  One round of loads reads the counts and every
+    // entry (self-validating: 0 = not written yet); rounds repeat until all
+    // are complete.  A rejected caller selection excludes every row.
+    const int mwp = (mask_words + 3) / 4 * 4;
+    auto load_bitmaps = [&](const int (&pairs)[kMaxBitmaps], int n, int level) {
+        for (int w = tid; w < n * mwp; w += kConsumers) bits[w] = 0u;
+        const int a_cnt = level == MASK_SUPER ? A_SCOUNT : A_COUNT;
+        const int a_ent = level == MASK_SUPER ? A_ENTRIES + p.topk : A_ENTRIES;
         const int cap = level == MASK_SUPER ? p.topk_super : p.topk;
         constexpr int kPer = (kMaxTopkEntries + kConsumers - 1) / kConsumers;
-        int e[kPer];
-        int cw = 0;
+        const int per = (cap + kConsumers - 1) / kConsumers;  // entries per thread and pair
+        int cw[kMaxBitmaps], e[kMaxBitmaps][kPer];
         const long long c0 = clock64(), lim = wait_cycles(p.wait_limit);
         bool missing;
         for (;;) {
-            cw = ld_relaxed(cnt_word);
 #pragma unroll
-            for (int j = 0; j < kPer; ++j) {
-                const int c = tid + kConsumers * j;
-                e[j] = c < cap ? ld_relaxed(ent + c) : 1;
+            for (int i = 0; i < kMaxBitmaps; ++i) {
+                cw[i] = i < n ? ld_relaxed(rec(a_cnt, pairs[i])) : 1;
+#pragma unroll
+                for (int j = 0; j < kPer; ++j) {
+                    const int c = tid + kConsumers * j;
+                    e[i][j] = (i < n && j < per && c < cap) ? ld_relaxed(rec(a_ent, pairs[i]) + c) : 1;
+                }
             }
-            const int k = (cw == 0 || (cw & kBadBit)) ? 0 : min((cw & (kBadBit - 1)) - 1, cap);
-            missing = cw == 0;
+            missing = false;
 #pragma unroll
-            for (int j = 0; j < kPer; ++j) missing |= (tid + kConsumers * j < k) && e[j] == 0;
+            for (int i = 0; i < kMaxBitmaps; ++i) {
+                const int k = (cw[i] == 0 || (cw[i] & kBadBit)) ? 0
+                                                               : min((cw[i] & (kBadBit - 1)) - 1, cap);
+                missing |= cw[i] == 0;
+#pragma unroll
+                for (int j = 0; j < kPer; ++j) missing |= (tid + kConsumers * j < k) && e[i][j] == 0;
+            }
             // every thread takes the same branch: the vote decides (the first
-            // vote also orders the clearing of the bitmap before the updates)
+            // vote also orders the clearing of the bitmaps before the updates)
             const bool expired = clock64() - c0 > lim;
             if (!csync.or_(missing && !expired)) break;
             __nanosleep(64);
         }
         if (missing) report_status(kStatusTimeout);
-        const int k = (cw == 0 || (cw & kBadBit)) ? 0 : min((cw & (kBadBit - 1)) - 1, cap);
 #pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            const int c = tid + kConsumers * j;
-            if (c < k && e[j] != 0) atomicOr(&bits[(e[j] - 1) >> 5], 1u << ((e[j] - 1) & 31));
+        for (int i = 0; i < kMaxBitmaps; ++i) {
+            if (i >= n) break;
+            uint32_t* bm = bits + i * mwp;
+            const int k = (cw[i] == 0 || (cw[i] & kBadBit)) ? 0 : min((cw[i] & (kBadBit - 1)) - 1, cap);
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int c = tid + kConsumers * j;
+                if (c < k && e[i][j] != 0)
+                    atomicOr(&bm[(e[i][j] - 1) >> 5], 1u << ((e[i][j] - 1) & 31));
+            }
+            if (cw[i] & kBadBit)
+                for (int w = tid; w < mask_words; w += kConsumers) bm[w] = ~0u;
         }
-        // a rejected caller selection excludes every summary row of the pair
-        if (cw & kBadBit)
-            for (int w = tid; w < mask_words; w += kConsumers) bits[w] = ~0u;
         csync();
+    };
+    // bitmaps loaded so far: their pairs and level
+    int bm_pair[kMaxBitmaps];
+    int bm_n = 0, bm_level = MASK_NONE;
+    uint32_t* cur_bits = bits;
+    // Makes cur_bits the bitmap of (pair, level): from the loaded ones, else
+    // loads the pairs of this block's share of the masked list, from `pair`
+    // on (several in one round when the selections are small).
+    auto select_bitmap = [&](int pair, int level) {
+        int slot = -1;
+        if (bm_level == level)
+            for (int i = 0; i < bm_n; ++i)
+                if (bm_pair[i] == pair) slot = i;
+        if (slot < 0) {
+            const int Lm = level == MASK_SUPER ? L_META : (p.logits ? L_SCORE : L_GIST);
+            const int cap = level == MASK_SUPER ? p.topk_super : p.topk;
+            const int nmax = cap <= kConsumers ? kMaxBitmaps : 1;
+            (void)nmax;
+            int lo, hi;
+            pv.share(Lm, cta, lo, hi);
+            bm_n = 0;
+            bm_pair[bm_n++] = pair;
+            for (int x = lo; x < hi && bm_n < nmax;) {
+                int pr2, first, count;
+                pv.locate(Lm, x, pr2, first, count);
+                if (pr2 > pair) bm_pair[bm_n++] = pr2;
+                x = first + count;
+            }
+            load_bitmaps(bm_pair, bm_n, level);
+            bm_level = level;
+            slot = 0;
+        }
+        cur_bits = bits + slot * mwp;
     };
 
     int stage = 0, round = 0;
@@ -1092,7 +1262,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!mbar_wait(&full[stage], (uint32_t)(round & 1), long_limit)) break;
         const StageMeta mt = meta[stage];
 #ifdef SSA_TRACE
-        const int tr_warp = (mt.kind == K_ATTN || mt.kind == K_SCORE) ? mt.owner : 0;
+        const int tr_warp = 0;
         if (lane == 0 && warp == tr_warp) trace_event(p, &misc[15], 15, mt.kind, round * NS + stage);
 #endif
         if (mt.kind == K_END) break;
@@ -1114,39 +1284,82 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         const int pair = mt.pair;
 
-        if (mt.kind == K_ATTN) {
+        if (mt.kind == K_ATTN || mt.kind == K_GISTV) {
             if (mt.flags & F_FIRST) {
                 if (tid == 0) SSA_TR(TR_C_SEG0, mt.a3, pair);
                 mrow[0] = mrow[1] = -INFINITY;
                 lrow[0] = lrow[1] = 0.f;
-#pragma unroll
-                for (int nt = 0; nt < D / 8; ++nt)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
-                seg_mask = mt.a1;
-                if (seg_mask != MASK_NONE) load_bitmap(pair, seg_mask);
+                zero_acc();
+                seg_mask = mt.kind == K_GISTV ? MASK_CHUNK : mt.a1;
+                if (seg_mask != MASK_NONE) select_bitmap(pair, seg_mask);
             }
-            if (warp == mt.owner && mt.nvalid > 0) {
-                // ---- this warp takes the whole 64-row tile: excluded rows (past
-                // the tile's valid rows, or in a selected chunk / superchunk),
-                // lane l tests rows l and l + 32
-                uint32_t ex_lo, ex_hi;
+            if (mt.kind == K_GISTV) {
+                // ---- values of up to 128 scored gist rows, logits kept in shared
+                // memory; warp w takes rows 16w.. (slot A) and 64 + 16w.. (slot B);
+                // lane l tests row 16w + l (l < 16) or 64 + 16w + l - 16
+                const int rb[2] = {16 * warp, 64 + 16 * warp};
+                bool e;
                 {
-                    bool e[2];
-#pragma unroll
-                    for (int hlf = 0; hlf < 2; ++hlf) {
-                        const int lr = lane + 32 * hlf;
-                        e[hlf] = lr >= mt.nvalid;
-                        if (!e[hlf] && seg_mask != MASK_NONE) {
-                            const int sid = (mt.a0 + lr) / mt.a2;
-                            e[hlf] = (bits[sid >> 5] >> (sid & 31)) & 1u;
-                        }
+                    const int lr = rb[lane >> 4] + (lane & 15);
+                    e = lr >= mt.nvalid;
+                    if (!e) {
+                        const int sid = (mt.a0 + lr) / mt.a2;
+                        e = (cur_bits[sid >> 5] >> (sid & 31)) & 1u;
                     }
-                    ex_lo = __ballot_sync(0xffffffffu, e[0]);
-                    ex_hi = __ballot_sync(0xffffffffu, e[1]);
                 }
-                attn_tile<D>(slotA, slotB, mt.nvalid, ex_lo, ex_hi, qa, mrow, lrow, acc, two_rows,
-                             scale_log2, lane);
+                const uint32_t ex = __ballot_sync(0xffffffffu, e);
+                float sc[2][2][4];
+                const float* lg = logits + mt.lrow;
+                const int ls = p.logit_stride;
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const int t = rb[i] + nt * 8 + 2 * tig;
+                        const float2 a = g8 < p.G ? *reinterpret_cast<const float2*>(lg + g8 * ls + t)
+                                                  : make_float2(0.f, 0.f);
+                        const float2 b2 = g8 + 8 < p.G
+                                              ? *reinterpret_cast<const float2*>(lg + (g8 + 8) * ls + t)
+                                              : make_float2(0.f, 0.f);
+                        const int tb = 16 * i + nt * 8 + 2 * tig;
+                        const bool x0 = (ex >> tb) & 1u, x1 = (ex >> (tb + 1)) & 1u;
+                        sc[i][nt][0] = x0 ? -INFINITY : a.x;
+                        sc[i][nt][1] = x1 ? -INFINITY : a.y;
+                        sc[i][nt][2] = x0 ? -INFINITY : b2.x;
+                        sc[i][nt][3] = x1 ? -INFINITY : b2.y;
+                    }
+                const uint32_t vs[2] = {slotA, slotB};
+                const int vr[2] = {16 * warp, 16 * warp};
+                const bool ok[2] = {rb[0] < mt.nvalid, rb[1] < mt.nvalid};
+                if (ok[0]) softmax_pv<D, 2>(sc, vs, vr, ok, mrow, lrow, acc, two_rows, lane);
+            } else if (16 * warp < mt.nvalid) {
+                // ---- 16 rows of a 64-row key / value tile per warp: excluded rows
+                // (past the tile's valid rows, or in a selected chunk / superchunk);
+                // lanes 0..15 test one row each
+                const int rbase = 16 * warp;
+                bool e = true;
+                if (lane < 16) {
+                    const int lr = rbase + lane;
+                    e = lr >= mt.nvalid;
+                    if (!e && seg_mask != MASK_NONE) {
+                        const int sid = (mt.a0 + lr) / mt.a2;
+                        e = (cur_bits[sid >> 5] >> (sid & 31)) & 1u;
+                    }
+                }
+                const uint32_t excl16 = __ballot_sync(0xffffffffu, e) & 0xffffu;
+                float sc[1][2][4];
+                qk16<D>(slotA, rbase, qa, sc[0], lane);
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int t = nt * 8 + 2 * tig + (c & 1);
+                        sc[0][nt][c] = ((excl16 >> t) & 1u) ? -INFINITY : sc[0][nt][c] * scale_log2;
+                    }
+                const uint32_t vs[1] = {slotB};
+                const int vr[1] = {rbase};
+                const bool ok[1] = {true};
+                softmax_pv<D, 1>(sc, vs, vr, ok, mrow, lrow, acc, two_rows, lane);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
@@ -1163,17 +1376,36 @@ __global__ void __launch_bounds__(kThreads, 2)
                     l += __shfl_xor_sync(0xffffffffu, l, 1);
                     l += __shfl_xor_sync(0xffffffffu, l, 2);
                     const int h = g8 + 8 * r;
-                    if (h < G) {
+                    if (h < G && tig == 0) {
                         float* mg = merge + ((size_t)warp * G + h) * (D + 2);
-                        if (tig == 0) {
-                            mg[0] = mrow[r];
-                            mg[1] = l;
-                        }
-#pragma unroll
-                        for (int nt = 0; nt < D / 8; ++nt)
-                            *reinterpret_cast<float2*>(mg + 2 + nt * 8 + 2 * tig) =
-                                make_float2(acc[nt][2 * r], acc[nt][2 * r + 1]);
+                        mg[0] = mrow[r];
+                        mg[1] = l;
                     }
+                }
+                if (kPvHeadsM) {
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const int h = g8 + 8 * r;
+                        if (h < G) {
+                            float* mg = merge + ((size_t)warp * G + h) * (D + 2);
+#pragma unroll
+                            for (int x = 0; x < D / 8; ++x)
+                                *reinterpret_cast<float2*>(mg + 2 + x * 8 + 2 * tig) =
+                                    make_float2(acc8<D>(acc, x)[2 * r], acc8<D>(acc, x)[2 * r + 1]);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int mm = 0; mm < D / 16; ++mm)
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const int h = 8 * nt + 2 * tig + (c & 1);
+                                const int dim = 16 * mm + g8 + 8 * (c >> 1);
+                                if (h < G)
+                                    merge[((size_t)warp * G + h) * (D + 2) + 2 + dim] = acc[nt][mm][c];
+                            }
                 }
                 csync();
                 for (int h = warp; h < G; h += kConsumerWarps) {
@@ -1209,12 +1441,15 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (tid == 0) SSA_TR(TR_C_SEG1, mt.a3, pair);
             }
         } else if (mt.kind == K_SCORE) {
-            if (warp == mt.owner) {
-                // ---- this warp scores all rows of the stage (two 64-row boxes)
+            {
+                // ---- warp w scores rows 16w.. of box 0 (slot A) and of box 1 (slot B)
+                float* lg = p.logits && mt.a5 == 0 ? logits + mt.lrow : nullptr;
                 if (two_rows)
-                    score_tile<D, 2>(slotA, slotB, mt.nvalid, p.G, qa, scale, rowmax + mt.a0, lane);
+                    score_rows2<D, 2>(slotA, slotB, warp, mt.nvalid, p.G, qa, scale, rowmax + mt.a0,
+                                      lg, p.logit_stride, scale_log2, lane);
                 else
-                    score_tile<D, 1>(slotA, slotB, mt.nvalid, p.G, qa, scale, rowmax + mt.a0, lane);
+                    score_rows2<D, 1>(slotA, slotB, warp, mt.nvalid, p.G, qa, scale, rowmax + mt.a0,
+                                      lg, p.logit_stride, scale_log2, lane);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
@@ -1349,7 +1584,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int b = pair / p.Hkv, j = pair % p.Hkv;
             int c0[3], nseg[3];
             pv.pair_blocks(L_META, pair, c0[0], nseg[0]);
-            pv.pair_blocks(L_GIST, pair, c0[1], nseg[1]);
+            pv.pair_blocks(p.logits ? L_SCORE : L_GIST, pair, c0[1], nseg[1]);
             pv.pair_blocks(L_RAW, pair, c0[2], nseg[2]);
             const int NP = nseg[0] + nseg[1] + nseg[2];
             if (tid == 0) {

@@ -32,6 +32,12 @@ struct Plan {
     int grid_cap = 0;
     int score_rows = 1024;
     int pair_ints = 0;
+    // ring stages of this launch; logits = 1: the scoring phase keeps the
+    // per-row logits of its gist rows in shared memory ([head][logit_stride])
+    // and the gist phase streams only the values of the same rows
+    int stages = 0;
+    int logits = 0;
+    int logit_stride = 0;
     int mask_words = 0, smask_words = 0;
 
     const void* q = nullptr;

@@ -91,7 +91,11 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int d) {
 }
 
 template <int D>
-static cudaError_t launch_fused_d(const Plan& p, cudaStream_t stream) {
+static cudaError_t launch_fused_d(const Plan& plan, cudaStream_t stream) {
+    Plan p = plan;
+    p.stages = fused::Cfg<D>::kStages;
+    p.logits = 0;
+    p.logit_stride = 0;
     CUtensorMap m[6];
     const uint64_t P = (uint64_t)p.n_pairs;
     bool ok = make_map(&m[2], p.k_gist, P * p.M_max * p.g, D);
@@ -125,6 +129,33 @@ static cudaError_t launch_fused_d(const Plan& p, cudaStream_t stream) {
                                                                   (size_t)L.total);
     if (e != cudaSuccess) return e;
     if (occ < 1) return cudaErrorInvalidConfiguration;
+    fused::SmemLayout Luse = L;
+    // Logits mode (single level, whole step, d = 64): one ring stage less for
+    // a shared-memory area that keeps the scored rows' logits, so the gist
+    // phase streams only values.  Taken when every block's score share fits
+    // and the blocks per SM stay the same.
+    if (D == 64 && !p.h2 && p.mode == kModeFull && fused::logit_rows_cap(p.G) > 0) {
+        Plan t = p;
+        t.logits = 1;
+        t.stages = fused::Cfg<D>::kStages - 1;
+        t.logit_stride = fused::logit_rows_cap(p.G) + 8;
+        const fused::SmemLayout Lt = fused::smem_layout<D>(t);
+        int occ_t = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_t, kern, fused::kThreads,
+                                                          (size_t)Lt.total);
+        if (e != cudaSuccess) return e;
+        long long grid_t = (long long)sm_count() * occ_t;
+        if (p.grid_cap > 0 && grid_t > p.grid_cap) grid_t = p.grid_cap;
+        if (grid_t > kFusedMaxGrid) grid_t = kFusedMaxGrid;
+        const long long chunks = (long long)p.n_pairs * p.M_max;
+        if (grid_t > chunks) grid_t = chunks;
+        const long long rows_max = grid_t > 0 ? (chunks + grid_t - 1) / grid_t * p.g : 0;
+        if (occ_t >= occ && grid_t > 0 && rows_max <= fused::logit_rows_cap(p.G)) {
+            p = t;
+            occ = occ_t;
+            Luse = Lt;
+        }
+    }
     // One block per co-resident slot: the static schedule waits across blocks,
     // so the launch is cooperative (all blocks resident at once).  Fewer
     // blocks when the call has little work (upper bound from n_max).
@@ -148,7 +179,7 @@ static cudaError_t launch_fused_d(const Plan& p, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(fused::kThreads);
-    cfg.dynamicSmemBytes = (size_t)L.total;
+    cfg.dynamicSmemBytes = (size_t)Luse.total;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;

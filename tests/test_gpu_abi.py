@@ -79,7 +79,9 @@ def test_bad_length_sets_status_and_zeroes(ssa, inp):
     assert ssa.ssa_get_device_status() == ssa.SSA_ERR_DEVICE_STATUS
     assert (out[1] == 0).all() and (sel[1] == -1).all()
     good, _ = run(ssa, inp)
-    assert torch.equal(out[0], good[0])
+    # the other sequence is unaffected; the split of the work over blocks
+    # depends on the whole batch, so only fp32 summation order may differ
+    assert (out[0] - good[0]).abs().max().item() <= 1e-5
     assert ssa.ssa_get_device_status() == 0
 
 
