@@ -61,9 +61,6 @@ constexpr int kBarConsumers = 1;      // named barrier id of the consumer warps
 constexpr int kMaxGrid = kFusedMaxGrid;
 constexpr int kMaxTopkEntries = 1024;  // largest topk / topk_super the library accepts
 constexpr int kLogitBytes = 16 * 1024; // shared memory for the kept logits (logits mode)
-// Selection bitmaps a block keeps.  One: loading the selections of several
-// pairs in one round makes the first segment wait for the latest of them.
-constexpr int kMaxBitmaps = 1;
 // P.V formulation: heads as the M rows of the MMA (false: heads as N, dims as M)
 #ifndef SSA_PV_HEADS_M
 #define SSA_PV_HEADS_M 1
@@ -155,8 +152,8 @@ __host__ __device__ inline SmemLayout smem_layout(const Plan& p) {
     L.plan = o;  // lengths [B], then per list prefixes [B + 1]
     o += (p.B + kNumLists * (p.B + 1)) * 4;
     o = (o + 15) / 16 * 16;
-    L.bits = o;  // selection bitmaps of the pairs of the block's masked segments
-    o += kMaxBitmaps * ((mask_words_for(p) + 3) / 4 * 4) * 4;
+    L.bits = o;  // selection bitmap of the current segment's pair
+    o += ((mask_words_for(p) + 3) / 4 * 4) * 4;
     L.uni = o;
     // the consumers use this area for one thing at a time
     int u = kRowmaxCap * 4;                                      // score rows
@@ -1162,95 +1159,49 @@ __global__ void __launch_bounds__(kThreads, 2)
     };
     zero_acc();
 
-    // Loads the published selections (chunks or superchunks) of pairs[0..n)
-    // into bitmap slots 0..n-1.  One round of loads reads the counts and every
-    // entry (self-validating: 0 = not written yet); rounds repeat until all
-    // are complete.  A rejected caller selection excludes every row.
-    const int mwp = (mask_words + 3) / 4 * 4;
-    auto load_bitmaps = [&](const int (&pairs)[kMaxBitmaps], int n, int level) {
-        for (int w = tid; w < n * mwp; w += kConsumers) bits[w] = 0u;
-        const int a_cnt = level == MASK_SUPER ? A_SCOUNT : A_COUNT;
-        const int a_ent = level == MASK_SUPER ? A_ENTRIES + p.topk : A_ENTRIES;
+    // Loads the published selection (chunks or superchunks) of `pair` into
+    // the shared bitmap.  One round of loads reads the count and every entry
+    // (self-validating: 0 = not written yet); rounds repeat until complete.
+    // A rejected caller selection excludes every row.  (Loading the
+    // selections of several pairs at once would make a segment wait for the
+    // latest of them.)
+    auto load_bitmap = [&](int pair, int level) {
+        for (int w = tid; w < mask_words; w += kConsumers) bits[w] = 0u;
+        const int* cnt_word = rec(level == MASK_SUPER ? A_SCOUNT : A_COUNT, pair);
+        const int* ent = rec(level == MASK_SUPER ? A_ENTRIES + p.topk : A_ENTRIES, pair);
         const int cap = level == MASK_SUPER ? p.topk_super : p.topk;
         constexpr int kPer = (kMaxTopkEntries + kConsumers - 1) / kConsumers;
-        const int per = (cap + kConsumers - 1) / kConsumers;  // entries per thread and pair
-        int cw[kMaxBitmaps], e[kMaxBitmaps][kPer];
+        int e[kPer];
+        int cw = 0;
         const long long c0 = clock64(), lim = wait_cycles(p.wait_limit);
         bool missing;
         for (;;) {
+            cw = ld_relaxed(cnt_word);
 #pragma unroll
-            for (int i = 0; i < kMaxBitmaps; ++i) {
-                cw[i] = i < n ? ld_relaxed(rec(a_cnt, pairs[i])) : 1;
-#pragma unroll
-                for (int j = 0; j < kPer; ++j) {
-                    const int c = tid + kConsumers * j;
-                    e[i][j] = (i < n && j < per && c < cap) ? ld_relaxed(rec(a_ent, pairs[i]) + c) : 1;
-                }
+            for (int j = 0; j < kPer; ++j) {
+                const int c = tid + kConsumers * j;
+                e[j] = c < cap ? ld_relaxed(ent + c) : 1;
             }
-            missing = false;
+            const int k = (cw == 0 || (cw & kBadBit)) ? 0 : min((cw & (kBadBit - 1)) - 1, cap);
+            missing = cw == 0;
 #pragma unroll
-            for (int i = 0; i < kMaxBitmaps; ++i) {
-                const int k = (cw[i] == 0 || (cw[i] & kBadBit)) ? 0
-                                                               : min((cw[i] & (kBadBit - 1)) - 1, cap);
-                missing |= cw[i] == 0;
-#pragma unroll
-                for (int j = 0; j < kPer; ++j) missing |= (tid + kConsumers * j < k) && e[i][j] == 0;
-            }
+            for (int j = 0; j < kPer; ++j) missing |= (tid + kConsumers * j < k) && e[j] == 0;
             // every thread takes the same branch: the vote decides (the first
-            // vote also orders the clearing of the bitmaps before the updates)
+            // vote also orders the clearing of the bitmap before the updates)
             const bool expired = clock64() - c0 > lim;
             if (!csync.or_(missing && !expired)) break;
             __nanosleep(64);
         }
         if (missing) report_status(kStatusTimeout);
+        const int k = (cw == 0 || (cw & kBadBit)) ? 0 : min((cw & (kBadBit - 1)) - 1, cap);
 #pragma unroll
-        for (int i = 0; i < kMaxBitmaps; ++i) {
-            if (i >= n) break;
-            uint32_t* bm = bits + i * mwp;
-            const int k = (cw[i] == 0 || (cw[i] & kBadBit)) ? 0 : min((cw[i] & (kBadBit - 1)) - 1, cap);
-#pragma unroll
-            for (int j = 0; j < kPer; ++j) {
-                const int c = tid + kConsumers * j;
-                if (c < k && e[i][j] != 0)
-                    atomicOr(&bm[(e[i][j] - 1) >> 5], 1u << ((e[i][j] - 1) & 31));
-            }
-            if (cw[i] & kBadBit)
-                for (int w = tid; w < mask_words; w += kConsumers) bm[w] = ~0u;
+        for (int j = 0; j < kPer; ++j) {
+            const int c = tid + kConsumers * j;
+            if (c < k && e[j] != 0) atomicOr(&bits[(e[j] - 1) >> 5], 1u << ((e[j] - 1) & 31));
         }
+        if (cw & kBadBit)
+            for (int w = tid; w < mask_words; w += kConsumers) bits[w] = ~0u;
         csync();
-    };
-    // bitmaps loaded so far: their pairs and level
-    int bm_pair[kMaxBitmaps];
-    int bm_n = 0, bm_level = MASK_NONE;
-    uint32_t* cur_bits = bits;
-    // Makes cur_bits the bitmap of (pair, level): from the loaded ones, else
-    // loads the pairs of this block's share of the masked list, from `pair`
-    // on (several in one round when the selections are small).
-    auto select_bitmap = [&](int pair, int level) {
-        int slot = -1;
-        if (bm_level == level)
-            for (int i = 0; i < bm_n; ++i)
-                if (bm_pair[i] == pair) slot = i;
-        if (slot < 0) {
-            const int Lm = level == MASK_SUPER ? L_META : (p.logits ? L_SCORE : L_GIST);
-            const int cap = level == MASK_SUPER ? p.topk_super : p.topk;
-            const int nmax = cap <= kConsumers ? kMaxBitmaps : 1;
-            (void)nmax;
-            int lo, hi;
-            pv.share(Lm, cta, lo, hi);
-            bm_n = 0;
-            bm_pair[bm_n++] = pair;
-            for (int x = lo; x < hi && bm_n < nmax;) {
-                int pr2, first, count;
-                pv.locate(Lm, x, pr2, first, count);
-                if (pr2 > pair) bm_pair[bm_n++] = pr2;
-                x = first + count;
-            }
-            load_bitmaps(bm_pair, bm_n, level);
-            bm_level = level;
-            slot = 0;
-        }
-        cur_bits = bits + slot * mwp;
     };
 
     int stage = 0, round = 0;
@@ -1291,7 +1242,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 lrow[0] = lrow[1] = 0.f;
                 zero_acc();
                 seg_mask = mt.kind == K_GISTV ? MASK_CHUNK : mt.a1;
-                if (seg_mask != MASK_NONE) select_bitmap(pair, seg_mask);
+                if (seg_mask != MASK_NONE) load_bitmap(pair, seg_mask);
             }
             if (mt.kind == K_GISTV) {
                 // ---- values of up to 128 scored gist rows, logits kept in shared
@@ -1300,11 +1251,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const int rb[2] = {16 * warp, 64 + 16 * warp};
                 bool e;
                 {
-                    const int lr = rb[lane >> 4] + (lane & 15);
+                    const int lr = (lane < 16 ? rb[0] : rb[1]) + (lane & 15);
                     e = lr >= mt.nvalid;
                     if (!e) {
                         const int sid = (mt.a0 + lr) / mt.a2;
-                        e = (cur_bits[sid >> 5] >> (sid & 31)) & 1u;
+                        e = (bits[sid >> 5] >> (sid & 31)) & 1u;
                     }
                 }
                 const uint32_t ex = __ballot_sync(0xffffffffu, e);
@@ -1343,7 +1294,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     e = lr >= mt.nvalid;
                     if (!e && seg_mask != MASK_NONE) {
                         const int sid = (mt.a0 + lr) / mt.a2;
-                        e = (cur_bits[sid >> 5] >> (sid & 31)) & 1u;
+                        e = (bits[sid >> 5] >> (sid & 31)) & 1u;
                     }
                 }
                 const uint32_t excl16 = __ballot_sync(0xffffffffu, e) & 0xffffu;
