@@ -1206,20 +1206,33 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     int stage = 0, round = 0;
     int seg_mask = MASK_NONE;
-    for (;;) {
-        // The producer's own waits are bounded and it always closes the ring
-        // with an END stage; this bound only ends the loop if it is gone, in
-        // which case no consumer warp receives another stage.
-        if (!mbar_wait(&full[stage], (uint32_t)(round & 1), long_limit)) break;
-        const StageMeta mt = meta[stage];
+    StageMeta mt;
+    const uint32_t ring_s = smem_u32(ring);
+    // Waits for the next stage and reads its description.  The producer's
+    // own waits are bounded and it always closes the ring with an END stage;
+    // this bound only fails if it is gone, and then no warp gets a stage.
+    auto wait_stage = [&]() -> bool {
+        if (!mbar_wait(&full[stage], (uint32_t)(round & 1), long_limit)) return false;
+        mt = meta[stage];
 #ifdef SSA_TRACE
-        const int tr_warp = 0;
-        if (lane == 0 && warp == tr_warp) trace_event(p, &misc[15], 15, mt.kind, round * NS + stage);
+        if (lane == 0 && warp == 0) trace_event(p, &misc[15], 15, mt.kind, round * NS + stage);
 #endif
-        if (mt.kind == K_END) break;
-        const uint32_t slotA = smem_u32(ring + (size_t)stage * Cfg<D>::kStageBytes);
-        const uint32_t slotB = slotA + Cfg<D>::kSlotBytes;
-        if (mt.flags & F_QLOAD) {
+        return true;
+    };
+    auto advance = [&]() {
+        if (++stage == NS) {
+            stage = 0;
+            ++round;
+        }
+    };
+    auto release = [&]() {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+#ifdef SSA_TRACE
+        if (lane == 0 && warp == 0) trace_event(p, &misc[15], 16, mt.kind, round * NS + stage);
+#endif
+    };
+    auto load_q = [&]() {
             const uint8_t* qs = qbuf + (size_t)stage * L.qbytes;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
@@ -1232,93 +1245,16 @@ __global__ void __launch_bounds__(kThreads, 2)
                         g8 + 8 < p.G ? *reinterpret_cast<const uint32_t*>(qs + ((g8 + 8) * D + col) * 2)
                                      : 0u;
                 }
-        }
-        const int pair = mt.pair;
-
-        if (mt.kind == K_ATTN || mt.kind == K_GISTV) {
-            if (mt.flags & F_FIRST) {
+    };
+    auto seg_start = [&](int pair) {
                 if (tid == 0) SSA_TR(TR_C_SEG0, mt.a3, pair);
                 mrow[0] = mrow[1] = -INFINITY;
                 lrow[0] = lrow[1] = 0.f;
                 zero_acc();
                 seg_mask = mt.kind == K_GISTV ? MASK_CHUNK : mt.a1;
                 if (seg_mask != MASK_NONE) load_bitmap(pair, seg_mask);
-            }
-            if (mt.kind == K_GISTV) {
-                // ---- values of up to 128 scored gist rows, logits kept in shared
-                // memory; warp w takes rows 16w.. (slot A) and 64 + 16w.. (slot B);
-                // lane l tests row 16w + l (l < 16) or 64 + 16w + l - 16
-                const int rb[2] = {16 * warp, 64 + 16 * warp};
-                bool e;
-                {
-                    const int lr = (lane < 16 ? rb[0] : rb[1]) + (lane & 15);
-                    e = lr >= mt.nvalid;
-                    if (!e) {
-                        const int sid = (mt.a0 + lr) / mt.a2;
-                        e = (bits[sid >> 5] >> (sid & 31)) & 1u;
-                    }
-                }
-                const uint32_t ex = __ballot_sync(0xffffffffu, e);
-                float sc[2][2][4];
-                const float* lg = logits + mt.lrow;
-                const int ls = p.logit_stride;
-#pragma unroll
-                for (int i = 0; i < 2; ++i)
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        const int t = rb[i] + nt * 8 + 2 * tig;
-                        const float2 a = g8 < p.G ? *reinterpret_cast<const float2*>(lg + g8 * ls + t)
-                                                  : make_float2(0.f, 0.f);
-                        const float2 b2 = g8 + 8 < p.G
-                                              ? *reinterpret_cast<const float2*>(lg + (g8 + 8) * ls + t)
-                                              : make_float2(0.f, 0.f);
-                        const int tb = 16 * i + nt * 8 + 2 * tig;
-                        const bool x0 = (ex >> tb) & 1u, x1 = (ex >> (tb + 1)) & 1u;
-                        sc[i][nt][0] = x0 ? -INFINITY : a.x;
-                        sc[i][nt][1] = x1 ? -INFINITY : a.y;
-                        sc[i][nt][2] = x0 ? -INFINITY : b2.x;
-                        sc[i][nt][3] = x1 ? -INFINITY : b2.y;
-                    }
-                const uint32_t vs[2] = {slotA, slotB};
-                const int vr[2] = {16 * warp, 16 * warp};
-                const bool ok[2] = {rb[0] < mt.nvalid, rb[1] < mt.nvalid};
-                if (ok[0]) softmax_pv<D, 2>(sc, vs, vr, ok, mrow, lrow, acc, two_rows, lane);
-            } else if (16 * warp < mt.nvalid) {
-                // ---- 16 rows of a 64-row key / value tile per warp: excluded rows
-                // (past the tile's valid rows, or in a selected chunk / superchunk);
-                // lanes 0..15 test one row each
-                const int rbase = 16 * warp;
-                bool e = true;
-                if (lane < 16) {
-                    const int lr = rbase + lane;
-                    e = lr >= mt.nvalid;
-                    if (!e && seg_mask != MASK_NONE) {
-                        const int sid = (mt.a0 + lr) / mt.a2;
-                        e = (bits[sid >> 5] >> (sid & 31)) & 1u;
-                    }
-                }
-                const uint32_t excl16 = __ballot_sync(0xffffffffu, e) & 0xffffu;
-                float sc[1][2][4];
-                qk16<D>(slotA, rbase, qa, sc[0], lane);
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int t = nt * 8 + 2 * tig + (c & 1);
-                        sc[0][nt][c] = ((excl16 >> t) & 1u) ? -INFINITY : sc[0][nt][c] * scale_log2;
-                    }
-                const uint32_t vs[1] = {slotB};
-                const int vr[1] = {rbase};
-                const bool ok[1] = {true};
-                softmax_pv<D, 1>(sc, vs, vr, ok, mrow, lrow, acc, two_rows, lane);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
-#ifdef SSA_TRACE
-            if (lane == 0 && warp == tr_warp) trace_event(p, &misc[15], 16, mt.kind, round * NS + stage);
-#endif
-
-            if (mt.flags & F_LAST) {
+    };
+    auto seg_end = [&](int pair) {
                 // ---- merge the 4 warps' states: one partial per head and segment
                 const int G = p.G;
 #pragma unroll
@@ -1390,8 +1326,151 @@ __global__ void __launch_bounds__(kThreads, 2)
                 csync();
                 if (tid == 0) red_release_add(rec(A_ATTN, pair), 1);
                 if (tid == 0) SSA_TR(TR_C_SEG1, mt.a3, pair);
-            }
-        } else if (mt.kind == K_SCORE) {
+    };
+
+    // Each kind of stage has its own loop over consecutive stages of that
+    // kind, so the code a data stage runs is one compact region.
+    bool alive = wait_stage();
+    while (alive && mt.kind != K_END) {
+        if (mt.kind == K_ATTN) {
+            // Two consecutive stages of one segment at a time: each warp then
+            // has two independent 16-row blocks (Q.K^T, one softmax update,
+            // P.V), which hides more of the tensor-core latency.
+            do {
+                const int pair = mt.pair;
+                if (mt.flags & F_QLOAD) load_q();
+                if (mt.flags & F_FIRST) seg_start(pair);
+                const int s0 = stage;
+                const StageMeta m0 = mt;
+                int s1 = -1;
+                StageMeta m1 = m0;
+                if (!(m0.flags & F_LAST)) {
+                    // the next stage belongs to the same segment
+                    advance();
+                    alive = wait_stage();
+                    if (alive) {
+                        s1 = stage;
+                        m1 = mt;
+                    }
+                }
+                const int rbase = 16 * warp;
+                const int nv1 = s1 >= 0 ? m1.nvalid : 0;
+                // excluded rows: lanes 0..15 test the first stage's rows,
+                // lanes 16..31 the second's
+                bool e;
+                {
+                    const StageMeta& mm = lane < 16 ? m0 : m1;
+                    const int nvx = lane < 16 ? m0.nvalid : nv1;
+                    const int lr = rbase + (lane & 15);
+                    e = lr >= nvx;
+                    if (!e && seg_mask != MASK_NONE) {
+                        const int sid = (mm.a0 + lr) / mm.a2;
+                        e = (bits[sid >> 5] >> (sid & 31)) & 1u;
+                    }
+                }
+                const uint32_t ex = __ballot_sync(0xffffffffu, e);
+                const uint32_t slotA0 = ring_s + s0 * Cfg<D>::kStageBytes;
+                const uint32_t slotA1 = s1 >= 0 ? ring_s + s1 * Cfg<D>::kStageBytes : slotA0;
+                const bool ok[2] = {rbase < m0.nvalid, rbase < nv1};
+                float sc[2][2][4];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    if (ok[i]) {
+                        qk16<D>(i ? slotA1 : slotA0, rbase, qa, sc[i], lane);
+                    } else {
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) sc[i][nt][c] = 0.f;
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int t = 16 * i + nt * 8 + 2 * tig + (c & 1);
+                            sc[i][nt][c] = ((ex >> t) & 1u) ? -INFINITY : sc[i][nt][c] * scale_log2;
+                        }
+                }
+                if (ok[0] || ok[1]) {
+                    const uint32_t vs[2] = {slotA0 + Cfg<D>::kSlotBytes, slotA1 + Cfg<D>::kSlotBytes};
+                    const int vr[2] = {rbase, rbase};
+                    softmax_pv<D, 2>(sc, vs, vr, ok, mrow, lrow, acc, two_rows, lane);
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&empty[s0]);
+                    if (s1 >= 0) mbar_arrive(&empty[s1]);
+                }
+#ifdef SSA_TRACE
+                if (lane == 0 && warp == 0) trace_event(p, &misc[15], 16, K_ATTN, round * NS + stage);
+#endif
+                if ((s1 >= 0 ? m1.flags : m0.flags) & F_LAST) seg_end(pair);
+                if (!alive) break;
+                advance();
+                alive = wait_stage();
+            } while (alive && mt.kind == K_ATTN);
+            continue;
+        }
+        if (mt.kind == K_GISTV) {
+            do {
+                const uint32_t slotA = ring_s + stage * Cfg<D>::kStageBytes;
+                const uint32_t slotB = slotA + Cfg<D>::kSlotBytes;
+                const int pair = mt.pair;
+                if (mt.flags & F_FIRST) seg_start(pair);
+                {
+                // ---- values of up to 128 scored gist rows, logits kept in shared
+                // memory; warp w takes rows 16w.. (slot A) and 64 + 16w.. (slot B);
+                // lane l tests row 16w + l (l < 16) or 64 + 16w + l - 16
+                const int rb[2] = {16 * warp, 64 + 16 * warp};
+                bool e;
+                {
+                    const int lr = (lane < 16 ? rb[0] : rb[1]) + (lane & 15);
+                    e = lr >= mt.nvalid;
+                    if (!e) {
+                        const int sid = (mt.a0 + lr) / mt.a2;
+                        e = (bits[sid >> 5] >> (sid & 31)) & 1u;
+                    }
+                }
+                const uint32_t ex = __ballot_sync(0xffffffffu, e);
+                float sc[2][2][4];
+                const float* lg = logits + mt.lrow;
+                const int ls = p.logit_stride;
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const int t = rb[i] + nt * 8 + 2 * tig;
+                        const float2 a = g8 < p.G ? *reinterpret_cast<const float2*>(lg + g8 * ls + t)
+                                                  : make_float2(0.f, 0.f);
+                        const float2 b2 = g8 + 8 < p.G
+                                              ? *reinterpret_cast<const float2*>(lg + (g8 + 8) * ls + t)
+                                              : make_float2(0.f, 0.f);
+                        const int tb = 16 * i + nt * 8 + 2 * tig;
+                        const bool x0 = (ex >> tb) & 1u, x1 = (ex >> (tb + 1)) & 1u;
+                        sc[i][nt][0] = x0 ? -INFINITY : a.x;
+                        sc[i][nt][1] = x1 ? -INFINITY : a.y;
+                        sc[i][nt][2] = x0 ? -INFINITY : b2.x;
+                        sc[i][nt][3] = x1 ? -INFINITY : b2.y;
+                    }
+                const uint32_t vs[2] = {slotA, slotB};
+                const int vr[2] = {16 * warp, 16 * warp};
+                const bool ok[2] = {rb[0] < mt.nvalid, rb[1] < mt.nvalid};
+                if (ok[0]) softmax_pv<D, 2>(sc, vs, vr, ok, mrow, lrow, acc, two_rows, lane);
+                }
+                release();
+                if (mt.flags & F_LAST) seg_end(pair);
+                advance();
+                alive = wait_stage();
+            } while (alive && mt.kind == K_GISTV);
+            continue;
+        }
+        if (mt.kind == K_SCORE) {
+            do {
+                const uint32_t slotA = ring_s + stage * Cfg<D>::kStageBytes;
+                const uint32_t slotB = slotA + Cfg<D>::kSlotBytes;
+                const int pair = mt.pair;
+                (void)pair;
+                if (mt.flags & F_QLOAD) load_q();
             {
                 // ---- warp w scores rows 16w.. of box 0 (slot A) and of box 1 (slot B)
                 float* lg = p.logits && mt.a5 == 0 ? logits + mt.lrow : nullptr;
@@ -1402,11 +1481,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     score_rows2<D, 1>(slotA, slotB, warp, mt.nvalid, p.G, qa, scale, rowmax + mt.a0,
                                       lg, p.logit_stride, scale_log2, lane);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
-#ifdef SSA_TRACE
-            if (lane == 0 && warp == tr_warp) trace_event(p, &misc[15], 16, mt.kind, round * NS + stage);
-#endif
+            release();
             if (mt.flags & F_LAST) {
                 csync();
                 // slot score = max over its summary rows (sec. 3.2)
@@ -1422,12 +1497,15 @@ __global__ void __launch_bounds__(kThreads, 2)
                 csync();
                 if (tid == 0) SSA_TR(TR_C_SCD, mt.a5, pair);
             }
-        } else if (mt.kind == K_SELECT) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
-#ifdef SSA_TRACE
-            if (lane == 0 && warp == tr_warp) trace_event(p, &misc[15], 16, mt.kind, round * NS + stage);
-#endif
+                advance();
+                alive = wait_stage();
+            } while (alive && mt.kind == K_SCORE);
+            continue;
+        }
+        {
+            const int pair = mt.pair;
+            if (mt.kind == K_SELECT) {
+            release();
             if (tid == 0) SSA_TR(TR_C_SEL0, mt.a0, pair);
             const PairSizes z = pair_sizes(p, nbv[pair / p.Hkv]);
             const int what = mt.a0;
@@ -1524,11 +1602,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             if (tid == 0) SSA_TR(TR_C_SEL1, what, pair);
         } else {  // K_COMBINE
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
-#ifdef SSA_TRACE
-            if (lane == 0 && warp == tr_warp) trace_event(p, &misc[15], 16, mt.kind, round * NS + stage);
-#endif
+            release();
             if (tid == 0) SSA_TR(TR_C_COMB0, 0, pair);
             // ---- combination of the pair's partial passes (sec. 3.6)
             const int G = p.G;
@@ -1637,10 +1711,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             if (tid == 0) SSA_TR(TR_C_COMB1, 0, pair);
         }
-        if (++stage == NS) {
-            stage = 0;
-            ++round;
         }
+        advance();
+        alive = wait_stage();
     }
     if (tid == 0) {
         SSA_TR(TR_KEND, 0, 0);
