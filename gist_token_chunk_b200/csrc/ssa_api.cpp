@@ -148,6 +148,8 @@ void plan_decompose(Plan& p) {
     p.smask_words = p.h2 ? (cdiv(p.S_max, 32) + 3) / 4 * 4 : 0;
 }
 
+bool seg_lists(const Plan& p) { return fused_path(p) && !p.h2 && p.topk <= kSegList; }
+
 int ctrl_words(const Plan& p) { return 64 + p.pair_ints * p.n_pairs; }  // see ssa_fused.cuh
 
 WsLayout plan_layout(const Plan& p) {
@@ -165,6 +167,7 @@ WsLayout plan_layout(const Plan& p) {
     L.cand_scores = take(p.h2 ? P * p.Mc_max * 4 : 0);
     L.chunk_mask = take(0);
     L.super_mask = take(0);
+    L.cands = take(seg_lists(p) ? (ssa::kFusedMaxGrid + P) * ssa::kSegList * 8 : 0);
     // one partial per (attention list, segment slot, query head)
     L.partials =
         take(fused_path(p) ? 3 * (ssa::kFusedMaxGrid + P) * p.G * (size_t)(p.d + 2) * 4 : 0);
@@ -184,6 +187,7 @@ void attach_ws(ssa::Plan& p, void* ws) {
     p.super_scores = p.h2 ? reinterpret_cast<float*>(base + L.super_scores) : nullptr;
     p.cand_scores = p.h2 ? reinterpret_cast<float*>(base + L.cand_scores) : nullptr;
     p.partials = reinterpret_cast<float*>(base + L.partials);
+    p.cands = ssa::seg_lists(p) ? reinterpret_cast<unsigned long long*>(base + L.cands) : nullptr;
 }
 
 // A fused call leaves its control words and its score areas zero (the

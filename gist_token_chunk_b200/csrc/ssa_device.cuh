@@ -315,6 +315,69 @@ struct NoProbe {
     __device__ void operator()(int) const {}
 };
 
+// ------------------------------------------------- warp-level ranking ---
+// Entries are 64-bit composites key << 32 | ~position (score_key order, ties
+// to the lower position: a larger composite ranks first).  A composite with a
+// zero key part (e.g. 1) is a placeholder below every real entry; 0 itself
+// means "not written yet" wherever entries are published.
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ unsigned long long cmax_u64(unsigned long long a, unsigned long long b) {
+    return a > b ? a : b;
+}
+__device__ __forceinline__ unsigned long long cmin_u64(unsigned long long a, unsigned long long b) {
+    return a < b ? a : b;
+}
+
+// Bitonic sort of the warp's 32 entries (one per lane) into descending order
+// (lane 0 holds the largest).
+__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long x, int lane) {
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const unsigned long long o = __shfl_xor_sync(0xffffffffu, x, j);
+            // runs with (lane & k) == 0 descend, the others ascend; the final
+            // run (k = 32) descends
+            const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+            x = keep_max ? cmax_u64(x, o) : cmin_u64(x, o);
+        }
+    return x;
+}
+
+// The 32 largest of two descending 32-entry lists a and b, descending: the
+// elementwise maximum of a and reversed b is a bitonic sequence holding them,
+// which one bitonic merge pass sorts.
+__device__ __forceinline__ unsigned long long warp_merge_desc(unsigned long long a,
+                                                              unsigned long long b, int lane) {
+    const unsigned long long br = __shfl_sync(0xffffffffu, b, 31 - lane);
+    unsigned long long x = cmax_u64(a, br);
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) {
+        const unsigned long long o = __shfl_xor_sync(0xffffffffu, x, j);
+        x = (lane & j) == 0 ? cmax_u64(x, o) : cmin_u64(x, o);
+    }
+    return x;
+}
+
+// Bitonic sort of the warp's 32 ints into ascending order.
+__device__ __forceinline__ int warp_sort_asc(int x, int lane) {
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const int o = __shfl_xor_sync(0xffffffffu, x, j);
+            const bool keep_min = ((lane & j) == 0) == ((lane & k) == 0);
+            x = keep_min ? min(x, o) : max(x, o);
+        }
+    return x;
+}
+
 constexpr int kTopkCandCap = 512;  // candidates the filtered selection ranks directly
 constexpr int kTopkRegPer = 16;    // values per thread the filtered selection holds
 

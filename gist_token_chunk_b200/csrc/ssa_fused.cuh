@@ -75,7 +75,8 @@ __host__ __device__ inline int logit_rows_cap(int G) {
 }
 
 enum : int { K_END = 0, K_SCORE = 1, K_ATTN = 2, K_SELECT = 3, K_COMBINE = 4, K_GISTV = 5 };
-enum : int { F_FIRST = 1, F_LAST = 2, F_QLOAD = 4 };
+// F_SEGBEG / F_SEGEND: a scoring sub-item is the first / last of its segment
+enum : int { F_FIRST = 1, F_LAST = 2, F_QLOAD = 4, F_SEGBEG = 8, F_SEGEND = 16 };
 enum : int { L_SCORE = 0, L_CAND = 1, L_META = 2, L_GIST = 3, L_RAW = 4, kNumLists = 5 };
 // what a K_SELECT stage does
 enum : int { SEL_CHUNKS = 0, SEL_SUPER = 1, SEL_CAND = 2, SEL_VALIDATE = 3 };
@@ -156,7 +157,7 @@ __host__ __device__ inline SmemLayout smem_layout(const Plan& p) {
     o += ((mask_words_for(p) + 3) / 4 * 4) * 4;
     L.uni = o;
     // the consumers use this area for one thing at a time
-    int u = kRowmaxCap * 4;                                      // score rows
+    int u = kRowmaxCap * 4 + kConsumerWarps * 32 * 8;           // score rows + lists
     const int tk = (int)sizeof(TopkScratch);                     // top-k
     u = u > tk ? u : tk;
     const int mg = kConsumerWarps * G * (D + 2) * 4;             // warp merge
@@ -642,11 +643,12 @@ struct Producer {
             const int ns = min(per, nslot - s0);
             const int np = (s0 + ns >= nslot) ? npad : 0;
             const int rows = ns * ntok;
+            const int segf = (s0 == 0 ? F_SEGBEG : 0) | (s0 + ns >= nslot ? F_SEGEND : 0);
             if (rows <= 0) {
                 StageMeta mt = {};
                 mt.kind = K_SCORE;
                 mt.pair = pair;
-                mt.flags = F_FIRST | F_LAST;
+                mt.flags = F_FIRST | F_LAST | segf;
                 mt.a2 = np;
                 mt.a3 = dst + s0;
                 mt.a4 = ntok;
@@ -665,7 +667,7 @@ struct Producer {
                     mt.pair = pair;
                     mt.nvalid = nv;
                     mt.flags = (first ? (F_FIRST | F_QLOAD) : 0) |
-                               (off + 2 * kBoxRows >= rows ? F_LAST : 0);
+                               (off + 2 * kBoxRows >= rows ? (F_LAST | segf) : 0);
                     mt.a0 = off;
                     mt.a1 = ns;
                     mt.a2 = np;
@@ -1143,6 +1145,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int mask_words = mask_words_for(p);
 
     uint32_t qa[D / 16][4];
+    // fast selection: this warp's 32 best chunks of the current scoring segment
+    unsigned long long segrun = 1ull;
+    unsigned long long* wlists = reinterpret_cast<unsigned long long*>(uni + kRowmaxCap * 4);
     float acc[2][D / 16][4];  // O^T: [head n tile][dim m tile][fragment]
     float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
 #pragma unroll
@@ -1484,15 +1489,45 @@ __global__ void __launch_bounds__(kThreads, 2)
             release();
             if (mt.flags & F_LAST) {
                 csync();
-                // slot score = max over its summary rows (sec. 3.2)
-                float* dst = mt.a5 == 1 ? p.cand_scores : p.h2 ? p.super_scores : p.scores;
-                for (int i = tid; i < mt.a1 + mt.a2; i += kConsumers) {
-                    float v = -INFINITY;
-                    if (i < mt.a1)
-                        for (int t = 0; t < mt.a4; ++t) v = fmaxf(v, rowmax[i * mt.a4 + t]);
-                    // for the selection, +0 is stored as -0 (same rank): an
-                    // all-zero word means "not written yet"
-                    dst[mt.a3 + i] = (so || v != 0.f) ? v : -0.f;
+                if (p.fastsel) {
+                    // slot score = max over its summary rows (sec. 3.2); the
+                    // segment keeps only its 32 best chunks (key, ~chunk):
+                    // no chunk outside them can be among the pair's top-k
+                    if (mt.flags & F_SEGBEG) segrun = 1ull;
+                    const uint32_t cbase = (uint32_t)(mt.a3 - pair * p.M_max);
+                    for (int i0 = 32 * warp; i0 < mt.a1; i0 += kConsumers) {
+                        const int i = i0 + lane;
+                        unsigned long long x = 1ull;
+                        if (i < mt.a1) {
+                            float v = -INFINITY;
+                            for (int t = 0; t < mt.a4; ++t) v = fmaxf(v, rowmax[i * mt.a4 + t]);
+                            x = ((unsigned long long)score_key(v) << 32) | (uint32_t)~(cbase + i);
+                        }
+                        segrun = warp_merge_desc(segrun, warp_sort_desc(x, lane), lane);
+                    }
+                    if (mt.flags & F_SEGEND) {
+                        wlists[warp * 32 + lane] = segrun;
+                        csync();
+                        if (warp == 0) {
+                            unsigned long long x = segrun;
+#pragma unroll 1
+                            for (int w = 1; w < kConsumerWarps; ++w)
+                                x = warp_merge_desc(x, wlists[w * 32 + lane], lane);
+                            // never 0 (a written entry); the selection polls for it
+                            p.cands[(size_t)(cta + pair) * kSegList + lane] = x;
+                        }
+                    }
+                } else {
+                    // slot score = max over its summary rows (sec. 3.2)
+                    float* dst = mt.a5 == 1 ? p.cand_scores : p.h2 ? p.super_scores : p.scores;
+                    for (int i = tid; i < mt.a1 + mt.a2; i += kConsumers) {
+                        float v = -INFINITY;
+                        if (i < mt.a1)
+                            for (int t = 0; t < mt.a4; ++t) v = fmaxf(v, rowmax[i * mt.a4 + t]);
+                        // for the selection, +0 is stored as -0 (same rank): an
+                        // all-zero word means "not written yet"
+                        dst[mt.a3 + i] = (so || v != 0.f) ? v : -0.f;
+                    }
                 }
                 csync();
                 if (tid == 0) SSA_TR(TR_C_SCD, mt.a5, pair);
@@ -1523,6 +1558,47 @@ __global__ void __launch_bounds__(kThreads, 2)
                                            p.sel_super + (size_t)pair * p.topk_super, tsc, csync,
                                            NoProbe(), rec(A_ENTRIES + p.topk, pair), p.wait_limit);
                     if (tid == 0) *rec(A_SCOUNT, pair) = z.ks + 1;
+                } else if (what == SEL_CHUNKS && p.fastsel) {
+                    // merge the 32-best lists of the pair's scoring segments;
+                    // the first k of the merged list are the pair's top-k
+                    vals = nullptr;
+                    nv = 0;
+                    int c0, nseg;
+                    pv.pair_blocks(L_SCORE, pair, c0, nseg);
+                    unsigned long long run = 1ull;
+                    const long long t0 = clock64(), lim = wait_cycles(p.wait_limit);
+                    bool late = false;
+                    for (int sg = warp; sg < nseg; sg += kConsumerWarps) {
+                        unsigned long long* src = p.cands + (size_t)(c0 + sg + pair) * kSegList;
+                        unsigned long long x = ld_relaxed_u64(src + lane);
+                        while (__any_sync(0xffffffffu, x == 0ull)) {
+                            if (__shfl_sync(0xffffffffu, (int)(clock64() - t0 > lim), 0)) {
+                                late = true;
+                                break;
+                            }
+                            __nanosleep(32);
+                            if (x == 0ull) x = ld_relaxed_u64(src + lane);
+                        }
+                        if (x == 0ull) x = 1ull;
+                        src[lane] = 0ull;  // cleared for the next call
+                        run = warp_merge_desc(run, x, lane);
+                    }
+                    if (late && lane == 0) report_status(kStatusTimeout);
+                    wlists[warp * 32 + lane] = run;
+                    csync();
+                    if (warp == 0) {
+#pragma unroll 1
+                        for (int w = 1; w < kConsumerWarps; ++w)
+                            run = warp_merge_desc(run, wlists[w * 32 + lane], lane);
+                        const int k = z.kc;
+                        int idx = lane < k ? (int)~(uint32_t)run : INT_MAX;
+                        idx = warp_sort_asc(idx, lane);
+                        int* out = p.sel_idx + (size_t)pair * p.topk;
+                        int* pub = rec(A_ENTRIES, pair);
+                        if (lane < p.topk) out[lane] = lane < k ? idx : -1;
+                        if (lane < k) pub[lane] = idx + 1;
+                        if (lane == 0) *rec(A_COUNT, pair) = k + 1;
+                    }
                 } else if (what == SEL_CHUNKS) {
                     vals = p.scores + (size_t)pair * p.M_max;
                     nv = z.M;

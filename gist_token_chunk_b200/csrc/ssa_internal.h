@@ -39,6 +39,10 @@ struct Plan {
     int logits = 0;
     int logit_stride = 0;
     int mask_words = 0, smask_words = 0;
+    // fused single-level decode with topk <= 32: every scoring segment
+    // publishes its 32 best chunks (descending composites key << 32 | ~chunk)
+    // and the top-k merges those lists instead of ranking every score
+    int fastsel = 0;
 
     const void* q = nullptr;
     const void* k_raw = nullptr;
@@ -56,6 +60,7 @@ struct Plan {
     uint32_t* chunk_mask = nullptr; // [P, mask_words]
     uint32_t* super_mask = nullptr; // [P, smask_words]
     float* partials = nullptr;      // [3, kFusedMaxGrid + P, G, d + 2]
+    unsigned long long* cands = nullptr;  // [kFusedMaxGrid + P, 32] segment lists
     float* out = nullptr;           // [B, Hq, d]
     int* ctrl = nullptr;            // control words
     long long wait_limit = 0;       // ns bound of every device-side wait
@@ -68,13 +73,18 @@ struct Plan {
 // Workspace layout for a plan (byte offsets from the workspace base).
 struct WsLayout {
     size_t ctrl = 0, scores = 0, super_scores = 0, cand_scores = 0, chunk_mask = 0,
-           super_mask = 0, partials = 0, total = 0;
+           super_mask = 0, cands = 0, partials = 0, total = 0;
 };
 
 // Fills the decomposition fields of `p` (needs shapes) and the layout.
 void plan_decompose(Plan& p);
 WsLayout plan_layout(const Plan& p);
 int ctrl_words(const Plan& p);
+
+// Segment candidate lists of the fused single-level top-k (entries per list).
+constexpr int kSegList = 32;
+// Whether a plan's layout holds the segment candidate lists.
+bool seg_lists(const Plan& p);
 
 // Fast fused path: bf16, d in {64, 128}.  Returns a cudaError_t.
 cudaError_t launch_fused(const Plan& p, cudaStream_t stream);

@@ -96,6 +96,7 @@ static cudaError_t launch_fused_d(const Plan& plan, cudaStream_t stream) {
     p.stages = fused::Cfg<D>::kStages;
     p.logits = 0;
     p.logit_stride = 0;
+    p.fastsel = (p.cands != nullptr && p.mode == kModeFull && !p.h2 && p.topk <= kSegList) ? 1 : 0;
     CUtensorMap m[6];
     const uint64_t P = (uint64_t)p.n_pairs;
     bool ok = make_map(&m[2], p.k_gist, P * p.M_max * p.g, D);
