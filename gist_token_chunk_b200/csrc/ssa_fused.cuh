@@ -66,6 +66,12 @@ constexpr int kLogitBytes = 16 * 1024; // shared memory for the kept logits (log
 #define SSA_PV_HEADS_M 1
 #endif
 constexpr bool kPvHeadsM = SSA_PV_HEADS_M != 0;
+// P in the P.V products: bf16 hi + lo parts (about 16 mantissa bits), or
+// the bf16 part alone (SSA_PV_LO=0: half the P.V tensor-core work)
+#ifndef SSA_PV_LO
+#define SSA_PV_LO 1
+#endif
+constexpr bool kPvLo = SSA_PV_LO != 0;
 
 // Rows of kept logits a block can hold for G query heads, and the row stride
 // of one head's logits (a multiple of 32 plus 8: conflict-free reads).
@@ -320,10 +326,10 @@ __device__ __forceinline__ void pvT16(uint32_t slot, int r0, const uint32_t (&ph
         ldsm_x4_trans(tile_addr<D>(slot, row, 2 * mm + csel), b0, b1, b2, b3);
         const uint32_t a[4] = {b0, b2, b1, b3};
         mma_bf16_16816(acc[0][mm], a, phi[0], phi[2]);
-        mma_bf16_16816(acc[0][mm], a, plo[0], plo[2]);
+        if (kPvLo) mma_bf16_16816(acc[0][mm], a, plo[0], plo[2]);
         if (two) {
             mma_bf16_16816(acc[1][mm], a, phi[1], phi[3]);
-            mma_bf16_16816(acc[1][mm], a, plo[1], plo[3]);
+            if (kPvLo) mma_bf16_16816(acc[1][mm], a, plo[1], plo[3]);
         }
     }
 }
@@ -347,9 +353,9 @@ __device__ __forceinline__ void pvM16(uint32_t slot, int r0, const uint32_t (&ph
         uint32_t b0, b1, b2, b3;
         ldsm_x4_trans(tile_addr<D>(slot, row, 2 * nn + csel), b0, b1, b2, b3);
         mma_bf16_16816(acc8<D>(acc, 2 * nn), phi, b0, b1);
-        mma_bf16_16816(acc8<D>(acc, 2 * nn), plo, b0, b1);
+        if (kPvLo) mma_bf16_16816(acc8<D>(acc, 2 * nn), plo, b0, b1);
         mma_bf16_16816(acc8<D>(acc, 2 * nn + 1), phi, b2, b3);
-        mma_bf16_16816(acc8<D>(acc, 2 * nn + 1), plo, b2, b3);
+        if (kPvLo) mma_bf16_16816(acc8<D>(acc, 2 * nn + 1), plo, b2, b3);
     }
 }
 
@@ -414,8 +420,13 @@ __device__ __forceinline__ void softmax_pv(float (&sc)[NSB][2][4], const uint32_
             const float p00 = exp2f(sc[i][0][2 * r] - ref), p01 = exp2f(sc[i][0][2 * r + 1] - ref);
             const float p10 = exp2f(sc[i][1][2 * r] - ref), p11 = exp2f(sc[i][1][2 * r + 1] - ref);
             lsum += (p00 + p01) + (p10 + p11);
-            split_bf16(p00, p01, phi[i][r], plo[i][r]);          // tokens 0..7
-            split_bf16(p10, p11, phi[i][2 + r], plo[i][2 + r]);  // tokens 8..15
+            if (kPvLo) {
+                split_bf16(p00, p01, phi[i][r], plo[i][r]);          // tokens 0..7
+                split_bf16(p10, p11, phi[i][2 + r], plo[i][2 + r]);  // tokens 8..15
+            } else {
+                phi[i][r] = pack_bf16(p00, p01);
+                phi[i][2 + r] = pack_bf16(p10, p11);
+            }
         }
         lrow[r] = lrow[r] * alpha + lsum;
         mrow[r] = mnew;
@@ -1444,12 +1455,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int i = 0; i < 2; ++i)
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
+                        // a segment's kept rows start at any row: the pair of rows is
+                        // read as one 8-byte word only where it is aligned
                         const int t = rb[i] + nt * 8 + 2 * tig;
-                        const float2 a = g8 < p.G ? *reinterpret_cast<const float2*>(lg + g8 * ls + t)
-                                                  : make_float2(0.f, 0.f);
-                        const float2 b2 = g8 + 8 < p.G
-                                              ? *reinterpret_cast<const float2*>(lg + (g8 + 8) * ls + t)
-                                              : make_float2(0.f, 0.f);
+                        const float* la = lg + g8 * ls + t;
+                        const float* lb = lg + (g8 + 8) * ls + t;
+                        float2 a = make_float2(0.f, 0.f), b2 = make_float2(0.f, 0.f);
+                        if (!(mt.lrow & 1)) {
+                            if (g8 < p.G) a = *reinterpret_cast<const float2*>(la);
+                            if (g8 + 8 < p.G) b2 = *reinterpret_cast<const float2*>(lb);
+                        } else {
+                            if (g8 < p.G) a = make_float2(la[0], la[1]);
+                            if (g8 + 8 < p.G) b2 = make_float2(lb[0], lb[1]);
+                        }
                         const int tb = 16 * i + nt * 8 + 2 * tig;
                         const bool x0 = (ex >> tb) & 1u, x1 = (ex >> (tb + 1)) & 1u;
                         sc[i][nt][0] = x0 ? -INFINITY : a.x;

@@ -72,6 +72,26 @@ def test_split_invariance(ssa, inp, blocks):
     assert (o - o0).abs().max().item() <= 1e-6
 
 
+W_ODD = Workload("odd_g", B=2, Hq=8, Hkv=2, d=64, n_max=4800, C=48, g=3, topk=7,
+                 seq_lens=(4799, 3001), planted=4)
+
+
+@pytest.mark.parametrize("blocks,rows", [(5, 128), (23, 0), (61, 64)])
+def test_split_invariance_odd_rows(ssa, blocks, rows):
+    """g = 3: a block's kept scoring rows of a second pair (or sub-item)
+    start at an odd row, so the gist pass reads them from any offset."""
+    i = {k: v.cuda() if k != "planted_idx" else v for k, v in make_inputs(W_ODD, seed=5).items()}
+    o0, s0 = run(ssa, i, w=W_ODD)
+    ssa.ssa_set_tuning(blocks, rows)
+    try:
+        o, s = run(ssa, i, w=W_ODD)
+    finally:
+        ssa.ssa_set_tuning(0, 0)
+    assert ssa.ssa_get_device_status() == 0
+    assert torch.equal(s, s0)
+    assert (o - o0).abs().max().item() <= 1e-5
+
+
 def test_bad_length_sets_status_and_zeroes(ssa, inp):
     bad = dict(inp)
     bad["seq_lens"] = torch.tensor([4096, 5000], dtype=torch.int32, device="cuda")  # > n_max
