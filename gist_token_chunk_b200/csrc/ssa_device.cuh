@@ -89,7 +89,7 @@ __device__ __forceinline__ bool wait_geq(const int* p, int target, long long lim
     unsigned sleep_ns = 32;
     for (;;) {
         __nanosleep(sleep_ns);
-        if (sleep_ns < 512) sleep_ns *= 2;
+        if (sleep_ns < 128) sleep_ns *= 2;
         if (ld_relaxed(p) >= target) {
             fence_acquire_gpu();
             return true;

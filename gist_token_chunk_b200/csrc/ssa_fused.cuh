@@ -1724,6 +1724,56 @@ __global__ void __launch_bounds__(kThreads, 2)
                 while (a < 2 && s >= nseg[a]) s -= nseg[a++];
                 return p.partials + partial_offset(p, a, c0[a] + s, pair, 0, D);
             };
+            // combinations of up to this many partials load in one round
+            constexpr int kCombineOne = D == 64 ? 16 : 8;
+            if (NP <= kCombineOne) {
+                // One round of loads: every lane reads the (m, l) of segment
+                // `lane` and its columns of every segment's output together.
+                for (int h = warp; h < G; h += kConsumerWarps) {
+                    float* op = p.out + ((size_t)b * p.Hq + (size_t)j * G + h) * D;
+                    float2 ml = make_float2(-INFINITY, 0.f);
+                    if (lane < NP)
+                        ml = __ldcg(reinterpret_cast<const float2*>(seg_base(lane) + (size_t)h * (D + 2)));
+                    float2 a[kCombineOne][D / 64];
+#pragma unroll
+                    for (int u = 0; u < kCombineOne; ++u) {
+                        if (u < NP) {
+                            const float* q = seg_base(u) + (size_t)h * (D + 2) + 2;
+#pragma unroll
+                            for (int t = 0; t < D / 64; ++t)
+                                a[u][t] = __ldcg(reinterpret_cast<const float2*>(q + 64 * t + 2 * lane));
+                        } else {
+#pragma unroll
+                            for (int t = 0; t < D / 64; ++t) a[u][t] = make_float2(0.f, 0.f);
+                        }
+                    }
+                    float mx = ml.x;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    const float ref = (mx == -INFINITY) ? 0.f : mx;
+                    const float fl = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - ref);
+                    float lsum = fl * ml.y;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+                    float ox[D / 64][2];
+#pragma unroll
+                    for (int t = 0; t < D / 64; ++t) ox[t][0] = ox[t][1] = 0.f;
+#pragma unroll
+                    for (int u = 0; u < kCombineOne; ++u) {
+                        const float f = __shfl_sync(0xffffffffu, fl, u);
+#pragma unroll
+                        for (int t = 0; t < D / 64; ++t) {
+                            ox[t][0] += f * a[u][t].x;
+                            ox[t][1] += f * a[u][t].y;
+                        }
+                    }
+                    const float inv = (!bad && lsum > 0.f) ? 1.f / lsum : 0.f;
+#pragma unroll
+                    for (int t = 0; t < D / 64; ++t)
+                        *reinterpret_cast<float2*>(op + 64 * t + 2 * lane) =
+                            make_float2(ox[t][0] * inv, ox[t][1] * inv);
+                }
+            } else
             for (int h = warp; h < G; h += kConsumerWarps) {
                 float* op = p.out + ((size_t)b * p.Hq + (size_t)j * G + h) * D;
                 float ox[D / 64][2];
