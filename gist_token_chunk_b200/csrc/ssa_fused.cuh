@@ -789,6 +789,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     const long long long_limit = 8 * p.wait_limit;
 
     // ---- prologue: barriers and the block-local plan (the same in every block)
+    if (warp == kConsumerWarps && lane == 0) {
+        // the tensor maps' descriptors are fetched while the lengths load
+        prefetch_tensormap(&tm_kraw);
+        prefetch_tensormap(&tm_vraw);
+        prefetch_tensormap(&tm_kgist);
+        prefetch_tensormap(&tm_vgist);
+        prefetch_tensormap(&tm_kmeta);
+        prefetch_tensormap(&tm_vmeta);
+    }
     if (threadIdx.x == 0) {
         misc[15] = 0;
         for (int s = 0; s < NS; ++s) {
@@ -833,8 +842,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (warp == kConsumerWarps) {
         Producer<D> pr{p,    {&tm_kraw, &tm_vraw, &tm_kgist, &tm_vgist, &tm_kmeta, &tm_vmeta},
                        ring, qbuf, L.qbytes, meta, full, empty, ctrl, lane, long_limit};
-        if (lane == 0)
-            for (int i = 0; i < 6; ++i) prefetch_tensormap(pr.tm[i]);
         pr.pol_once = l2_policy_evict_first();
         pr.trace_ctr = &misc[15];
         pr.pol_keep = so ? pr.pol_once : l2_policy_evict_last();

@@ -96,7 +96,7 @@ static cudaError_t launch_fused_d(const Plan& plan, cudaStream_t stream) {
     p.stages = fused::Cfg<D>::kStages;
     p.logits = 0;
     p.logit_stride = 0;
-    p.fastsel = (p.cands != nullptr && p.mode == kModeFull && !p.h2 && p.topk <= kSegList) ? 1 : 0;
+    p.fastsel = 0;
     CUtensorMap m[6];
     const uint64_t P = (uint64_t)p.n_pairs;
     bool ok = make_map(&m[2], p.k_gist, P * p.M_max * p.g, D);
@@ -152,6 +152,9 @@ static cudaError_t launch_fused_d(const Plan& plan, cudaStream_t stream) {
         if (grid_t > chunks) grid_t = chunks;
         const long long rows_max = grid_t > 0 ? (chunks + grid_t - 1) / grid_t * p.g : 0;
         if (occ_t >= occ && grid_t > 0 && rows_max <= fused::logit_rows_cap(p.G)) {
+            // the merged segment lists replace the full top-k where a block's
+            // segments are short (one sub-item each)
+            t.fastsel = (p.cands != nullptr && p.topk <= kSegList) ? 1 : 0;
             p = t;
             occ = occ_t;
             Luse = Lt;
