@@ -148,7 +148,9 @@ void plan_decompose(Plan& p) {
     p.smask_words = p.h2 ? (cdiv(p.S_max, 32) + 3) / 4 * 4 : 0;
 }
 
-bool seg_lists(const Plan& p) { return fused_path(p) && !p.h2 && p.topk <= kSegList; }
+bool seg_lists(const Plan& p) {
+    return fused_path(p) && p.topk <= kSegList && (!p.h2 || p.topk_super <= kSegList);
+}
 
 int ctrl_words(const Plan& p) { return 64 + p.pair_ints * p.n_pairs; }  // see ssa_fused.cuh
 
@@ -167,7 +169,8 @@ WsLayout plan_layout(const Plan& p) {
     L.cand_scores = take(p.h2 ? P * p.Mc_max * 4 : 0);
     L.chunk_mask = take(0);
     L.super_mask = take(0);
-    L.cands = take(seg_lists(p) ? (ssa::kFusedMaxGrid + P) * ssa::kSegList * 8 : 0);
+    // one set of segment lists per selection level
+    L.cands = take(seg_lists(p) ? (p.h2 ? 2 : 1) * (ssa::kFusedMaxGrid + P) * ssa::kSegList * 8 : 0);
     // one partial per (attention list, segment slot, query head)
     L.partials =
         take(fused_path(p) ? 3 * (ssa::kFusedMaxGrid + P) * p.G * (size_t)(p.d + 2) * 4 : 0);

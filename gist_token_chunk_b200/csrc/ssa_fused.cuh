@@ -646,15 +646,19 @@ struct Producer {
     // Scores `nslot` consecutive summary slots of `ntok` rows each, starting
     // at global row y0 of map m, into dst[0..nslot), then writes `npad` slots
     // of -inf.  Split into sub-items of at most `per_rows` rows.
+    // (seg_first / seg_last: this run starts / ends its block's segment of
+    // the pair; a candidate segment is several runs)
     __device__ void score_run(int pair, int level, const CUtensorMap* m, int y0, int nslot,
-                              int npad, int dst, int ntok, int per_rows, int lrow0) {
+                              int npad, int dst, int ntok, int per_rows, int lrow0,
+                              bool seg_first = true, bool seg_last = true) {
         const int per = max(1, per_rows / ntok);  // slots per sub-item
         int s0 = 0;
         do {
             const int ns = min(per, nslot - s0);
             const int np = (s0 + ns >= nslot) ? npad : 0;
             const int rows = ns * ntok;
-            const int segf = (s0 == 0 ? F_SEGBEG : 0) | (s0 + ns >= nslot ? F_SEGEND : 0);
+            const int segf = (seg_first && s0 == 0 ? F_SEGBEG : 0) |
+                             (seg_last && s0 + ns >= nslot ? F_SEGEND : 0);
             if (rows <= 0) {
                 StageMeta mt = {};
                 mt.kind = K_SCORE;
@@ -887,7 +891,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                             run = i1 - c;
                         }
                         pr.score_run(pair, 1, &tm_kgist, (pair * p.M_max + chunk0) * p.g, run, 0,
-                                     pair * p.Mc_max + c, p.g, score_rows, 0);
+                                     pair * p.Mc_max + c, p.g, score_rows, 0, c == i0, c + run >= i1);
                         c += run;
                     }
                 }
@@ -1519,7 +1523,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                     // segment keeps only its 32 best chunks (key, ~chunk):
                     // no chunk outside them can be among the pair's top-k
                     if (mt.flags & F_SEGBEG) segrun = 1ull;
-                    const uint32_t cbase = (uint32_t)(mt.a3 - pair * p.M_max);
+                    // slot index in the pair's list of this level (chunk, superchunk
+                    // or candidate position)
+                    const int lstride = mt.a5 == 1 ? p.Mc_max : p.h2 ? p.S_max : p.M_max;
+                    const uint32_t cbase = (uint32_t)(mt.a3 - pair * lstride);
                     for (int i0 = 32 * warp; i0 < mt.a1; i0 += kConsumers) {
                         const int i = i0 + lane;
                         unsigned long long x = 1ull;
@@ -1539,7 +1546,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                             for (int w = 1; w < kConsumerWarps; ++w)
                                 x = warp_merge_desc(x, wlists[w * 32 + lane], lane);
                             // never 0 (a written entry); the selection polls for it
-                            p.cands[(size_t)(cta + pair) * kSegList + lane] = x;
+                            p.cands[((size_t)mt.a5 * (kMaxGrid + P) + cta + pair) * kSegList + lane] = x;
                         }
                     }
                 } else {
@@ -1576,25 +1583,20 @@ __global__ void __launch_bounds__(kThreads, 2)
                 // afterwards this block clears them for the next call.
                 float* vals;
                 int nv;
-                if (what == SEL_SUPER) {
-                    vals = p.super_scores + (size_t)pair * p.S_max;
-                    nv = z.S;
-                    block_topk<kConsumers>(vals, nv, p.topk_super,
-                                           p.sel_super + (size_t)pair * p.topk_super, tsc, csync,
-                                           NoProbe(), rec(A_ENTRIES + p.topk, pair), p.wait_limit);
-                    if (tid == 0) *rec(A_SCOUNT, pair) = z.ks + 1;
-                } else if (what == SEL_CHUNKS && p.fastsel) {
-                    // merge the 32-best lists of the pair's scoring segments;
-                    // the first k of the merged list are the pair's top-k
+                if (p.fastsel) {
+                    // merge the 32-best lists of the pair's scoring segments of
+                    // this level; the first k of the merged list are the top-k
                     vals = nullptr;
                     nv = 0;
+                    const int lvl = what == SEL_CAND ? 1 : 0;
                     int c0, nseg;
-                    pv.pair_blocks(L_SCORE, pair, c0, nseg);
+                    pv.pair_blocks(lvl ? L_CAND : L_SCORE, pair, c0, nseg);
                     unsigned long long run = 1ull;
                     const long long t0 = clock64(), lim = wait_cycles(p.wait_limit);
                     bool late = false;
                     for (int sg = warp; sg < nseg; sg += kConsumerWarps) {
-                        unsigned long long* src = p.cands + (size_t)(c0 + sg + pair) * kSegList;
+                        unsigned long long* src =
+                            p.cands + ((size_t)lvl * (kMaxGrid + P) + c0 + sg + pair) * kSegList;
                         unsigned long long x = ld_relaxed_u64(src + lane);
                         while (__any_sync(0xffffffffu, x == 0ull)) {
                             if (__shfl_sync(0xffffffffu, (int)(clock64() - t0 > lim), 0)) {
@@ -1615,15 +1617,43 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll 1
                         for (int w = 1; w < kConsumerWarps; ++w)
                             run = warp_merge_desc(run, wlists[w * 32 + lane], lane);
-                        const int k = z.kc;
+                        const bool sup_level = what == SEL_SUPER;
+                        const int k = sup_level ? z.ks : z.kc;
                         int idx = lane < k ? (int)~(uint32_t)run : INT_MAX;
                         idx = warp_sort_asc(idx, lane);
-                        int* out = p.sel_idx + (size_t)pair * p.topk;
-                        int* pub = rec(A_ENTRIES, pair);
-                        if (lane < p.topk) out[lane] = lane < k ? idx : -1;
+                        if (what == SEL_CAND && lane < k) {
+                            // candidate position -> chunk id (an increasing map); the
+                            // superchunks come from their published copy (entry + 1)
+                            const int pos = idx;
+                            if (pos < z.ks * p.J) {
+                                const int* sup = rec(A_ENTRIES + p.topk, pair);
+                                int e = ld_relaxed(sup + pos / p.J);
+                                const long long c1 = clock64();
+                                while (e == 0 && clock64() - c1 < lim) {
+                                    __nanosleep(64);
+                                    e = ld_relaxed(sup + pos / p.J);
+                                }
+                                if (e == 0) report_status(kStatusTimeout);
+                                idx = (e - 1) * p.J + pos % p.J;
+                            } else {
+                                idx = z.S * p.J + (pos - z.ks * p.J);
+                            }
+                        }
+                        const int cap = sup_level ? p.topk_super : p.topk;
+                        int* out = sup_level ? p.sel_super + (size_t)pair * p.topk_super
+                                             : p.sel_idx + (size_t)pair * p.topk;
+                        int* pub = rec(sup_level ? A_ENTRIES + p.topk : A_ENTRIES, pair);
+                        if (lane < cap) out[lane] = lane < k ? idx : -1;
                         if (lane < k) pub[lane] = idx + 1;
-                        if (lane == 0) *rec(A_COUNT, pair) = k + 1;
+                        if (lane == 0) *rec(sup_level ? A_SCOUNT : A_COUNT, pair) = k + 1;
                     }
+                } else if (what == SEL_SUPER) {
+                    vals = p.super_scores + (size_t)pair * p.S_max;
+                    nv = z.S;
+                    block_topk<kConsumers>(vals, nv, p.topk_super,
+                                           p.sel_super + (size_t)pair * p.topk_super, tsc, csync,
+                                           NoProbe(), rec(A_ENTRIES + p.topk, pair), p.wait_limit);
+                    if (tid == 0) *rec(A_SCOUNT, pair) = z.ks + 1;
                 } else if (what == SEL_CHUNKS) {
                     vals = p.scores + (size_t)pair * p.M_max;
                     nv = z.M;

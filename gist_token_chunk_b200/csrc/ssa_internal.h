@@ -39,9 +39,10 @@ struct Plan {
     int logits = 0;
     int logit_stride = 0;
     int mask_words = 0, smask_words = 0;
-    // fused single-level decode with topk <= 32: every scoring segment
-    // publishes its 32 best chunks (descending composites key << 32 | ~chunk)
-    // and the top-k merges those lists instead of ranking every score
+    // topk (and topk_super) <= 32, single level in logits mode or two
+    // level: every scoring segment publishes its 32 best slots (descending
+    // composites key << 32 | ~slot) and the top-k merges those lists
+    // instead of ranking every score
     int fastsel = 0;
 
     const void* q = nullptr;
@@ -60,7 +61,7 @@ struct Plan {
     uint32_t* chunk_mask = nullptr; // [P, mask_words]
     uint32_t* super_mask = nullptr; // [P, smask_words]
     float* partials = nullptr;      // [3, kFusedMaxGrid + P, G, d + 2]
-    unsigned long long* cands = nullptr;  // [kFusedMaxGrid + P, 32] segment lists
+    unsigned long long* cands = nullptr;  // [levels, kFusedMaxGrid + P, 32] segment lists
     float* out = nullptr;           // [B, Hq, d]
     int* ctrl = nullptr;            // control words
     long long wait_limit = 0;       // ns bound of every device-side wait

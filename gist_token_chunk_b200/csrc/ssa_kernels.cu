@@ -96,7 +96,11 @@ static cudaError_t launch_fused_d(const Plan& plan, cudaStream_t stream) {
     p.stages = fused::Cfg<D>::kStages;
     p.logits = 0;
     p.logit_stride = 0;
-    p.fastsel = 0;
+    // two levels: the merged segment lists at both selections
+    p.fastsel = (p.cands != nullptr && p.h2 && p.mode == kModeFull && p.topk <= kSegList &&
+                 p.topk_super <= kSegList)
+                    ? 1
+                    : 0;
     CUtensorMap m[6];
     const uint64_t P = (uint64_t)p.n_pairs;
     bool ok = make_map(&m[2], p.k_gist, P * p.M_max * p.g, D);
