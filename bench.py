@@ -441,29 +441,46 @@ def main():
 
     # ---- end to end through the public call, host buffers
     ek = max(NS, min(args.steps, args.e2e_steps)) if args.e2e_steps > 0 else 0
-    q_host = [x["q"].cpu().pin_memory() for x in sets]
-    len_host = [x["seq_lens"].cpu().pin_memory() for x in sets]
-    q_dev = [torch.empty_like(x["q"]) for x in sets]
-    len_dev = [torch.empty_like(x["seq_lens"]) for x in sets]
-    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-    sel_host = [torch.empty(s.shape, dtype=s.dtype).pin_memory() for s in sels]
+    # one pinned staging buffer per direction and set: the query and the
+    # lengths go up in one copy, the output and the selection come back in one
+    def packed(tensors, device):
+        sizes = [(t.numel() * t.element_size() + 15) // 16 * 16 for t in tensors]
+        buf = torch.empty(sum(sizes), dtype=torch.uint8, device=device)
+        if device == "cpu":
+            buf = buf.pin_memory()
+        views, off = [], 0
+        for t, n in zip(tensors, sizes):
+            nb = t.numel() * t.element_size()
+            views.append(buf[off:off + nb].view(t.dtype).view(t.shape))
+            off += n
+        return buf, views
+
+    up_host, up_dev, down_host, down_dev = [], [], [], []
+    for s in range(NS):
+        hb, (qh, lh) = packed([sets[s]["q"], sets[s]["seq_lens"]], "cpu")
+        qh.copy_(sets[s]["q"].cpu())
+        lh.copy_(sets[s]["seq_lens"].cpu())
+        up_host.append(hb)
+        up_dev.append(packed([sets[s]["q"], sets[s]["seq_lens"]], dev))
+        down_dev.append(packed([outs[s], sels[s]], dev))
+        down_host.append(packed([outs[s], sels[s]], "cpu")[0])
 
     def e2e_step(i):
         s = i % NS
-        q_dev[s].copy_(q_host[s], non_blocking=True)
-        len_dev[s].copy_(len_host[s], non_blocking=True)
-        x = dict(sets[s], q=q_dev[s], seq_lens=len_dev[s])
+        dbuf, (q_dev, len_dev) = up_dev[s]
+        dbuf.copy_(up_host[s], non_blocking=True)
+        x = dict(sets[s], q=q_dev, seq_lens=len_dev)
+        obuf, (o_dev, s_dev) = down_dev[s]
         if w.two_level:
             ssa.ssa_decode_h2(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
                               x["k_meta"], x["v_meta"], x["seq_lens"], w.C, w.g, w.J, w.gm,
-                              w.topk_super, w.topk, out=outs[s], sel_super=sups[s],
-                              sel_idx=sels[s], ws=ws, stream=stream)
+                              w.topk_super, w.topk, out=o_dev, sel_super=sups[s],
+                              sel_idx=s_dev, ws=ws, stream=stream)
         else:
             ssa.ssa_decode(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
-                           x["seq_lens"], w.C, w.g, w.topk, out=outs[s], sel_idx=sels[s], ws=ws,
+                           x["seq_lens"], w.C, w.g, w.topk, out=o_dev, sel_idx=s_dev, ws=ws,
                            stream=stream)
-        out_host[s].copy_(outs[s], non_blocking=True)
-        sel_host[s].copy_(sels[s], non_blocking=True)
+        down_host[s].copy_(obuf, non_blocking=True)
 
     e2e_value = None
     if ek > 0:
@@ -504,7 +521,7 @@ def main():
         "gpu_launches": args.steps,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": ek,
-                "path": "ssa_decode per step (Python binding -> C ABI) with pinned host copies"},
+                "path": "ssa_decode per step (Python binding -> C ABI); query and lengths up in one pinned copy, output and selection back in one"},
     }
     clk = sampler.summary()
     if clk is not None:
