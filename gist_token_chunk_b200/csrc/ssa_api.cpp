@@ -145,6 +145,9 @@ void plan_decompose(Plan& p) {
     // counters line, published-count line, then the published selection(s)
     p.pair_ints = 64 + (p.topk + (p.h2 ? p.topk_super : 0) + 31) / 32 * 32;
     p.mask_words = (cdiv(p.M_max, 32) + 3) / 4 * 4;
+    p.g_shift = -1;
+    for (int sh = 0; sh < 11; ++sh)
+        if (p.g == (1 << sh)) p.g_shift = sh;
     p.smask_words = p.h2 ? (cdiv(p.S_max, 32) + 3) / 4 * 4 : 0;
 }
 

@@ -1451,17 +1451,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const int rb[2] = {16 * warp, 64 + 16 * warp};
                 bool e;
                 {
+                    // (branch-free: the row's slot word is read for every lane)
                     const int lr = (lane < 16 ? rb[0] : rb[1]) + (lane & 15);
-                    e = lr >= mt.nvalid;
-                    if (!e) {
-                        const int sid = (mt.a0 + lr) / mt.a2;
-                        e = (bits[sid >> 5] >> (sid & 31)) & 1u;
-                    }
+                    const int row = mt.a0 + min(lr, max(mt.nvalid - 1, 0));
+                    const int sid = p.g_shift >= 0 ? row >> p.g_shift : row / mt.a2;
+                    e = (lr >= mt.nvalid) | ((bits[sid >> 5] >> (sid & 31)) & 1u);
                 }
                 const uint32_t ex = __ballot_sync(0xffffffffu, e);
                 float sc[2][2][4];
                 const float* lg = logits + mt.lrow;
                 const int ls = p.logit_stride;
+                // lanes of heads past G read head 0's logits (their P rows are
+                // never used): no divergent loads
+                const int ha = g8 < p.G ? g8 : 0, hb = g8 + 8 < p.G ? g8 + 8 : 0;
 #pragma unroll
                 for (int i = 0; i < 2; ++i)
 #pragma unroll
@@ -1469,15 +1471,15 @@ __global__ void __launch_bounds__(kThreads, 2)
                         // a segment's kept rows start at any row: the pair of rows is
                         // read as one 8-byte word only where it is aligned
                         const int t = rb[i] + nt * 8 + 2 * tig;
-                        const float* la = lg + g8 * ls + t;
-                        const float* lb = lg + (g8 + 8) * ls + t;
-                        float2 a = make_float2(0.f, 0.f), b2 = make_float2(0.f, 0.f);
+                        const float* la = lg + ha * ls + t;
+                        const float* lb = lg + hb * ls + t;
+                        float2 a, b2 = make_float2(0.f, 0.f);
                         if (!(mt.lrow & 1)) {
-                            if (g8 < p.G) a = *reinterpret_cast<const float2*>(la);
-                            if (g8 + 8 < p.G) b2 = *reinterpret_cast<const float2*>(lb);
+                            a = *reinterpret_cast<const float2*>(la);
+                            if (two_rows) b2 = *reinterpret_cast<const float2*>(lb);
                         } else {
-                            if (g8 < p.G) a = make_float2(la[0], la[1]);
-                            if (g8 + 8 < p.G) b2 = make_float2(lb[0], lb[1]);
+                            a = make_float2(la[0], la[1]);
+                            if (two_rows) b2 = make_float2(lb[0], lb[1]);
                         }
                         const int tb = 16 * i + nt * 8 + 2 * tig;
                         const bool x0 = (ex >> tb) & 1u, x1 = (ex >> (tb + 1)) & 1u;

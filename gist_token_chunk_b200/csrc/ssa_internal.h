@@ -39,6 +39,7 @@ struct Plan {
     int logits = 0;
     int logit_stride = 0;
     int mask_words = 0, smask_words = 0;
+    int g_shift = -1;      // log2(g) when g is a power of two, else -1
     // topk (and topk_super) <= 32, single level in logits mode or two
     // level: every scoring segment publishes its 32 best slots (descending
     // composites key << 32 | ~slot) and the top-k merges those lists
