@@ -1534,7 +1534,15 @@ __global__ void __launch_bounds__(kThreads, 2)
                         unsigned long long x = 1ull;
                         if (i < mt.a1) {
                             float v = -INFINITY;
-                            for (int t = 0; t < mt.a4; ++t) v = fmaxf(v, rowmax[i * mt.a4 + t]);
+                            if (mt.a4 == 8) {
+                                // 8 summary rows per slot: two 16-byte loads
+                                const float4* r4 = reinterpret_cast<const float4*>(rowmax + i * 8);
+                                const float4 u = r4[0], w = r4[1];
+                                v = fmaxf(fmaxf(fmaxf(u.x, u.y), fmaxf(u.z, u.w)),
+                                          fmaxf(fmaxf(w.x, w.y), fmaxf(w.z, w.w)));
+                            } else {
+                                for (int t = 0; t < mt.a4; ++t) v = fmaxf(v, rowmax[i * mt.a4 + t]);
+                            }
                             x = ((unsigned long long)score_key(v) << 32) | (uint32_t)~(cbase + i);
                         }
                         segrun = warp_merge_desc(segrun, warp_sort_desc(x, lane), lane);
@@ -1556,8 +1564,15 @@ __global__ void __launch_bounds__(kThreads, 2)
                     float* dst = mt.a5 == 1 ? p.cand_scores : p.h2 ? p.super_scores : p.scores;
                     for (int i = tid; i < mt.a1 + mt.a2; i += kConsumers) {
                         float v = -INFINITY;
-                        if (i < mt.a1)
+                        if (i < mt.a1 && mt.a4 == 8) {
+                            // 8 summary rows per slot: two 16-byte loads
+                            const float4* r4 = reinterpret_cast<const float4*>(rowmax + i * 8);
+                            const float4 u = r4[0], w = r4[1];
+                            v = fmaxf(fmaxf(fmaxf(u.x, u.y), fmaxf(u.z, u.w)),
+                                      fmaxf(fmaxf(w.x, w.y), fmaxf(w.z, w.w)));
+                        } else if (i < mt.a1) {
                             for (int t = 0; t < mt.a4; ++t) v = fmaxf(v, rowmax[i * mt.a4 + t]);
+                        }
                         // for the selection, +0 is stored as -0 (same rank): an
                         // all-zero word means "not written yet"
                         dst[mt.a3 + i] = (so || v != 0.f) ? v : -0.f;
