@@ -1,6 +1,6 @@
 """CUDA path (through the C ABI) against the fp64 oracle, element by element.
 
-Bars (the benchmark spec criteria, applied in tests/parity.py): selections bit-exact
+Bars (the accuracy criteria of this path, applied in tests/parity.py): selections bit-exact
 unless the oracle's k-th/(k+1)-th score gap is <= 1e-4 (then the GPU's choice
 must be a valid top-k and the oracle is re-run on it); outputs within max-abs
 1e-2 and mean-abs 1e-3 of the oracle.
