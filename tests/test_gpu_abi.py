@@ -92,6 +92,32 @@ def test_split_invariance_odd_rows(ssa, blocks, rows):
     assert (o - o0).abs().max().item() <= 1e-5
 
 
+W_TIE = Workload("ties", B=2, Hq=8, Hkv=2, d=64, n_max=8192, C=64, g=8, topk=16,
+                 seq_lens=(8192, 5000), planted=0)
+
+
+@pytest.mark.parametrize("blocks,rows", [(0, 0), (37, 0), (5, 128)])
+def test_equal_scores_select_lowest_chunks(ssa, blocks, rows):
+    """Every gist key of a pair equal: every chunk scores the same, so the
+    selection is chunks 0..k-1 (ties to the lower index), however the chunks
+    are split into scoring segments and sub-items."""
+    i = {k: v.cuda() if k != "planted_idx" else v for k, v in make_inputs(W_TIE, seed=9).items()}
+    kg = i["k_gist"]
+    i["k_gist"] = kg[:, :, :1, :1, :].expand_as(kg).contiguous()
+    ssa.ssa_set_tuning(blocks, rows)
+    try:
+        out, sel = run(ssa, i, w=W_TIE)
+    finally:
+        ssa.ssa_set_tuning(0, 0)
+    assert ssa.ssa_get_device_status() == 0
+    s = sel.cpu()
+    for b, n in enumerate(W_TIE.seq_lens):
+        k = min(W_TIE.topk, n // W_TIE.C)
+        want = list(range(k)) + [-1] * (W_TIE.topk - k)
+        for j in range(W_TIE.Hkv):
+            assert s[b, j].tolist() == want, (b, j)
+
+
 def test_bad_length_sets_status_and_zeroes(ssa, inp):
     bad = dict(inp)
     bad["seq_lens"] = torch.tensor([4096, 5000], dtype=torch.int32, device="cuda")  # > n_max
