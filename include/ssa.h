@@ -61,8 +61,9 @@
  * bytes.  Pass ws = NULL, ws_bytes = 0 to let the library allocate it
  * stream-ordered (cudaMallocAsync) for that one call.  A caller-owned
  * workspace must be zeroed once with ssa_workspace_init() (or cudaMemset 0)
- * before its first use; every call leaves the state it used (control words
- * and score scratch) zeroed again, so it can be reused by later calls on the
+ * before its first use; every call leaves the state it used (control words,
+ * score scratch and the scoring segments' candidate lists) zeroed again, so
+ * it can be reused by later calls on the
  * same stream, for any sizes that fit, without re-initialising (when a call
  * lays the workspace out differently from the workspace's previous call, the
  * library zeroes the part it needs stream-ordered first).
