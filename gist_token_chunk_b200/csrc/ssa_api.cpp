@@ -157,7 +157,7 @@ bool seg_lists(const Plan& p) {
 
 int ctrl_words(const Plan& p) { return 64 + p.pair_ints * p.n_pairs; }  // see ssa_fused.cuh
 
-WsLayout plan_layout(const Plan& p) {
+static WsLayout fused_layout(const Plan& p) {
     WsLayout L;
     size_t o = 0;
     auto take = [&](size_t bytes) {
@@ -181,6 +181,46 @@ WsLayout plan_layout(const Plan& p) {
     return L;
 }
 
+// The streaming path's areas (p prepared by stream_prepare); the header with
+// the epoch sits at offset 0 in every size, so any two calls of this path
+// agree on it.
+static WsLayout stream_layout(const Plan& p) {
+    WsLayout L;
+    size_t hdr, sc, sel, sum, part;
+    stream_ws_sizes(p, &hdr, &sc, &sel, &sum, &part);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o += (bytes + 255) / 256 * 256;
+        return at;
+    };
+    L.stream = true;
+    L.st_hdr = take(hdr);
+    L.st_scores = take(sc);
+    L.st_sel = take(sel);
+    L.st_sum = take(sum);
+    L.st_part = take(part);
+    L.total = o;
+    return L;
+}
+
+WsLayout plan_layout(const Plan& p) {
+    Plan q = p;
+    if (stream_prepare(q)) return stream_layout(q);
+    return fused_layout(p);
+}
+
+size_t plan_bytes_any(const Plan& p) {
+    size_t a = fused_layout(p).total;
+    Plan q = p;
+    q.mode = kModeFull;
+    if (stream_prepare(q)) {
+        const size_t b = stream_layout(q).total;
+        if (b > a) a = b;
+    }
+    return a;
+}
+
 }  // namespace ssa
 
 namespace {
@@ -188,6 +228,14 @@ namespace {
 void attach_ws(ssa::Plan& p, void* ws) {
     const ssa::WsLayout L = ssa::plan_layout(p);
     char* base = static_cast<char*>(ws);
+    if (L.stream) {
+        p.st_hdr = reinterpret_cast<unsigned*>(base + L.st_hdr);
+        p.st_scores = reinterpret_cast<unsigned long long*>(base + L.st_scores);
+        p.st_sel = reinterpret_cast<unsigned long long*>(base + L.st_sel);
+        p.st_sum = reinterpret_cast<unsigned long long*>(base + L.st_sum);
+        p.st_part = base + L.st_part;
+        return;
+    }
     p.ctrl = reinterpret_cast<int*>(base + L.ctrl);
     p.scores = reinterpret_cast<float*>(base + L.scores);
     p.super_scores = p.h2 ? reinterpret_cast<float*>(base + L.super_scores) : nullptr;
@@ -204,7 +252,9 @@ void attach_ws(ssa::Plan& p, void* ws) {
 // layout is not already known to be zero, it zeroes that prefix
 // (stream-ordered).
 struct WsState {
-    int kind = 0;      // 0: zero up to `bytes`; 1: fused layout; 2: unknown
+    int kind = 0;      // 0: zero up to `bytes`; 1: fused layout; 2: unknown;
+                       // 3: streaming path (up to `bytes`: zero or written by
+                       //    that path, whose words carry an older epoch)
     size_t bytes = 0;  // kind 0: zeroed bytes; kind 1: zero prefix of the layout
     size_t ctrl = 0;   // kind 1: control bytes of the layout
 };
@@ -245,9 +295,56 @@ cudaError_t prepare_ws(void* ws, bool fused, size_t ctrl_bytes, size_t clean_byt
     return zero ? cudaMemsetAsync(ws, 0, clean_bytes, stream) : cudaSuccess;
 }
 
+// Before a streaming-path call: its areas must hold zeros or words of an
+// earlier launch of that path (whatever its sizes: the epoch header is at
+// offset 0 and only grows), so the workspace is zeroed only when it comes
+// from another path or is larger than what is known.
+cudaError_t prepare_ws_stream(void* ws, size_t need, cudaStream_t stream) {
+    bool zero = false;
+    {
+        std::lock_guard<std::mutex> lk(g_ws_mu);
+        auto it = g_ws.find(ws);
+        WsState next;
+        next.kind = 3;
+        next.bytes = need;
+        if (it != g_ws.end()) {
+            const WsState& st = it->second;
+            if ((st.kind == 0 || st.kind == 3) && st.bytes >= need)
+                next.bytes = st.bytes;
+            else
+                zero = true;
+        }
+        g_ws[ws] = next;
+    }
+    return zero ? cudaMemsetAsync(ws, 0, need, stream) : cudaSuccess;
+}
+
+// After a device wait ran out, a fused-layout workspace may hold non-zero
+// control words: its next call zeroes it.
+void note_timeout() {
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    for (auto& kv : g_ws)
+        if (kv.second.kind == 1) kv.second.kind = 2;
+}
+
+void note_ws_unknown(const void* ws) {
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    WsState st;
+    st.kind = 2;
+    g_ws[ws] = st;
+}
+
+cudaError_t launch_plan(const ssa::Plan& p, cudaStream_t stream) {
+    if (p.st_rcap > 0) return ssa::launch_stream(p, stream);
+    return fused_path(p) ? ssa::launch_fused(p, stream) : ssa::launch_generic(p, stream);
+}
+
 // Runs a workspace-using plan: caller workspace, or a stream-ordered one.
 ssa_status run_with_ws(ssa::Plan& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
-    const size_t need = ssa::plan_layout(p).total;
+    ssa::stream_prepare(p);
+    // a caller workspace must hold ssa_workspace_size() bytes, which cover
+    // every path a call of these sizes can take
+    const size_t need = p.h2 ? ssa::plan_layout(p).total : ssa::plan_bytes_any(p);
     void* own = nullptr;
     if (ws == nullptr) {
         if (ws_bytes != 0) return fail(SSA_ERR_WORKSPACE, "ws is NULL but ws_bytes != 0");
@@ -267,11 +364,12 @@ ssa_status run_with_ws(ssa::Plan& p, void* ws, size_t ws_bytes, cudaStream_t str
     attach_ws(p, ws);
     if (!own) {
         const ssa::WsLayout L = ssa::plan_layout(p);
-        cudaError_t e = prepare_ws(ws, fused_path(p), (size_t)ssa::ctrl_words(p) * 4, L.partials,
-                                   stream);
+        cudaError_t e = L.stream ? prepare_ws_stream(ws, L.total, stream)
+                                 : prepare_ws(ws, fused_path(p), (size_t)ssa::ctrl_words(p) * 4,
+                                              L.partials, stream);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(control words)");
     }
-    cudaError_t e = fused_path(p) ? ssa::launch_fused(p, stream) : ssa::launch_generic(p, stream);
+    cudaError_t e = launch_plan(p, stream);
     if (own) cudaFreeAsync(own, stream);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return SSA_OK;
@@ -413,6 +511,7 @@ ssa_status ssa_decode_noalloc(const ssa_shape* shape, const void* q, const void*
     st = check_tensors(p, {q, k_raw, v_raw, k_gist, v_gist, seq_lens, out});
     if (st != SSA_OK) return st;
     if (topk > 0 && !sel_idx) return fail(SSA_ERR_INVALID_ARG, "sel_idx is NULL");
+    ssa::stream_prepare(p);
     const ssa::WsLayout L = ssa::plan_layout(p);
     if (L.total > ssa::kBuiltinWsBytes)
         return fail(SSA_ERR_WORKSPACE,
@@ -432,11 +531,18 @@ ssa_status ssa_decode_noalloc(const ssa_shape* shape, const void* q, const void*
     p.sel_idx = sel_idx;
     p.out = out;
     attach_ws(p, ws);
-    // the area keeps whatever the previous call left: clear the part that
-    // must start at zero (control words and scores), stream-ordered
-    e = cudaMemsetAsync(ws, 0, L.partials, stream);
+    if (L.stream) {
+        // the streaming path's words carry the epoch of the launch that wrote
+        // them: the area is cleared only when another path used it last
+        e = prepare_ws_stream(ws, L.total, stream);
+    } else {
+        // the area keeps whatever the previous call left: clear the part
+        // that must start at zero (control words and scores), stream-ordered
+        note_ws_unknown(ws);
+        e = cudaMemsetAsync(ws, 0, L.partials, stream);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(built-in scratch)");
-    e = fused_path(p) ? ssa::launch_fused(p, stream) : ssa::launch_generic(p, stream);
+    e = launch_plan(p, stream);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return SSA_OK;
 }
@@ -475,7 +581,7 @@ ssa_status ssa_workspace_size(const ssa_shape* shape, int32_t C, int32_t g, int3
     ssa::Plan p;
     ssa_status st = build_single(p, shape, C, g, topk);
     if (st != SSA_OK) return st;
-    *bytes = ssa::plan_layout(p).total;
+    *bytes = ssa::plan_bytes_any(p);
     return SSA_OK;
 }
 
@@ -503,6 +609,7 @@ ssa_status ssa_get_device_status(int32_t* host_code, cudaStream_t stream) {
     int v = 0;
     cudaError_t e = ssa::read_device_status(&v, stream);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
+    if (v == SSA_ERR_DEVICE_TIMEOUT) note_timeout();
     *host_code = v;
     return SSA_OK;
 }

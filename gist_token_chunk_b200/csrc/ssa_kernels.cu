@@ -9,6 +9,7 @@
 #include "ssa_fused.cuh"
 #include "ssa_generic.cuh"
 #include "ssa_internal.h"
+#include "ssa_stream.cuh"
 
 namespace ssa {
 
@@ -24,14 +25,22 @@ int sm_count() {
     return n;
 }
 
+// The status word is taken (read and cleared) by one atomic exchange on the
+// device, so a status that a kernel on another stream sets in between is
+// either returned now or kept for the next read, never lost.
+static __device__ int g_status_taken = 0;
+
+__global__ void take_status_kernel() { g_status_taken = atomicExch(&g_device_status, 0); }
+
 cudaError_t read_device_status(int* code, cudaStream_t stream) {
-    cudaError_t e = cudaStreamSynchronize(stream);
+    take_status_kernel<<<1, 1, 0, stream>>>();
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     int v = 0;
-    e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
+    e = cudaMemcpyFromSymbolAsync(&v, g_status_taken, sizeof(int), 0, cudaMemcpyDeviceToHost,
+                                  stream);
     if (e != cudaSuccess) return e;
-    const int zero = 0;
-    e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+    e = cudaStreamSynchronize(stream);
     *code = v;
     return e;
 }
@@ -41,20 +50,42 @@ cudaError_t read_device_status(int* code, cudaStream_t stream) {
 // that entry point never allocates.  Every call shares it.
 static __device__ __align__(256) unsigned char g_builtin_ws[kBuiltinWsBytes];
 
+// The driver's current context: the area's device address belongs to it (a
+// device reset or a new primary context gives the area a new address).
+static void* current_context() {
+    using GetCtx = CUresult (*)(CUcontext*);
+    static GetCtx fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void* f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<GetCtx>(f);
+    });
+    CUcontext c = nullptr;
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
 cudaError_t builtin_workspace(void** ptr) {
     static std::mutex mu;
+    static void* ctx[64] = {nullptr};
     static void* addr[64] = {nullptr};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    void* c = current_context();
     std::lock_guard<std::mutex> lk(mu);
-    if (!addr[dev]) {
-        // first use on this device (which is current): look up the address
+    if (!addr[dev] || c == nullptr || ctx[dev] != c) {
+        // first use in this context (its device is current): look it up
+        // (the query also makes the device's primary context current)
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_builtin_ws);
         if (e != cudaSuccess) return e;
         addr[dev] = p;
+        ctx[dev] = current_context();
     }
     *ptr = addr[dev];
     return cudaSuccess;
@@ -76,13 +107,15 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// A [rows, d] bf16 row-major tensor as 64 x 64 boxes with 128-byte swizzle.
-static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int d) {
+// A [rows, d] bf16 row-major tensor as boxes of 64 columns x box_rows rows
+// with the 128-byte swizzle.
+static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int d,
+                     int box_rows = fused::kBoxRows) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)fused::kBoxRows};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -195,6 +228,81 @@ static cudaError_t launch_fused_d(const Plan& plan, cudaStream_t stream) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, p, m[0], m[1], m[2], m[3], m[4], m[5]);
+}
+
+// ------------------------------------------------------------- streaming ---
+
+bool stream_prepare(Plan& p) {
+    p.st_rcap = 0;
+    if (p.mode != kModeFull || p.h2 || p.dtype != 0 || p.d != stream::kD) return false;
+    if (p.G > stream::kMaxG || p.topk > stream::kMaxTopk || p.M_max > stream::kMaxChunks)
+        return false;
+    // opt-in while the per-warp streaming kernel is slower than the fused one
+    if (p.B > kFusedMaxB || !(p.debug_flags & 4)) return false;
+    const int nsm = sm_count();
+    if (nsm > stream::kMaxBlocks) return false;
+    // kept-logit rows of the largest chunk share (all sequences at n_max);
+    // with odd g every segment may take one row of alignment padding
+    const long long chunks = (long long)p.n_pairs * p.M_max;
+    const long long W = (long long)nsm * stream::kWorkers;
+    const long long parts = chunks < W ? chunks : W;
+    const long long per = parts > 0 ? (chunks + parts - 1) / parts : 1;
+    long long rows = per * (p.g + (p.g & 1));
+    if (rows < 32) rows = 32;
+    rows = (rows + 31) / 32 * 32;
+    if (rows > (1 << 16)) return false;
+    p.st_rcap = (int)rows;
+    p.st_sel_stride = stream::sel_stride(p.topk);
+    p.st_slot_bytes = stream::kRecBytes;
+    p.st_part_slots = stream::kMaxBlocks * stream::kWorkers + p.n_pairs;
+    if (stream::layout(p).total > 227 * 1024) {
+        p.st_rcap = 0;
+        return false;
+    }
+    return true;
+}
+
+void stream_ws_sizes(const Plan& p, size_t* hdr, size_t* scores, size_t* sel, size_t* sum,
+                     size_t* part) {
+    const size_t P = (size_t)p.n_pairs;
+    *hdr = 256;
+    *scores = P * stream::score_stride(p.M_max) * 8;
+    *sel = P * p.st_sel_stride * 8;
+    *sum = (size_t)p.st_part_slots * 8;
+    *part = 2 * (size_t)p.G * p.st_part_slots * p.st_slot_bytes;
+}
+
+cudaError_t launch_stream(const Plan& p, cudaStream_t stream) {
+    CUtensorMap m[4];
+    const uint64_t P = (uint64_t)p.n_pairs;
+    const bool ok = make_map(&m[0], p.k_gist, P * p.M_max * p.g, stream::kD, stream::kGistRows) &&
+                    make_map(&m[1], p.v_gist, P * p.M_max * p.g, stream::kD, stream::kGistRows) &&
+                    make_map(&m[2], p.k_raw, P * p.n_max, stream::kD, stream::kRawRows) &&
+                    make_map(&m[3], p.v_raw, P * p.n_max, stream::kD, stream::kRawRows);
+    if (!ok) return cudaErrorInvalidValue;
+    const int smem = stream::layout(p).total;
+    auto kern = stream::stream_kernel;
+    static int attr_done[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_done[dev] = 1;
+    }
+    // one block per SM, all resident at once (blocks wait on each other)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)sm_count());
+    cfg.blockDim = dim3(stream::kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p, m[0], m[1], m[2], m[3]);
 }
 
 cudaError_t launch_fused(const Plan& p, cudaStream_t stream) {
