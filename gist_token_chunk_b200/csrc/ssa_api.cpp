@@ -181,24 +181,23 @@ static WsLayout fused_layout(const Plan& p) {
     return L;
 }
 
-// The streaming path's areas (p prepared by stream_prepare); the header with
-// the epoch sits at offset 0 in every size, so any two calls of this path
-// agree on it.
-static WsLayout stream_layout(const Plan& p) {
+// The pipeline's areas (p prepared by pipe_prepare); the epoch header sits
+// at offset 0 in every size, so any two calls of this path agree on it.
+static WsLayout pipe_layout(const Plan& p) {
     WsLayout L;
-    size_t hdr, sc, sel, sum, part;
-    stream_ws_sizes(p, &hdr, &sc, &sel, &sum, &part);
+    size_t hdr, sc, lg, sel, part;
+    pipe_ws_sizes(p, &hdr, &sc, &lg, &sel, &part);
     size_t o = 0;
     auto take = [&](size_t bytes) {
         size_t at = o;
         o += (bytes + 255) / 256 * 256;
         return at;
     };
-    L.stream = true;
+    L.pipe = true;
     L.st_hdr = take(hdr);
-    L.st_scores = take(sc);
+    L.pp_scores = take(sc);
+    L.pp_logits = take(lg);
     L.st_sel = take(sel);
-    L.st_sum = take(sum);
     L.st_part = take(part);
     L.total = o;
     return L;
@@ -206,7 +205,7 @@ static WsLayout stream_layout(const Plan& p) {
 
 WsLayout plan_layout(const Plan& p) {
     Plan q = p;
-    if (stream_prepare(q)) return stream_layout(q);
+    if (pipe_prepare(q)) return pipe_layout(q);
     return fused_layout(p);
 }
 
@@ -214,8 +213,8 @@ size_t plan_bytes_any(const Plan& p) {
     size_t a = fused_layout(p).total;
     Plan q = p;
     q.mode = kModeFull;
-    if (stream_prepare(q)) {
-        const size_t b = stream_layout(q).total;
+    if (pipe_prepare(q)) {
+        const size_t b = pipe_layout(q).total;
         if (b > a) a = b;
     }
     return a;
@@ -228,11 +227,11 @@ namespace {
 void attach_ws(ssa::Plan& p, void* ws) {
     const ssa::WsLayout L = ssa::plan_layout(p);
     char* base = static_cast<char*>(ws);
-    if (L.stream) {
+    if (L.pipe) {
         p.st_hdr = reinterpret_cast<unsigned*>(base + L.st_hdr);
-        p.st_scores = reinterpret_cast<unsigned long long*>(base + L.st_scores);
+        p.pp_scores = reinterpret_cast<float*>(base + L.pp_scores);
+        p.pp_logits = reinterpret_cast<float*>(base + L.pp_logits);
         p.st_sel = reinterpret_cast<unsigned long long*>(base + L.st_sel);
-        p.st_sum = reinterpret_cast<unsigned long long*>(base + L.st_sum);
         p.st_part = base + L.st_part;
         return;
     }
@@ -253,7 +252,7 @@ void attach_ws(ssa::Plan& p, void* ws) {
 // (stream-ordered).
 struct WsState {
     int kind = 0;      // 0: zero up to `bytes`; 1: fused layout; 2: unknown;
-                       // 3: streaming path (up to `bytes`: zero or written by
+                       // 3: pipeline (up to `bytes`: zero or written by
                        //    that path, whose words carry an older epoch)
     size_t bytes = 0;  // kind 0: zeroed bytes; kind 1: zero prefix of the layout
     size_t ctrl = 0;   // kind 1: control bytes of the layout
@@ -295,11 +294,11 @@ cudaError_t prepare_ws(void* ws, bool fused, size_t ctrl_bytes, size_t clean_byt
     return zero ? cudaMemsetAsync(ws, 0, clean_bytes, stream) : cudaSuccess;
 }
 
-// Before a streaming-path call: its areas must hold zeros or words of an
+// Before a pipeline call: its areas must hold zeros or words of an
 // earlier launch of that path (whatever its sizes: the epoch header is at
 // offset 0 and only grows), so the workspace is zeroed only when it comes
 // from another path or is larger than what is known.
-cudaError_t prepare_ws_stream(void* ws, size_t need, cudaStream_t stream) {
+cudaError_t prepare_ws_pipe(void* ws, size_t need, cudaStream_t stream) {
     bool zero = false;
     {
         std::lock_guard<std::mutex> lk(g_ws_mu);
@@ -335,13 +334,13 @@ void note_ws_unknown(const void* ws) {
 }
 
 cudaError_t launch_plan(const ssa::Plan& p, cudaStream_t stream) {
-    if (p.st_rcap > 0) return ssa::launch_stream(p, stream);
+    if (p.pp_w3 > 0) return ssa::launch_pipe(p, stream);
     return fused_path(p) ? ssa::launch_fused(p, stream) : ssa::launch_generic(p, stream);
 }
 
 // Runs a workspace-using plan: caller workspace, or a stream-ordered one.
 ssa_status run_with_ws(ssa::Plan& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
-    ssa::stream_prepare(p);
+    ssa::pipe_prepare(p);
     // a caller workspace must hold ssa_workspace_size() bytes, which cover
     // every path a call of these sizes can take
     const size_t need = p.h2 ? ssa::plan_layout(p).total : ssa::plan_bytes_any(p);
@@ -364,7 +363,7 @@ ssa_status run_with_ws(ssa::Plan& p, void* ws, size_t ws_bytes, cudaStream_t str
     attach_ws(p, ws);
     if (!own) {
         const ssa::WsLayout L = ssa::plan_layout(p);
-        cudaError_t e = L.stream ? prepare_ws_stream(ws, L.total, stream)
+        cudaError_t e = L.pipe ? prepare_ws_pipe(ws, L.total, stream)
                                  : prepare_ws(ws, fused_path(p), (size_t)ssa::ctrl_words(p) * 4,
                                               L.partials, stream);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(control words)");
@@ -511,7 +510,7 @@ ssa_status ssa_decode_noalloc(const ssa_shape* shape, const void* q, const void*
     st = check_tensors(p, {q, k_raw, v_raw, k_gist, v_gist, seq_lens, out});
     if (st != SSA_OK) return st;
     if (topk > 0 && !sel_idx) return fail(SSA_ERR_INVALID_ARG, "sel_idx is NULL");
-    ssa::stream_prepare(p);
+    ssa::pipe_prepare(p);
     const ssa::WsLayout L = ssa::plan_layout(p);
     if (L.total > ssa::kBuiltinWsBytes)
         return fail(SSA_ERR_WORKSPACE,
@@ -531,10 +530,10 @@ ssa_status ssa_decode_noalloc(const ssa_shape* shape, const void* q, const void*
     p.sel_idx = sel_idx;
     p.out = out;
     attach_ws(p, ws);
-    if (L.stream) {
-        // the streaming path's words carry the epoch of the launch that wrote
+    if (L.pipe) {
+        // the pipeline's words carry the epoch of the launch that wrote
         // them: the area is cleared only when another path used it last
-        e = prepare_ws_stream(ws, L.total, stream);
+        e = prepare_ws_pipe(ws, L.total, stream);
     } else {
         // the area keeps whatever the previous call left: clear the part
         // that must start at zero (control words and scores), stream-ordered
@@ -573,6 +572,20 @@ ssa_status ssa_decode_h2(const ssa_shape* shape, const void* q, const void* k_ra
     p.sel_super = sel_super;
     p.out = out;
     return run_with_ws(p, ws, ws_bytes, stream);
+}
+
+ssa_status ssa_decode_path(const ssa_shape* shape, int32_t C, int32_t g, int32_t topk,
+                           int32_t* path) {
+    if (!path) return fail(SSA_ERR_INVALID_ARG, "path is NULL");
+    ssa::Plan p;
+    ssa_status st = build_single(p, shape, C, g, topk);
+    if (st != SSA_OK) return st;
+    p.mode = ssa::kModeFull;
+    if (ssa::pipe_prepare(p))
+        *path = SSA_PATH_PIPELINE;
+    else
+        *path = fused_path(p) ? SSA_PATH_FUSED : SSA_PATH_GENERIC;
+    return SSA_OK;
 }
 
 ssa_status ssa_workspace_size(const ssa_shape* shape, int32_t C, int32_t g, int32_t topk,

@@ -65,15 +65,16 @@ struct Plan {
     unsigned long long* cands = nullptr;  // [levels, kFusedMaxGrid + P, 32] segment lists
     float* out = nullptr;           // [B, Hq, d]
     int* ctrl = nullptr;            // control words
-    // streaming kernel (ssa_stream.cuh; st_rcap > 0 when a call takes it):
+    // two-kernel pipeline (ssa_pipe.cuh; pp_w3 > 0 when a call takes it):
     // workspace areas whose words carry the launch's epoch
     unsigned* st_hdr = nullptr;               // [0] epoch of the last launch, [1] blocks done
-    unsigned long long* st_scores = nullptr;  // [P, M_max rounded up to even] epoch << 32 | score
     unsigned long long* st_sel = nullptr;     // [P, st_sel_stride] epoch << 32 | chunk
-    unsigned long long* st_sum = nullptr;     // [st_part_slots] epoch << 32 | segment's 2nd key
     char* st_part = nullptr;                  // [2, G, st_part_slots] records of st_slot_bytes
     int st_sel_stride = 0, st_part_slots = 0, st_slot_bytes = 0;
-    int st_rcap = 0;                          // kept-logit rows per worker warp
+    int st_rcap = 0;                          // kept-logit rows per scoring worker warp
+    float* pp_scores = nullptr;               // [P, M_max rounded up to 8] chunk scores
+    float* pp_logits = nullptr;               // [P * M_max * g + 64, logit stride] kept logits
+    int pp_w1 = 0, pp_w3 = 0;                 // worker warps per block: scoring, attention
     long long wait_limit = 0;       // ns bound of every device-side wait
     int debug_flags = 0;
     // timeline trace (only written by builds compiled with SSA_TRACE)
@@ -85,13 +86,15 @@ struct Plan {
 struct WsLayout {
     size_t ctrl = 0, scores = 0, super_scores = 0, cand_scores = 0, chunk_mask = 0,
            super_mask = 0, cands = 0, partials = 0, total = 0;
-    // streaming path (stream = true): header, scores, selections, partials
-    bool stream = false;
-    size_t st_hdr = 0, st_scores = 0, st_sel = 0, st_sum = 0, st_part = 0;
+    // pipeline (pipe = true): epoch header, chunk scores, kept logits,
+    // selections, partials
+    bool pipe = false;
+    size_t st_hdr = 0, st_sel = 0, st_part = 0;
+    size_t pp_scores = 0, pp_logits = 0;
 };
 
 // Fills the decomposition fields of `p` (needs shapes) and the layout.  The
-// layout is the streaming path's when the plan takes it, else the fused or
+// layout is the pipeline's when the plan takes it, else the fused or
 // generic path's.
 void plan_decompose(Plan& p);
 WsLayout plan_layout(const Plan& p);
@@ -104,15 +107,14 @@ constexpr int kSegList = 32;
 // Whether a plan's layout holds the segment candidate lists.
 bool seg_lists(const Plan& p);
 
-// Streaming path (single level, bf16, d = 64, G <= 8, topk <= 128, at most
-// 2048 chunks per sequence): fills the st_* sizes of `p` and returns true
-// when the call takes it on the current device.
-bool stream_prepare(Plan& p);
-cudaError_t launch_stream(const Plan& p, cudaStream_t stream);
-// Workspace bytes of the streaming path's areas (header, scores, selections,
-// partials) for a prepared plan.
-void stream_ws_sizes(const Plan& p, size_t* hdr, size_t* scores, size_t* sel, size_t* sum,
-                     size_t* part);
+// Two-kernel pipeline (single level, bf16, d = 64, G <= 8, topk <= 128):
+// fills the pp_* and st_* sizes of `p` and returns true when the call takes
+// it on the current device.
+bool pipe_prepare(Plan& p);
+cudaError_t launch_pipe(const Plan& p, cudaStream_t stream);
+// Workspace bytes of the pipeline's areas for a prepared plan.
+void pipe_ws_sizes(const Plan& p, size_t* hdr, size_t* scores, size_t* logits, size_t* sel,
+                   size_t* part);
 
 // Fast fused path: bf16, d in {64, 128}.  Returns a cudaError_t.
 cudaError_t launch_fused(const Plan& p, cudaStream_t stream);

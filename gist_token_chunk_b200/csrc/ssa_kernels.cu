@@ -9,7 +9,7 @@
 #include "ssa_fused.cuh"
 #include "ssa_generic.cuh"
 #include "ssa_internal.h"
-#include "ssa_stream.cuh"
+#include "ssa_pipe.cuh"
 
 namespace ssa {
 
@@ -109,8 +109,28 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // A [rows, d] bf16 row-major tensor as boxes of 64 columns x box_rows rows
 // with the 128-byte swizzle.
+// A descriptor is a pure function of (base, rows, d, box rows): each host
+// thread keeps the last few it encoded, so a decode loop over the same
+// buffers encodes none.
+struct MapEntry {
+    const void* base;
+    uint64_t rows;
+    int d, box_rows;
+    CUtensorMap map;
+};
+constexpr int kMapCache = 16;
+thread_local MapEntry t_maps[kMapCache];
+thread_local int t_map_n = 0, t_map_next = 0;
+
 static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int d,
                      int box_rows = fused::kBoxRows) {
+    for (int i = 0; i < t_map_n; ++i) {
+        const MapEntry& e = t_maps[i];
+        if (e.base == base && e.rows == rows && e.d == d && e.box_rows == box_rows) {
+            *m = e.map;
+            return true;
+        }
+    }
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
@@ -120,7 +140,16 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int d,
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    if (r != CUDA_SUCCESS) return false;
+    MapEntry& e = t_maps[t_map_next];
+    e.base = base;
+    e.rows = rows;
+    e.d = d;
+    e.box_rows = box_rows;
+    e.map = *m;
+    t_map_next = (t_map_next + 1) % kMapCache;
+    if (t_map_n < kMapCache) ++t_map_n;
+    return true;
 }
 
 template <int D>
@@ -230,79 +259,98 @@ static cudaError_t launch_fused_d(const Plan& plan, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, kern, p, m[0], m[1], m[2], m[3], m[4], m[5]);
 }
 
-// ------------------------------------------------------------- streaming ---
+// -------------------------------------------------------------- pipeline ---
 
-bool stream_prepare(Plan& p) {
-    p.st_rcap = 0;
-    if (p.mode != kModeFull || p.h2 || p.dtype != 0 || p.d != stream::kD) return false;
-    if (p.G > stream::kMaxG || p.topk > stream::kMaxTopk || p.M_max > stream::kMaxChunks)
-        return false;
-    // opt-in while the per-warp streaming kernel is slower than the fused one
-    if (p.B > kFusedMaxB || !(p.debug_flags & 4)) return false;
+bool pipe_prepare(Plan& p) {
+    p.pp_w1 = p.pp_w3 = 0;
+    if (p.mode != kModeFull || p.h2 || p.dtype != 0 || p.d != pipe::kD) return false;
+    if (p.G > pipe::kMaxG || p.topk > 128 || p.M_max > 8192 || p.B > kFusedMaxB) return false;
+    if (p.debug_flags & 2) return false;  // the fused kernel, for comparisons
     const int nsm = sm_count();
-    if (nsm > stream::kMaxBlocks) return false;
-    // kept-logit rows of the largest chunk share (all sequences at n_max);
-    // with odd g every segment may take one row of alignment padding
+    if (nsm > pipe::kMaxBlocks) return false;
+    // scoring: 8 worker warps per block when the ring fits, else fewer; the
+    // row maxima of the largest chunk share stay in shared memory
     const long long chunks = (long long)p.n_pairs * p.M_max;
-    const long long W = (long long)nsm * stream::kWorkers;
-    const long long parts = chunks < W ? chunks : W;
-    const long long per = parts > 0 ? (chunks + parts - 1) / parts : 1;
-    long long rows = per * (p.g + (p.g & 1));
-    if (rows < 32) rows = 32;
-    rows = (rows + 31) / 32 * 32;
-    if (rows > (1 << 16)) return false;
-    p.st_rcap = (int)rows;
-    p.st_sel_stride = stream::sel_stride(p.topk);
-    p.st_slot_bytes = stream::kRecBytes;
-    p.st_part_slots = stream::kMaxBlocks * stream::kWorkers + p.n_pairs;
-    if (stream::layout(p).total > 227 * 1024) {
-        p.st_rcap = 0;
+    for (int w1 = pipe::kMaxWorkers; w1 >= 4; --w1) {
+        const long long W = (long long)nsm * w1;
+        const long long parts = chunks < W ? chunks : W;
+        const long long per = parts > 0 ? (chunks + parts - 1) / parts : 1;
+        const long long rows = (per * p.g + 31) / 32 * 32;
+        if (rows > (1 << 16)) return false;
+        p.st_rcap = (int)rows;
+        if (pipe::score_layout(p, w1).total <= 227 * 1024) {
+            p.pp_w1 = w1;
+            break;
+        }
+    }
+    for (int w3 = 6; w3 >= 3; --w3)
+        if (pipe::attn_layout(p, w3).total <= 227 * 1024) {
+            p.pp_w3 = w3;
+            break;
+        }
+    if (p.pp_w1 == 0 || p.pp_w3 == 0) {
+        p.pp_w1 = p.pp_w3 = 0;
         return false;
     }
+    p.st_slot_bytes = pipe::kRecBytes;
+    p.st_part_slots = pipe::kMaxBlocks * pipe::kMaxWorkers + p.n_pairs;
+    p.st_sel_stride = pipe::sel_stride(p.topk);
     return true;
 }
 
-void stream_ws_sizes(const Plan& p, size_t* hdr, size_t* scores, size_t* sel, size_t* sum,
-                     size_t* part) {
+void pipe_ws_sizes(const Plan& p, size_t* hdr, size_t* scores, size_t* logits, size_t* sel,
+                   size_t* part) {
     const size_t P = (size_t)p.n_pairs;
     *hdr = 256;
-    *scores = P * stream::score_stride(p.M_max) * 8;
+    *scores = P * pipe::score_row(p.M_max) * 4;
+    *logits = (P * p.M_max * p.g + 64) * pipe::logit_stride(p.G) * 4;
     *sel = P * p.st_sel_stride * 8;
-    *sum = (size_t)p.st_part_slots * 8;
     *part = 2 * (size_t)p.G * p.st_part_slots * p.st_slot_bytes;
 }
 
-cudaError_t launch_stream(const Plan& p, cudaStream_t stream) {
+cudaError_t launch_pipe(const Plan& p, cudaStream_t stream) {
     CUtensorMap m[4];
     const uint64_t P = (uint64_t)p.n_pairs;
-    const bool ok = make_map(&m[0], p.k_gist, P * p.M_max * p.g, stream::kD, stream::kGistRows) &&
-                    make_map(&m[1], p.v_gist, P * p.M_max * p.g, stream::kD, stream::kGistRows) &&
-                    make_map(&m[2], p.k_raw, P * p.n_max, stream::kD, stream::kRawRows) &&
-                    make_map(&m[3], p.v_raw, P * p.n_max, stream::kD, stream::kRawRows);
+    const bool ok = make_map(&m[0], p.k_gist, P * p.M_max * p.g, pipe::kD, pipe::kGistRows) &&
+                    make_map(&m[1], p.v_gist, P * p.M_max * p.g, pipe::kD, pipe::kGistRows) &&
+                    make_map(&m[2], p.k_raw, P * p.n_max, pipe::kD, pipe::kRawRows) &&
+                    make_map(&m[3], p.v_raw, P * p.n_max, pipe::kD, pipe::kRawRows);
     if (!ok) return cudaErrorInvalidValue;
-    const int smem = stream::layout(p).total;
-    auto kern = stream::stream_kernel;
     static int attr_done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        cudaError_t e = cudaFuncSetAttribute(pipe::score_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(pipe::attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     227 * 1024);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = 1;
     }
-    // one block per SM, all resident at once (blocks wait on each other)
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)sm_count());
-    cfg.blockDim = dim3(stream::kThreads);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, p, m[0], m[1], m[2], m[3]);
+    const unsigned nsm = (unsigned)sm_count();
+    // scoring: an ordinary launch (it follows whatever came before on the
+    // stream); attention: may start as scoring drains (programmatic
+    // dependent launch) and waits for it on the device before it reads the
+    // scoring results
+    cudaLaunchConfig_t c1 = {};
+    c1.gridDim = dim3(nsm);
+    c1.blockDim = dim3(32 * p.pp_w1);
+    c1.dynamicSmemBytes = (size_t)pipe::score_layout(p, p.pp_w1).total;
+    c1.stream = stream;
+    cudaError_t e = cudaLaunchKernelEx(&c1, pipe::score_kernel, p, m[0]);
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t c3 = {};
+    c3.gridDim = dim3(nsm);
+    c3.blockDim = dim3(32 * (p.pp_w3 + 1));
+    c3.dynamicSmemBytes = (size_t)pipe::attn_layout(p, p.pp_w3).total;
+    c3.stream = stream;
+    c3.attrs = pdl;
+    c3.numAttrs = 1;
+    return cudaLaunchKernelEx(&c3, pipe::attend_kernel, p, m[1], m[2], m[3]);
 }
 
 cudaError_t launch_fused(const Plan& p, cudaStream_t stream) {

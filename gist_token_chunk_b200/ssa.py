@@ -39,6 +39,10 @@ SSA_ERR_DEVICE_TIMEOUT = 6
 SSA_BF16 = 0
 SSA_FP32 = 1
 SSA_DEBUG_SKIP_PUBLISH = 1
+SSA_DEBUG_FUSED_PATH = 2
+SSA_PATH_GENERIC = 0
+SSA_PATH_FUSED = 1
+SSA_PATH_PIPELINE = 2
 
 
 class Shape(ctypes.Structure):
@@ -59,6 +63,7 @@ lib.ssa_decode_noalloc.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, 
 lib.ssa_decode_h2.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P,
                               _P, _P, _P, _S, _P]
 lib.ssa_workspace_size.argtypes = [_SH, _I, _I, _I, ctypes.POINTER(_S)]
+lib.ssa_decode_path.argtypes = [_SH, _I, _I, _I, ctypes.POINTER(_I)]
 lib.ssa_workspace_size_h2.argtypes = [_SH, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_S)]
 lib.ssa_workspace_init.argtypes = [_P, _S, _P]
 lib.ssa_get_device_status.argtypes = [ctypes.POINTER(_I), _P]
@@ -74,8 +79,8 @@ lib.ssa_last_error.argtypes = []
 lib.ssa_last_error.restype = ctypes.c_char_p
 lib.ssa_version.restype = _I
 for _f in ("ssa_score_gists", "ssa_topk_chunks", "ssa_sparse_decode", "ssa_decode",
-           "ssa_decode_noalloc", "ssa_decode_h2", "ssa_workspace_size", "ssa_workspace_size_h2",
-           "ssa_workspace_init", "ssa_get_device_status"):
+           "ssa_decode_path", "ssa_decode_noalloc", "ssa_decode_h2", "ssa_workspace_size",
+           "ssa_workspace_size_h2", "ssa_workspace_init", "ssa_get_device_status"):
     getattr(lib, _f).restype = _I
 
 
@@ -124,6 +129,15 @@ def _stream(stream) -> Optional[int]:
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
     return int(stream)
+
+
+def ssa_decode_path(shape: Shape, C: int, g: int, topk: int) -> int:
+    """SSA_PATH_PIPELINE, SSA_PATH_FUSED or SSA_PATH_GENERIC: the kernels
+    ssa_decode runs for these sizes on the current device."""
+    v = _I(0)
+    _check(lib.ssa_decode_path(ctypes.byref(shape), C, g, topk, ctypes.byref(v)),
+           "ssa_decode_path")
+    return int(v.value)
 
 
 def ssa_workspace_size(shape: Shape, C: int, g: int, topk: int) -> int:

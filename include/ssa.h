@@ -197,6 +197,25 @@ SSA_API ssa_status ssa_decode_h2(const ssa_shape* shape, const void* q, const vo
                          int32_t topk_chunk, float* out, int32_t* sel_super, int32_t* sel_idx,
                          void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/*
+ * ssa_decode_path -- which kernels ssa_decode runs for these sizes on the
+ * current device (a host-side query; nothing is launched):
+ *   SSA_PATH_PIPELINE  two kernels on the stream: gist scoring, then top-k,
+ *                      hybrid attention and combination (bf16, d = 64,
+ *                      G <= 8, topk <= 128, M_max <= 8192, B <= 128);
+ *   SSA_PATH_FUSED     one kernel for the whole step (other bf16 shapes with
+ *                      d = 64 or 128 and B <= 128);
+ *   SSA_PATH_GENERIC   the portable kernels (fp32, other d, larger B).
+ * All three compute the same selection and output up to fp32 summation
+ * order.  Errors: those of ssa_decode's size checks; path NULL ->
+ * SSA_ERR_INVALID_ARG.
+ */
+#define SSA_PATH_GENERIC 0
+#define SSA_PATH_FUSED 1
+#define SSA_PATH_PIPELINE 2
+SSA_API ssa_status ssa_decode_path(const ssa_shape* shape, int32_t C, int32_t g, int32_t topk,
+                                   int32_t* path);
+
 /* Workspace bytes needed by ssa_decode / ssa_sparse_decode for these sizes. */
 SSA_API ssa_status ssa_workspace_size(const ssa_shape* shape, int32_t C, int32_t g, int32_t topk,
                               size_t* bytes);
@@ -237,12 +256,18 @@ SSA_API void ssa_set_wait_limit(int64_t ns);
 SSA_API void ssa_set_tuning(int32_t max_blocks, int32_t rows_per_score_item);
 
 /*
- * Test hook: with SSA_DEBUG_SKIP_PUBLISH set, the selection step of
- * ssa_sparse_decode never publishes its "selection ready" flag, so every
- * attention block waits until its wait limit and the call reports
- * SSA_ERR_DEVICE_TIMEOUT through ssa_get_device_status.  0 disables.
+ * Test hooks (bit flags, process-wide, later launches; 0 disables all):
+ * SSA_DEBUG_SKIP_PUBLISH: the selection step of ssa_sparse_decode never
+ *   publishes its selection, so every attention worker waits until its wait
+ *   limit and the call reports SSA_ERR_DEVICE_TIMEOUT through
+ *   ssa_get_device_status.
+ * SSA_DEBUG_FUSED_PATH: single-level bf16 calls that would take the
+ *   two-kernel pipeline (d = 64, G <= 8, topk <= 128, M_max <= 8192) take the
+ *   one-kernel fused path instead, so the two can be compared.  Both compute
+ *   the same selection and the same output up to fp32 summation order.
  */
 #define SSA_DEBUG_SKIP_PUBLISH 1
+#define SSA_DEBUG_FUSED_PATH 2
 SSA_API void ssa_set_debug_flags(int32_t flags);
 
 SSA_API const char* ssa_status_string(ssa_status status);

@@ -44,6 +44,30 @@ def test_workspace_size_scales_with_problem():
     assert h2 > 0
 
 
+@pytest.mark.parametrize("kw,C,g,topk,flags,path", [
+    (dict(), 128, 8, 32, 0, ssa.SSA_PATH_PIPELINE),                   # the 128K batch workload
+    (dict(B=2, n_max=524288), 256, 8, 64, 0, ssa.SSA_PATH_PIPELINE),  # 512K
+    (dict(), 128, 8, 32, ssa.SSA_DEBUG_FUSED_PATH, ssa.SSA_PATH_FUSED),
+    (dict(d=128), 128, 8, 32, 0, ssa.SSA_PATH_FUSED),                 # d = 128
+    (dict(Hq=64, Hkv=4), 128, 8, 32, 0, ssa.SSA_PATH_FUSED),          # G = 16
+    (dict(dtype=ssa.SSA_FP32), 128, 8, 32, 0, ssa.SSA_PATH_GENERIC),
+    (dict(B=200, n_max=8192), 128, 8, 32, 0, ssa.SSA_PATH_GENERIC),   # B > 128
+])
+def test_decode_path(kw, C, g, topk, flags, path):
+    ssa.ssa_set_debug_flags(flags)
+    try:
+        assert ssa.ssa_decode_path(shape(**kw), C, g, topk) == path
+    finally:
+        ssa.ssa_set_debug_flags(0)
+
+
+def test_decode_path_rejects_bad_sizes():
+    v = ctypes.c_int32(-1)
+    assert ssa.lib.ssa_decode_path(ctypes.byref(shape(d=96)), 128, 8, 32,
+                                   ctypes.byref(v)) == ssa.SSA_ERR_UNSUPPORTED
+    assert ssa.lib.ssa_decode_path(ctypes.byref(shape()), 128, 8, 32, None) == ssa.SSA_ERR_INVALID_ARG
+
+
 @pytest.mark.parametrize("kw,C,g,topk,code", [
     (dict(Hq=30), 128, 8, 32, ssa.SSA_ERR_INVALID_ARG),          # Hq % Hkv
     (dict(d=96), 128, 8, 32, ssa.SSA_ERR_UNSUPPORTED),           # bf16 head dim

@@ -1,6 +1,6 @@
 """ssa_decode_noalloc (the entry point that uses the library's built-in
-scratch instead of a workspace) against ssa_decode, through the C ABI, on two
-calls in a row; and its size limit.  Collected last on purpose: it must pass
+scratch instead of a workspace) against the oracle and against ssa_decode,
+through the C ABI, on two calls in a row; and its size limit.  Collected last on purpose: it must pass
 alone in a fresh process and after every other test."""
 import ctypes
 
@@ -8,6 +8,7 @@ import pytest
 import torch
 
 from gist_token_chunk_b200.inputs import Workload, make_inputs
+from parity import check_single
 
 pytestmark = pytest.mark.gpu
 
@@ -24,14 +25,10 @@ def ssa():
     return mod
 
 
-def _inputs(seed):
-    x = make_inputs(W, seed=seed)
-    return {k: v.cuda() for k, v in x.items() if k != "planted_idx"}
-
-
-def test_noalloc_matches_decode_twice_in_a_row(ssa):
+def test_noalloc_matches_oracle_twice_in_a_row(ssa, orc):
     for seed in (5, 6):  # two calls in a row; the second finds the first's leftovers
-        x = _inputs(seed)
+        h = make_inputs(W, seed=seed)
+        x = {k: v.cuda() for k, v in h.items() if k != "planted_idx"}
         o_ref, s_ref = ssa.ssa_decode(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
                                       x["seq_lens"], W.C, W.g, W.topk)
         out = torch.empty(W.B, W.Hq, W.d, dtype=torch.float32, device="cuda")
@@ -40,6 +37,7 @@ def test_noalloc_matches_decode_twice_in_a_row(ssa):
                                x["seq_lens"], W.C, W.g, W.topk, out, sel)
         torch.cuda.synchronize()
         assert ssa.ssa_get_device_status() == 0
+        check_single(orc, h, W.C, W.g, W.topk, out, sel)
         assert torch.equal(sel, s_ref)
         assert (out - o_ref).abs().max().item() <= 1e-5
 
