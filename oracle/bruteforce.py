@@ -28,6 +28,12 @@ def _rank_key(scores: np.ndarray, i: int):
     return (v, -i)
 
 
+def _score_max(x: np.ndarray, axis=None):
+    """Maximum over logits in which a NaN never wins: the largest non-NaN
+    value, -inf when there is none (the NaN reading of the chunk score)."""
+    return np.where(np.isnan(x), -np.inf, x).max(axis=axis)
+
+
 def topk_subsets(scores: np.ndarray, cand, k: int):
     """Return the unique k-subset of ``cand`` that outranks its complement."""
     cand = list(cand)
@@ -77,7 +83,7 @@ def decode(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C, g, topk, sel=None):
             if M:
                 gk = k_gist[b, j, :M].reshape(M * g, d)        # [M*g, d]
                 s = (qg @ gk.T / np.sqrt(d)).reshape(G, M, g)  # [G, M, g]
-                scores[b, j, :M] = s.max(axis=(0, 2))
+                scores[b, j, :M] = _score_max(s, axis=(0, 2))
             if sel is None:
                 chosen = topk_subsets(scores[b, j], range(M), topk)
             else:
@@ -128,12 +134,12 @@ def decode_h2(q, k_raw, v_raw, k_gist, v_gist, k_meta, v_meta, seq_lens, C, g, J
             qg = q[b, j * G:(j + 1) * G]
             if S:
                 mk = k_meta[b, j, :S].reshape(S * gm, d)
-                s2[b, j, :S] = (qg @ mk.T / np.sqrt(d)).reshape(G, S, gm).max(axis=(0, 2))
+                s2[b, j, :S] = _score_max((qg @ mk.T / np.sqrt(d)).reshape(G, S, gm), axis=(0, 2))
             sup = topk_subsets(s2[b, j], range(S), topk_super)
             ss_out[b, j, :len(sup)] = sup
             cand = [x * J + i for x in sup for i in range(J)] + list(range(S * J, M))
             for m in cand:
-                s1[b, j, m] = (qg @ k_gist[b, j, m].T / np.sqrt(d)).max()
+                s1[b, j, m] = _score_max(qg @ k_gist[b, j, m].T / np.sqrt(d))
             chosen = topk_subsets(s1[b, j], cand, topk_chunk)
             sl_out[b, j, :len(chosen)] = chosen
             keys, vals = [], []

@@ -305,9 +305,49 @@ def pin_bad_length(orc):
     assert np.isfinite(o["out"][0]).all() and (o["sel_idx"][0] >= 0).all()
 
 
+def pin_nan_gist_key(orc):
+    """A NaN logit never wins a chunk's score maximum, and a chunk whose every
+    logit is NaN scores -inf, ranks last and is selected only when k reaches
+    it (ties to the lower index among the -inf chunks)."""
+    rng = np.random.default_rng(21)
+    B, Hq, Hkv, d, C, g, n_max = 1, 2, 1, 8, 4, 2, 32
+    c = _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, [31])   # M = 7, tail of 3
+    q = c["q"][0]
+    boost = (q.sum(0) / np.linalg.norm(q.sum(0))).astype(np.float32) * 6.0
+    # chunk 2: one gist row NaN, the other the clear winner -> still selected
+    c["k_gist"][0, 0, 2, 0] = boost
+    c["k_gist"][0, 0, 2, 1, 3] = np.nan
+    # chunk 5: every gist key NaN -> score -inf
+    c["k_gist"][0, 0, 5] = np.nan
+    o = orc.decode(*_args(c), C=C, g=g, topk=2)
+    r = bruteforce.decode(*_args(c), C=C, g=g, topk=2)
+    s = o["scores"][0, 0]
+    assert np.isfinite(s[2]) and s[2] == s.max()
+    assert s[5] == -np.inf
+    assert 2 in o["sel_idx"][0, 0] and 5 not in o["sel_idx"][0, 0]
+    assert np.array_equal(o["sel_idx"], r["sel_idx"]), (o["sel_idx"], r["sel_idx"])
+    # chunk 5's NaN gist keys are in the context (unselected): the output is NaN
+    assert np.isnan(o["out"]).all() and np.isnan(r["out"]).all()
+    # k = 6 of 7: chunk 5 is the one left out; k = 7: all chunks, a finite output
+    o6 = orc.decode(*_args(c), C=C, g=g, topk=6)
+    assert list(o6["sel_idx"][0, 0]) == [0, 1, 2, 3, 4, 6]
+    r6 = bruteforce.decode(*_args(c), C=C, g=g, topk=6)
+    assert np.array_equal(o6["sel_idx"], r6["sel_idx"])
+    o7 = orc.decode(*_args(c), C=C, g=g, topk=7)
+    r7 = bruteforce.decode(*_args(c), C=C, g=g, topk=7)
+    assert list(o7["sel_idx"][0, 0]) == list(range(7))
+    _close(o7["out"], r7["out"], 1e-12, "all selected around NaN gists")
+    # two all-NaN chunks tie at -inf: the lower index goes first
+    c["k_gist"][0, 0, 1] = np.nan
+    o6 = orc.decode(*_args(c), C=C, g=g, topk=6)
+    assert list(o6["sel_idx"][0, 0]) == [0, 1, 2, 3, 4, 6]
+    r6 = bruteforce.decode(*_args(c), C=C, g=g, topk=6)
+    assert np.array_equal(o6["sel_idx"], r6["sel_idx"])
+
+
 ALL_PINS = [
     pin_bruteforce_single, pin_given_selection, pin_ties, pin_dense_when_all_selected,
     pin_gists_when_none_selected, pin_single_token, pin_equal_keys_mean, pin_context_size,
     pin_parallel_query, pin_hand_example, pin_bruteforce_h2, pin_h2_reduces_to_single,
-    pin_bad_length,
+    pin_bad_length, pin_nan_gist_key,
 ]
