@@ -51,6 +51,7 @@ UNIT = "queries/s"
 DEFAULT_CONFIG = "llama1b_128k_var"
 NSETS = 4
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0  # B200 HBM3e as specified (DGX figure), for the spec-based fraction
 
 
 def log(*a):
@@ -249,6 +250,18 @@ def oracle_cores(pairs: int) -> int:
     return max(1, min(avail, pairs))
 
 
+def run_config(w, world: int, nsets: int) -> dict:
+    """The `config` of both arms' JSON lines (identical, so the two lines
+    describe the same workload and measurement)."""
+    return dict(config_of(w), global_batch=w.B * world,
+                l2=f"inputs larger than L2: {nsets} input sets rotate, each step follows "
+                   f"{nsets - 1} steps over other sets",
+                timing="GPU arm: CUDA-graph replays of the decode step, CUDA events on the "
+                       "launching stream, max over ranks; reference arm: wall clock around "
+                       "whole-batch oracle calls",
+                parallelism=f"dp{world} (independent sequences per GPU, no collective)")
+
+
 def config_of(w) -> dict:
     cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "n_max": w.n_max,
            "C": w.C, "g": w.g, "topk": w.topk}
@@ -264,7 +277,14 @@ def config_of(w) -> dict:
 # -------------------------------------------------------- reference arm ---
 
 def run_reference(args):
+    """The reference arm: the fp64 CPU oracle, as it stands, on the host
+    cores.  A step is one oracle call over a sample of the batch's sequences
+    (all their KV heads; OpenMP over the (sequence, KV head) pairs on every
+    core): the whole batch unless (steps + warmup) whole-batch calls would
+    exceed the time budget, then the fewest leading sequences (at least one)
+    that fit it."""
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
     w = WORKLOADS[args.config]
@@ -276,33 +296,43 @@ def run_reference(args):
             if k not in ("seq_lens", "planted_idx")}
     lens = inp["seq_lens"].numpy()
 
-    def step(i):
-        b = i % w.B
-        sl = {k: v[b:b + 1] for k, v in host.items()}
+    def call(nseq):
+        sl = {k: v[:nseq] for k, v in host.items()}
         if w.two_level:
             orc.decode_h2(sl["q"], sl["k_raw"], sl["v_raw"], sl["k_gist"], sl["v_gist"],
-                          sl["k_meta"], sl["v_meta"], lens[b:b + 1], C=w.C, g=w.g, J=w.J, gm=w.gm,
-                          topk_super=w.topk_super, topk_chunk=w.topk)
+                          sl["k_meta"], sl["v_meta"], lens[:nseq], C=w.C, g=w.g, J=w.J,
+                          gm=w.gm, topk_super=w.topk_super, topk_chunk=w.topk)
         else:
             orc.decode(sl["q"], sl["k_raw"], sl["v_raw"], sl["k_gist"], sl["v_gist"],
-                       lens[b:b + 1], C=w.C, g=w.g, topk=w.topk)
+                       lens[:nseq], C=w.C, g=w.g, topk=w.topk)
 
-    for i in range(args.warmup):
-        step(i)
     t0 = time.perf_counter()
-    for i in range(args.steps):
-        step(i)
+    call(w.B)  # one whole-batch call sizes the sample
+    t_batch = time.perf_counter() - t0
+    calls = args.steps + args.warmup
+    nseq = w.B
+    if calls * t_batch > args.ref_budget:
+        nseq = max(1, int(w.B * args.ref_budget / (calls * t_batch)))
+    for _ in range(args.warmup):
+        call(nseq)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        call(nseq)
     el = time.perf_counter() - t0
-    value = args.steps / el
-    cores = oracle_cores(w.Hkv)
+    value = args.steps * nseq / el
+    cores = oracle_cores(nseq * w.Hkv)
+    if nseq == w.B:
+        sample = f"each step = one oracle call over the whole batch ({w.B} sequences, all KV heads)"
+    else:
+        sample = (f"each step = one oracle call over the first {nseq} of the batch's {w.B} "
+                  "sequences (all KV heads)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": dict(config_of(w), parallelism="host cores (OpenMP over KV heads)"),
+            "config": run_config(w, world, args.sets),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": "each step = one sequence (all KV heads) of the workload, "
-                                       "cycling through the batch"},
+                             "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -320,6 +350,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
     ap.add_argument("--seed", type=int, default=1003)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-budget", type=float, default=150.0,
+                    help="reference arm: seconds its warm-up and timed calls may take")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=1000,
                     help="steps of the end-to-end measurement (0: skip it)")
@@ -378,6 +410,15 @@ def main():
             ssa.ssa_decode(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
                            x["seq_lens"], w.C, w.g, w.topk, out=outs[s], sel_idx=sels[s], ws=ws,
                            stream=stream)
+
+    if w.two_level:
+        path, kernel_name, launches_per_step = None, "ssa::fused::fused_kernel<64>", 1
+    else:
+        path = ssa.ssa_decode_path(shape, w.C, w.g, w.topk)
+        kernel_name, launches_per_step = {
+            ssa.SSA_PATH_PIPELINE: ("ssa::pipe::score_kernel + ssa::pipe::attend_kernel", 2),
+            ssa.SSA_PATH_FUSED: (f"ssa::fused::fused_kernel<{w.d}>", 1),
+        }.get(path, ("ssa::gen score, top-k and attend kernels", 3))
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize(dev)
@@ -465,10 +506,27 @@ def main():
         down_dev.append(packed([outs[s], sels[s]], dev))
         down_host.append(packed([outs[s], sels[s]], "cpu")[0])
 
+    # Copies run on their own streams so that step i+1's upload and step i's
+    # download overlap the decode kernels; events keep each set's buffers
+    # ordered: upload -> decode -> download -> the set's next upload/decode.
+    up_stream = torch.cuda.Stream(device=dev)
+    down_stream = torch.cuda.Stream(device=dev)
+    up_done = [torch.cuda.Event() for _ in range(NS)]
+    dec_done = [torch.cuda.Event() for _ in range(NS)]
+    down_done = [torch.cuda.Event() for _ in range(NS)]
+    for s in range(NS):
+        dec_done[s].record(stream)
+        down_done[s].record(stream)
+
     def e2e_step(i):
         s = i % NS
         dbuf, (q_dev, len_dev) = up_dev[s]
-        dbuf.copy_(up_host[s], non_blocking=True)
+        up_stream.wait_event(dec_done[s])       # the set's last decode has read q
+        with torch.cuda.stream(up_stream):
+            dbuf.copy_(up_host[s], non_blocking=True)
+        up_done[s].record(up_stream)
+        stream.wait_event(up_done[s])
+        stream.wait_event(down_done[s])         # the set's last output has been read back
         x = dict(sets[s], q=q_dev, seq_lens=len_dev)
         obuf, (o_dev, s_dev) = down_dev[s]
         if w.two_level:
@@ -480,21 +538,28 @@ def main():
             ssa.ssa_decode(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
                            x["seq_lens"], w.C, w.g, w.topk, out=o_dev, sel_idx=s_dev, ws=ws,
                            stream=stream)
-        down_host[s].copy_(obuf, non_blocking=True)
+        dec_done[s].record(stream)
+        down_stream.wait_event(dec_done[s])
+        with torch.cuda.stream(down_stream):
+            down_host[s].copy_(obuf, non_blocking=True)
+        down_done[s].record(down_stream)
 
     e2e_value = None
     if ek > 0:
         with torch.cuda.stream(stream):
             for i in range(NS):
                 e2e_step(i)
-        stream.synchronize()
+        torch.cuda.synchronize(dev)
         if pg:
             pg.barrier()
         torch.cuda.synchronize(dev)
         with torch.cuda.stream(stream):
             ev0.record(stream)
+            up_stream.wait_event(ev0)
             for i in range(ek):
                 e2e_step(i)
+            for s in range(NS):
+                stream.wait_event(down_done[s])
             ev1.record(stream)
         ev1.synchronize()
         e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), pg, dev)
@@ -507,21 +572,21 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": dict(config_of(w), global_batch=w.B * world,
-                       l2=f"{NS} input sets rotate (each step follows {NS - 1} steps over "
-                          "other sets; inputs larger than L2)",
-                       timing="CUDA-graph replays of the fused kernel, CUDA events, max over ranks",
-                       parallelism=f"dp{world} (independent sequences per GPU, no collective)"),
+        "config": run_config(w, world, NS),
         "hbm_gbs": achieved, "hbm_frac_of_peak": achieved / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_src} copy bandwidth",
+                     "spec_peak": SPEC_HBM_GBS, "frac_of_spec": achieved / SPEC_HBM_GBS,
                      "algorithmic_bytes_per_launch": int(bytes_per_launch),
                      "traffic": profiled_traffic(args.config),
-                     "kernel": "ssa::fused::fused_kernel<64>"},
-        "gpu_launches": args.steps,
+                     "kernel": kernel_name,
+                     "per": "decode step (every kernel of the step; their launches overlap)"},
+        "gpu_launches": args.steps * launches_per_step,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": ek,
-                "path": "ssa_decode per step (Python binding -> C ABI); query and lengths up in one pinned copy, output and selection back in one"},
+                "path": "ssa_decode per step (Python binding -> C ABI); query and lengths up "
+                        "in one pinned copy, output and selection back in one, each on its own "
+                        "stream so copies overlap the neighbouring steps' kernels"},
     }
     clk = sampler.summary()
     if clk is not None:

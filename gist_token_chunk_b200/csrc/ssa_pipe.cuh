@@ -325,6 +325,91 @@ __host__ __device__ inline AttnLayout attn_layout(const Plan& p, int workers) {
 
 // ------------------------------------------------------------ score kernel ---
 
+// Scoring on the CUDA cores (builds with SSA_SCORE_CUDA_CORES=1; the
+// default build scores on the tensor cores).  Eight lanes share a gist row,
+// each holding 8 of its 64 dims (one 16-byte load from the swizzled box) and
+// the same 8 dims of every head's query in fp32; four rows per pass, 16
+// passes per 64-row stage.  The 8 lanes' partial dot products are reduced
+// and spread by a butterfly of warp shuffles, so lane c of the row ends with
+// head c's logit; the row maximum over heads takes three more shuffles.
+#ifndef SSA_SCORE_CUDA_CORES
+#define SSA_SCORE_CUDA_CORES 0
+#endif
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
+// One 64-row stage: writes the kept logits of rows < nv (heads < G, log2
+// domain) and their row maxima (q.k / sqrt(d)).  NG: 4 or 8 (G <= NG).
+template <int NG>
+__device__ __forceinline__ void score_stage_cuda_cores(const Plan& p, uint32_t box, const float (&qv)[8][8],
+                                                       int nv, int G, int GP, float* lgrow,
+                                                       float* rmax_seg, float scale, float scale_log2) {
+    const int lane = threadIdx.x & 31, rq = lane >> 3, c = lane & 7;
+#pragma unroll 2
+    for (int t = 0; t < 16; ++t) {
+        const int r = 4 * t + rq;
+        const uint4 kw = lds_v4(box + swz(r, c));
+        float k[8];
+        k[0] = bf_lo(kw.x); k[1] = bf_hi(kw.x); k[2] = bf_lo(kw.y); k[3] = bf_hi(kw.y);
+        k[4] = bf_lo(kw.z); k[5] = bf_hi(kw.z); k[6] = bf_lo(kw.w); k[7] = bf_hi(kw.w);
+        float acc[NG];
+#pragma unroll
+        for (int h = 0; h < NG; ++h) {
+            float a = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) a = fmaf(k[i], qv[h][i], a);
+            acc[h] = a;
+        }
+        // butterfly reduce-scatter over the row's 8 lanes: lane c keeps head c
+        // (NG = 8) or head c & 3 (NG = 4) with the sum over all 64 dims
+        float x;
+        if constexpr (NG == 8) {
+            float v4[4], v2[2];
+            const bool b4 = c & 4, b2 = c & 2, b1 = c & 1;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float keep = b4 ? acc[i + 4] : acc[i], send = b4 ? acc[i] : acc[i + 4];
+                v4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float keep = b2 ? v4[i + 2] : v4[i], send = b2 ? v4[i] : v4[i + 2];
+                v2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+            }
+            const float keep = b1 ? v2[1] : v2[0], send = b1 ? v2[0] : v2[1];
+            x = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+        } else {
+            float v2[2];
+            const bool b2 = c & 2, b1 = c & 1;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float keep = b2 ? acc[i + 2] : acc[i], send = b2 ? acc[i] : acc[i + 2];
+                v2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+            }
+            const float keep = b1 ? v2[1] : v2[0], send = b1 ? v2[0] : v2[1];
+            x = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+            x += __shfl_xor_sync(0xffffffffu, x, 4);
+        }
+        const int h = NG == 8 ? c : (c & 3);
+        const bool valid = h < G && (NG == 8 || c < 4);
+        if (valid && r < nv) lgrow[(size_t)r * GP + h] = x * scale_log2;
+        float m = valid ? x : -INFINITY;
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        if (c == 0 && r < nv) rmax_seg[r] = m * scale;
+    }
+}
+
+
 // Grid: one block per SM, workers = blockDim.x / 32.  Each worker scores its
 // share of the CHUNKS list: per 64-row stage of gist keys, S^T = K.Q^T on the
 // tensor cores (keys as the M rows, the group's heads as N); each row's
@@ -374,9 +459,17 @@ __global__ void __launch_bounds__(256, 1)
     v.share(0, w, cur.x, cur.hi);
     int lbase = 0, ni = 0, nc = 0;
     bool more = true, dead = false;
+#if SSA_SCORE_CUDA_CORES
+    float qv[8][8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qv[h][i] = 0.f;
+#else
     uint32_t qf[4][2];
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) qf[kk][0] = qf[kk][1] = 0u;
+#endif
 
     for (;;) {
         while (more && !dead && ni < nc + kScoreStages) {
@@ -430,6 +523,24 @@ __global__ void __launch_bounds__(256, 1)
         const Desc d = desc[s];
         const uint32_t box = ring_s + s * kSlotBytes;
         const int nv = d.nvalid;
+#if SSA_SCORE_CUDA_CORES
+        if (d.flags & F_Q) {
+            const __nv_bfloat16* qsm = reinterpret_cast<const __nv_bfloat16*>(qs + s * L.qbytes);
+            const int c8 = 8 * (lane & 7);
+#pragma unroll
+            for (int h = 0; h < 8; ++h)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    qv[h][i] = h < G ? __bfloat162float(qsm[h * kD + c8 + i]) : 0.f;
+        }
+        {
+            float* lgrow = p.pp_logits + ((size_t)(d.pair * p.M_max + d.c0) * p.g + d.off) * GP;
+            if (G <= 4)
+                score_stage_cuda_cores<4>(p, box, qv, nv, G, GP, lgrow, rmax + d.lrow, scale, scale_log2);
+            else
+                score_stage_cuda_cores<8>(p, box, qv, nv, G, GP, lgrow, rmax + d.lrow, scale, scale_log2);
+        }
+#else
         if (d.flags & F_Q) {
             const uint8_t* qsm = qs + s * L.qbytes;
 #pragma unroll
@@ -493,6 +604,7 @@ __global__ void __launch_bounds__(256, 1)
                 if (rb < nv) rmax[d.lrow + rb] = vb[blk] * scale;
             }
         }
+#endif
         // the chunks whose last gist row this stage scored
         const int cb = p.g_shift >= 0 ? d.off >> p.g_shift : d.off / p.g;
         const int ce = (d.flags & F_LAST) ? d.nch
