@@ -56,13 +56,19 @@ def topk_subsets(scores: np.ndarray, cand, k: int):
 
 def _softmax_attend(qh: np.ndarray, K: np.ndarray, V: np.ndarray):
     d = qh.shape[-1]
+    if K.shape[0] == 0:  # an empty context attends to nothing
+        return np.zeros(d), -np.inf
     logits = K @ qh / np.sqrt(d)
     mx = logits.max()
     w = np.exp(logits - mx)
     return (w[:, None] * V).sum(0) / w.sum(), mx + np.log(w.sum())
 
 
-def decode(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C, g, topk, sel=None):
+def decode(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C, g, topk, sel=None, context=0, select=0):
+    """context 0: unselected gists + selected raw + tail; 1: selected gists +
+    selected raw + tail.  select 0: one top-k per KV head over the group's
+    maximum; 1: each query head's own top-k (its own query only), union over
+    the group (scores then per query head, sel_idx of G*topk entries)."""
     q = np.asarray(q, np.float64)
     k_raw, v_raw = np.asarray(k_raw, np.float64), np.asarray(v_raw, np.float64)
     k_gist, v_gist = np.asarray(k_gist, np.float64), np.asarray(v_gist, np.float64)
@@ -70,8 +76,9 @@ def decode(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C, g, topk, sel=None):
     Hkv, n_max = k_raw.shape[1], k_raw.shape[2]
     G = Hq // Hkv
     M_max = n_max // C
-    scores = np.full((B, Hkv, M_max), -np.inf)
-    sel_out = np.full((B, Hkv, topk), -1, np.int32)
+    cap = G * topk if select else topk
+    scores = np.full((B, Hq if select else Hkv, M_max), -np.inf)
+    sel_out = np.full((B, Hkv, cap), -1, np.int32)
     out = np.zeros((B, Hq, d))
     lse = np.full((B, Hq), -np.inf)
     ctx = np.zeros((B, Hkv), np.int32)
@@ -83,20 +90,27 @@ def decode(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C, g, topk, sel=None):
             if M:
                 gk = k_gist[b, j, :M].reshape(M * g, d)        # [M*g, d]
                 s = (qg @ gk.T / np.sqrt(d)).reshape(G, M, g)  # [G, M, g]
-                scores[b, j, :M] = _score_max(s, axis=(0, 2))
-            if sel is None:
-                chosen = topk_subsets(scores[b, j], range(M), topk)
-            else:
+                if select:
+                    scores[b, j * G:(j + 1) * G, :M] = _score_max(s, axis=2)
+                else:
+                    scores[b, j, :M] = _score_max(s, axis=(0, 2))
+            if sel is not None:
                 chosen = [int(c) for c in sel[b, j] if c >= 0]
+            elif select:
+                chosen = sorted(set().union(*[topk_subsets(scores[b, j * G + r], range(M), topk)
+                                              for r in range(G)]))
+            else:
+                chosen = topk_subsets(scores[b, j], range(M), topk)
             sel_out[b, j, :len(chosen)] = chosen
             keys, vals = [], []
             for m in range(M):
-                if m in chosen:
-                    keys.append(k_raw[b, j, m * C:(m + 1) * C])
-                    vals.append(v_raw[b, j, m * C:(m + 1) * C])
-                else:
+                picked = m in chosen
+                if context == 0 and not picked or context == 1 and picked:
                     keys.append(k_gist[b, j, m])
                     vals.append(v_gist[b, j, m])
+                if picked:
+                    keys.append(k_raw[b, j, m * C:(m + 1) * C])
+                    vals.append(v_raw[b, j, m * C:(m + 1) * C])
             keys.append(k_raw[b, j, M * C:n])
             vals.append(v_raw[b, j, M * C:n])
             K = np.concatenate(keys, 0)

@@ -27,6 +27,17 @@
  *     the remainder chunks that belong to no complete superchunk) + raw K/V
  *     of the selected chunks + tail;
  *   - seq_lens counts every cached raw token; all of them are visible.
+ * Variants (oracle_decode_v):
+ *   - context "selected only" (the sec. 3.3 wording "each selected chunk's
+ *     gist and raw tokens while excluding unselected chunks"): gist K/V and
+ *     raw K/V of the selected chunks + raw K/V of the tail; unselected
+ *     chunks contribute nothing;
+ *   - selection "per head + union" (App. A, "each head selecting chunks
+ *     independently before their union"): every query head scores the
+ *     chunks with its own query only (max over the chunk's g gist tokens of
+ *     q_h.k / sqrt(d)) and keeps its own top-k (ties to the lower index); the
+ *     KV head's selection is the union of its group's selections, ascending,
+ *     and every head of the group attends over the context it defines.
  *
  * Inputs are fp32 arrays (bf16 values convert to fp32 exactly); every sum,
  * product and exponential is fp64.  Layouts (row-major):
@@ -114,6 +125,21 @@ static double chunk_score(const oshape* s, const float* q, const float* k_gist, 
     double v = slot_score(s, q, b, j, r, s->g);
     free((void*)r);
     return v;
+}
+
+/* Per-head score of chunk m of KV head j (selection variant "per head +
+ * union", App. A): max over the chunk's g gist tokens of q_h.k * scale for
+ * the single query head h of the group. */
+static double head_score(const oshape* s, const float* q, const float* k_gist, int b, int j,
+                         int h, int m) {
+    const double sc = scale_of(s->d);
+    const float* qh = q + ((size_t)b * s->Hq + h) * s->d;
+    double best = -INFINITY;
+    for (int t = 0; t < s->g; ++t) {
+        double v = dot(qh, gist_row(s, k_gist, b, j, m, t), s->d) * sc;
+        if (v > best) best = v;
+    }
+    return best;
 }
 
 static double super_score(const oshape* s, const float* q, const float* k_meta, int S_max,
@@ -219,39 +245,50 @@ static int is_in(const int* sorted, int k, int m) {
 /* ----------------------------------------------------- single level path --- */
 
 /*
- * oracle_decode: the whole single-level decode step.
- *   scores  [B,Hkv,M_max]  chunk scores (-inf for m >= M_b)         (out)
- *   sel     [B,Hkv,topk]   selected chunks ascending, -1 padded     (in/out)
+ * oracle_decode_v: the whole single-level decode step, with the context and
+ * selection readings chosen by context_mode (0: unselected gists + selected
+ * raw + tail; 1: selected gists + selected raw + tail) and select_mode (0:
+ * one selection per KV head from the max over its group's heads; 1: per-head
+ * top-k, union over the group).
+ *   scores  [B,Hkv,M_max] (select_mode 0) or [B,Hq,M_max] (select_mode 1):
+ *           chunk scores, -inf for m >= M_b                          (out)
+ *   sel     [B,Hkv,cap]    selected chunks ascending, -1 padded; cap = topk
+ *                          (select_mode 0) or G * topk (select_mode 1) (in/out)
  *   out     [B,Hq,d]       attention output                         (out)
  *   lse     [B,Hq]         natural log-sum-exp of the logits         (out)
  *   ctx     [B,Hkv]        context size |X| of each (b, j)           (out)
  * force_sel != 0: `sel` is an input (a given selection, e.g. the GPU's at a
  * near tie) and only the attention step runs on it.
- * Returns 0, or -1 for a bad shape, or 1 + b for a bad seq_lens[b] (that
- * sequence's outputs are zero, its selections -1).
+ * Returns 0, or -1 for a bad shape or mode, or 1 + b for a bad seq_lens[b]
+ * (that sequence's outputs are zero, its selections -1).
  */
-int oracle_decode(int B, int Hq, int Hkv, int d, int n_max, int C, int g, int topk,
-                  const float* q, const float* k_raw, const float* v_raw, const float* k_gist,
-                  const float* v_gist, const int32_t* seq_lens, int force_sel, double* scores,
-                  int32_t* sel, double* out, double* lse, int32_t* ctx) {
+int oracle_decode_v(int B, int Hq, int Hkv, int d, int n_max, int C, int g, int topk,
+                    int context_mode, int select_mode, const float* q, const float* k_raw,
+                    const float* v_raw, const float* k_gist, const float* v_gist,
+                    const int32_t* seq_lens, int force_sel, double* scores, int32_t* sel,
+                    double* out, double* lse, int32_t* ctx) {
     oshape s = {B, Hq, Hkv, d, n_max, C, g};
     if (!ok_shape(&s) || topk < 0) return -1;
+    if (context_mode < 0 || context_mode > 1 || select_mode < 0 || select_mode > 1) return -1;
     const int G = Hq / Hkv;
     const int M_max = n_max / C;
+    const int cap = select_mode ? G * topk : topk;
     int bad = 0;
 #pragma omp parallel for collapse(2) schedule(dynamic)
     for (int b = 0; b < B; ++b) {
         for (int j = 0; j < Hkv; ++j) {
             const int n = seq_len(&s, seq_lens, b);
             const size_t pj = (size_t)b * Hkv + j;
-            double* sc = scores ? scores + pj * M_max : NULL;
-            int32_t* sl = sel + pj * (size_t)topk;
+            /* score rows of this pair: one (select_mode 0) or G (one per head) */
+            const int nrows = select_mode ? G : 1;
+            double* sc = scores ? scores + pj * (size_t)nrows * M_max : NULL;
+            int32_t* sl = sel + pj * (size_t)cap;
             if (n < 0) {
 #pragma omp critical
                 if (!bad || b + 1 < bad) bad = b + 1;
-                for (int m = 0; m < M_max && sc; ++m) sc[m] = -INFINITY;
+                for (int m = 0; m < nrows * M_max && sc; ++m) sc[m] = -INFINITY;
                 if (!force_sel)
-                    for (int c = 0; c < topk; ++c) sl[c] = -1;
+                    for (int c = 0; c < cap; ++c) sl[c] = -1;
                 for (int gh = 0; gh < G; ++gh) {
                     const size_t h = (size_t)b * Hq + (size_t)j * G + gh;
                     for (int i = 0; i < d; ++i) out[h * d + i] = 0.0;
@@ -263,31 +300,52 @@ int oracle_decode(int B, int Hq, int Hkv, int d, int n_max, int C, int g, int to
             const int M = n / C;       /* complete chunks */
             const int tail0 = M * C;   /* first tail token */
             double* own = (double*)malloc(sizeof(double) * (size_t)(M_max > 0 ? M_max : 1));
-            for (int m = 0; m < M_max; ++m) own[m] = -INFINITY;
-            for (int m = 0; m < M; ++m) own[m] = chunk_score(&s, q, k_gist, b, j, m);
-            if (sc)
-                for (int m = 0; m < M_max; ++m) sc[m] = own[m];
-            int* chosen = (int*)malloc(sizeof(int) * (size_t)(topk > 0 ? topk : 1));
-            int k;
-            if (force_sel) {
-                k = 0;
-                for (int c = 0; c < topk; ++c)
-                    if (sl[c] >= 0) chosen[k++] = sl[c];
-            } else {
-                int* all = (int*)malloc(sizeof(int) * (size_t)(M > 0 ? M : 1));
-                for (int m = 0; m < M; ++m) all[m] = m;
-                k = topk_of(own, all, M, topk, chosen, topk);
-                for (int c = 0; c < topk; ++c) sl[c] = chosen[c];
-                free(all);
+            int* chosen = (int*)malloc(sizeof(int) * (size_t)(cap > 0 ? cap : 1));
+            int* all = (int*)malloc(sizeof(int) * (size_t)(M > 0 ? M : 1));
+            for (int m = 0; m < M; ++m) all[m] = m;
+            if (!force_sel)
+                for (int c = 0; c < cap; ++c) sl[c] = -1;
+            int nch = 0; /* select_mode 1: size of the union so far, in chosen[] */
+            for (int r = 0; r < nrows; ++r) {
+                /* select_mode 0: the group's score; 1: query head j*G + r's own */
+                for (int m = 0; m < M_max; ++m) own[m] = -INFINITY;
+                for (int m = 0; m < M; ++m)
+                    own[m] = select_mode ? head_score(&s, q, k_gist, b, j, j * G + r, m)
+                                         : chunk_score(&s, q, k_gist, b, j, m);
+                if (sc)
+                    for (int m = 0; m < M_max; ++m) sc[(size_t)r * M_max + m] = own[m];
+                if (force_sel) continue;
+                if (!select_mode) {
+                    topk_of(own, all, M, topk, sl, topk);
+                } else if (r == 0 || !MUT(12)) { /* mutant 12: union of head 0 only */
+                    int* mine = (int*)malloc(sizeof(int) * (size_t)(topk > 0 ? topk : 1));
+                    const int kh = topk_of(own, all, M, topk, mine, topk);
+                    for (int c = 0; c < kh; ++c)
+                        if (!is_in(chosen, nch, mine[c])) chosen[nch++] = mine[c];
+                    free(mine);
+                }
             }
-            /* context list (sec. 3.3, reading above) */
-            const int cap = (M * g) + k * C + C + 8;
-            const float** ks = (const float**)malloc(sizeof(float*) * (size_t)cap);
-            const float** vs = (const float**)malloc(sizeof(float*) * (size_t)cap);
+            if (select_mode && !force_sel) {
+                qsort(chosen, (size_t)nch, sizeof(int), cmp_int);
+                for (int c = 0; c < cap; ++c) sl[c] = c < nch ? chosen[c] : -1;
+            }
+            int k = 0;
+            for (int c = 0; c < cap; ++c)
+                if (sl[c] >= 0) chosen[k++] = sl[c];
+            free(all);
+            /* context list (sec. 3.3, reading above, or the variant) */
+            const int xcap = (M * g) + M * C + C + 8;
+            const float** ks = (const float**)malloc(sizeof(float*) * (size_t)xcap);
+            const float** vs = (const float**)malloc(sizeof(float*) * (size_t)xcap);
             int nx = 0;
             for (int m = 0; m < M; ++m) {
                 const int selected = is_in(chosen, k, m);
-                if (!selected || MUT(4)) { /* mutant 4: selected chunks keep their gists */
+                int gists;
+                if (!context_mode)
+                    gists = !selected || MUT(4); /* mutant 4: selected chunks keep their gists */
+                else
+                    gists = selected && !MUT(13); /* mutant 13: variant drops selected gists */
+                if (gists) {
                     for (int t = 0; t < g; ++t) {
                         ks[nx] = gist_row(&s, k_gist, b, j, m, t);
                         vs[nx] = gist_row(&s, v_gist, b, j, m, t);
@@ -312,6 +370,16 @@ int oracle_decode(int B, int Hq, int Hkv, int d, int n_max, int C, int g, int to
         }
     }
     return bad;
+}
+
+/* oracle_decode: the step under the default readings (context_mode 0,
+ * select_mode 0), sel [B,Hkv,topk]. */
+int oracle_decode(int B, int Hq, int Hkv, int d, int n_max, int C, int g, int topk,
+                  const float* q, const float* k_raw, const float* v_raw, const float* k_gist,
+                  const float* v_gist, const int32_t* seq_lens, int force_sel, double* scores,
+                  int32_t* sel, double* out, double* lse, int32_t* ctx) {
+    return oracle_decode_v(B, Hq, Hkv, d, n_max, C, g, topk, 0, 0, q, k_raw, v_raw, k_gist,
+                           v_gist, seq_lens, force_sel, scores, sel, out, lse, ctx);
 }
 
 /* ------------------------------------------------------- two level path --- */

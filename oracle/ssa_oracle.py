@@ -79,6 +79,7 @@ class Oracle:
         self.path = path or build(mutant)
         self.lib = ctypes.CDLL(self.path)
         self.lib.oracle_decode.restype = ctypes.c_int
+        self.lib.oracle_decode_v.restype = ctypes.c_int
         self.lib.oracle_decode_h2.restype = ctypes.c_int
         self.lib.oracle_mutant_id.restype = ctypes.c_int
 
@@ -87,28 +88,36 @@ class Oracle:
         return int(self.lib.oracle_mutant_id())
 
     def decode(self, q, k_raw, v_raw, k_gist, v_gist, seq_lens, C: int, g: int, topk: int,
-               sel: Optional[np.ndarray] = None) -> dict:
-        """Single-level decode step.  ``sel`` given => attend on that selection."""
+               sel: Optional[np.ndarray] = None, context: int = 0, select: int = 0) -> dict:
+        """Single-level decode step.  ``sel`` given => attend on that selection.
+
+        context 0: unselected gists + selected raw + tail; 1: selected gists +
+        selected raw + tail (sec. 3.3 wording).  select 0: one selection per KV
+        head (max over the group's heads); 1: per-head top-k, union over the
+        group (App. A) -- then scores are per query head [B,Hq,M_max] and
+        sel_idx has G*topk entries per KV head."""
         q, k_raw, v_raw = _f32(q), _f32(k_raw), _f32(v_raw)
         k_gist, v_gist = _f32(k_gist), _f32(v_gist)
         lens = _i32(seq_lens)
         B, Hq, d = q.shape
         Hkv, n_max = k_raw.shape[1], k_raw.shape[2]
         M_max = n_max // C
+        G = Hq // Hkv
         assert k_gist.shape == (B, Hkv, M_max, g, d), (k_gist.shape, (B, Hkv, M_max, g, d))
-        scores = np.empty((B, Hkv, M_max), np.float64)
+        scores = np.empty((B, Hq if select else Hkv, M_max), np.float64)
         out = np.empty((B, Hq, d), np.float64)
         lse = np.empty((B, Hq), np.float64)
         ctx = np.empty((B, Hkv), np.int32)
+        cap = G * topk if select else topk
         force = sel is not None
-        sel_arr = (_i32(sel).copy() if force else np.empty((B, Hkv, topk), np.int32))
-        assert sel_arr.shape == (B, Hkv, topk)
-        rc = self.lib.oracle_decode(
-            B, Hq, Hkv, d, n_max, C, g, topk, _p(q, _F), _p(k_raw, _F), _p(v_raw, _F),
-            _p(k_gist, _F), _p(v_gist, _F), _p(lens, _I), int(force), _p(scores, _D),
-            _p(sel_arr, _I), _p(out, _D), _p(lse, _D), _p(ctx, _I))
+        sel_arr = (_i32(sel).copy() if force else np.empty((B, Hkv, cap), np.int32))
+        assert sel_arr.shape == (B, Hkv, cap), (sel_arr.shape, (B, Hkv, cap))
+        rc = self.lib.oracle_decode_v(
+            B, Hq, Hkv, d, n_max, C, g, topk, int(context), int(select), _p(q, _F),
+            _p(k_raw, _F), _p(v_raw, _F), _p(k_gist, _F), _p(v_gist, _F), _p(lens, _I),
+            int(force), _p(scores, _D), _p(sel_arr, _I), _p(out, _D), _p(lse, _D), _p(ctx, _I))
         if rc < 0:
-            raise ValueError("oracle_decode: bad shape or topk")
+            raise ValueError("oracle_decode_v: bad shape, topk or mode")
         return {"scores": scores, "sel_idx": sel_arr, "out": out, "lse": lse, "ctx": ctx,
                 "bad_seq": rc}
 

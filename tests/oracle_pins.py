@@ -345,9 +345,117 @@ def pin_nan_gist_key(orc):
     assert np.array_equal(o6["sel_idx"], r6["sel_idx"])
 
 
+VARIANT_CASES = [
+    # (B, Hq, Hkv, d, C, g, n_max, seq_lens, topk)
+    (1, 4, 1, 8, 4, 2, 32, [30], 2),
+    (2, 4, 2, 8, 4, 2, 40, [40, 27], 3),
+    (1, 6, 2, 8, 5, 3, 45, [44], 2),
+    (2, 2, 2, 8, 3, 2, 30, [30, 7], 20),   # topk > M: every chunk
+    (1, 4, 2, 8, 4, 2, 16, [3], 2),        # M = 0: tail only
+    (2, 8, 2, 8, 4, 2, 24, [23, 24], 0),   # topk = 0
+]
+
+
+def pin_variants_bruteforce(orc):
+    """Both context readings and both selection readings against the brute
+    force (dense scoring, subset-enumeration top-k, explicit token list)."""
+    rng = np.random.default_rng(4321)
+    for (B, Hq, Hkv, d, C, g, n_max, lens, topk) in VARIANT_CASES:
+        c = _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, lens)
+        for context in (0, 1):
+            for select in (0, 1):
+                o = orc.decode(*_args(c), C=C, g=g, topk=topk, context=context, select=select)
+                r = bruteforce.decode(*_args(c), C=C, g=g, topk=topk, context=context,
+                                      select=select)
+                what = f"context={context} select={select} case={(B, Hq, Hkv, C, g, lens, topk)}"
+                _close(o["scores"], r["scores"], 1e-12, "scores " + what)
+                assert np.array_equal(o["sel_idx"], r["sel_idx"]), ("sel " + what, o["sel_idx"],
+                                                                   r["sel_idx"])
+                assert np.array_equal(o["ctx"], r["ctx"]), ("ctx " + what, o["ctx"], r["ctx"])
+                _close(o["out"], r["out"], 1e-12, "out " + what)
+                _close(o["lse"], r["lse"], 1e-12, "lse " + what)
+
+
+def pin_selected_only_closed_forms(orc):
+    """Context "selected only": |X| = k (C + g) + T; with k = M it is textbook
+    attention over every raw token and every gist token; with k = 0 it is
+    attention over the tail alone (an empty context gives 0 and lse -inf)."""
+    rng = np.random.default_rng(77)
+    B, Hq, Hkv, d, C, g, n_max = 2, 4, 2, 8, 4, 2, 40
+    c = _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, [38, 32])
+    G = Hq // Hkv
+    for topk in (0, 2, 5, 10):
+        o = orc.decode(*_args(c), C=C, g=g, topk=topk, context=1)
+        for b, n in enumerate(c["seq_lens"]):
+            M, T = int(n) // C, int(n) % C
+            k = min(topk, M)
+            assert (o["ctx"][b] == k * (C + g) + T).all(), (topk, b, o["ctx"][b])
+    o = orc.decode(*_args(c), C=C, g=g, topk=10, context=1)
+    for b, n in enumerate(c["seq_lens"]):
+        n = int(n)
+        M = n // C
+        for h in range(Hq):
+            j = h // G
+            K = np.concatenate([c["k_raw"][b, j, :n], c["k_gist"][b, j, :M].reshape(-1, d)])
+            V = np.concatenate([c["v_raw"][b, j, :n], c["v_gist"][b, j, :M].reshape(-1, d)])
+            ref, lse = _sdpa(c["q"][b, h], K, V)
+            _close(o["out"][b, h], ref, 1e-12, "selected-only, k = M")
+            _close(o["lse"][b, h], lse, 1e-12, "selected-only lse, k = M")
+    o0 = orc.decode(*_args(c), C=C, g=g, topk=0, context=1)
+    for b, n in enumerate(c["seq_lens"]):
+        n = int(n)
+        M = n // C
+        for h in range(Hq):
+            j = h // G
+            if n == M * C:
+                assert (o0["out"][b, h] == 0).all() and o0["lse"][b, h] == -np.inf
+            else:
+                ref, _ = _sdpa(c["q"][b, h], c["k_raw"][b, j, M * C:n], c["v_raw"][b, j, M * C:n])
+                _close(o0["out"][b, h], ref, 1e-12, "selected-only, k = 0")
+
+
+def pin_union_reductions(orc):
+    """Per-head selection + union: with one query head per KV head it is the
+    shared selection; with equal queries in a group every head picks the
+    shared top-k, so the union is it; in general the union holds every head's
+    own top-k of its own scores and has between k and min(G k, M) chunks."""
+    rng = np.random.default_rng(5)
+    # G = 1
+    c = _rand_case(rng, 2, 3, 3, 8, 4, 2, 40, [40, 29])
+    for context in (0, 1):
+        a = orc.decode(*_args(c), C=4, g=2, topk=3, context=context, select=0)
+        u = orc.decode(*_args(c), C=4, g=2, topk=3, context=context, select=1)
+        assert np.array_equal(a["sel_idx"], u["sel_idx"])
+        _close(u["out"], a["out"], 1e-12, "union with G = 1")
+        _close(u["scores"], a["scores"], 1e-12, "per-head scores with G = 1")
+    # equal queries in each group
+    c = _rand_case(rng, 1, 8, 2, 8, 4, 2, 48, [46])
+    c["q"][0, 1:4] = c["q"][0, 0]
+    c["q"][0, 5:8] = c["q"][0, 4]
+    a = orc.decode(*_args(c), C=4, g=2, topk=4, select=0)
+    u = orc.decode(*_args(c), C=4, g=2, topk=4, select=1)
+    assert np.array_equal(u["sel_idx"][..., :4], a["sel_idx"]) and (u["sel_idx"][..., 4:] == -1).all()
+    _close(u["out"], a["out"], 1e-12, "union of equal heads")
+    # general: containment and size
+    c = _rand_case(rng, 2, 8, 2, 8, 4, 2, 64, [64, 50])
+    topk = 3
+    u = orc.decode(*_args(c), C=4, g=2, topk=topk, select=1)
+    G = 4
+    for b, n in enumerate(c["seq_lens"]):
+        M = int(n) // 4
+        for j in range(2):
+            chosen = [int(x) for x in u["sel_idx"][b, j] if x >= 0]
+            assert chosen == sorted(set(chosen))
+            assert min(topk, M) <= len(chosen) <= min(G * topk, M)
+            for r in range(G):
+                own = bruteforce.topk_subsets(u["scores"][b, j * G + r], range(M), topk)
+                assert set(own) <= set(chosen), (b, j, r, own, chosen)
+
+
 ALL_PINS = [
     pin_bruteforce_single, pin_given_selection, pin_ties, pin_dense_when_all_selected,
     pin_gists_when_none_selected, pin_single_token, pin_equal_keys_mean, pin_context_size,
     pin_parallel_query, pin_hand_example, pin_bruteforce_h2, pin_h2_reduces_to_single,
-    pin_bad_length, pin_nan_gist_key,
+    pin_bad_length, pin_nan_gist_key, pin_variants_bruteforce, pin_selected_only_closed_forms,
+    pin_union_reductions,
 ]
