@@ -178,3 +178,68 @@ def decode_h2(q, k_raw, v_raw, k_gist, v_gist, k_meta, v_meta, seq_lens, C, g, J
                 out[b, h], lse[b, h] = _softmax_attend(q[b, h], K, V)
     return {"super_scores": s2, "scores": s1, "sel_super": ss_out, "sel_idx": sl_out,
             "out": out, "lse": lse, "ctx": ctx}
+
+
+def decode_hier(q, k_raw, v_raw, k_gist, v_gist, k_sum, v_sum, seq_lens, C, g, J, topks):
+    """t-level coarse-to-fine step, written as a recursion over kept units:
+    a unit is scored when its parent was kept (or it is a top-level unit, or
+    a remainder unit that lies in no complete parent), each level keeps its
+    top-k by subset enumeration, and the context is built as an explicit
+    token list (summaries of unkept candidates, gists of unkept candidate
+    chunks, raw tokens of kept chunks, the tail)."""
+    q = np.asarray(q, np.float64)
+    k_raw, v_raw = np.asarray(k_raw, np.float64), np.asarray(v_raw, np.float64)
+    k_gist, v_gist = np.asarray(k_gist, np.float64), np.asarray(v_gist, np.float64)
+    k_sum = [np.asarray(x, np.float64) for x in k_sum]
+    v_sum = [np.asarray(x, np.float64) for x in v_sum]
+    t = len(topks)
+    B, Hq, d = q.shape
+    Hkv, n_max = k_raw.shape[1], k_raw.shape[2]
+    G = Hq // Hkv
+    sels = [np.full((B, Hkv, k), -1, np.int32) for k in topks]
+    out = np.zeros((B, Hq, d))
+    ctx = np.zeros((B, Hkv), np.int32)
+    for b in range(B):
+        n = int(seq_lens[b])
+        M = n // C
+        U = [M]
+        for _ in range(1, t):
+            U.append(U[-1] // J)
+        for j in range(Hkv):
+            qg = q[b, j * G:(j + 1) * G]
+
+            def keys_of(level, x):  # level 1-based
+                return k_gist[b, j, x] if level == 1 else k_sum[level - 2][b, j, x]
+
+            def vals_of(level, x):
+                return v_gist[b, j, x] if level == 1 else v_sum[level - 2][b, j, x]
+
+            keys, vals = [], []
+            kept = []
+            for level in range(t, 0, -1):
+                if level == t:
+                    cand = list(range(U[level - 1]))
+                else:
+                    cand = [x * J + i for x in kept for i in range(J)]
+                    cand += list(range(U[level] * J, U[level - 1]))
+                sc = np.full(max(U[level - 1], 1), -np.inf)
+                for x in cand:
+                    sc[x] = _score_max(qg @ keys_of(level, x).T / np.sqrt(d))
+                keep = topk_subsets(sc, cand, topks[level - 1])
+                sels[level - 1][b, j, :len(keep)] = keep
+                for x in cand:
+                    if level == 1 and x in keep:
+                        keys.append(k_raw[b, j, x * C:(x + 1) * C])
+                        vals.append(v_raw[b, j, x * C:(x + 1) * C])
+                    elif x not in keep:
+                        keys.append(keys_of(level, x))
+                        vals.append(vals_of(level, x))
+                kept = keep
+            keys.append(k_raw[b, j, M * C:n])
+            vals.append(v_raw[b, j, M * C:n])
+            K = np.concatenate(keys, 0)
+            V = np.concatenate(vals, 0)
+            ctx[b, j] = K.shape[0]
+            for gh in range(G):
+                out[b, j * G + gh] = _softmax_attend(q[b, j * G + gh], K, V)[0]
+    return {"sels": sels, "out": out, "ctx": ctx}

@@ -526,4 +526,159 @@ int oracle_decode_h2(int B, int Hq, int Hkv, int d, int n_max, int C, int g, int
     return bad;
 }
 
+/* ------------------------------------------------------ t level path --- */
+
+/*
+ * oracle_decode_hier: coarse-to-fine selection over `levels` = t levels
+ * (sec. 3.5, "additional hierarchy levels can be added as context grows";
+ * App. B.2, t = ceil(log_J M) levels), the two-level reading applied level by
+ * level.  Level-1 units are the chunks (g gist tokens each).  A level-l unit
+ * (l >= 2) groups J level-(l-1) units and has gs[l-2] summary tokens in
+ * k_sum[l-2], v_sum[l-2] laid out [B,Hkv,Umax(l),gs[l-2],d] with Umax(l) =
+ * M_max / J^(l-1).  Complete units: U_1 = M_b, U_l = floor(U_{l-1} / J).
+ * From the top: the candidates of level t are its U_t units; those of level
+ * l < t are the J children of every unit kept at level l+1 (ascending), then
+ * the remainder units U_{l+1} J .. U_l - 1, which lie in no complete parent.
+ * Each level keeps the topks[l-1] best candidates (score = max over the
+ * group's query heads and the unit's summary tokens of q.k/sqrt(d); ties to
+ * the lower index).  Context: the summary tokens of every unkept candidate
+ * at levels >= 2, the gists of the unkept candidate chunks, the raw tokens of
+ * the kept chunks and the raw tail.
+ *   scores[l-1] [B,Hkv,Umax(l)]  candidate scores, -inf elsewhere      (out)
+ *   sels[l-1]   [B,Hkv,topks[l-1]] kept units ascending, -1 padded  (in/out)
+ *   out, lse, ctx as in oracle_decode.  force_sel != 0: every level's
+ *   selection is given in sels.
+ * Returns 0, -1 for bad arguments, or 1 + b for a bad seq_lens[b].
+ */
+#define ORACLE_MAX_LEVELS 8
+int oracle_decode_hier(int B, int Hq, int Hkv, int d, int n_max, int C, int g, int J, int levels,
+                       const int32_t* gs, const int32_t* topks, const float* q,
+                       const float* k_raw, const float* v_raw, const float* k_gist,
+                       const float* v_gist, const float* const* k_sum,
+                       const float* const* v_sum, const int32_t* seq_lens, int force_sel,
+                       double* const* scores, int32_t* const* sels, double* out, double* lse,
+                       int32_t* ctx) {
+    oshape s = {B, Hq, Hkv, d, n_max, C, g};
+    if (!ok_shape(&s) || J < 1 || levels < 1 || levels > ORACLE_MAX_LEVELS) return -1;
+    for (int l = 0; l < levels; ++l)
+        if (topks[l] < 0 || (l > 0 && gs[l - 1] < 1)) return -1;
+    const int G = Hq / Hkv;
+    const int M_max = n_max / C;
+    int umax[ORACLE_MAX_LEVELS];
+    umax[0] = M_max;
+    for (int l = 1; l < levels; ++l) umax[l] = umax[l - 1] / J;
+    int bad = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int j = 0; j < Hkv; ++j) {
+            const int n = seq_len(&s, seq_lens, b);
+            const size_t pj = (size_t)b * Hkv + j;
+            if (n < 0) {
+#pragma omp critical
+                if (!bad || b + 1 < bad) bad = b + 1;
+                for (int l = 0; l < levels; ++l) {
+                    for (int x = 0; x < umax[l] && scores && scores[l]; ++x)
+                        scores[l][pj * (size_t)umax[l] + x] = -INFINITY;
+                    if (!force_sel)
+                        for (int c = 0; c < topks[l]; ++c) sels[l][pj * (size_t)topks[l] + c] = -1;
+                }
+                for (int gh = 0; gh < G; ++gh) {
+                    const size_t h = (size_t)b * Hq + (size_t)j * G + gh;
+                    for (int i = 0; i < d; ++i) out[h * d + i] = 0.0;
+                    if (lse) lse[h] = -INFINITY;
+                }
+                if (ctx) ctx[pj] = 0;
+                continue;
+            }
+            const int M = n / C;
+            int U[ORACLE_MAX_LEVELS];
+            U[0] = M;
+            for (int l = 1; l < levels; ++l) U[l] = U[l - 1] / J;
+            /* context capacity: every candidate's summaries or raw tokens */
+            size_t xcap = (size_t)M * (g + C) + C + 8;
+            for (int l = 1; l < levels; ++l) xcap += (size_t)(U[l - 1] + 1) * gs[l - 1];
+            const float** kx = (const float**)malloc(sizeof(float*) * xcap);
+            const float** vx = (const float**)malloc(sizeof(float*) * xcap);
+            int nx = 0;
+            int* kept = NULL;   /* units kept at the level above, ascending */
+            int nkept = 0;
+            for (int l = levels - 1; l >= 0; --l) {
+                /* candidates of level l + 1 (1-based) */
+                const int ncap = (l == levels - 1) ? U[l] : nkept * J + U[l];
+                int* cand = (int*)malloc(sizeof(int) * (size_t)(ncap > 0 ? ncap : 1));
+                int nc = 0;
+                if (l == levels - 1) {
+                    for (int x = 0; x < U[l]; ++x) cand[nc++] = x;
+                } else {
+                    for (int c = 0; c < nkept; ++c)
+                        for (int i = 0; i < J; ++i) cand[nc++] = kept[c] * J + i;
+                    if (!MUT(14)) /* mutant 14: remainder units never candidates */
+                        for (int x = U[l + 1] * J; x < U[l]; ++x) cand[nc++] = x;
+                }
+                double* sc = (double*)malloc(sizeof(double) * (size_t)(umax[l] > 0 ? umax[l] : 1));
+                for (int x = 0; x < umax[l]; ++x) sc[x] = -INFINITY;
+                for (int c = 0; c < nc; ++c) {
+                    const int x = cand[c];
+                    sc[x] = l == 0 ? chunk_score(&s, q, k_gist, b, j, x)
+                                   : super_score(&s, q, k_sum[l - 1], umax[l], gs[l - 1], b, j, x);
+                }
+                if (scores && scores[l])
+                    for (int x = 0; x < umax[l]; ++x) scores[l][pj * (size_t)umax[l] + x] = sc[x];
+                int32_t* sl = sels[l] + pj * (size_t)topks[l];
+                int* keep = (int*)malloc(sizeof(int) * (size_t)(topks[l] > 0 ? topks[l] : 1));
+                int nk;
+                if (force_sel) {
+                    nk = 0;
+                    for (int c = 0; c < topks[l]; ++c)
+                        if (sl[c] >= 0) keep[nk++] = sl[c];
+                } else {
+                    nk = topk_of(sc, cand, nc, topks[l], keep, topks[l]);
+                    for (int c = 0; c < topks[l]; ++c) sl[c] = keep[c];
+                }
+                /* context of this level */
+                for (int c = 0; c < nc; ++c) {
+                    const int x = cand[c];
+                    const int picked = is_in(keep, nk, x);
+                    if (l == 0) {
+                        if (picked) {
+                            nx = push_raw(&s, k_raw, v_raw, b, j, x * C, x * C + C, kx, vx, nx);
+                        } else {
+                            for (int t = 0; t < g; ++t) {
+                                kx[nx] = gist_row(&s, k_gist, b, j, x, t);
+                                vx[nx] = gist_row(&s, v_gist, b, j, x, t);
+                                ++nx;
+                            }
+                        }
+                    } else if (!picked) {
+                        for (int t = 0; t < gs[l - 1]; ++t) {
+                            const size_t r =
+                                ((((size_t)b * Hkv + j) * umax[l] + x) * gs[l - 1] + t) * d;
+                            kx[nx] = k_sum[l - 1] + r;
+                            vx[nx] = v_sum[l - 1] + r;
+                            ++nx;
+                        }
+                    }
+                }
+                free(sc);
+                free(cand);
+                free(kept);
+                kept = keep;
+                nkept = nk;
+            }
+            free(kept);
+            nx = push_raw(&s, k_raw, v_raw, b, j, M * C, n, kx, vx, nx);
+            if (ctx) ctx[pj] = nx;
+            for (int gh = 0; gh < G; ++gh) {
+                const size_t h = (size_t)b * Hq + (size_t)j * G + gh;
+                double l2;
+                attend_list(q + h * d, d, kx, vx, nx, out + h * d, &l2);
+                if (lse) lse[h] = l2;
+            }
+            free(kx);
+            free(vx);
+        }
+    }
+    return bad;
+}
+
 int oracle_mutant_id(void) { return ORACLE_MUTANT; }

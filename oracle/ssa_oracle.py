@@ -80,6 +80,7 @@ class Oracle:
         self.lib = ctypes.CDLL(self.path)
         self.lib.oracle_decode.restype = ctypes.c_int
         self.lib.oracle_decode_v.restype = ctypes.c_int
+        self.lib.oracle_decode_hier.restype = ctypes.c_int
         self.lib.oracle_decode_h2.restype = ctypes.c_int
         self.lib.oracle_mutant_id.restype = ctypes.c_int
 
@@ -159,6 +160,51 @@ class Oracle:
         if rc < 0:
             raise ValueError("oracle_decode_h2: bad shape or topk")
         return {"super_scores": s2[:, :, :S_max], "scores": s1, "sel_super": ss, "sel_idx": sl,
+                "out": out, "lse": lse, "ctx": ctx, "bad_seq": rc}
+
+
+    def decode_hier(self, q, k_raw, v_raw, k_gist, v_gist, k_sum, v_sum, seq_lens, C: int,
+                    g: int, J: int, topks, sels=None) -> dict:
+        """t-level coarse-to-fine decode step, t = len(topks): level 1 = chunks
+        (gists), level l >= 2 = units of J level-(l-1) units with summaries
+        k_sum[l-2], v_sum[l-2] [B,Hkv,Umax(l),gs,d]; topks[l-1] kept at level
+        l.  ``sels`` (one array per level) given => attend on those."""
+        q, k_raw, v_raw = _f32(q), _f32(k_raw), _f32(v_raw)
+        k_gist, v_gist = _f32(k_gist), _f32(v_gist)
+        k_sum = [_f32(x) for x in k_sum]
+        v_sum = [_f32(x) for x in v_sum]
+        lens = _i32(seq_lens)
+        t = len(topks)
+        assert len(k_sum) == len(v_sum) == t - 1
+        B, Hq, d = q.shape
+        Hkv, n_max = k_raw.shape[1], k_raw.shape[2]
+        umax = [n_max // C]
+        for _ in range(1, t):
+            umax.append(umax[-1] // J)
+        gs = np.asarray([x.shape[3] for x in k_sum] or [0], np.int32)
+        for l in range(1, t):
+            assert k_sum[l - 1].shape == (B, Hkv, umax[l], int(gs[l - 1]), d), (l, k_sum[l - 1].shape)
+        tk = np.asarray(list(topks), np.int32)
+        scores = [np.empty((B, Hkv, max(u, 1)), np.float64) for u in umax]
+        force = sels is not None
+        sel_arr = ([_i32(x).copy() for x in sels] if force
+                   else [np.empty((B, Hkv, max(int(k), 1)), np.int32) for k in topks])
+        out = np.empty((B, Hq, d), np.float64)
+        lse = np.empty((B, Hq), np.float64)
+        ctx = np.empty((B, Hkv), np.int32)
+        FP = ctypes.POINTER(ctypes.c_float)
+        ksp = (FP * max(t - 1, 1))(*[_p(x, _F) for x in k_sum])
+        vsp = (FP * max(t - 1, 1))(*[_p(x, _F) for x in v_sum])
+        scp = (_D * t)(*[_p(x, _D) for x in scores])
+        slp = (_I * t)(*[_p(x, _I) for x in sel_arr])
+        rc = self.lib.oracle_decode_hier(
+            B, Hq, Hkv, d, n_max, C, g, J, t, _p(gs, _I), _p(tk, _I), _p(q, _F), _p(k_raw, _F),
+            _p(v_raw, _F), _p(k_gist, _F), _p(v_gist, _F), ksp, vsp, _p(lens, _I), int(force),
+            scp, slp, _p(out, _D), _p(lse, _D), _p(ctx, _I))
+        if rc < 0:
+            raise ValueError("oracle_decode_hier: bad arguments")
+        return {"scores": [sc[:, :, :u] for sc, u in zip(scores, umax)],
+                "sels": [x[:, :, :int(k)] for x, k in zip(sel_arr, topks)],
                 "out": out, "lse": lse, "ctx": ctx, "bad_seq": rc}
 
 

@@ -452,10 +452,95 @@ def pin_union_reductions(orc):
                 assert set(own) <= set(chosen), (b, j, r, own, chosen)
 
 
+def _hier_case(rng, B, Hq, Hkv, d, C, g, n_max, lens, J, gs):
+    """Random inputs with one summary tensor per level >= 2 (gs[l-2] tokens)."""
+    c = _rand_case(rng, B, Hq, Hkv, d, C, g, n_max, lens)
+    umax = n_max // C
+    c["k_sum"], c["v_sum"] = [], []
+    for gl in gs:
+        umax //= J
+        c["k_sum"].append(rng.standard_normal((B, Hkv, umax, gl, d)).astype(np.float32))
+        c["v_sum"].append(rng.standard_normal((B, Hkv, umax, gl, d)).astype(np.float32))
+    return c
+
+
+HIER_CASES = [
+    # (B, Hq, Hkv, d, C, g, n_max, seq_lens, J, gs (levels 2..t), topks (levels 1..t))
+    (1, 4, 2, 8, 2, 2, 32, [31], 2, [2, 3], [2, 1, 1]),       # 15 chunks: remainders at 2 levels
+    (2, 2, 1, 8, 2, 1, 36, [36, 25], 3, [2], [3, 1]),
+    (1, 4, 1, 8, 2, 2, 34, [34], 2, [1, 2, 2], [3, 2, 1, 1]),  # four levels
+    (2, 4, 2, 8, 3, 2, 42, [41, 13], 2, [2, 2], [0, 2, 1]),   # topk 0 at the chunk level
+    (1, 2, 1, 8, 2, 2, 28, [27], 3, [2], [20, 9]),           # every unit kept
+]
+
+
+def pin_hier_bruteforce(orc):
+    """t-level selection against the recursive brute force (subset top-k per
+    level, explicit context list), for t = 2, 3, 4 with remainder units."""
+    rng = np.random.default_rng(2468)
+    for (B, Hq, Hkv, d, C, g, n_max, lens, J, gs, topks) in HIER_CASES:
+        c = _hier_case(rng, B, Hq, Hkv, d, C, g, n_max, lens, J, gs)
+        o = orc.decode_hier(*_args(c)[:5], c["k_sum"], c["v_sum"], c["seq_lens"], C=C, g=g, J=J,
+                            topks=topks)
+        r = bruteforce.decode_hier(*_args(c)[:5], c["k_sum"], c["v_sum"], c["seq_lens"], C, g, J,
+                                   topks)
+        for l in range(len(topks)):
+            assert np.array_equal(o["sels"][l], r["sels"][l]), (l, o["sels"][l], r["sels"][l])
+        assert np.array_equal(o["ctx"], r["ctx"]), (o["ctx"], r["ctx"])
+        _close(o["out"], r["out"], 1e-12, f"hier out J={J} topks={topks}")
+
+
+def pin_hier_reductions(orc):
+    """One level is the single-level step; two levels are the two-level step;
+    t levels whose top level keeps every unit are the t-1 levels below it."""
+    rng = np.random.default_rng(1357)
+    B, Hq, Hkv, d, C, g, n_max, J = 2, 4, 2, 8, 2, 2, 64, 2
+    c = _hier_case(rng, B, Hq, Hkv, d, C, g, n_max, [64, 45], J, [2, 3, 2])
+    a = _args(c)
+    one = orc.decode_hier(*a[:5], [], [], c["seq_lens"], C=C, g=g, J=J, topks=[5])
+    ref = orc.decode(*a, C=C, g=g, topk=5)
+    assert np.array_equal(one["sels"][0], ref["sel_idx"])
+    _close(one["out"], ref["out"], 1e-12, "one level")
+    two = orc.decode_hier(*a[:5], c["k_sum"][:1], c["v_sum"][:1], c["seq_lens"], C=C, g=g, J=J,
+                          topks=[4, 3])
+    ref2 = orc.decode_h2(*a[:5], c["k_sum"][0], c["v_sum"][0], c["seq_lens"], C=C, g=g, J=J,
+                         gm=2, topk_super=3, topk_chunk=4)
+    assert np.array_equal(two["sels"][0], ref2["sel_idx"])
+    assert np.array_equal(two["sels"][1], ref2["sel_super"])
+    _close(two["out"], ref2["out"], 1e-12, "two levels")
+    for t in (3, 4):
+        lower = orc.decode_hier(*a[:5], c["k_sum"][:t - 2], c["v_sum"][:t - 2], c["seq_lens"],
+                                C=C, g=g, J=J, topks=[4, 3, 2][:t - 1])
+        upper = orc.decode_hier(*a[:5], c["k_sum"][:t - 1], c["v_sum"][:t - 1], c["seq_lens"],
+                                C=C, g=g, J=J, topks=[4, 3, 2][:t - 1] + [1000])
+        for l in range(t - 1):
+            assert np.array_equal(upper["sels"][l], lower["sels"][l]), (t, l)
+        _close(upper["out"], lower["out"], 1e-12, f"{t} levels, top kept")
+        # the context counts: candidates' summaries or raw tokens, plus the tail
+        for b, n in enumerate(c["seq_lens"]):
+            M = int(n) // C
+            U = [M]
+            for _ in range(1, t):
+                U.append(U[-1] // J)
+            for j in range(Hkv):
+                size = int(n) - M * C
+                kept = []
+                gl = [g, 2, 3, 2]
+                for lv in range(t, 0, -1):
+                    cand = (list(range(U[lv - 1])) if lv == t else
+                            [x * J + i for x in kept for i in range(J)] + list(range(U[lv] * J, U[lv - 1])))
+                    keep = [int(x) for x in upper["sels"][lv - 1][b, j] if x >= 0]
+                    assert set(keep) <= set(cand)
+                    size += sum(C if (lv == 1 and x in keep) else (0 if x in keep else gl[lv - 1])
+                                for x in cand)
+                    kept = keep
+                assert upper["ctx"][b, j] == size, (t, b, j, upper["ctx"][b, j], size)
+
+
 ALL_PINS = [
     pin_bruteforce_single, pin_given_selection, pin_ties, pin_dense_when_all_selected,
     pin_gists_when_none_selected, pin_single_token, pin_equal_keys_mean, pin_context_size,
     pin_parallel_query, pin_hand_example, pin_bruteforce_h2, pin_h2_reduces_to_single,
     pin_bad_length, pin_nan_gist_key, pin_variants_bruteforce, pin_selected_only_closed_forms,
-    pin_union_reductions,
+    pin_union_reductions, pin_hier_bruteforce, pin_hier_reductions,
 ]

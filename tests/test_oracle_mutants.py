@@ -7,13 +7,14 @@ The mutants live behind ``-DORACLE_MUTANT=<n>`` in ``oracle/ssa_oracle.c``:
  7 tail starts one token late               8 query head -> KV head map wrong
 10 gist rows indexed token-major           11 selection not re-sorted by index
 12 per-head union keeps head 0 only        13 selected-only context drops the gists
+14 t levels: remainder units never candidates
 """
 import pytest
 
 from oracle import ssa_oracle
 from oracle_pins import ALL_PINS
 
-MUTANTS = [1, 2, 3, 4, 5, 6, 7, 8, 10, 11, 12, 13]
+MUTANTS = [1, 2, 3, 4, 5, 6, 7, 8, 10, 11, 12, 13, 14]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS)
