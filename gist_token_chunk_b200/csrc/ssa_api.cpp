@@ -101,6 +101,7 @@ void fill_shape(ssa::Plan& p, const ssa_shape* s, int C, int g, int topk) {
     p.g = g;
     p.M_max = s->n_max / C;
     p.topk = topk;
+    p.sel_stride = topk;
     p.n_pairs = s->B * s->Hkv;
     long long lim = g_wait_limit.load();
     p.wait_limit = lim > 0 ? lim : kDefaultWaitLimitNs;
@@ -414,6 +415,35 @@ ssa_status build_h2(ssa::Plan& p, const ssa_shape* shape, int C, int g, int J, i
     return check_sizes(p);
 }
 
+// Variant step (generic kernels): layout = chunk scores (per head under the
+// union reading) + the per-head selections.
+static size_t variant_layout(const ssa::Plan& p, size_t* scores_off, size_t* head_sel_off) {
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o += (bytes + 255) / 256 * 256;
+        return at;
+    };
+    const size_t rows = p.sel_mode ? (size_t)p.B * p.Hq : (size_t)p.n_pairs;
+    *scores_off = take(rows * p.M_max * 4);
+    *head_sel_off = take(p.sel_mode ? (size_t)p.B * p.Hq * (p.topk > 0 ? p.topk : 1) * 4 : 0);
+    return o;
+}
+
+static ssa_status build_variant(ssa::Plan& p, const ssa_shape* shape, int C, int g, int topk,
+                                int context, int select) {
+    if (context != SSA_CONTEXT_UNSELECTED_GISTS && context != SSA_CONTEXT_SELECTED_ONLY)
+        return fail(SSA_ERR_INVALID_ARG, "context = %d is not a context reading", context);
+    if (select != SSA_SELECT_GROUP_MAX && select != SSA_SELECT_HEAD_UNION)
+        return fail(SSA_ERR_INVALID_ARG, "select = %d is not a selection reading", select);
+    ssa_status st = build_single(p, shape, C, g, topk);
+    if (st != SSA_OK) return st;
+    p.ctx_mode = context;
+    p.sel_mode = select;
+    p.sel_stride = select == SSA_SELECT_HEAD_UNION ? p.G * topk : topk;
+    return SSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -476,6 +506,61 @@ ssa_status ssa_sparse_decode(const ssa_shape* shape, const void* q, const void* 
     p.sel_idx = const_cast<int32_t*>(sel_idx);
     p.out = out;
     return run_with_ws(p, ws, ws_bytes, stream);
+}
+
+ssa_status ssa_workspace_size_variant(const ssa_shape* shape, int32_t C, int32_t g, int32_t topk,
+                                      int32_t context, int32_t select, size_t* bytes) {
+    if (!bytes) return fail(SSA_ERR_INVALID_ARG, "bytes is NULL");
+    ssa::Plan p;
+    ssa_status st = build_variant(p, shape, C, g, topk, context, select);
+    if (st != SSA_OK) return st;
+    size_t a, b;
+    *bytes = variant_layout(p, &a, &b);
+    return SSA_OK;
+}
+
+ssa_status ssa_decode_variant(const ssa_shape* shape, const void* q, const void* k_raw,
+                              const void* v_raw, const void* k_gist, const void* v_gist,
+                              const int32_t* seq_lens, int32_t C, int32_t g, int32_t topk,
+                              int32_t context, int32_t select, float* out, int32_t* sel_idx,
+                              void* ws, size_t ws_bytes, cudaStream_t stream) {
+    ssa::Plan p;
+    ssa_status st = build_variant(p, shape, C, g, topk, context, select);
+    if (st != SSA_OK) return st;
+    st = check_tensors(p, {q, k_raw, v_raw, k_gist, v_gist, seq_lens, out});
+    if (st != SSA_OK) return st;
+    if (topk > 0 && !sel_idx) return fail(SSA_ERR_INVALID_ARG, "sel_idx is NULL");
+    p.mode = ssa::kModeFull;
+    p.q = q;
+    p.k_raw = k_raw;
+    p.v_raw = v_raw;
+    p.k_gist = k_gist;
+    p.v_gist = v_gist;
+    p.seq_lens = seq_lens;
+    p.sel_idx = sel_idx;
+    p.out = out;
+    size_t so, ho;
+    const size_t need = variant_layout(p, &so, &ho);
+    void* own = nullptr;
+    if (ws == nullptr) {
+        if (ws_bytes != 0) return fail(SSA_ERR_WORKSPACE, "ws is NULL but ws_bytes != 0");
+        cudaError_t e = cudaMallocAsync(&own, need, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+        ws = own;
+    } else if (ws_bytes < need) {
+        return fail(SSA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+    } else if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) {
+        return fail(SSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    } else {
+        note_ws_unknown(ws);  // the generic kernels leave it holding scores
+    }
+    char* base = static_cast<char*>(ws);
+    p.scores = reinterpret_cast<float*>(base + so);
+    p.head_sel = p.sel_mode ? reinterpret_cast<int32_t*>(base + ho) : nullptr;
+    cudaError_t e = ssa::launch_generic(p, stream);
+    if (own) cudaFreeAsync(own, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return SSA_OK;
 }
 
 ssa_status ssa_decode(const ssa_shape* shape, const void* q, const void* k_raw, const void* v_raw,

@@ -97,6 +97,38 @@ __global__ void score_kernel(Plan p, int level, float* dst, int stride, int n_sl
     }
 }
 
+// Per-head chunk scores (selection reading "per head + union", App. A):
+// dst[row * M_max + m] = max over the chunk's g gist rows of q_h.k/sqrt(d)
+// for row = b * Hq + h, m < M_b; -inf for M_b <= m < M_max.
+template <class T>
+__global__ void head_score_kernel(Plan p, float* dst) {
+    extern __shared__ float qs[];  // [d]
+    const int row = blockIdx.y;
+    const int b = row / p.Hq, h = row % p.Hq, j = h / p.G;
+    const int pr = b * p.Hkv + j;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const T* q = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * p.d;
+    for (int i = threadIdx.x; i < p.d; i += blockDim.x) qs[i] = to_f(q[i]);
+    __syncthreads();
+    const int n = checked_len(p, b);
+    const int M = n > 0 ? n / p.C : 0;
+    const T* keys = static_cast<const T*>(p.k_gist) + (size_t)pr * p.M_max * p.g * p.d;
+    const float scale = rsqrtf((float)p.d);
+    const int nw = blockDim.x >> 5;
+    for (int m = blockIdx.x * nw + warp; m < p.M_max; m += gridDim.x * nw) {
+        float best = -INFINITY;
+        if (m < M) {
+            const T* kr = keys + (size_t)m * p.g * p.d;
+            for (int t = 0; t < p.g; ++t) {
+                float acc = 0.f;
+                for (int i = lane; i < p.d; i += 32) acc += qs[i] * to_f(kr[(size_t)t * p.d + i]);
+                best = fmaxf(best, warp_sum(acc) * scale);
+            }
+        }
+        if (lane == 0) dst[(size_t)row * p.M_max + m] = best;
+    }
+}
+
 struct BlockSync {
     __device__ void operator()() const { __syncthreads(); }
     __device__ bool or_(bool pred) const { return __syncthreads_or(pred) != 0; }
@@ -130,6 +162,52 @@ __global__ void topk_kernel(Plan p, int level, const float* vals, int stride) {
             if (pos >= 0) out[c] = cand_chunk(p, pr, pos, ks, S);
         }
     }
+}
+
+// Per-head top-k (block of 128 per row b * Hq + h) into head_sel.
+__global__ void head_topk_kernel(Plan p, const float* vals) {
+    __shared__ TopkScratch sc;
+    const int row = blockIdx.x;
+    const int b = row / p.Hq;
+    int n = p.seq_lens[b];
+    if (n < 1 || n > p.n_max) n = 0;  // reported by the scoring kernel
+    block_topk<128>(vals + (size_t)row * p.M_max, n / p.C, p.topk,
+                    p.head_sel + (size_t)row * p.topk, sc, BlockSync());
+}
+
+// Union of the group's per-head selections (App. A): sel_idx[pr] = the
+// chunks any head of KV head j selected, ascending, then -1 up to sel_stride.
+// One block of 128 per pair; a chunk bitmap in shared memory.
+__global__ void union_kernel(Plan p) {
+    extern __shared__ uint32_t bits[];  // [mask_words]
+    __shared__ int base[129];
+    const int pr = blockIdx.x;
+    const int b = pr / p.Hkv, j = pr % p.Hkv;
+    for (int i = threadIdx.x; i < p.mask_words; i += blockDim.x) bits[i] = 0u;
+    __syncthreads();
+    for (int e = threadIdx.x; e < p.G * p.topk; e += blockDim.x) {
+        const int h = j * p.G + e / p.topk;
+        const int m = p.head_sel[((size_t)b * p.Hq + h) * p.topk + e % p.topk];
+        if (m >= 0) atomicOr(&bits[m >> 5], 1u << (m & 31));
+    }
+    __syncthreads();
+    // thread t owns words [t * per, (t + 1) * per): count, scan, then write
+    const int per = (p.mask_words + 127) / 128;
+    const int w0 = threadIdx.x * per, w1 = min(w0 + per, p.mask_words);
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
+    base[threadIdx.x + 1] = cnt;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        base[0] = 0;
+        for (int t = 1; t <= 128; ++t) base[t] += base[t - 1];
+    }
+    __syncthreads();
+    int32_t* out = p.sel_idx + (size_t)pr * p.sel_stride;
+    int at = base[threadIdx.x];
+    for (int w = w0; w < w1; ++w)
+        for (uint32_t x = bits[w]; x; x &= x - 1) out[at++] = w * 32 + __ffs(x) - 1;
+    for (int i = base[128] + threadIdx.x; i < p.sel_stride; i += blockDim.x) out[i] = -1;
 }
 
 // Checks a caller-given selection (ssa_sparse_decode): strictly ascending
@@ -191,8 +269,9 @@ __global__ void attend_kernel(Plan p, const int* bad) {
     const int S = p.h2 ? M / p.J : 0;
     const int ks = p.h2 ? kept_super(p, S) : 0;
     if (threadIdx.x == 0) {
-        for (int c = 0; c < p.topk; ++c) {
-            int m = p.sel_idx[(size_t)pr * p.topk + c];
+        const int ns = p.sel_stride > 0 ? p.sel_stride : p.topk;
+        for (int c = 0; c < ns; ++c) {
+            int m = p.sel_idx[(size_t)pr * ns + c];
             if (m >= 0) cbits[m >> 5] |= 1u << (m & 31);
         }
         for (int c = 0; c < ks; ++c) {
@@ -232,11 +311,16 @@ __global__ void attend_kernel(Plan p, const int* bad) {
             m_run = mn;
         }
     };
+    // ctx_mode 0: a selected chunk contributes its raw tokens, an unselected
+    // one its gists; ctx_mode 1: a selected chunk its gists and raw tokens,
+    // an unselected one nothing
     auto chunk_unit = [&](int m) {
-        if (cbits[m >> 5] >> (m & 31) & 1u)
-            visit(kr + (size_t)m * p.C * p.d, vr + (size_t)m * p.C * p.d, p.C);
-        else
-            visit(kg + (size_t)m * p.g * p.d, vg + (size_t)m * p.g * p.d, p.g);
+        const bool selected = cbits[m >> 5] >> (m & 31) & 1u;
+        if (selected || p.ctx_mode == 0) {
+            if (!selected || p.ctx_mode == 1)
+                visit(kg + (size_t)m * p.g * p.d, vg + (size_t)m * p.g * p.d, p.g);
+            if (selected) visit(kr + (size_t)m * p.C * p.d, vr + (size_t)m * p.C * p.d, p.C);
+        }
     };
     // units: single level -> chunks 0..M-1 then the tail;
     // two level -> superchunks 0..S-1, remainder chunks, then the tail.

@@ -75,10 +75,15 @@ struct Plan {
     float* pp_scores = nullptr;               // [P, M_max rounded up to 8] chunk scores
     float* pp_logits = nullptr;               // [P * M_max * g + 64, logit stride] kept logits
     int pp_w1 = 0, pp_w3 = 0;                 // worker warps per block: scoring, attention
+    // context / selection readings (ssa_decode_variant; 0, 0 everywhere else):
+    // ctx_mode 1 = selected gists + selected raw + tail; sel_mode 1 = per-head
+    // top-k, union over the group.  sel_stride = entries per pair in sel_idx.
+    int ctx_mode = 0, sel_mode = 0, sel_stride = 0;
+    int32_t* head_sel = nullptr;    // sel_mode 1: [B, Hq, topk] per-head selections
     long long wait_limit = 0;       // ns bound of every device-side wait
     int debug_flags = 0;
     // timeline trace (only written by builds compiled with SSA_TRACE)
-    uint4* trace = nullptr;         // [gridDim.x][trace_cap] events
+    uint4* trace = nullptr;         // events: pipeline [gridDim.x][16][trace_cap], fused [gridDim.x][trace_cap]
     int trace_cap = 0;
 };
 
@@ -128,7 +133,7 @@ cudaError_t read_device_status(int* code, cudaStream_t stream);
 // Built-in scratch of ssa_decode_noalloc: a fixed device array in the
 // library's device code (no allocation).  Its device address for the current
 // device, looked up once per device.
-constexpr size_t kBuiltinWsBytes = size_t(8) << 20;
+constexpr size_t kBuiltinWsBytes = size_t(16) << 20;
 cudaError_t builtin_workspace(void** ptr);
 
 // Query the SM count of the current device (cached per device).

@@ -283,7 +283,9 @@ bool pipe_prepare(Plan& p) {
             break;
         }
     }
-    for (int w3 = 6; w3 >= 3; --w3)
+    // attention: as many worker warps as fit (at least the four that run a
+    // block's top-k)
+    for (int w3 = pipe::kAttnWorkers; w3 >= 4; --w3)
         if (pipe::attn_layout(p, w3).total <= 227 * 1024) {
             p.pp_w3 = w3;
             break;
@@ -293,7 +295,8 @@ bool pipe_prepare(Plan& p) {
         return false;
     }
     p.st_slot_bytes = pipe::kRecBytes;
-    p.st_part_slots = pipe::kMaxBlocks * pipe::kMaxWorkers + p.n_pairs;
+    // one partial slot per (attention worker + pair) index of the launch
+    p.st_part_slots = nsm * p.pp_w3 + p.n_pairs;
     p.st_sel_stride = pipe::sel_stride(p.topk);
     return true;
 }
@@ -385,6 +388,14 @@ static cudaError_t launch_generic_t(const Plan& p, cudaStream_t stream) {
     }
     if (p.mode == kModeAttnOnly) {
         gen::validate_kernel<<<(P + 127) / 128, 128, 0, stream>>>(p, bad);
+    } else if (!p.h2 && p.sel_mode == 1) {
+        // per-head scores and top-k, union over each group (App. A)
+        const int rows = p.B * p.Hq;
+        const int gx = (p.M_max + 3) / 4;
+        gen::head_score_kernel<T><<<dim3(gx > 0 ? gx : 1, rows), 128, (size_t)p.d * sizeof(float),
+                                    stream>>>(p, p.scores);
+        gen::head_topk_kernel<<<rows, 128, 0, stream>>>(p, p.scores);
+        gen::union_kernel<<<P, 128, (size_t)p.mask_words * sizeof(uint32_t), stream>>>(p);
     } else if (!p.h2) {
         score(0, p.scores, p.M_max, p.M_max);
         gen::topk_kernel<<<P, 128, 0, stream>>>(p, 0, p.scores, p.M_max);

@@ -176,16 +176,17 @@ __device__ __forceinline__ char* part_rec(const Plan& p, int L, int h, int w, in
 }
 
 // Timeline trace: builds compiled with SSA_TRACE record per warp (clock64,
-// global timer, event | a << 8, b) into Plan::trace; the product build
+// global timer, event | a << 8, b) into Plan::trace, laid out [block][16
+// warps][trace_cap] (warps past 16 record nothing); the product build
 // compiles these to nothing.
 #ifdef SSA_TRACE
 // events 1 (warp start) and 29 (warp end) also carry the global timer (ns)
 #define ST_TR(ev, a, b)                                                                       \
     do {                                                                                      \
-        if (p.trace && lane == 0 && tr_n < p.trace_cap) {                                      \
+        if (p.trace && lane == 0 && tr_n < p.trace_cap && warp < 16) {                         \
             const unsigned long long c_ = clock64();                                           \
             const uint32_t g_ = ((ev) == 1 || (ev) == 29) ? (uint32_t)now_ns() : 0u;           \
-            p.trace[((size_t)blockIdx.x * 8 + warp) * p.trace_cap + tr_n] =                    \
+            p.trace[((size_t)blockIdx.x * 16 + warp) * p.trace_cap + tr_n] =                   \
                 make_uint4((uint32_t)c_, g_, (uint32_t)(ev) | ((uint32_t)(a) << 8), (uint32_t)(b)); \
         }                                                                                     \
         ++tr_n;                                                                               \
@@ -196,9 +197,39 @@ __device__ __forceinline__ char* part_rec(const Plan& p, int L, int h, int w, in
 
 // -------------------------------------------------------------- pipeline ---
 
-constexpr int kScoreStages = 3;   // ring stages per scoring worker
-constexpr int kAttnStages = 3;    // ring stages per attention worker
-constexpr int kMaxWorkers = 8;    // worker warps per block (sizes the partial slots)
+// Build-time shape of the two kernels: ring stages per worker warp and the
+// thread bound each is compiled for (registers per thread follow from it),
+// the most attention workers a block runs, whether P enters P.V as bf16 hi +
+// lo parts (about 16 significant bits) or as bf16 alone, and whether the
+// scoring kernel prefetches the gist values of the rows it scores into L2.
+#ifndef SSA_SCORE_STAGES
+#define SSA_SCORE_STAGES 3
+#endif
+#ifndef SSA_SCORE_THREADS
+#define SSA_SCORE_THREADS 256
+#endif
+#ifndef SSA_ATTN_STAGES
+#define SSA_ATTN_STAGES 2
+#endif
+#ifndef SSA_ATTN_THREADS
+#define SSA_ATTN_THREADS 384
+#endif
+#ifndef SSA_ATTN_WORKERS
+#define SSA_ATTN_WORKERS 11
+#endif
+#ifndef SSA_PIPE_PV_LO
+#define SSA_PIPE_PV_LO 1
+#endif
+#ifndef SSA_PREFETCH_GISTV
+#define SSA_PREFETCH_GISTV 0
+#endif
+constexpr int kScoreStages = SSA_SCORE_STAGES;  // ring stages per scoring worker
+constexpr int kScoreThreads = SSA_SCORE_THREADS;
+constexpr int kAttnStages = SSA_ATTN_STAGES;    // ring stages per attention worker
+constexpr int kAttnThreads = SSA_ATTN_THREADS;
+constexpr int kAttnWorkers = SSA_ATTN_WORKERS < SSA_ATTN_THREADS / 32 - 1 ? SSA_ATTN_WORKERS
+                                                                           : SSA_ATTN_THREADS / 32 - 1;
+constexpr int kMaxWorkers = kScoreThreads / 32;  // scoring worker warps per block
 
 // Kept-logit row stride (floats): G rounded up to 4, so every row is a
 // 16-byte unit and a stage's rows are one bulk copy.
@@ -206,6 +237,12 @@ __host__ __device__ inline int logit_stride(int G) { return (G + 3) & ~3; }
 // Chunk-score row stride (floats) of a pair: M_max rounded up to 8, so each
 // thread of the top-k reads its 8 chunks as two aligned 16-byte loads.
 __host__ __device__ inline int score_row(int M_max) { return (M_max + 7) & ~7; }
+
+// L2 prefetch of `bytes` (a multiple of 16) from a 16-byte aligned address.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes, uint64_t pol) {
+    asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;"
+                 ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "l"(pol) : "memory");
+}
 
 __device__ __forceinline__ void launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -416,7 +453,7 @@ __device__ __forceinline__ void score_stage_cuda_cores(const Plan& p, uint32_t b
 // per-head logits q.k / sqrt(d) * log2(e) go to the workspace's kept logits,
 // and the chunks whose last row the stage holds get their score (the
 // maximum over their rows and heads of q.k / sqrt(d)).
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ Plan p, const __grid_constant__ CUtensorMap tm_kg) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -453,6 +490,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     __syncwarp();
     const uint64_t pol = l2_policy_evict_first();
+    const uint64_t pol_keep = l2_policy_evict_last();
     const uint32_t ring_s = smem_u32(ring);
 
     Cursor cur;
@@ -508,6 +546,9 @@ __global__ void __launch_bounds__(256, 1)
                     bulk_load(qs + s * L.qbytes, src, (uint32_t)(G * kD * 2), &full[s]);
                 }
                 tma_load_2d_hint(ring + s * kSlotBytes, &tm_kg, 0, y, &full[s], pol);
+                if (SSA_PREFETCH_GISTV)
+                    bulk_prefetch_l2(static_cast<const __nv_bfloat16*>(p.v_gist) + (size_t)y * kD,
+                                     (uint32_t)d.nvalid * kD * 2, pol_keep);
             }
             __syncwarp();
             ++ni;
@@ -747,7 +788,7 @@ __device__ __forceinline__ bool fast_topk128(const float* scores, int M, int top
 // first word; a control warp combines the partials of its (pair, query
 // head) tasks as they complete (every wait bounded); the last block to
 // finish moves the epoch on.
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kAttnThreads, 1)
     attend_kernel(const __grid_constant__ Plan p, const __grid_constant__ CUtensorMap tm_vg,
                   const __grid_constant__ CUtensorMap tm_kr,
                   const __grid_constant__ CUtensorMap tm_vr) {
@@ -908,8 +949,14 @@ __global__ void __launch_bounds__(256, 1)
         // acc (dims as M, heads as N) += V^T (16 rows at r0 of a value box) . P^T
         auto pv16 = [&](uint32_t vbox, int r0, float p00, float p01, float p10, float p11) {
             uint32_t hi0, lo0, hi1, lo1;
+#if SSA_PIPE_PV_LO
             split_bf16(p00, p01, hi0, lo0);
             split_bf16(p10, p11, hi1, lo1);
+#else
+            hi0 = pack_bf16(p00, p01);
+            hi1 = pack_bf16(p10, p11);
+            lo0 = lo1 = 0u;
+#endif
             const int row = r0 + (lane & 7) + ((lane >> 4) << 3);
             const int csel = (lane >> 3) & 1;
 #pragma unroll
@@ -917,7 +964,7 @@ __global__ void __launch_bounds__(256, 1)
                 uint32_t a[4];
                 ldsm_x4_trans(vbox + swz(row, 2 * mt + csel), a[0], a[1], a[2], a[3]);
                 mma_bf16_16816(acc[mt], a, hi0, hi1);
-                mma_bf16_16816(acc[mt], a, lo0, lo1);
+                if (SSA_PIPE_PV_LO) mma_bf16_16816(acc[mt], a, lo0, lo1);
             }
         };
         // One partial per query head of the segment (list Lp, pair); each
@@ -1087,7 +1134,7 @@ __global__ void __launch_bounds__(256, 1)
                 if (phase == 3 || dead) break;
                 continue;  // the next raw tile waited for a selection: retry
             }
-            ST_TR(43, ni | (phase << 24), nc);
+            ST_TR(43, phase, nc);
 
             // ---- consume the oldest stage
             const int s = nc % kAttnStages;
@@ -1097,6 +1144,7 @@ __global__ void __launch_bounds__(256, 1)
                 continue;
             }
             const Desc d = desc[s];
+            ST_TR(46, d.kind, d.pair);
             const uint32_t box = ring_s + s * kSlotBytes;
             const int nv = d.nvalid;
             if (d.kind == K_GISTV) {
@@ -1197,6 +1245,7 @@ __global__ void __launch_bounds__(256, 1)
                     reset_state();
                 }
             }
+            ST_TR(47, d.kind, d.flags);
             __syncwarp();
             ++nc;
         }

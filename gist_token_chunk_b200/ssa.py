@@ -43,6 +43,10 @@ SSA_DEBUG_FUSED_PATH = 2
 SSA_PATH_GENERIC = 0
 SSA_PATH_FUSED = 1
 SSA_PATH_PIPELINE = 2
+SSA_CONTEXT_UNSELECTED_GISTS = 0
+SSA_CONTEXT_SELECTED_ONLY = 1
+SSA_SELECT_GROUP_MAX = 0
+SSA_SELECT_HEAD_UNION = 1
 
 
 class Shape(ctypes.Structure):
@@ -64,6 +68,9 @@ lib.ssa_decode_h2.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _
                               _P, _P, _P, _S, _P]
 lib.ssa_workspace_size.argtypes = [_SH, _I, _I, _I, ctypes.POINTER(_S)]
 lib.ssa_decode_path.argtypes = [_SH, _I, _I, _I, ctypes.POINTER(_I)]
+lib.ssa_decode_variant.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P,
+                                   _S, _P]
+lib.ssa_workspace_size_variant.argtypes = [_SH, _I, _I, _I, _I, _I, ctypes.POINTER(_S)]
 lib.ssa_workspace_size_h2.argtypes = [_SH, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_S)]
 lib.ssa_workspace_init.argtypes = [_P, _S, _P]
 lib.ssa_get_device_status.argtypes = [ctypes.POINTER(_I), _P]
@@ -79,7 +86,8 @@ lib.ssa_last_error.argtypes = []
 lib.ssa_last_error.restype = ctypes.c_char_p
 lib.ssa_version.restype = _I
 for _f in ("ssa_score_gists", "ssa_topk_chunks", "ssa_sparse_decode", "ssa_decode",
-           "ssa_decode_path", "ssa_decode_noalloc", "ssa_decode_h2", "ssa_workspace_size",
+           "ssa_decode_path", "ssa_decode_variant", "ssa_workspace_size_variant",
+           "ssa_decode_noalloc", "ssa_decode_h2", "ssa_workspace_size",
            "ssa_workspace_size_h2", "ssa_workspace_init", "ssa_get_device_status"):
     getattr(lib, _f).restype = _I
 
@@ -212,6 +220,36 @@ def ssa_decode(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C: int, g: int, topk: 
     _check(lib.ssa_decode(ctypes.byref(shape), _ptr(q), _ptr(k_raw), _ptr(v_raw), _ptr(k_gist),
                           _ptr(v_gist), _ptr(seq_lens), C, g, topk, _ptr(out), _ptr(sel_idx),
                           _ptr(ws), nbytes, _stream(stream)), "ssa_decode")
+    return out, sel_idx
+
+
+def ssa_workspace_size_variant(shape: Shape, C: int, g: int, topk: int, context: int,
+                               select: int) -> int:
+    n = _S(0)
+    _check(lib.ssa_workspace_size_variant(ctypes.byref(shape), C, g, topk, context, select,
+                                          ctypes.byref(n)), "ssa_workspace_size_variant")
+    return int(n.value)
+
+
+def ssa_decode_variant(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C: int, g: int, topk: int,
+                       context: int = SSA_CONTEXT_UNSELECTED_GISTS,
+                       select: int = SSA_SELECT_GROUP_MAX, out=None, sel_idx=None, ws=None,
+                       stream=None):
+    """The decode step under another context or selection reading (see
+    include/ssa.h); sel_idx holds G * topk entries per KV head under the
+    head-union selection."""
+    shape = shape_of(q, k_raw)
+    B, Hq, Hkv = q.shape[0], q.shape[1], k_raw.shape[1]
+    cap = (Hq // Hkv) * topk if select == SSA_SELECT_HEAD_UNION else topk
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    if sel_idx is None:
+        sel_idx = torch.empty((B, Hkv, cap), dtype=torch.int32, device=q.device)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib.ssa_decode_variant(ctypes.byref(shape), _ptr(q), _ptr(k_raw), _ptr(v_raw),
+                                  _ptr(k_gist), _ptr(v_gist), _ptr(seq_lens), C, g, topk,
+                                  context, select, _ptr(out), _ptr(sel_idx), _ptr(ws), nbytes,
+                                  _stream(stream)), "ssa_decode_variant")
     return out, sel_idx
 
 

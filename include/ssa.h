@@ -160,17 +160,20 @@ SSA_API ssa_status ssa_decode(const ssa_shape* shape, const void* q, const void*
  * over only the tensors.  The pages have no counterpart; this is a library
  * convenience, not a step of the method.
  * Same arguments and results as ssa_decode without ws / ws_bytes.  It
- * allocates nothing: its scratch is a fixed 8 MiB area inside the library's
+ * allocates nothing: its scratch is a fixed 16 MiB area inside the library's
  * device code (enough for the 32K, 128K and 512K batch workloads of this
  * library's tests; larger sizes return SSA_ERR_WORKSPACE with the byte count
  * in ssa_last_error(); use ssa_decode with a workspace then).
  * The first call on each device, with that device current, looks up the
  * area's device address (a CUDA runtime query); make that first call before
- * any stream capture.  Every call clears the part of the area that must start
- * at zero (a stream-ordered memset) before the kernel runs.  All calls share
- * the one area and it keeps the last call's contents, so two calls whose work
- * overlaps on the GPU (different streams without ordering, several host
- * threads) race on it: order them on one stream.
+ * any stream capture.  Before the kernels run, a call clears what must start
+ * at zero (a stream-ordered memset): on the two-kernel path only when the
+ * area was last used by another path, or by a call that used less of it (its
+ * words carry the launch's epoch and need no clearing), on the other paths
+ * the control and score part every time.  All calls share the one area and it
+ * keeps the last call's contents, so two calls whose work overlaps on the GPU
+ * (different streams without ordering, several host threads) race on it:
+ * order them on one stream.
  */
 SSA_API ssa_status ssa_decode_noalloc(const ssa_shape* shape, const void* q, const void* k_raw,
                               const void* v_raw, const void* k_gist, const void* v_gist,
@@ -196,6 +199,47 @@ SSA_API ssa_status ssa_decode_h2(const ssa_shape* shape, const void* q, const vo
                          int32_t C, int32_t g, int32_t J, int32_t gm, int32_t topk_super,
                          int32_t topk_chunk, float* out, int32_t* sel_super, int32_t* sel_idx,
                          void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * ssa_decode_variant -- the decode step under the pages' other readings of
+ * the context and of the selection (the default readings are those of
+ * ssa_decode):
+ *   context SSA_CONTEXT_UNSELECTED_GISTS: gist K/V of the unselected complete
+ *     chunks + raw K/V of the selected chunks + raw tail (ssa_decode);
+ *   context SSA_CONTEXT_SELECTED_ONLY: gist K/V and raw K/V of the selected
+ *     chunks + raw tail; unselected chunks contribute nothing (sec. 3.3,
+ *     "each selected chunk's gist and raw tokens while excluding unselected
+ *     chunks": |X| = k (C + g) + T);
+ *   select SSA_SELECT_GROUP_MAX: one top-k per KV head over the max of its
+ *     group's query heads (ssa_decode);
+ *   select SSA_SELECT_HEAD_UNION: every query head scores the chunks with its
+ *     own query (max over the chunk's g gists of q_h.k / sqrt(d)) and keeps
+ *     its own top-k (ties to the lower index); the KV head's selection is the
+ *     union over its group, and all heads of the group attend over the
+ *     context it defines (App. A, "each head selecting chunks independently
+ *     before their union").
+ * Out: out fp32 [B,Hq,d]; sel_idx int32 [B,Hkv,cap], the selection ascending
+ * and -1 padded, cap = topk (group max) or G * topk (head union).
+ * Runs on the library's portable kernels (every dtype and head dim the
+ * library accepts).  Needs ssa_workspace_size_variant() bytes of workspace
+ * (ws = NULL: allocated stream-ordered).  Errors as ssa_decode; an unknown
+ * context or select value -> SSA_ERR_INVALID_ARG.
+ */
+#define SSA_CONTEXT_UNSELECTED_GISTS 0
+#define SSA_CONTEXT_SELECTED_ONLY 1
+#define SSA_SELECT_GROUP_MAX 0
+#define SSA_SELECT_HEAD_UNION 1
+SSA_API ssa_status ssa_decode_variant(const ssa_shape* shape, const void* q, const void* k_raw,
+                                      const void* v_raw, const void* k_gist, const void* v_gist,
+                                      const int32_t* seq_lens, int32_t C, int32_t g, int32_t topk,
+                                      int32_t context, int32_t select, float* out,
+                                      int32_t* sel_idx, void* ws, size_t ws_bytes,
+                                      cudaStream_t stream);
+
+/* Workspace bytes needed by ssa_decode_variant for these sizes and readings. */
+SSA_API ssa_status ssa_workspace_size_variant(const ssa_shape* shape, int32_t C, int32_t g,
+                                              int32_t topk, int32_t context, int32_t select,
+                                              size_t* bytes);
 
 /*
  * ssa_decode_path -- which kernels ssa_decode runs for these sizes on the

@@ -126,3 +126,15 @@ def test_h2_argument_checks():
                                          ctypes.byref(n)) == ssa.SSA_ERR_UNSUPPORTED  # J*g > 1024
     assert ssa.lib.ssa_workspace_size_h2(ctypes.byref(sh), 64, 8, 16, 8, -1, 16,
                                          ctypes.byref(n)) == ssa.SSA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("context,select,code", [
+    (2, 0, ssa.SSA_ERR_INVALID_ARG), (0, -1, ssa.SSA_ERR_INVALID_ARG), (1, 1, ssa.SSA_OK)])
+def test_variant_workspace_and_bad_readings(context, select, code):
+    n = ctypes.c_size_t(0)
+    st = ssa.lib.ssa_workspace_size_variant(ctypes.byref(shape()), 128, 8, 32, context, select,
+                                            ctypes.byref(n))
+    assert st == code
+    if code == ssa.SSA_OK:
+        # per-head scores (B*Hq rows) and per-head selections
+        assert n.value >= 4 * 32 * 1024 * 4 + 4 * 32 * 32 * 4

@@ -43,11 +43,29 @@ def test_noalloc_matches_oracle_twice_in_a_row(ssa, orc):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(ssa):
-    # 128 sequences x 8 KV heads at 128K need far more than the built-in 8 MiB:
-    # the call must fail on the host, before anything is enqueued.
-    sh = ssa.make_shape(128, 32, 8, 64, 131072, 0)
-    buf = torch.zeros(1024, dtype=torch.uint8, device="cuda")
-    p = buf.data_ptr()
-    st = ssa.lib.ssa_decode_noalloc(ctypes.byref(sh), p, p, p, p, p, p, 128, 8, 32, p, p, None)
+    # 16 sequences x 8 KV heads at 64K with C=64, g=8 take the two-kernel path,
+    # whose kept logits alone need ~16.8 MB, more than the built-in 16 MiB:
+    # the call must fail on the host, before anything is enqueued.  The
+    # tensors are real, full-size allocations, so the call would stay in
+    # bounds even if the host check were wrong.
+    B, Hq, Hkv, d, n_max, C, g, topk = 16, 32, 8, 64, 65536, 64, 8, 16
+    sh = ssa.make_shape(B, Hq, Hkv, d, n_max, ssa.SSA_BF16)
+    assert ssa.ssa_decode_path(sh, C, g, topk) == ssa.SSA_PATH_PIPELINE
+    assert ssa.ssa_workspace_size(sh, C, g, topk) > 16 << 20
+    bf = torch.bfloat16
+    q = torch.zeros(B, Hq, d, dtype=bf, device="cuda")
+    k_raw = torch.empty(B, Hkv, n_max, d, dtype=bf, device="cuda")
+    v_raw = torch.empty_like(k_raw)
+    k_gist = torch.zeros(B, Hkv, n_max // C, g, d, dtype=bf, device="cuda")
+    v_gist = torch.zeros_like(k_gist)
+    lens = torch.full((B,), n_max, dtype=torch.int32, device="cuda")
+    out = torch.empty(B, Hq, d, dtype=torch.float32, device="cuda")
+    sel = torch.empty(B, Hkv, topk, dtype=torch.int32, device="cuda")
+    st = ssa.lib.ssa_decode_noalloc(ctypes.byref(sh), q.data_ptr(), k_raw.data_ptr(),
+                                    v_raw.data_ptr(), k_gist.data_ptr(), v_gist.data_ptr(),
+                                    lens.data_ptr(), C, g, topk, out.data_ptr(), sel.data_ptr(),
+                                    None)
     assert st == 3  # SSA_ERR_WORKSPACE
     assert b"built-in" in ssa.lib.ssa_last_error()
+    del k_raw, v_raw, k_gist, v_gist
+    torch.cuda.empty_cache()
