@@ -444,9 +444,117 @@ static ssa_status build_variant(ssa::Plan& p, const ssa_shape* shape, int C, int
     return SSA_OK;
 }
 
+// t-level plan: the single-level shape plus the levels' sizes (host arrays
+// of levels - 1 summary token counts and levels top-k's).
+static ssa_status build_hier(ssa::Plan& p, ssa::HierLevels& hl, const ssa_shape* shape, int C,
+                             int g, int J, int levels, const int32_t* g_sum,
+                             const int32_t* topk) {
+    if (levels < 1 || levels > ssa::kMaxLevels)
+        return fail(SSA_ERR_INVALID_ARG, "levels = %d outside [1, %d]", levels, ssa::kMaxLevels);
+    if (J < 1) return fail(SSA_ERR_INVALID_ARG, "J must be >= 1");
+    if (!topk || (levels > 1 && !g_sum)) return fail(SSA_ERR_INVALID_ARG, "topk or g_sum is NULL");
+    ssa_status st = build_single(p, shape, C, g, topk[0]);
+    if (st != SSA_OK) return st;
+    p.J = J;
+    hl.levels = levels;
+    hl.mask_words = 0;
+    for (int l = 0; l < levels; ++l) {
+        if (topk[l] < 0 || topk[l] > kMaxTopk)
+            return fail(topk[l] < 0 ? SSA_ERR_INVALID_ARG : SSA_ERR_UNSUPPORTED,
+                        "topk[%d] = %d outside [0, %d]", l, topk[l], kMaxTopk);
+        hl.topk[l] = topk[l];
+        hl.umax[l] = l == 0 ? p.M_max : hl.umax[l - 1] / J;
+        hl.gs[l] = l == 0 ? g : g_sum[l - 1];
+        if (hl.gs[l] < 1 || hl.gs[l] > 1024)
+            return fail(SSA_ERR_INVALID_ARG, "g_sum[%d] = %d outside [1, 1024]", l - 1, hl.gs[l]);
+        if ((long long)p.n_pairs * hl.umax[l] * hl.gs[l] >= (1ll << 31))
+            return fail(SSA_ERR_UNSUPPORTED, "level %d rows too large for 32-bit indices", l + 1);
+        hl.mask_words += (hl.umax[l] + 31) / 32;
+    }
+    return SSA_OK;
+}
+
+// Workspace of a t-level step: each level's candidate scores.
+static size_t hier_layout(const ssa::Plan& p, const ssa::HierLevels& hl, size_t* off) {
+    size_t o = 0;
+    for (int l = 0; l < hl.levels; ++l) {
+        off[l] = o;
+        o += ((size_t)p.n_pairs * (hl.umax[l] > 0 ? hl.umax[l] : 1) * 4 + 255) / 256 * 256;
+    }
+    return o;
+}
+
 }  // namespace
 
 extern "C" {
+
+ssa_status ssa_workspace_size_hier(const ssa_shape* shape, int32_t C, int32_t g, int32_t J,
+                                   int32_t levels, const int32_t* g_sum, const int32_t* topk,
+                                   size_t* bytes) {
+    if (!bytes) return fail(SSA_ERR_INVALID_ARG, "bytes is NULL");
+    ssa::Plan p;
+    ssa::HierLevels hl;
+    ssa_status st = build_hier(p, hl, shape, C, g, J, levels, g_sum, topk);
+    if (st != SSA_OK) return st;
+    size_t off[ssa::kMaxLevels];
+    *bytes = hier_layout(p, hl, off);
+    return SSA_OK;
+}
+
+ssa_status ssa_decode_hier(const ssa_shape* shape, const void* q, const void* k_raw,
+                           const void* v_raw, const void* k_gist, const void* v_gist,
+                           const int32_t* seq_lens, int32_t C, int32_t g, int32_t J,
+                           int32_t levels, const void* const* k_sum, const void* const* v_sum,
+                           const int32_t* g_sum, const int32_t* topk, float* out,
+                           int32_t* const* sel, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    ssa::Plan p;
+    ssa::HierLevels hl;
+    ssa_status st = build_hier(p, hl, shape, C, g, J, levels, g_sum, topk);
+    if (st != SSA_OK) return st;
+    st = check_tensors(p, {q, k_raw, v_raw, k_gist, v_gist, seq_lens, out});
+    if (st != SSA_OK) return st;
+    if (!sel || (levels > 1 && (!k_sum || !v_sum)))
+        return fail(SSA_ERR_INVALID_ARG, "sel, k_sum or v_sum is NULL");
+    for (int l = 0; l < levels; ++l) {
+        if (topk[l] > 0 && !sel[l]) return fail(SSA_ERR_INVALID_ARG, "sel[%d] is NULL", l);
+        hl.sel[l] = sel[l];
+        if (l > 0) {
+            if (!k_sum[l - 1] || !v_sum[l - 1])
+                return fail(SSA_ERR_INVALID_ARG, "k_sum[%d] or v_sum[%d] is NULL", l - 1, l - 1);
+            hl.k_sum[l] = k_sum[l - 1];
+            hl.v_sum[l] = v_sum[l - 1];
+        }
+    }
+    p.mode = ssa::kModeFull;
+    p.q = q;
+    p.k_raw = k_raw;
+    p.v_raw = v_raw;
+    p.k_gist = k_gist;
+    p.v_gist = v_gist;
+    p.seq_lens = seq_lens;
+    p.out = out;
+    size_t off[ssa::kMaxLevels];
+    const size_t need = hier_layout(p, hl, off);
+    void* own = nullptr;
+    if (ws == nullptr) {
+        if (ws_bytes != 0) return fail(SSA_ERR_WORKSPACE, "ws is NULL but ws_bytes != 0");
+        cudaError_t e = cudaMallocAsync(&own, need, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+        ws = own;
+    } else if (ws_bytes < need) {
+        return fail(SSA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+    } else if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) {
+        return fail(SSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    } else {
+        note_ws_unknown(ws);
+    }
+    for (int l = 0; l < levels; ++l)
+        hl.cscore[l] = reinterpret_cast<float*>(static_cast<char*>(ws) + off[l]);
+    cudaError_t e = ssa::launch_hier(p, hl, stream);
+    if (own) cudaFreeAsync(own, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return SSA_OK;
+}
 
 ssa_status ssa_score_gists(const ssa_shape* shape, const void* q, const void* k_gist,
                            const int32_t* seq_lens, int32_t C, int32_t g, float* scores,

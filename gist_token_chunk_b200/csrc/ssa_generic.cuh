@@ -362,5 +362,199 @@ __global__ void attend_kernel(Plan p, const int* bad) {
     }
 }
 
+// ------------------------------------------------------------- t levels ---
+
+// Complete units of every level of pair `pr`'s sequence (U[0] = M).
+__device__ __forceinline__ void hier_units(const Plan& p, const HierLevels& hl, int n, int* U) {
+    U[0] = n > 0 ? n / p.C : 0;
+    for (int l = 1; l < hl.levels; ++l) U[l] = U[l - 1] / p.J;
+}
+
+// Candidates of level l for pair pr: the top level's complete units; below,
+// the J children of each unit kept one level up (ascending), then the
+// remainder units U[l+1] J .. U[l] - 1.  Returns the count; cand_unit maps a
+// candidate position to its unit (an increasing map).
+__device__ __forceinline__ int hier_count(const HierLevels& hl, int l, int pr, const int* U,
+                                          int J, int& nkept) {
+    if (l == hl.levels - 1) {
+        nkept = 0;
+        return U[l];
+    }
+    const int32_t* up = hl.sel[l + 1] + (size_t)pr * hl.topk[l + 1];
+    nkept = 0;
+    while (nkept < hl.topk[l + 1] && up[nkept] >= 0) ++nkept;
+    return nkept * J + (U[l] - U[l + 1] * J);
+}
+__device__ __forceinline__ int hier_unit(const HierLevels& hl, int l, int pr, const int* U, int J,
+                                         int nkept, int c) {
+    if (l == hl.levels - 1) return c;
+    if (c < nkept * J) return hl.sel[l + 1][(size_t)pr * hl.topk[l + 1] + c / J] * J + c % J;
+    return U[l + 1] * J + (c - nkept * J);
+}
+
+// Scores of level l's candidates: max over the group's heads and the unit's
+// summary tokens (gists at level 0) of q.k/sqrt(d), into cscore[l].
+template <class T>
+__global__ void hier_score_kernel(Plan p, HierLevels hl, int l) {
+    extern __shared__ float qs[];  // [G][d]
+    const int pr = blockIdx.y;
+    const int b = pr / p.Hkv, j = pr % p.Hkv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const T* q = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)j * p.G) * p.d;
+    for (int i = threadIdx.x; i < p.G * p.d; i += blockDim.x) qs[i] = to_f(q[i]);
+    __syncthreads();
+    int U[kMaxLevels];
+    hier_units(p, hl, checked_len(p, b), U);
+    int nkept;
+    const int nc = hier_count(hl, l, pr, U, p.J, nkept);
+    const int ntok = l == 0 ? p.g : hl.gs[l];
+    const T* keys = l == 0 ? static_cast<const T*>(p.k_gist) + (size_t)pr * p.M_max * p.g * p.d
+                           : static_cast<const T*>(hl.k_sum[l]) +
+                                 (size_t)pr * hl.umax[l] * hl.gs[l] * p.d;
+    const float scale = rsqrtf((float)p.d);
+    const int nw = blockDim.x >> 5;
+    for (int c = blockIdx.x * nw + warp; c < nc; c += gridDim.x * nw) {
+        const T* kr = keys + (size_t)hier_unit(hl, l, pr, U, p.J, nkept, c) * ntok * p.d;
+        float best = -INFINITY;
+        for (int t = 0; t < ntok; ++t)
+            for (int h = 0; h < p.G; ++h) {
+                float acc = 0.f;
+                for (int i = lane; i < p.d; i += 32) acc += qs[h * p.d + i] * to_f(kr[(size_t)t * p.d + i]);
+                best = fmaxf(best, warp_sum(acc) * scale);
+            }
+        if (lane == 0) hl.cscore[l][(size_t)pr * hl.umax[l] + c] = best;
+    }
+}
+
+// Level l's top-k over its candidates (ties to the lower position, which is
+// the lower unit: the candidate map increases), mapped to unit ids.
+__global__ void hier_topk_kernel(Plan p, HierLevels hl, int l) {
+    __shared__ TopkScratch sc;
+    const int pr = blockIdx.x;
+    const int b = pr / p.Hkv;
+    int n = p.seq_lens[b];
+    if (n < 1 || n > p.n_max) n = 0;  // reported by the scoring kernel
+    int U[kMaxLevels];
+    hier_units(p, hl, n, U);
+    int nkept;
+    const int nc = hier_count(hl, l, pr, U, p.J, nkept);
+    int* out = hl.sel[l] + (size_t)pr * hl.topk[l];
+    block_topk<128>(hl.cscore[l] + (size_t)pr * hl.umax[l], nc, hl.topk[l], out, sc, BlockSync());
+    __syncthreads();
+    for (int c = threadIdx.x; c < hl.topk[l]; c += blockDim.x) {
+        const int pos = out[c];
+        if (pos >= 0) out[c] = hier_unit(hl, l, pr, U, p.J, nkept, pos);
+    }
+}
+
+// Attention over the t-level context, one block per (query head, sequence):
+// the summaries of every unkept candidate at levels >= 1, the gists of
+// unkept candidate chunks, the raw tokens of kept chunks, the tail.
+template <class T>
+__global__ void hier_attend_kernel(Plan p, HierLevels hl) {
+    extern __shared__ float sm[];
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int j = h / p.G;
+    const int pr = b * p.Hkv + j;
+    const int nw = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float* qs = sm;                                   // [d]
+    float* wm = qs + p.d;                             // [nw]
+    float* wl = wm + nw;                              // [nw]
+    float* wacc = wl + nw;                            // [nw][d]
+    uint32_t* bits = reinterpret_cast<uint32_t*>(wacc + nw * p.d);  // kept units, per level
+    float* outp = p.out + ((size_t)b * p.Hq + h) * p.d;
+    const int n = p.seq_lens[b];
+    if (n < 1 || n > p.n_max) {
+        report_status(kStatusBadInput);
+        for (int i = threadIdx.x; i < p.d; i += blockDim.x) outp[i] = 0.f;
+        return;
+    }
+    const T* qg = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * p.d;
+    for (int i = threadIdx.x; i < p.d; i += blockDim.x) qs[i] = to_f(qg[i]);
+    for (int i = threadIdx.x; i < hl.mask_words; i += blockDim.x) bits[i] = 0u;
+    __syncthreads();
+    int off[kMaxLevels];
+    {
+        int o = 0;
+        for (int l = 0; l < hl.levels; ++l) {
+            off[l] = o;
+            o += (hl.umax[l] + 31) / 32;
+        }
+    }
+    if (threadIdx.x == 0)
+        for (int l = 0; l < hl.levels; ++l)
+            for (int c = 0; c < hl.topk[l]; ++c) {
+                const int x = hl.sel[l][(size_t)pr * hl.topk[l] + c];
+                if (x >= 0) bits[off[l] + (x >> 5)] |= 1u << (x & 31);
+            }
+    __syncthreads();
+    int U[kMaxLevels];
+    hier_units(p, hl, n, U);
+    const int M = U[0];
+    const float scale = rsqrtf((float)p.d) * 1.4426950408889634f;  // log2 domain
+    const T* kr = static_cast<const T*>(p.k_raw) + (size_t)pr * p.n_max * p.d;
+    const T* vr = static_cast<const T*>(p.v_raw) + (size_t)pr * p.n_max * p.d;
+    float m_run = -INFINITY, l_run = 0.f;
+    float acc[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) acc[r] = 0.f;
+    auto visit = [&](const T* kbase, const T* vbase, int rows) {
+        for (int t = 0; t < rows; ++t) {
+            float x = 0.f;
+            for (int i = lane; i < p.d; i += 32) x += qs[i] * to_f(kbase[(size_t)t * p.d + i]);
+            x = warp_sum(x) * scale;
+            const float mn = fmaxf(m_run, x);
+            const float a = exp2f(m_run - mn);
+            const float e = exp2f(x - mn);
+            l_run = l_run * a + e;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int i = lane + 32 * r;
+                if (i < p.d) acc[r] = acc[r] * a + e * to_f(vbase[(size_t)t * p.d + i]);
+            }
+            m_run = mn;
+        }
+    };
+    for (int l = hl.levels - 1; l >= 0; --l) {
+        int nkept;
+        const int nc = hier_count(hl, l, pr, U, p.J, nkept);
+        const int ntok = l == 0 ? p.g : hl.gs[l];
+        const T* ks = l == 0 ? static_cast<const T*>(p.k_gist) + (size_t)pr * p.M_max * p.g * p.d
+                             : static_cast<const T*>(hl.k_sum[l]) + (size_t)pr * hl.umax[l] * ntok * p.d;
+        const T* vs = l == 0 ? static_cast<const T*>(p.v_gist) + (size_t)pr * p.M_max * p.g * p.d
+                             : static_cast<const T*>(hl.v_sum[l]) + (size_t)pr * hl.umax[l] * ntok * p.d;
+        for (int c = warp; c < nc; c += nw) {
+            const int x = hier_unit(hl, l, pr, U, p.J, nkept, c);
+            const bool kept = bits[off[l] + (x >> 5)] >> (x & 31) & 1u;
+            if (!kept)
+                visit(ks + (size_t)x * ntok * p.d, vs + (size_t)x * ntok * p.d, ntok);
+            else if (l == 0)
+                visit(kr + (size_t)x * p.C * p.d, vr + (size_t)x * p.C * p.d, p.C);
+        }
+    }
+    if (warp == nw - 1) visit(kr + (size_t)M * p.C * p.d, vr + (size_t)M * p.C * p.d, n - M * p.C);
+    if (lane == 0) {
+        wm[warp] = m_run;
+        wl[warp] = l_run;
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int i = lane + 32 * r;
+        if (i < p.d) wacc[warp * p.d + i] = acc[r];
+    }
+    __syncthreads();
+    float mx = -INFINITY;
+    for (int w = 0; w < nw; ++w) mx = fmaxf(mx, wm[w]);
+    float L = 0.f;
+    for (int w = 0; w < nw; ++w) L += (wm[w] == -INFINITY) ? 0.f : wl[w] * exp2f(wm[w] - mx);
+    for (int i = threadIdx.x; i < p.d; i += blockDim.x) {
+        float o = 0.f;
+        for (int w = 0; w < nw; ++w)
+            if (wm[w] != -INFINITY) o += wacc[w * p.d + i] * exp2f(wm[w] - mx);
+        outp[i] = L > 0.f ? o / L : 0.f;
+    }
+}
+
 }  // namespace gen
 }  // namespace ssa

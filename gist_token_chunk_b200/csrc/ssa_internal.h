@@ -87,6 +87,25 @@ struct Plan {
     int trace_cap = 0;
 };
 
+// Coarse-to-fine selection over t levels (ssa_decode_hier): level 0 is the
+// chunks (gists), level l >= 1 groups J level-(l-1) units and has gs[l]
+// summary tokens in k_sum[l], v_sum[l] [B,Hkv,umax[l],gs[l],d].  cscore[l]
+// holds each pair's candidate scores (umax[l] per pair), sel[l] the kept
+// units [B,Hkv,topk[l]].
+constexpr int kMaxLevels = 8;
+struct HierLevels {
+    int levels = 0;
+    const void* k_sum[kMaxLevels] = {};
+    const void* v_sum[kMaxLevels] = {};
+    int gs[kMaxLevels] = {};
+    int topk[kMaxLevels] = {};
+    int umax[kMaxLevels] = {};
+    float* cscore[kMaxLevels] = {};
+    int32_t* sel[kMaxLevels] = {};
+    int mask_words = 0;  // sum over levels of ceil(umax / 32)
+};
+cudaError_t launch_hier(const Plan& p, const HierLevels& hl, cudaStream_t stream);
+
 // Workspace layout for a plan (byte offsets from the workspace base).
 struct WsLayout {
     size_t ctrl = 0, scores = 0, super_scores = 0, cand_scores = 0, chunk_mask = 0,

@@ -416,6 +416,29 @@ static cudaError_t launch_generic_t(const Plan& p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+template <class T>
+static cudaError_t launch_hier_t(const Plan& p, const HierLevels& hl, cudaStream_t stream) {
+    const int P = p.n_pairs;
+    const size_t qsm = (size_t)p.G * p.d * sizeof(float);
+    for (int l = hl.levels - 1; l >= 0; --l) {
+        const int gx = (hl.umax[l] + 3) / 4;
+        gen::hier_score_kernel<T><<<dim3(gx > 0 ? gx : 1, P), 128, qsm, stream>>>(p, hl, l);
+        gen::hier_topk_kernel<<<P, 128, 0, stream>>>(p, hl, l);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int nw = 8;
+    const size_t sm = (size_t)(p.d + 2 * nw + nw * p.d) * sizeof(float) +
+                      (size_t)hl.mask_words * sizeof(uint32_t);
+    gen::hier_attend_kernel<T><<<dim3(p.Hq, p.B), 32 * nw, sm, stream>>>(p, hl);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_hier(const Plan& p, const HierLevels& hl, cudaStream_t stream) {
+    return p.dtype == 0 ? launch_hier_t<__nv_bfloat16>(p, hl, stream)
+                        : launch_hier_t<float>(p, hl, stream);
+}
+
 cudaError_t launch_generic(const Plan& p, cudaStream_t stream) {
     if (p.dtype == 1) return launch_generic_t<float>(p, stream);
     return launch_generic_t<__nv_bfloat16>(p, stream);

@@ -211,3 +211,22 @@ def small_variant(w: Workload, n_max: int, B: Optional[int] = None, seq_lens=Non
         seq_lens = (n_max,) * B
     return w.with_(name=w.name + f"_n{n_max}", B=B, n_max=n_max, seq_lens=tuple(seq_lens),
                    seq_range=None, **kw)
+
+
+def make_level_summaries(w: Workload, J: int, g_sum, seed: int, device="cpu"):
+    """Summary K/V of levels 2 .. len(g_sum) + 1 for a t-level step: level l's
+    tensors are [B,Hkv,Umax(l),g_sum[l-2],d] with Umax(l) = (n_max / C) /
+    J^(l-1), N(0, 1) in the workload's storage dtype (seeded; input
+    synthesis only).  Returns (k_sum, v_sum) lists."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    dt = _torch_dtype(w.dtype)
+    umax = w.M_max
+    k_sum, v_sum = [], []
+    for gl in g_sum:
+        umax //= J
+        shape = (w.B, w.Hkv, umax, int(gl), w.d)
+        k_sum.append(_normal(gen, shape, device).to(dt))
+        v_sum.append(_normal(gen, shape, device).to(dt))
+    return k_sum, v_sum

@@ -71,6 +71,11 @@ lib.ssa_decode_path.argtypes = [_SH, _I, _I, _I, ctypes.POINTER(_I)]
 lib.ssa_decode_variant.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P,
                                    _S, _P]
 lib.ssa_workspace_size_variant.argtypes = [_SH, _I, _I, _I, _I, _I, ctypes.POINTER(_S)]
+_PP = ctypes.POINTER(ctypes.c_void_p)
+_IP = ctypes.POINTER(ctypes.c_int32)
+lib.ssa_decode_hier.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _PP, _PP, _IP, _IP,
+                                _P, _PP, _P, _S, _P]
+lib.ssa_workspace_size_hier.argtypes = [_SH, _I, _I, _I, _I, _IP, _IP, ctypes.POINTER(_S)]
 lib.ssa_workspace_size_h2.argtypes = [_SH, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_S)]
 lib.ssa_workspace_init.argtypes = [_P, _S, _P]
 lib.ssa_get_device_status.argtypes = [ctypes.POINTER(_I), _P]
@@ -87,6 +92,7 @@ lib.ssa_last_error.restype = ctypes.c_char_p
 lib.ssa_version.restype = _I
 for _f in ("ssa_score_gists", "ssa_topk_chunks", "ssa_sparse_decode", "ssa_decode",
            "ssa_decode_path", "ssa_decode_variant", "ssa_workspace_size_variant",
+           "ssa_decode_hier", "ssa_workspace_size_hier",
            "ssa_decode_noalloc", "ssa_decode_h2", "ssa_workspace_size",
            "ssa_workspace_size_h2", "ssa_workspace_init", "ssa_get_device_status"):
     getattr(lib, _f).restype = _I
@@ -251,6 +257,44 @@ def ssa_decode_variant(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C: int, g: int
                                   context, select, _ptr(out), _ptr(sel_idx), _ptr(ws), nbytes,
                                   _stream(stream)), "ssa_decode_variant")
     return out, sel_idx
+
+
+def _i32_array(xs):
+    return (ctypes.c_int32 * max(len(xs), 1))(*[int(x) for x in xs])
+
+
+def ssa_workspace_size_hier(shape: Shape, C: int, g: int, J: int, g_sum, topk) -> int:
+    n = _S(0)
+    _check(lib.ssa_workspace_size_hier(ctypes.byref(shape), C, g, J, len(topk), _i32_array(g_sum),
+                                       _i32_array(topk), ctypes.byref(n)),
+           "ssa_workspace_size_hier")
+    return int(n.value)
+
+
+def ssa_decode_hier(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C: int, g: int, J: int, k_sum,
+                    v_sum, topk, out=None, sels=None, ws=None, stream=None):
+    """Coarse-to-fine decode step over t = len(topk) levels (see include/ssa.h):
+    k_sum, v_sum are the t-1 summary tensors of levels 2..t [B,Hkv,Umax,g_l,d];
+    returns out and one selection tensor per level [B,Hkv,topk[l]]."""
+    shape = shape_of(q, k_raw)
+    B, Hkv = q.shape[0], k_raw.shape[1]
+    t = len(topk)
+    assert len(k_sum) == len(v_sum) == t - 1
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    if sels is None:
+        sels = [torch.empty((B, Hkv, max(int(k), 1)), dtype=torch.int32, device=q.device)
+                for k in topk]
+    g_sum = [int(x.shape[3]) for x in k_sum]
+    kp = (ctypes.c_void_p * max(t - 1, 1))(*[_ptr(x) for x in k_sum])
+    vp = (ctypes.c_void_p * max(t - 1, 1))(*[_ptr(x) for x in v_sum])
+    sp = (ctypes.c_void_p * t)(*[_ptr(x) for x in sels])
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib.ssa_decode_hier(ctypes.byref(shape), _ptr(q), _ptr(k_raw), _ptr(v_raw),
+                               _ptr(k_gist), _ptr(v_gist), _ptr(seq_lens), C, g, J, t, kp, vp,
+                               _i32_array(g_sum), _i32_array(topk), _ptr(out), sp, _ptr(ws),
+                               nbytes, _stream(stream)), "ssa_decode_hier")
+    return out, [s[:, :, :int(k)] for s, k in zip(sels, topk)]
 
 
 def ssa_decode_noalloc(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C: int, g: int, topk: int,

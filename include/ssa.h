@@ -242,6 +242,45 @@ SSA_API ssa_status ssa_workspace_size_variant(const ssa_shape* shape, int32_t C,
                                               size_t* bytes);
 
 /*
+ * ssa_decode_hier -- coarse-to-fine selection over t = levels levels (sec.
+ * 3.5, "additional hierarchy levels can be added as context grows"; App.
+ * B.2, t = ceil(log_J M)), the two-level reading of ssa_decode_h2 applied
+ * level by level.  Level 1 is the chunks with their g gists (k_gist,
+ * v_gist).  A level-l unit (l >= 2) groups J level-(l-1) units and has
+ * g_sum[l-2] summary tokens in k_sum[l-2], v_sum[l-2], bf16/fp32 like the
+ * rest, laid out [B,Hkv,Umax(l),g_sum[l-2],d] with Umax(l) = (n_max / C) /
+ * J^(l-1) (integer divisions, level by level).  A sequence has U_1 = M_b
+ * complete chunks and U_l = floor(U_{l-1} / J) complete level-l units.
+ * Selection, from the top: level t's candidates are its U_t units; level
+ * l < t's are the J children of each unit kept at level l+1 (ascending),
+ * then the remainder units U_{l+1} J .. U_l - 1, which lie in no complete
+ * parent; each level keeps its topk[l-1] best candidates (score = max over
+ * the group's query heads and the unit's summary tokens of q.k / sqrt(d),
+ * ties to the lower index) into sel[l-1] [B,Hkv,topk[l-1]], ascending, -1
+ * padded.  Context: the summary tokens of every unkept candidate at levels
+ * >= 2, the gists of unkept candidate chunks, the raw tokens of kept chunks
+ * and the raw tail.  levels = 1 is ssa_decode's step, levels = 2 is
+ * ssa_decode_h2's.
+ * k_sum, v_sum, g_sum (levels - 1 entries) and topk, sel (levels entries)
+ * are HOST arrays; the tensors they point to are device memory.  1 <= levels
+ * <= 8, J >= 1, 1 <= g_sum <= 1024, 0 <= topk <= 1024.  Runs on the
+ * library's portable kernels.  Needs ssa_workspace_size_hier() bytes of
+ * workspace (ws = NULL: allocated stream-ordered).
+ */
+SSA_API ssa_status ssa_decode_hier(const ssa_shape* shape, const void* q, const void* k_raw,
+                                   const void* v_raw, const void* k_gist, const void* v_gist,
+                                   const int32_t* seq_lens, int32_t C, int32_t g, int32_t J,
+                                   int32_t levels, const void* const* k_sum,
+                                   const void* const* v_sum, const int32_t* g_sum,
+                                   const int32_t* topk, float* out, int32_t* const* sel, void* ws,
+                                   size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes needed by ssa_decode_hier for these sizes. */
+SSA_API ssa_status ssa_workspace_size_hier(const ssa_shape* shape, int32_t C, int32_t g, int32_t J,
+                                           int32_t levels, const int32_t* g_sum,
+                                           const int32_t* topk, size_t* bytes);
+
+/*
  * ssa_decode_path -- which kernels ssa_decode runs for these sizes on the
  * current device (a host-side query; nothing is launched):
  *   SSA_PATH_PIPELINE  two kernels on the stream: gist scoring, then top-k,

@@ -180,3 +180,39 @@ def check_variant(orc, inp: dict, C: int, g: int, topk: int, context: int, selec
         ref = orc.decode(*args, C=C, g=g, topk=topk, context=context, select=select, sel=sel)
     mx, mean = assert_outputs_close(out, ref["out"])
     return {"max_abs": mx, "mean_abs": mean, "near_ties": near}
+
+
+def check_hier(orc, inp: dict, k_sum, v_sum, C: int, g: int, J: int, topks, gpu_out,
+               gpu_sels) -> dict:
+    """Compare a t-level step with the oracle: every level's selection
+    bit-exact away from near ties (there the GPU's choice must be a valid
+    top-k of the oracle's candidate scores, and the oracle is re-run on the
+    GPU's selections of every level); outputs within the bars."""
+    args = (inp["q"], inp["k_raw"], inp["v_raw"], inp["k_gist"], inp["v_gist"])
+    ref = orc.decode_hier(*args, k_sum, v_sum, inp["seq_lens"], C=C, g=g, J=J, topks=topks)
+    sels = [host(s).astype(np.int32) for s in gpu_sels]
+    out = host(gpu_out)
+    t = len(topks)
+    near = 0
+    B, Hkv = sels[0].shape[:2]
+    for b in range(B):
+        for j in range(Hkv):
+            for l in range(t - 1, -1, -1):
+                sc = ref["scores"][l][b, j]
+                cand = [x for x in range(sc.shape[0]) if np.isfinite(sc[x])]
+                k = min(topks[l], len(cand))
+                if np.array_equal(sels[l][b, j], ref["sels"][l][b, j]):
+                    continue
+                # a different choice is allowed only at a near tie; the levels
+                # below then see other candidates, so stop comparing this pair
+                assert kth_gap(sc, cand, k) <= NEAR_TIE, (
+                    f"level {l + 1} selection differs at (b={b}, j={j}): gpu {sels[l][b, j]} vs "
+                    f"oracle {ref['sels'][l][b, j]}")
+                assert selection_is_valid_topk(sc, cand, sels[l][b, j], k)
+                near += 1
+                break
+    if near:
+        ref = orc.decode_hier(*args, k_sum, v_sum, inp["seq_lens"], C=C, g=g, J=J, topks=topks,
+                              sels=sels)
+    mx, mean = assert_outputs_close(out, ref["out"])
+    return {"max_abs": mx, "mean_abs": mean, "near_ties": near}

@@ -138,3 +138,18 @@ def test_variant_workspace_and_bad_readings(context, select, code):
     if code == ssa.SSA_OK:
         # per-head scores (B*Hq rows) and per-head selections
         assert n.value >= 4 * 32 * 1024 * 4 + 4 * 32 * 32 * 4
+
+
+def test_hier_workspace_and_bad_levels():
+    sh = shape(B=1, n_max=1 << 20)
+    n = ssa.ssa_workspace_size_hier(sh, 64, 8, 16, [8, 8], [16, 8, 4])
+    # candidate scores of every level: 8 pairs x (16384 + 1024 + 64) floats
+    assert n >= 8 * (16384 + 1024 + 64) * 4
+    v = ctypes.c_size_t(0)
+    nine = (ctypes.c_int32 * 9)(*([8] * 9))
+    assert ssa.lib.ssa_workspace_size_hier(ctypes.byref(sh), 64, 8, 16, 9, nine, nine,
+                                           ctypes.byref(v)) == ssa.SSA_ERR_INVALID_ARG
+    bad_g = (ctypes.c_int32 * 2)(0, 8)
+    tk = (ctypes.c_int32 * 3)(16, 8, 4)
+    assert ssa.lib.ssa_workspace_size_hier(ctypes.byref(sh), 64, 8, 16, 3, bad_g, tk,
+                                           ctypes.byref(v)) == ssa.SSA_ERR_INVALID_ARG
