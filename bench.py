@@ -58,6 +58,9 @@ def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
+VARIANTS = {"none": None, "selected_only": (1, 0), "head_union": (0, 1),
+            "selected_union": (1, 1)}
+
 # ------------------------------------------------------------ bytes model ---
 
 def algorithmic_bytes(w, seq_lens) -> int:
@@ -87,6 +90,101 @@ def algorithmic_bytes(w, seq_lens) -> int:
         tot += w.Hkv * rows * w.d * e
     sel_k = w.topk + (w.topk_super if w.two_level else 0)
     tot += w.B * w.Hq * w.d * e + w.B * w.Hq * w.d * 4 + w.B * w.Hkv * sel_k * 4 + w.B * 4
+    return tot
+
+
+# ------------------------------------------------------------ host cost ---
+
+def host_call_cost(ssa, w, x, out, sel, sup, ws, stream, calls: int = 200) -> dict:
+    """Host microseconds one decode call costs: through the Python binding,
+    and through the C ABI alone (ctypes with the arguments prepared once).
+    Each call enqueues a real step; the stream is drained before and after."""
+    import ctypes
+
+    torch.cuda.synchronize()
+    sp = stream.cuda_stream
+    sh = ssa.shape_of(x["q"], x["k_raw"])
+    if w.two_level:
+        def bind():
+            ssa.ssa_decode_h2(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
+                              x["k_meta"], x["v_meta"], x["seq_lens"], w.C, w.g, w.J, w.gm,
+                              w.topk_super, w.topk, out=out, sel_super=sup, sel_idx=sel, ws=ws,
+                              stream=stream)
+        cargs = (ctypes.byref(sh), x["q"].data_ptr(), x["k_raw"].data_ptr(), x["v_raw"].data_ptr(),
+                 x["k_gist"].data_ptr(), x["v_gist"].data_ptr(), x["k_meta"].data_ptr(),
+                 x["v_meta"].data_ptr(), x["seq_lens"].data_ptr(), w.C, w.g, w.J, w.gm,
+                 w.topk_super, w.topk, out.data_ptr(), sup.data_ptr(), sel.data_ptr(),
+                 ws.data_ptr(), ws.numel(), sp)
+        cfn = ssa.lib.ssa_decode_h2
+    else:
+        def bind():
+            ssa.ssa_decode(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
+                           x["seq_lens"], w.C, w.g, w.topk, out=out, sel_idx=sel, ws=ws,
+                           stream=stream)
+        cargs = (ctypes.byref(sh), x["q"].data_ptr(), x["k_raw"].data_ptr(), x["v_raw"].data_ptr(),
+                 x["k_gist"].data_ptr(), x["v_gist"].data_ptr(), x["seq_lens"].data_ptr(), w.C,
+                 w.g, w.topk, out.data_ptr(), sel.data_ptr(), ws.data_ptr(), ws.numel(), sp)
+        cfn = ssa.lib.ssa_decode
+    if cfn(*cargs) != 0:
+        raise SystemExit("host cost: the C ABI call failed: " + ssa.lib.ssa_last_error().decode())
+    res = {}
+    for name, fn in (("binding", bind), ("c_abi", lambda: cfn(*cargs))):
+        fn()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(calls):
+            fn()
+        res[name] = 1e6 * (time.perf_counter() - t0) / calls
+        torch.cuda.synchronize()
+    return res
+
+
+def variant_bytes(w, seq_lens, sel, context: int) -> int:
+    """Bytes one variant step must move, each read once: per (sequence, KV
+    head) the gist keys of all complete chunks, the gist values of the
+    unselected chunks (context 0) or of the selected ones (context 1), the
+    raw K/V of the selected chunks (k_u = the selection's size) and the tail;
+    plus q, out, selection and lengths."""
+    e = 2 if w.dtype == "bf16" else 4
+    tot = 0
+    for b, n in enumerate(seq_lens):
+        n = int(n)
+        M = n // w.C
+        T = n - M * w.C
+        for j in range(w.Hkv):
+            ku = int((sel[b, j] >= 0).sum())
+            gv = (M - ku) * w.g if context == 0 else ku * w.g
+            tot += (M * w.g + gv + 2 * ku * w.C + 2 * T) * w.d * e
+    tot += w.B * w.Hq * w.d * e + w.B * w.Hq * w.d * 4 + sel.size * 4 + w.B * 4
+    return tot
+
+
+def hier_bytes(w, seq_lens, sels, J: int, g_sum, topks) -> int:
+    """Bytes of a t-level step, each read once: per (sequence, KV head) and
+    level, the summary keys of every candidate (scored) and the summary
+    values of the unkept ones; the raw K/V of the kept chunks; the tail."""
+    e = 2 if w.dtype == "bf16" else 4
+    t = len(topks)
+    gl = [w.g] + list(g_sum)
+    tot = 0
+    for b, n in enumerate(seq_lens):
+        n = int(n)
+        U = [n // w.C]
+        for _ in range(1, t):
+            U.append(U[-1] // J)
+        T = n - U[0] * w.C
+        for j in range(w.Hkv):
+            kept_above = 0
+            rows = 2 * T
+            for l in range(t - 1, -1, -1):
+                nc = U[l] if l == t - 1 else kept_above * J + (U[l] - U[l + 1] * J)
+                kept = int((sels[l][b, j] >= 0).sum())
+                rows += nc * gl[l] + (nc - kept) * gl[l]
+                if l == 0:
+                    rows += 2 * kept * w.C
+                kept_above = kept
+            tot += rows * w.d * e
+    tot += w.B * w.Hq * w.d * e + w.B * w.Hq * w.d * 4 + sum(s.size for s in sels) * 4 + w.B * 4
     return tot
 
 
@@ -214,8 +312,9 @@ class ClockSampler:
 
 # ------------------------------------------------------------- cpu oracle ---
 
-def oracle_time(inp, w, min_seconds: float, max_reps: int = 1000):
-    """Time the fp64 oracle on whole decode steps of `inp` (host tensors)."""
+def oracle_time(inp, w, min_seconds: float, max_reps: int = 1000, variant=None, hier=None):
+    """Time the fp64 oracle on whole decode steps of `inp` (host tensors),
+    under the same reading (variant) or levels (hier) as the GPU arm."""
     from oracle import ssa_oracle
 
     orc = ssa_oracle.default()
@@ -226,9 +325,17 @@ def oracle_time(inp, w, min_seconds: float, max_reps: int = 1000):
 
     args = [_np.ascontiguousarray(a.float().numpy()) for a in args]
     lens = inp["seq_lens"].numpy()
+    if hier:
+        ks = [_np.ascontiguousarray(x.float().numpy()) for x in inp["k_sum"]]
+        vs = [_np.ascontiguousarray(x.float().numpy()) for x in inp["v_sum"]]
 
     def one():
-        if w.two_level:
+        if hier:
+            orc.decode_hier(*args, ks, vs, lens, C=w.C, g=w.g, J=hier[0], topks=hier[2])
+        elif variant:
+            orc.decode(*args, lens, C=w.C, g=w.g, topk=w.topk, context=variant[0],
+                       select=variant[1])
+        elif w.two_level:
             orc.decode_h2(*args, lens, C=w.C, g=w.g, J=w.J, gm=w.gm, topk_super=w.topk_super,
                           topk_chunk=w.topk)
         else:
@@ -357,6 +464,10 @@ def main():
                     help="steps of the end-to-end measurement (0: skip it)")
     ap.add_argument("--sets", type=int, default=NSETS,
                     help="rotating input sets (fewer only for profiling runs)")
+    ap.add_argument("--variant", default="none", choices=sorted(VARIANTS),
+                    help="another context / selection reading (ssa_decode_variant)")
+    ap.add_argument("--levels", default="",
+                    help="coarse-to-fine over t levels (ssa_decode_hier): 'J:g2,..,gt:k1,..,kt'")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -388,30 +499,73 @@ def main():
     for s in sets:
         s.pop("planted_idx", None)
     shape = ssa.shape_of(sets[0]["q"], sets[0]["k_raw"])
-    if w.two_level:
+    variant = VARIANTS[args.variant]
+    hier = None
+    if args.levels:
+        if w.two_level or variant:
+            ap.error("--levels takes a single-level workload and no --variant")
+        J_s, g_s, k_s = args.levels.split(":")
+        hier = (int(J_s), [int(x) for x in g_s.split(",") if x], [int(x) for x in k_s.split(",")])
+        if len(hier[1]) != len(hier[2]) - 1:
+            ap.error("--levels: t-1 summary sizes and t top-k's")
+    if variant and w.two_level:
+        ap.error("--variant takes a single-level workload")
+    if hier:
+        nbytes = ssa.ssa_workspace_size_hier(shape, w.C, w.g, hier[0], hier[1], hier[2])
+    elif variant:
+        nbytes = ssa.ssa_workspace_size_variant(shape, w.C, w.g, w.topk, *variant)
+    elif w.two_level:
         nbytes = ssa.ssa_workspace_size_h2(shape, w.C, w.g, w.J, w.gm, w.topk_super, w.topk)
     else:
         nbytes = ssa.ssa_workspace_size(shape, w.C, w.g, w.topk)
     ws = ssa.workspace(nbytes, device=dev)
+    cap = w.topk * (w.G if variant and variant[1] else 1)
     outs = [torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev) for _ in range(NS)]
-    sels = [torch.empty(w.B, w.Hkv, w.topk, dtype=torch.int32, device=dev) for _ in range(NS)]
+    sels = [torch.empty(w.B, w.Hkv, max(cap, 1), dtype=torch.int32, device=dev)
+            for _ in range(NS)]
     sups = [torch.empty(w.B, w.Hkv, max(w.topk_super, 1), dtype=torch.int32, device=dev)
             for _ in range(NS)]
+    if hier:
+        from gist_token_chunk_b200.inputs import make_level_summaries
+
+        for s_i, x in enumerate(sets):
+            x["k_sum"], x["v_sum"] = make_level_summaries(
+                w, hier[0], hier[1], seed=rank_seed(args.seed, s_i, rank) + 17, device=dev)
+        hsels = [[torch.empty(w.B, w.Hkv, max(k, 1), dtype=torch.int32, device=dev)
+                  for k in hier[2]] for _ in range(NS)]
+
+    def decode_call(x, s, out, sel, stream):
+        """One decode step of set s's inputs x through the public call."""
+        if hier:
+            ssa.ssa_decode_hier(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
+                                x["seq_lens"], w.C, w.g, hier[0], x["k_sum"], x["v_sum"],
+                                hier[2], out=out, sels=hsels[s], ws=ws, stream=stream)
+        elif variant:
+            ssa.ssa_decode_variant(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
+                                   x["seq_lens"], w.C, w.g, w.topk, variant[0], variant[1],
+                                   out=out, sel_idx=sel, ws=ws, stream=stream)
+        elif w.two_level:
+            ssa.ssa_decode_h2(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
+                              x["k_meta"], x["v_meta"], x["seq_lens"], w.C, w.g, w.J, w.gm,
+                              w.topk_super, w.topk, out=out, sel_super=sups[s], sel_idx=sel,
+                              ws=ws, stream=stream)
+        else:
+            ssa.ssa_decode(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
+                           x["seq_lens"], w.C, w.g, w.topk, out=out, sel_idx=sel, ws=ws,
+                           stream=stream)
 
     def step(i, stream=None):
         s = i % NS
-        x = sets[s]
-        if w.two_level:
-            ssa.ssa_decode_h2(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
-                              x["k_meta"], x["v_meta"], x["seq_lens"], w.C, w.g, w.J, w.gm,
-                              w.topk_super, w.topk, out=outs[s], sel_super=sups[s],
-                              sel_idx=sels[s], ws=ws, stream=stream)
-        else:
-            ssa.ssa_decode(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
-                           x["seq_lens"], w.C, w.g, w.topk, out=outs[s], sel_idx=sels[s], ws=ws,
-                           stream=stream)
+        decode_call(sets[s], s, outs[s], sels[s], stream)
 
-    if w.two_level:
+    if hier:
+        kernel_name = "ssa::gen hier_score, hier_topk (per level) and hier_attend kernels"
+        launches_per_step = 2 * len(hier[2]) + 1
+    elif variant:
+        kernel_name = ("ssa::gen head_score, head_topk, union and attend kernels" if variant[1]
+                       else "ssa::gen score, top-k and attend kernels")
+        launches_per_step = 4 if variant[1] else 3
+    elif w.two_level:
         path, kernel_name, launches_per_step = None, "ssa::fused::fused_kernel<64>", 1
     else:
         path = ssa.ssa_decode_path(shape, w.C, w.g, w.topk)
@@ -474,8 +628,17 @@ def main():
     value = queries / (ms / 1e3)
     ms_step = ms / args.steps
     # bytes model, averaged over the rotating sets
-    bytes_per_launch = statistics.mean(
-        algorithmic_bytes(w, s["seq_lens"].cpu().tolist()) for s in sets)
+    if hier:
+        bytes_per_launch = statistics.mean(
+            hier_bytes(w, sets[s]["seq_lens"].cpu().tolist(), [x.cpu().numpy() for x in hsels[s]],
+                       *hier) for s in range(NS))
+    elif variant:
+        bytes_per_launch = statistics.mean(
+            variant_bytes(w, sets[s]["seq_lens"].cpu().tolist(), sels[s].cpu().numpy(), variant[0])
+            for s in range(NS))
+    else:
+        bytes_per_launch = statistics.mean(
+            algorithmic_bytes(w, s["seq_lens"].cpu().tolist()) for s in sets)
     per_launch_s = (ms / 1e3) / args.steps
     achieved = bytes_per_launch / per_launch_s / 1e9
     peak, peak_src = hbm_peak()
@@ -529,15 +692,7 @@ def main():
         stream.wait_event(down_done[s])         # the set's last output has been read back
         x = dict(sets[s], q=q_dev, seq_lens=len_dev)
         obuf, (o_dev, s_dev) = down_dev[s]
-        if w.two_level:
-            ssa.ssa_decode_h2(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
-                              x["k_meta"], x["v_meta"], x["seq_lens"], w.C, w.g, w.J, w.gm,
-                              w.topk_super, w.topk, out=o_dev, sel_super=sups[s],
-                              sel_idx=s_dev, ws=ws, stream=stream)
-        else:
-            ssa.ssa_decode(x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"],
-                           x["seq_lens"], w.C, w.g, w.topk, out=o_dev, sel_idx=s_dev, ws=ws,
-                           stream=stream)
+        decode_call(x, s, o_dev, s_dev, stream)
         dec_done[s].record(stream)
         down_stream.wait_event(dec_done[s])
         with torch.cuda.stream(down_stream):
@@ -556,14 +711,18 @@ def main():
         with torch.cuda.stream(stream):
             ev0.record(stream)
             up_stream.wait_event(ev0)
+            h0 = time.perf_counter()
             for i in range(ek):
                 e2e_step(i)
+            host_issue_s = time.perf_counter() - h0
             for s in range(NS):
                 stream.wait_event(down_done[s])
             ev1.record(stream)
         ev1.synchronize()
         e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), pg, dev)
         e2e_value = ek * w.B * world / (e2e_ms / 1e3)
+        host_cost = (None if hier or variant else
+                     host_call_cost(ssa, w, sets[0], outs[0], sels[0], sups[0], ws, stream))
     h2d = sets[0]["q"].numel() * sets[0]["q"].element_size() + sets[0]["seq_lens"].numel() * 4
     d2h = outs[0].numel() * 4 + sels[0].numel() * 4
 
@@ -572,7 +731,9 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": run_config(w, world, NS),
+        "config": dict(run_config(w, world, NS),
+                       **({"reading": args.variant} if variant else {}),
+                       **({"levels": args.levels} if hier else {})),
         "hbm_gbs": achieved, "hbm_frac_of_peak": achieved / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_src} copy bandwidth",
@@ -584,6 +745,8 @@ def main():
         "gpu_launches": args.steps * launches_per_step,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": ek,
+                "host_issue_us_per_step": (1e6 * host_issue_s / ek) if ek > 0 else None,
+                "host_us_per_call": host_cost if ek > 0 else None,
                 "path": "ssa_decode per step (Python binding -> C ABI); query and lengths up "
                         "in one pinned copy, output and selection back in one, each on its own "
                         "stream so copies overlap the neighbouring steps' kernels"},
@@ -594,8 +757,9 @@ def main():
 
     # ---- CPU baseline: the oracle on the host (rank 0, N = 1 only)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        host = {k: v.cpu() for k, v in sets[0].items()}
-        reps, el = oracle_time(host, w, args.cpu_seconds)
+        host = {k: ([x.cpu() for x in v] if isinstance(v, list) else v.cpu())
+                for k, v in sets[0].items()}
+        reps, el = oracle_time(host, w, args.cpu_seconds, variant=variant, hier=hier)
         line["cpu_baseline"] = {
             "value": reps * w.B / el, "unit": UNIT, "cores": oracle_cores(w.B * w.Hkv),
             "kind": "oracle",
