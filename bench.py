@@ -747,9 +747,9 @@ def main():
                 "d2h_bytes_per_step": int(d2h), "steps": ek,
                 "host_issue_us_per_step": (1e6 * host_issue_s / ek) if ek > 0 else None,
                 "host_us_per_call": host_cost if ek > 0 else None,
-                "path": "ssa_decode per step (Python binding -> C ABI); query and lengths up "
-                        "in one pinned copy, output and selection back in one, each on its own "
-                        "stream so copies overlap the neighbouring steps' kernels"},
+                "path": "the step's call per step (Python binding -> C ABI); query and lengths "
+                        "up in one pinned copy, output and selection back in one, each on its "
+                        "own stream so copies overlap the neighbouring steps' kernels"},
     }
     clk = sampler.summary()
     if clk is not None:

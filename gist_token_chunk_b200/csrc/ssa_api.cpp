@@ -624,6 +624,11 @@ ssa_status ssa_workspace_size_variant(const ssa_shape* shape, int32_t C, int32_t
     if (st != SSA_OK) return st;
     size_t a, b;
     *bytes = variant_layout(p, &a, &b);
+    // the group-max selection may run on the two-kernel pipeline
+    if (select == SSA_SELECT_GROUP_MAX && ssa::pipe_prepare(p)) {
+        const size_t pb = ssa::plan_bytes_any(p);
+        if (pb > *bytes) *bytes = pb;
+    }
     return SSA_OK;
 }
 
@@ -647,6 +652,9 @@ ssa_status ssa_decode_variant(const ssa_shape* shape, const void* q, const void*
     p.seq_lens = seq_lens;
     p.sel_idx = sel_idx;
     p.out = out;
+    // group max on a pipeline shape: the two-kernel path, whose attention
+    // kernel applies either context's keep predicate
+    if (p.sel_mode == 0 && ssa::pipe_prepare(p)) return run_with_ws(p, ws, ws_bytes, stream);
     size_t so, ho;
     const size_t need = variant_layout(p, &so, &ho);
     void* own = nullptr;
@@ -691,6 +699,71 @@ ssa_status ssa_decode(const ssa_shape* shape, const void* q, const void* k_raw, 
     p.sel_idx = sel_idx;
     p.out = out;
     return run_with_ws(p, ws, ws_bytes, stream);
+}
+
+// Device copies of a host-buffer step's small tensors, after the decode's
+// own workspace: q, seq_lens, out, sel_idx (256-byte aligned).
+static size_t host_staging(const ssa::Plan& p, size_t base, size_t* off) {
+    size_t o = (base + 255) / 256 * 256;
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o += (bytes + 255) / 256 * 256;
+        return at;
+    };
+    const size_t e = p.dtype == SSA_BF16 ? 2 : 4;
+    off[0] = take((size_t)p.B * p.Hq * p.d * e);
+    off[1] = take((size_t)p.B * 4);
+    off[2] = take((size_t)p.B * p.Hq * p.d * 4);
+    off[3] = take((size_t)p.n_pairs * (p.topk > 0 ? p.topk : 1) * 4);
+    return o;
+}
+
+ssa_status ssa_workspace_size_host(const ssa_shape* shape, int32_t C, int32_t g, int32_t topk,
+                                   size_t* bytes) {
+    if (!bytes) return fail(SSA_ERR_INVALID_ARG, "bytes is NULL");
+    ssa::Plan p;
+    ssa_status st = build_single(p, shape, C, g, topk);
+    if (st != SSA_OK) return st;
+    size_t off[4];
+    *bytes = host_staging(p, ssa::plan_bytes_any(p), off);
+    return SSA_OK;
+}
+
+ssa_status ssa_decode_host(const ssa_shape* shape, const void* q_host, const void* k_raw,
+                           const void* v_raw, const void* k_gist, const void* v_gist,
+                           const int32_t* seq_lens_host, int32_t C, int32_t g, int32_t topk,
+                           float* out_host, int32_t* sel_idx_host, void* ws, size_t ws_bytes,
+                           cudaStream_t stream) {
+    ssa::Plan p;
+    ssa_status st = build_single(p, shape, C, g, topk);
+    if (st != SSA_OK) return st;
+    if (!q_host || !seq_lens_host || !out_host || (topk > 0 && !sel_idx_host))
+        return fail(SSA_ERR_INVALID_ARG, "a host buffer is NULL");
+    if (!ws) return fail(SSA_ERR_WORKSPACE, "ssa_decode_host needs a workspace");
+    const size_t base = ssa::plan_bytes_any(p);
+    size_t off[4];
+    const size_t need = host_staging(p, base, off);
+    if (ws_bytes < need)
+        return fail(SSA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+    char* w = static_cast<char*>(ws);
+    const size_t e = p.dtype == SSA_BF16 ? 2 : 4;
+    const size_t qb = (size_t)p.B * p.Hq * p.d * e, ob = (size_t)p.B * p.Hq * p.d * 4;
+    const size_t sb = (size_t)p.n_pairs * topk * 4;
+    cudaError_t ce = cudaMemcpyAsync(w + off[0], q_host, qb, cudaMemcpyHostToDevice, stream);
+    if (ce == cudaSuccess)
+        ce = cudaMemcpyAsync(w + off[1], seq_lens_host, (size_t)p.B * 4, cudaMemcpyHostToDevice,
+                             stream);
+    if (ce != cudaSuccess) return cuda_fail(ce, "cudaMemcpyAsync(host to device)");
+    st = ssa_decode(shape, w + off[0], k_raw, v_raw, k_gist, v_gist,
+                    reinterpret_cast<const int32_t*>(w + off[1]), C, g, topk,
+                    reinterpret_cast<float*>(w + off[2]), reinterpret_cast<int32_t*>(w + off[3]),
+                    ws, base, stream);
+    if (st != SSA_OK) return st;
+    ce = cudaMemcpyAsync(out_host, w + off[2], ob, cudaMemcpyDeviceToHost, stream);
+    if (ce == cudaSuccess && sb > 0)
+        ce = cudaMemcpyAsync(sel_idx_host, w + off[3], sb, cudaMemcpyDeviceToHost, stream);
+    if (ce != cudaSuccess) return cuda_fail(ce, "cudaMemcpyAsync(device to host)");
+    return SSA_OK;
 }
 
 ssa_status ssa_decode_noalloc(const ssa_shape* shape, const void* q, const void* k_raw,

@@ -1164,13 +1164,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     __syncwarp();
                 }
                 // excluded rows: past the valid rows, or in a selected chunk
+                // (the selected-only context excludes the unselected ones)
+                const bool keep_selected = p.ctx_mode == 1;
                 uint32_t ex[2];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const int r = lane + 32 * hh;
                     const int sr = d.off + r;
                     const int c = min(p.g_shift >= 0 ? (sr >> p.g_shift) : sr / p.g, d.nch - 1);
-                    const bool e = (r >= nv) | (((bits[c >> 5] >> (c & 31)) & 1u) != 0u);
+                    const bool in_sel = ((bits[c >> 5] >> (c & 31)) & 1u) != 0u;
+                    const bool e = (r >= nv) | (in_sel != keep_selected);
                     ex[hh] = __ballot_sync(0xffffffffu, e);
                 }
                 // head g8's kept logits of rows r0 + 2 tig, + 1, + 8, + 9

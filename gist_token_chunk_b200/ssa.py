@@ -73,6 +73,8 @@ lib.ssa_decode_variant.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, 
 lib.ssa_workspace_size_variant.argtypes = [_SH, _I, _I, _I, _I, _I, ctypes.POINTER(_S)]
 _PP = ctypes.POINTER(ctypes.c_void_p)
 _IP = ctypes.POINTER(ctypes.c_int32)
+lib.ssa_decode_host.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _S, _P]
+lib.ssa_workspace_size_host.argtypes = [_SH, _I, _I, _I, ctypes.POINTER(_S)]
 lib.ssa_decode_hier.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _PP, _PP, _IP, _IP,
                                 _P, _PP, _P, _S, _P]
 lib.ssa_workspace_size_hier.argtypes = [_SH, _I, _I, _I, _I, _IP, _IP, ctypes.POINTER(_S)]
@@ -92,7 +94,8 @@ lib.ssa_last_error.restype = ctypes.c_char_p
 lib.ssa_version.restype = _I
 for _f in ("ssa_score_gists", "ssa_topk_chunks", "ssa_sparse_decode", "ssa_decode",
            "ssa_decode_path", "ssa_decode_variant", "ssa_workspace_size_variant",
-           "ssa_decode_hier", "ssa_workspace_size_hier",
+           "ssa_decode_hier", "ssa_workspace_size_hier", "ssa_decode_host",
+           "ssa_workspace_size_host",
            "ssa_decode_noalloc", "ssa_decode_h2", "ssa_workspace_size",
            "ssa_workspace_size_h2", "ssa_workspace_init", "ssa_get_device_status"):
     getattr(lib, _f).restype = _I
@@ -295,6 +298,27 @@ def ssa_decode_hier(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C: int, g: int, J
                                _i32_array(g_sum), _i32_array(topk), _ptr(out), sp, _ptr(ws),
                                nbytes, _stream(stream)), "ssa_decode_hier")
     return out, [s[:, :, :int(k)] for s, k in zip(sels, topk)]
+
+
+def ssa_workspace_size_host(shape: Shape, C: int, g: int, topk: int) -> int:
+    n = _S(0)
+    _check(lib.ssa_workspace_size_host(ctypes.byref(shape), C, g, topk, ctypes.byref(n)),
+           "ssa_workspace_size_host")
+    return int(n.value)
+
+
+def ssa_decode_host(q_host, k_raw, v_raw, k_gist, v_gist, seq_lens_host, C: int, g: int,
+                    topk: int, out_host, sel_idx_host, ws, stream=None):
+    """ssa_decode with q, seq_lens, out and sel_idx in (pinned) host memory;
+    the copies and the step are stream-ordered (see include/ssa.h)."""
+    B, Hq, d = q_host.shape
+    shape = make_shape(B, Hq, k_raw.shape[1], d, k_raw.shape[2], _dtype_code(q_host))
+    _check(lib.ssa_decode_host(ctypes.byref(shape), _ptr(q_host), _ptr(k_raw), _ptr(v_raw),
+                               _ptr(k_gist), _ptr(v_gist), _ptr(seq_lens_host), C, g, topk,
+                               _ptr(out_host), _ptr(sel_idx_host), _ptr(ws),
+                               ws.numel() * ws.element_size(), _stream(stream)),
+           "ssa_decode_host")
+    return out_host, sel_idx_host
 
 
 def ssa_decode_noalloc(q, k_raw, v_raw, k_gist, v_gist, seq_lens, C: int, g: int, topk: int,

@@ -154,6 +154,31 @@ SSA_API ssa_status ssa_decode(const ssa_shape* shape, const void* q, const void*
                       int32_t* sel_idx, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * ssa_decode_host -- ssa_decode with the step's small tensors in HOST memory:
+ * q_host [B,Hq,d] (the shape's dtype) and seq_lens_host [B] are copied to the
+ * device, the step runs, and out_host fp32 [B,Hq,d] and sel_idx_host int32
+ * [B,Hkv,topk] are copied back, all stream-ordered on `stream` (one
+ * cudaMemcpyAsync per tensor).  The KV cache (k_raw, v_raw, k_gist, v_gist)
+ * is device memory, as in ssa_decode.  The device copies live in the
+ * workspace, which must hold ssa_workspace_size_host() bytes (ws must not be
+ * NULL).  Host buffers should be page-locked for the copies to be
+ * asynchronous; pageable ones work, but their copies block the host.  The
+ * host outputs are complete once the stream has passed this call
+ * (synchronize, or wait on an event recorded after it).  A library
+ * convenience for callers whose per-step tensors live on the host; the pages
+ * have no counterpart.
+ */
+SSA_API ssa_status ssa_decode_host(const ssa_shape* shape, const void* q_host, const void* k_raw,
+                                   const void* v_raw, const void* k_gist, const void* v_gist,
+                                   const int32_t* seq_lens_host, int32_t C, int32_t g,
+                                   int32_t topk, float* out_host, int32_t* sel_idx_host, void* ws,
+                                   size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes needed by ssa_decode_host for these sizes. */
+SSA_API ssa_status ssa_workspace_size_host(const ssa_shape* shape, int32_t C, int32_t g,
+                                           int32_t topk, size_t* bytes);
+
+/*
  * ssa_decode_noalloc -- ssa_decode for callers that cannot allocate device
  * memory and cannot pass a workspace: for example an engine that reserves all
  * device memory for itself before serving, or a plugin interface that hands
@@ -220,10 +245,12 @@ SSA_API ssa_status ssa_decode_h2(const ssa_shape* shape, const void* q, const vo
  *     before their union").
  * Out: out fp32 [B,Hq,d]; sel_idx int32 [B,Hkv,cap], the selection ascending
  * and -1 padded, cap = topk (group max) or G * topk (head union).
- * Runs on the library's portable kernels (every dtype and head dim the
- * library accepts).  Needs ssa_workspace_size_variant() bytes of workspace
- * (ws = NULL: allocated stream-ordered).  Errors as ssa_decode; an unknown
- * context or select value -> SSA_ERR_INVALID_ARG.
+ * The group-max selection on a shape the two-kernel pipeline takes (see
+ * ssa_decode_path) runs there, either context; everything else runs on the
+ * library's portable kernels (every dtype and head dim the library accepts).
+ * Needs ssa_workspace_size_variant() bytes of workspace (ws = NULL:
+ * allocated stream-ordered).  Errors as ssa_decode; an unknown context or
+ * select value -> SSA_ERR_INVALID_ARG.
  */
 #define SSA_CONTEXT_UNSELECTED_GISTS 0
 #define SSA_CONTEXT_SELECTED_ONLY 1

@@ -181,3 +181,24 @@ def test_fused_equals_components(ssa, inp):
     out2 = ssa.ssa_sparse_decode(inp["q"], inp["k_raw"], inp["v_raw"], inp["k_gist"],
                                  inp["v_gist"], inp["seq_lens"], W1.C, W1.g, W1.topk, sel2)
     assert (out - out2).abs().max().item() <= 1e-6
+
+
+def test_decode_host_buffers_equal_device_call(ssa, inp):
+    """ssa_decode_host (pinned and pageable host buffers) gives ssa_decode's
+    results."""
+    out_d, sel_d = run(ssa, inp)
+    sh = ssa.shape_of(inp["q"], inp["k_raw"])
+    ws = ssa.workspace(ssa.ssa_workspace_size_host(sh, W1.C, W1.g, W1.topk))
+    for pin in (True, False):
+        q = inp["q"].cpu()
+        lens = inp["seq_lens"].cpu()
+        out = torch.empty(out_d.shape, dtype=torch.float32)
+        sel = torch.empty(sel_d.shape, dtype=torch.int32)
+        if pin:
+            q, lens, out, sel = q.pin_memory(), lens.pin_memory(), out.pin_memory(), sel.pin_memory()
+        ssa.ssa_decode_host(q, inp["k_raw"], inp["v_raw"], inp["k_gist"], inp["v_gist"], lens,
+                            W1.C, W1.g, W1.topk, out, sel, ws)
+        torch.cuda.synchronize()
+        assert ssa.ssa_get_device_status() == 0
+        assert torch.equal(sel, sel_d.cpu())
+        assert (out - out_d.cpu()).abs().max().item() <= 1e-6
