@@ -29,6 +29,7 @@ Multi-GPU: one process per GPU (torchrun); each rank decodes its own batch
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import math
@@ -94,6 +95,38 @@ def algorithmic_bytes(w, seq_lens) -> int:
 
 
 # ------------------------------------------------------------ host cost ---
+
+def cuda_runtime():
+    """The CUDA runtime that torch loaded, through ctypes (copies and events
+    for the end-to-end leg, at a microsecond per call)."""
+    import ctypes
+
+    names = ["libcudart.so.12", "libcudart.so"]
+    try:
+        import nvidia.cuda_runtime as ncr
+
+        names.insert(0, os.path.join(list(ncr.__path__)[0], "lib", "libcudart.so.12"))
+    except Exception:
+        pass
+    lib = None
+    for n in names:
+        try:
+            lib = ctypes.CDLL(n)
+            break
+        except OSError:
+            continue
+    if lib is None:
+        raise SystemExit("CUDA runtime library not found")
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    lib.cudaMemcpyAsync.argtypes = [vp, vp, sz, ctypes.c_int, vp]
+    lib.cudaEventRecord.argtypes = [vp, vp]
+    lib.cudaStreamWaitEvent.argtypes = [vp, vp, ctypes.c_uint]
+    lib.cudaEventCreateWithFlags.argtypes = [ctypes.POINTER(vp), ctypes.c_uint]
+    for f in ("cudaMemcpyAsync", "cudaEventRecord", "cudaStreamWaitEvent",
+              "cudaEventCreateWithFlags"):
+        getattr(lib, f).restype = ctypes.c_int
+    return lib
+
 
 def host_call_cost(ssa, w, x, out, sel, sup, ws, stream, calls: int = 200) -> dict:
     """Host microseconds one decode call costs: through the Python binding,
@@ -561,6 +594,12 @@ def main():
     if hier:
         kernel_name = "ssa::gen hier_score, hier_topk (per level) and hier_attend kernels"
         launches_per_step = 2 * len(hier[2]) + 1
+    elif variant and (ssa.ssa_decode_path(shape, w.C, w.g, w.topk) == ssa.SSA_PATH_PIPELINE
+                      and w.G * w.topk <= 1024):
+        # the variants run on the pipeline wherever ssa_decode does
+        kernel_name = ("ssa::pipe::score_kernel + ssa::pipe::attend_kernel<true>" if variant[1]
+                       else "ssa::pipe::score_kernel + ssa::pipe::attend_kernel<false>")
+        launches_per_step = 2
     elif variant:
         kernel_name = ("ssa::gen head_score, head_topk, union and attend kernels" if variant[1]
                        else "ssa::gen score, top-k and attend kernels")
@@ -570,7 +609,7 @@ def main():
     else:
         path = ssa.ssa_decode_path(shape, w.C, w.g, w.topk)
         kernel_name, launches_per_step = {
-            ssa.SSA_PATH_PIPELINE: ("ssa::pipe::score_kernel + ssa::pipe::attend_kernel", 2),
+            ssa.SSA_PATH_PIPELINE: ("ssa::pipe::score_kernel + ssa::pipe::attend_kernel<false>", 2),
             ssa.SSA_PATH_FUSED: (f"ssa::fused::fused_kernel<{w.d}>", 1),
         }.get(path, ("ssa::gen score, top-k and attend kernels", 3))
 
@@ -672,32 +711,47 @@ def main():
     # Copies run on their own streams so that step i+1's upload and step i's
     # download overlap the decode kernels; events keep each set's buffers
     # ordered: upload -> decode -> download -> the set's next upload/decode.
+    # The copies and the event operations go straight to the CUDA runtime
+    # (ctypes), a microsecond each, so that the host issues a step faster
+    # than the device runs it; the decode itself is the public call.
+    cr = cuda_runtime()
     up_stream = torch.cuda.Stream(device=dev)
     down_stream = torch.cuda.Stream(device=dev)
-    up_done = [torch.cuda.Event() for _ in range(NS)]
-    dec_done = [torch.cuda.Event() for _ in range(NS)]
-    down_done = [torch.cuda.Event() for _ in range(NS)]
-    for s in range(NS):
-        dec_done[s].record(stream)
-        down_done[s].record(stream)
+    sh_main, sh_up, sh_down = stream.cuda_stream, up_stream.cuda_stream, down_stream.cuda_stream
+
+    def new_event():
+        ev = ctypes.c_void_p()
+        if cr.cudaEventCreateWithFlags(ctypes.byref(ev), 2) != 0:  # cudaEventDisableTiming
+            raise SystemExit("cudaEventCreateWithFlags failed")
+        return ev
+
+    up_done = [new_event() for _ in range(NS)]
+    dec_done = [new_event() for _ in range(NS)]
+    down_done = [new_event() for _ in range(NS)]
+    for s_i in range(NS):
+        cr.cudaEventRecord(dec_done[s_i], sh_main)
+        cr.cudaEventRecord(down_done[s_i], sh_main)
+    e2e_x, e2e_bufs = [], []
+    for s_i in range(NS):
+        dbuf, (q_dev, len_dev) = up_dev[s_i]
+        obuf, (o_dev, s_dev) = down_dev[s_i]
+        e2e_x.append(dict(sets[s_i], q=q_dev, seq_lens=len_dev))
+        e2e_bufs.append((dbuf.data_ptr(), up_host[s_i].data_ptr(), dbuf.numel(), o_dev, s_dev,
+                         down_host[s_i].data_ptr(), obuf.data_ptr(), obuf.numel()))
 
     def e2e_step(i):
-        s = i % NS
-        dbuf, (q_dev, len_dev) = up_dev[s]
-        up_stream.wait_event(dec_done[s])       # the set's last decode has read q
-        with torch.cuda.stream(up_stream):
-            dbuf.copy_(up_host[s], non_blocking=True)
-        up_done[s].record(up_stream)
-        stream.wait_event(up_done[s])
-        stream.wait_event(down_done[s])         # the set's last output has been read back
-        x = dict(sets[s], q=q_dev, seq_lens=len_dev)
-        obuf, (o_dev, s_dev) = down_dev[s]
-        decode_call(x, s, o_dev, s_dev, stream)
-        dec_done[s].record(stream)
-        down_stream.wait_event(dec_done[s])
-        with torch.cuda.stream(down_stream):
-            down_host[s].copy_(obuf, non_blocking=True)
-        down_done[s].record(down_stream)
+        s_i = i % NS
+        dptr, hptr, nup, o_dev, s_dev, hout, optr, ndown = e2e_bufs[s_i]
+        cr.cudaStreamWaitEvent(sh_up, dec_done[s_i], 0)      # the set's last decode read q
+        cr.cudaMemcpyAsync(dptr, hptr, nup, 1, sh_up)        # host to device
+        cr.cudaEventRecord(up_done[s_i], sh_up)
+        cr.cudaStreamWaitEvent(sh_main, up_done[s_i], 0)
+        cr.cudaStreamWaitEvent(sh_main, down_done[s_i], 0)   # its last output was read back
+        decode_call(e2e_x[s_i], s_i, o_dev, s_dev, stream)
+        cr.cudaEventRecord(dec_done[s_i], sh_main)
+        cr.cudaStreamWaitEvent(sh_down, dec_done[s_i], 0)
+        cr.cudaMemcpyAsync(hout, optr, ndown, 2, sh_down)    # device to host
+        cr.cudaEventRecord(down_done[s_i], sh_down)
 
     e2e_value = None
     if ek > 0:
@@ -715,8 +769,8 @@ def main():
             for i in range(ek):
                 e2e_step(i)
             host_issue_s = time.perf_counter() - h0
-            for s in range(NS):
-                stream.wait_event(down_done[s])
+            for s_i in range(NS):
+                cr.cudaStreamWaitEvent(sh_main, down_done[s_i], 0)
             ev1.record(stream)
         ev1.synchronize()
         e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), pg, dev)

@@ -625,7 +625,7 @@ ssa_status ssa_workspace_size_variant(const ssa_shape* shape, int32_t C, int32_t
     size_t a, b;
     *bytes = variant_layout(p, &a, &b);
     // the group-max selection may run on the two-kernel pipeline
-    if (select == SSA_SELECT_GROUP_MAX && ssa::pipe_prepare(p)) {
+    if (ssa::pipe_prepare(p)) {
         const size_t pb = ssa::plan_bytes_any(p);
         if (pb > *bytes) *bytes = pb;
     }
@@ -652,9 +652,9 @@ ssa_status ssa_decode_variant(const ssa_shape* shape, const void* q, const void*
     p.seq_lens = seq_lens;
     p.sel_idx = sel_idx;
     p.out = out;
-    // group max on a pipeline shape: the two-kernel path, whose attention
-    // kernel applies either context's keep predicate
-    if (p.sel_mode == 0 && ssa::pipe_prepare(p)) return run_with_ws(p, ws, ws_bytes, stream);
+    // a pipeline shape: the two-kernel path, whose attention kernel applies
+    // either context's keep predicate and either selection
+    if (ssa::pipe_prepare(p)) return run_with_ws(p, ws, ws_bytes, stream);
     size_t so, ho;
     const size_t need = variant_layout(p, &so, &ho);
     void* own = nullptr;

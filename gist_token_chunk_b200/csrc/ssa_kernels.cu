@@ -265,6 +265,7 @@ bool pipe_prepare(Plan& p) {
     p.pp_w1 = p.pp_w3 = 0;
     if (p.mode != kModeFull || p.h2 || p.dtype != 0 || p.d != pipe::kD) return false;
     if (p.G > pipe::kMaxG || p.topk > 128 || p.M_max > 8192 || p.B > kFusedMaxB) return false;
+    if (p.sel_stride > 1024) return false;  // published selection entries
     if (p.debug_flags & 2) return false;  // the fused kernel, for comparisons
     const int nsm = sm_count();
     if (nsm > pipe::kMaxBlocks) return false;
@@ -297,7 +298,7 @@ bool pipe_prepare(Plan& p) {
     p.st_slot_bytes = pipe::kRecBytes;
     // one partial slot per (attention worker + pair) index of the launch
     p.st_part_slots = nsm * p.pp_w3 + p.n_pairs;
-    p.st_sel_stride = pipe::sel_stride(p.topk);
+    p.st_sel_stride = pipe::sel_stride(p.sel_stride);
     return true;
 }
 
@@ -326,8 +327,11 @@ cudaError_t launch_pipe(const Plan& p, cudaStream_t stream) {
         cudaError_t e = cudaFuncSetAttribute(pipe::score_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(pipe::attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     227 * 1024);
+            e = cudaFuncSetAttribute(pipe::attend_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(pipe::attend_kernel<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = 1;
     }
@@ -353,7 +357,8 @@ cudaError_t launch_pipe(const Plan& p, cudaStream_t stream) {
     c3.stream = stream;
     c3.attrs = pdl;
     c3.numAttrs = 1;
-    return cudaLaunchKernelEx(&c3, pipe::attend_kernel, p, m[1], m[2], m[3]);
+    return p.sel_mode == 1 ? cudaLaunchKernelEx(&c3, pipe::attend_kernel<true>, p, m[1], m[2], m[3])
+                           : cudaLaunchKernelEx(&c3, pipe::attend_kernel<false>, p, m[1], m[2], m[3]);
 }
 
 cudaError_t launch_fused(const Plan& p, cudaStream_t stream) {

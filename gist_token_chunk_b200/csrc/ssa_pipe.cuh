@@ -109,7 +109,9 @@ __device__ __forceinline__ int list_count(const Plan& p, int L, int n) {
     if (L == 0) return M;
     const int T = n - M * p.C;
     const int tpc = (p.C + kRawRows - 1) / kRawRows;
-    return min(p.topk, M) * tpc + (T + kRawRows - 1) / kRawRows;
+    // selected chunks: k, or at most G k under the per-head union (unused
+    // slots become empty tiles)
+    return min(p.sel_stride, M) * tpc + (T + kRawRows - 1) / kRawRows;
 }
 
 // The plan every block computes from seq_lens: lengths and per-list prefix
@@ -330,7 +332,7 @@ __host__ __device__ inline ScoreLayout score_layout(const Plan& p, int workers) 
 }
 
 struct AttnLayout {
-    int ring, lgs, qs, bars, desc, bits, sel, tk, selout, plan, misc, total;
+    int ring, lgs, qs, bars, desc, bits, sel, tk, selout, ubits, plan, misc, total;
     int lgbytes, qbytes, bwords, kcap;
 };
 __host__ __device__ inline AttnLayout attn_layout(const Plan& p, int workers) {
@@ -350,10 +352,11 @@ __host__ __device__ inline AttnLayout attn_layout(const Plan& p, int workers) {
     L.desc = take(workers * kAttnStages * (int)sizeof(Desc));
     L.bwords = (p.M_max + 31) / 32;
     L.bits = take(workers * L.bwords * 4);
-    L.kcap = p.topk > 0 ? p.topk : 1;
+    L.kcap = p.sel_stride > 0 ? p.sel_stride : 1;  // entries of a published selection
     L.sel = take(workers * 2 * L.kcap * 4);
     L.tk = take((int)sizeof(TopkScratch));
     L.selout = take(L.kcap * 4);
+    L.ubits = take(p.sel_mode ? L.bwords * 4 : 0);  // per-head union: chunk bitmap
     L.plan = take((p.B + 2 * (p.B + 1)) * 4);
     L.misc = take(64);
     L.total = o + 1024;
@@ -788,6 +791,9 @@ __device__ __forceinline__ bool fast_topk128(const float* scores, int M, int top
 // first word; a control warp combines the partials of its (pair, query
 // head) tasks as they complete (every wait bounded); the last block to
 // finish moves the epoch on.
+// kUnion: the per-head union selection (a separate instantiation, so that
+// its code does not weigh on the registers of the default one).
+template <bool kUnion>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attend_kernel(const __grid_constant__ Plan p, const __grid_constant__ CUtensorMap tm_vg,
                   const __grid_constant__ CUtensorMap tm_kr,
@@ -860,7 +866,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (cpair1 == pair) return 1;
             const int e = (cpair0 == keep && keep >= 0) ? 1 : 0;
             int* dst = selc + e * L.kcap;
-            const int k = min(p.topk, nb[pair / p.Hkv] / p.C);
+            const int k = min(p.sel_stride, nb[pair / p.Hkv] / p.C);
             const unsigned long long* src = p.st_sel + (size_t)pair * p.st_sel_stride;
             const long long c0 = clock64();
             for (;;) {
@@ -876,12 +882,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     __syncwarp();
                     if (!done && !blocking) return -1;
                     if (give_up && lane == 0) report_status(kStatusTimeout);
+                    // the chunks are the leading non-negative entries (a
+                    // per-head union pads its slots with -1)
+                    int cnt = 0;
+                    for (int i = lane; i < k; i += 32) cnt += dst[i] >= 0;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
                     if (e == 0) {
                         cpair0 = pair;
-                        ccount0 = done ? k : 0;
+                        ccount0 = done ? cnt : 0;
                     } else {
                         cpair1 = pair;
-                        ccount1 = done ? k : 0;
+                        ccount1 = done ? cnt : 0;
                     }
                     return e;
                 }
@@ -1004,18 +1016,59 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         bool selected = false;
         int* selout = reinterpret_cast<int*>(smem + L.selout);
         TopkScratch& tks = *reinterpret_cast<TopkScratch*>(smem + L.tk);
+        // Per-head union (App. A): each head of the group ranks the chunks by
+        // its own score, the max over the chunk's gist rows of its kept logit
+        // (log2 domain: the same order as q.k / sqrt(d)), written over the
+        // pair's group-max scores one head at a time; the heads' top-k's are
+        // ORed into a chunk bitmap and compacted in chunk order.
+        uint32_t* ubits = reinterpret_cast<uint32_t*>(smem + L.ubits);
+        auto union_selection = [&](int pr, int M) {
+            const int t = threadIdx.x;
+            float* hs = p.pp_scores + (size_t)pr * score_row(p.M_max);
+            const int W = (M + 31) >> 5;
+            for (int i = t; i < W; i += 128) ubits[i] = 0u;
+            for (int h = 0; h < G; ++h) {
+                const float* lg = p.pp_logits + (size_t)pr * p.M_max * p.g * GP + h;
+                for (int m = t; m < M; m += 128) {
+                    float best = -INFINITY;
+                    for (int r = 0; r < p.g; ++r) best = fmaxf(best, __ldcg(lg + ((size_t)m * p.g + r) * GP));
+                    hs[m] = best;
+                }
+                named_sync(1, 128);
+                if (M > 1024 || !fast_topk128(hs, M, p.topk, selout, tks))
+                    block_topk<128>(hs, M, p.topk, selout, tks, Sync128());
+                named_sync(1, 128);
+                for (int i = t; i < min(p.topk, M); i += 128)
+                    atomicOr(&ubits[selout[i] >> 5], 1u << (selout[i] & 31));
+                named_sync(1, 128);
+            }
+            const int per = (W + 127) / 128;
+            const int w0 = t * per, w1 = min(w0 + per, W);
+            int cnt = 0;
+            for (int i = w0; i < w1; ++i) cnt += __popc(ubits[i]);
+            int tot;
+            int at = scan128(cnt, tks.scan, tot);
+            for (int i = w0; i < w1; ++i)
+                for (uint32_t x = ubits[i]; x; x &= x - 1) selout[at++] = i * 32 + __ffs(x) - 1;
+            for (int i = tot + t; i < p.sel_stride; i += 128) selout[i] = -1;
+            named_sync(1, 128);
+        };
         auto run_selection = [&]() {
             if (warp >= 4 || p.topk <= 0 || (int)blockIdx.x >= p.n_pairs) return;
             for (int pr = blockIdx.x; pr < p.n_pairs; pr += gridDim.x) {
                 const int M = nb[pr / p.Hkv] / p.C;
-                const int k = min(p.topk, M);
-                const float* sc = p.pp_scores + (size_t)pr * score_row(p.M_max);
-                if (M > 1024 || !fast_topk128(sc, M, p.topk, selout, tks))
-                    block_topk<128>(sc, M, p.topk, selout, tks, Sync128());
-                named_sync(1, 128);
+                const int k = min(p.sel_stride, M);  // published entries
+                if constexpr (kUnion) {
+                    union_selection(pr, M);
+                } else {
+                    const float* sc = p.pp_scores + (size_t)pr * score_row(p.M_max);
+                    if (M > 1024 || !fast_topk128(sc, M, p.topk, selout, tks))
+                        block_topk<128>(sc, M, p.topk, selout, tks, Sync128());
+                    named_sync(1, 128);
+                }
                 unsigned long long* pub = p.st_sel + (size_t)pr * p.st_sel_stride;
-                int32_t* user = p.sel_idx + (size_t)pr * p.topk;
-                for (int i = threadIdx.x; i < p.topk; i += 128) {
+                int32_t* user = p.sel_idx + (size_t)pr * p.sel_stride;
+                for (int i = threadIdx.x; i < p.sel_stride; i += 128) {
                     const int c = selout[i];
                     user[i] = c;
                     if (i < k && !(p.debug_flags & 1))
@@ -1058,7 +1111,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     const int pr = cr.pair;
                     const int n = nb[pr / p.Hkv];
                     const int M = n / p.C;
-                    const int kc = min(p.topk, M);
+                    const int kc = min(p.sel_stride, M);
                     const int u = cr.i0 + cr.off;
                     int r0, nv;
                     if (u < kc * tpc) {
@@ -1106,16 +1159,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         bulk_load(lgs + s * L.lgbytes, p.pp_logits + (size_t)y * GP,
                                   (uint32_t)L.lgbytes, &full[s]);
                     } else {
+                        // an empty tile (an unused slot of a per-head union)
+                        // loads nothing but the query
                         const bool wq = (d.flags & F_Q) != 0;
-                        mbar_arrive_expect_tx(&full[s], (uint32_t)(kSlotBytes + (wq ? G * kD * 2 : 0)));
+                        const bool any = d.nvalid > 0;
+                        mbar_arrive_expect_tx(&full[s], (uint32_t)((any ? kSlotBytes : 0) +
+                                                                   (wq ? G * kD * 2 : 0)));
                         if (wq) {
                             const int b = d.pair / p.Hkv, j = d.pair - b * p.Hkv;
                             const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.q) +
                                                        ((size_t)b * p.Hq + (size_t)j * G) * kD;
                             bulk_load(qs + s * L.qbytes, src, (uint32_t)(G * kD * 2), &full[s]);
                         }
-                        tma_load_2d_hint(dst, &tm_kr, 0, y, &full[s], pol);
-                        tma_load_2d_hint(dst + kSlotBytes / 2, &tm_vr, 0, y, &full[s], pol);
+                        if (any) {
+                            tma_load_2d_hint(dst, &tm_kr, 0, y, &full[s], pol);
+                            tma_load_2d_hint(dst + kSlotBytes / 2, &tm_vr, 0, y, &full[s], pol);
+                        }
                     }
                 }
                 __syncwarp();

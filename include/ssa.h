@@ -245,8 +245,8 @@ SSA_API ssa_status ssa_decode_h2(const ssa_shape* shape, const void* q, const vo
  *     before their union").
  * Out: out fp32 [B,Hq,d]; sel_idx int32 [B,Hkv,cap], the selection ascending
  * and -1 padded, cap = topk (group max) or G * topk (head union).
- * The group-max selection on a shape the two-kernel pipeline takes (see
- * ssa_decode_path) runs there, either context; everything else runs on the
+ * On a shape the two-kernel pipeline takes (see ssa_decode_path) both
+ * readings run there, when G * topk <= 1024; everything else runs on the
  * library's portable kernels (every dtype and head dim the library accepts).
  * Needs ssa_workspace_size_variant() bytes of workspace (ws = NULL:
  * allocated stream-ordered).  Errors as ssa_decode; an unknown context or
