@@ -97,6 +97,58 @@ __global__ void score_kernel(Plan p, int level, float* dst, int stride, int n_sl
     }
 }
 
+// Online softmax of one query (qs, fp32 in shared memory, log2-domain scale)
+// over `rows` key/value rows, by one warp, 32 rows at a time: lane j takes
+// the dot product of row r0 + j (its loads independent of the other lanes'),
+// the warp shares one maximum and one sum per group, and each lane
+// accumulates its dims (lane + 32 r) over the group's rows.  m_run, l_run,
+// acc are the warp's running state (same values in every lane).
+template <class T>
+__device__ __forceinline__ void attend_rows(const float* qs, const T* kbase, const T* vbase,
+                                            int rows, int d, float scale, float& m_run,
+                                            float& l_run, float (&acc)[8]) {
+    const int lane = threadIdx.x & 31;
+    for (int r0 = 0; r0 < rows; r0 += 32) {
+        const int r = r0 + lane;
+        const int nr = min(32, rows - r0);
+        float x = -INFINITY;
+        if (r < rows) {
+            const T* kr = kbase + (size_t)r * d;
+            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+            int i = 0;
+            for (; i + 4 <= d; i += 4) {
+                s0 += qs[i] * to_f(kr[i]);
+                s1 += qs[i + 1] * to_f(kr[i + 1]);
+                s2 += qs[i + 2] * to_f(kr[i + 2]);
+                s3 += qs[i + 3] * to_f(kr[i + 3]);
+            }
+            for (; i < d; ++i) s0 += qs[i] * to_f(kr[i]);
+            x = (s0 + s1 + s2 + s3) * scale;
+        }
+        float mx = x;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float mn = fmaxf(m_run, mx);
+        const float ref = mn == -INFINITY ? 0.f : mn;
+        const float a = exp2f(m_run - ref);
+        const float e = r < rows ? exp2f(x - ref) : 0.f;
+        l_run = l_run * a + warp_sum(e);
+        m_run = mn;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] *= a;
+#pragma unroll 4
+        for (int j = 0; j < nr; ++j) {
+            const float ej = __shfl_sync(0xffffffffu, e, j);
+            const T* vr = vbase + (size_t)(r0 + j) * d;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int i = lane + 32 * q;
+                if (i < d) acc[q] += ej * to_f(vr[i]);
+            }
+        }
+    }
+}
+
 // Per-head chunk scores (selection reading "per head + union", App. A):
 // dst[row * M_max + m] = max over the chunk's g gist rows of q_h.k/sqrt(d)
 // for row = b * Hq + h, m < M_b; -inf for M_b <= m < M_max.
@@ -295,21 +347,7 @@ __global__ void attend_kernel(Plan p, const int* bad) {
     for (int r = 0; r < 8; ++r) acc[r] = 0.f;
 
     auto visit = [&](const T* kbase, const T* vbase, int rows) {
-        for (int t = 0; t < rows; ++t) {
-            float x = 0.f;
-            for (int i = lane; i < p.d; i += 32) x += qs[i] * to_f(kbase[(size_t)t * p.d + i]);
-            x = warp_sum(x) * scale;
-            float mn = fmaxf(m_run, x);
-            float a = exp2f(m_run - mn);
-            float e = exp2f(x - mn);
-            l_run = l_run * a + e;
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                int i = lane + 32 * r;
-                if (i < p.d) acc[r] = acc[r] * a + e * to_f(vbase[(size_t)t * p.d + i]);
-            }
-            m_run = mn;
-        }
+        attend_rows<T>(qs, kbase, vbase, rows, p.d, scale, m_run, l_run, acc);
     };
     // ctx_mode 0: a selected chunk contributes its raw tokens, an unselected
     // one its gists; ctx_mode 1: a selected chunk its gists and raw tokens,
@@ -500,21 +538,7 @@ __global__ void hier_attend_kernel(Plan p, HierLevels hl) {
 #pragma unroll
     for (int r = 0; r < 8; ++r) acc[r] = 0.f;
     auto visit = [&](const T* kbase, const T* vbase, int rows) {
-        for (int t = 0; t < rows; ++t) {
-            float x = 0.f;
-            for (int i = lane; i < p.d; i += 32) x += qs[i] * to_f(kbase[(size_t)t * p.d + i]);
-            x = warp_sum(x) * scale;
-            const float mn = fmaxf(m_run, x);
-            const float a = exp2f(m_run - mn);
-            const float e = exp2f(x - mn);
-            l_run = l_run * a + e;
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const int i = lane + 32 * r;
-                if (i < p.d) acc[r] = acc[r] * a + e * to_f(vbase[(size_t)t * p.d + i]);
-            }
-            m_run = mn;
-        }
+        attend_rows<T>(qs, kbase, vbase, rows, p.d, scale, m_run, l_run, acc);
     };
     for (int l = hl.levels - 1; l >= 0; --l) {
         int nkept;
