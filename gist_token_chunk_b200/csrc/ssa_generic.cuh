@@ -108,9 +108,22 @@ __device__ __forceinline__ void attend_rows(const float* qs, const T* kbase, con
                                             int rows, int d, float scale, float& m_run,
                                             float& l_run, float (&acc)[8]) {
     const int lane = threadIdx.x & 31;
+    const int row_bytes = d * (int)sizeof(T);
+    // L2 prefetch of row r's key and value lines (each lane one row)
+    auto prefetch_row = [&](int r) {
+        if (r >= rows) return;
+        const char* kp = reinterpret_cast<const char*>(kbase + (size_t)r * d);
+        const char* vp = reinterpret_cast<const char*>(vbase + (size_t)r * d);
+        for (int o = 0; o < row_bytes; o += 128) {
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(kp + o));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(vp + o));
+        }
+    };
+    prefetch_row(lane);
     for (int r0 = 0; r0 < rows; r0 += 32) {
         const int r = r0 + lane;
         const int nr = min(32, rows - r0);
+        prefetch_row(r + 32);  // the next group's rows, while this one computes
         float x = -INFINITY;
         if (r < rows) {
             const T* kr = kbase + (size_t)r * d;
@@ -136,7 +149,7 @@ __device__ __forceinline__ void attend_rows(const float* qs, const T* kbase, con
         m_run = mn;
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] *= a;
-#pragma unroll 4
+#pragma unroll 8
         for (int j = 0; j < nr; ++j) {
             const float ej = __shfl_sync(0xffffffffu, e, j);
             const T* vr = vbase + (size_t)(r0 + j) * d;
@@ -412,16 +425,18 @@ __device__ __forceinline__ void hier_units(const Plan& p, const HierLevels& hl, 
 // the J children of each unit kept one level up (ascending), then the
 // remainder units U[l+1] J .. U[l] - 1.  Returns the count; cand_unit maps a
 // candidate position to its unit (an increasing map).
+// Every level keeps exactly min(topk, candidates) units, so the counts
+// follow from the unit counts alone: no selection needs to be read.
 __device__ __forceinline__ int hier_count(const HierLevels& hl, int l, int pr, const int* U,
                                           int J, int& nkept) {
-    if (l == hl.levels - 1) {
-        nkept = 0;
-        return U[l];
-    }
-    const int32_t* up = hl.sel[l + 1] + (size_t)pr * hl.topk[l + 1];
+    (void)pr;
+    int nc = U[hl.levels - 1];
     nkept = 0;
-    while (nkept < hl.topk[l + 1] && up[nkept] >= 0) ++nkept;
-    return nkept * J + (U[l] - U[l + 1] * J);
+    for (int m = hl.levels - 2; m >= l; --m) {
+        nkept = min(hl.topk[m + 1], nc);
+        nc = nkept * J + (U[m] - U[m + 1] * J);
+    }
+    return nc;
 }
 __device__ __forceinline__ int hier_unit(const HierLevels& hl, int l, int pr, const int* U, int J,
                                          int nkept, int c) {

@@ -426,7 +426,14 @@ static cudaError_t launch_hier_t(const Plan& p, const HierLevels& hl, cudaStream
     const int P = p.n_pairs;
     const size_t qsm = (size_t)p.G * p.d * sizeof(float);
     for (int l = hl.levels - 1; l >= 0; --l) {
-        const int gx = (hl.umax[l] + 3) / 4;
+        // candidates: every unit at the top; below, the kept parents'
+        // children and fewer than J remainder units
+        long long bound = hl.umax[l];
+        if (l < hl.levels - 1) {
+            const long long b2 = (long long)hl.topk[l + 1] * p.J + p.J;
+            if (b2 < bound) bound = b2;
+        }
+        const int gx = (int)((bound + 3) / 4);
         gen::hier_score_kernel<T><<<dim3(gx > 0 ? gx : 1, P), 128, qsm, stream>>>(p, hl, l);
         gen::hier_topk_kernel<<<P, 128, 0, stream>>>(p, hl, l);
     }

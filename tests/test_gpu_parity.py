@@ -273,3 +273,19 @@ def test_nan_gist_keys(ssa, orc, flags):
     assert np.array_equal(np.isnan(o), nan_ref)
     err = np.abs(o[~nan_ref] - ref["out"][~nan_ref])
     assert err.max() <= 1e-2 and err.mean() <= 1e-3
+
+
+def test_pipeline_at_its_chunk_limit(ssa, orc):
+    """8192 chunks per sequence (512K tokens, C = 64), the most the two-kernel
+    pipeline takes: its top-k falls back from the 128-candidate path to the
+    radix path, and the score rows are longest."""
+    w = Workload("chunk_limit", B=1, Hq=32, Hkv=8, d=64, n_max=524288, C=64, g=8, topk=64,
+                 seq_lens=(524288 - 37,), planted=64)
+    sh = ssa.make_shape(w.B, w.Hq, w.Hkv, w.d, w.n_max, ssa.SSA_BF16)
+    assert ssa.ssa_decode_path(sh, w.C, w.g, w.topk) == ssa.SSA_PATH_PIPELINE
+    inp = make_inputs(w, seed=8192, device="cuda")
+    out, sel = ssa.ssa_decode(inp["q"], inp["k_raw"], inp["v_raw"], inp["k_gist"],
+                              inp["v_gist"], inp["seq_lens"], w.C, w.g, w.topk)
+    assert ssa.ssa_get_device_status() == 0
+    stats = check_single(orc, sample_seq(inp, 0), w.C, w.g, w.topk, out, sel)
+    print("chunk_limit", stats)
