@@ -97,6 +97,37 @@ __global__ void score_kernel(Plan p, int level, float* dst, int stride, int n_sl
     }
 }
 
+// q . k for one key row: 16-byte loads when the row allows them (each lane
+// reads its own row, so wide loads keep the L1 requests per row few), else
+// element loads.
+__device__ __forceinline__ float bf_lo32(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf_hi32(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+template <class T>
+__device__ __forceinline__ float dot_row(const float* qs, const T* kr, int d) {
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    int i = 0;
+    if ((reinterpret_cast<uintptr_t>(kr) & 15u) == 0) {
+        const uint4* k4 = reinterpret_cast<const uint4*>(kr);
+        constexpr int per = 16 / (int)sizeof(T);
+        for (; i + per <= d; i += per) {
+            const uint4 w = k4[i / per];
+            if constexpr (sizeof(T) == 2) {
+                s0 += qs[i] * bf_lo32(w.x) + qs[i + 1] * bf_hi32(w.x);
+                s1 += qs[i + 2] * bf_lo32(w.y) + qs[i + 3] * bf_hi32(w.y);
+                s2 += qs[i + 4] * bf_lo32(w.z) + qs[i + 5] * bf_hi32(w.z);
+                s3 += qs[i + 6] * bf_lo32(w.w) + qs[i + 7] * bf_hi32(w.w);
+            } else {
+                s0 += qs[i] * __uint_as_float(w.x);
+                s1 += qs[i + 1] * __uint_as_float(w.y);
+                s2 += qs[i + 2] * __uint_as_float(w.z);
+                s3 += qs[i + 3] * __uint_as_float(w.w);
+            }
+        }
+    }
+    for (; i < d; ++i) s0 += qs[i] * to_f(kr[i]);
+    return (s0 + s1) + (s2 + s3);
+}
+
 // Online softmax of one query (qs, fp32 in shared memory, log2-domain scale)
 // over `rows` key/value rows, by one warp, 32 rows at a time: lane j takes
 // the dot product of row r0 + j (its loads independent of the other lanes'),
@@ -125,19 +156,7 @@ __device__ __forceinline__ void attend_rows(const float* qs, const T* kbase, con
         const int nr = min(32, rows - r0);
         prefetch_row(r + 32);  // the next group's rows, while this one computes
         float x = -INFINITY;
-        if (r < rows) {
-            const T* kr = kbase + (size_t)r * d;
-            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-            int i = 0;
-            for (; i + 4 <= d; i += 4) {
-                s0 += qs[i] * to_f(kr[i]);
-                s1 += qs[i + 1] * to_f(kr[i + 1]);
-                s2 += qs[i + 2] * to_f(kr[i + 2]);
-                s3 += qs[i + 3] * to_f(kr[i + 3]);
-            }
-            for (; i < d; ++i) s0 += qs[i] * to_f(kr[i]);
-            x = (s0 + s1 + s2 + s3) * scale;
-        }
+        if (r < rows) x = dot_row<T>(qs, kbase + (size_t)r * d, d) * scale;
         float mx = x;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -333,15 +352,15 @@ __global__ void attend_kernel(Plan p, const int* bad) {
     const int M = n / p.C;
     const int S = p.h2 ? M / p.J : 0;
     const int ks = p.h2 ? kept_super(p, S) : 0;
-    if (threadIdx.x == 0) {
+    {
         const int ns = p.sel_stride > 0 ? p.sel_stride : p.topk;
-        for (int c = 0; c < ns; ++c) {
-            int m = p.sel_idx[(size_t)pr * ns + c];
-            if (m >= 0) cbits[m >> 5] |= 1u << (m & 31);
+        for (int c = threadIdx.x; c < ns; c += blockDim.x) {
+            const int m = p.sel_idx[(size_t)pr * ns + c];
+            if (m >= 0) atomicOr(&cbits[m >> 5], 1u << (m & 31));
         }
-        for (int c = 0; c < ks; ++c) {
-            int x = p.sel_super[(size_t)pr * p.topk_super + c];
-            sbits[x >> 5] |= 1u << (x & 31);
+        for (int c = threadIdx.x; c < ks; c += blockDim.x) {
+            const int x = p.sel_super[(size_t)pr * p.topk_super + c];
+            atomicOr(&sbits[x >> 5], 1u << (x & 31));
         }
     }
     __syncthreads();
@@ -359,8 +378,15 @@ __global__ void attend_kernel(Plan p, const int* bad) {
 #pragma unroll
     for (int r = 0; r < 8; ++r) acc[r] = 0.f;
 
+    // Every warp walks every unit in the same order and numbers its 32-row
+    // groups the same way; warp w attends the groups numbered w mod (warps),
+    // so the rows spread evenly whatever the unit sizes.
+    int gi = 0;
     auto visit = [&](const T* kbase, const T* vbase, int rows) {
-        attend_rows<T>(qs, kbase, vbase, rows, p.d, scale, m_run, l_run, acc);
+        for (int r0 = 0; r0 < rows; r0 += 32, ++gi)
+            if (gi % nw == warp)
+                attend_rows<T>(qs, kbase + (size_t)r0 * p.d, vbase + (size_t)r0 * p.d,
+                               min(32, rows - r0), p.d, scale, m_run, l_run, acc);
     };
     // ctx_mode 0: a selected chunk contributes its raw tokens, an unselected
     // one its gists; ctx_mode 1: a selected chunk its gists and raw tokens,
@@ -376,7 +402,7 @@ __global__ void attend_kernel(Plan p, const int* bad) {
     // units: single level -> chunks 0..M-1 then the tail;
     // two level -> superchunks 0..S-1, remainder chunks, then the tail.
     const int n_units = p.h2 ? S + (M - S * p.J) + 1 : M + 1;
-    for (int u = warp; u < n_units; u += nw) {
+    for (int u = 0; u < n_units; ++u) {
         if (u == n_units - 1) {
             visit(kr + (size_t)M * p.C * p.d, vr + (size_t)M * p.C * p.d, n - M * p.C);
         } else if (!p.h2) {
@@ -502,7 +528,11 @@ __global__ void hier_topk_kernel(Plan p, HierLevels hl, int l) {
 
 // Attention over the t-level context, one block per (query head, sequence):
 // the summaries of every unkept candidate at levels >= 1, the gists of
-// unkept candidate chunks, the raw tokens of kept chunks, the tail.
+// unkept candidate chunks, the raw tokens of kept chunks, the tail.  Every
+// warp walks the same list of candidates (each level's selection is first
+// copied to shared memory, so the walk reads no global memory) and numbers
+// their 32-row groups in the same order; warp w attends the groups whose
+// number is w mod (warps), so the rows spread evenly whatever the unit sizes.
 template <class T>
 __global__ void hier_attend_kernel(Plan p, HierLevels hl) {
     extern __shared__ float sm[];
@@ -516,6 +546,7 @@ __global__ void hier_attend_kernel(Plan p, HierLevels hl) {
     float* wl = wm + nw;                              // [nw]
     float* wacc = wl + nw;                            // [nw][d]
     uint32_t* bits = reinterpret_cast<uint32_t*>(wacc + nw * p.d);  // kept units, per level
+    int* sels = reinterpret_cast<int*>(bits + hl.mask_words);        // every level's selection
     float* outp = p.out + ((size_t)b * p.Hq + h) * p.d;
     const int n = p.seq_lens[b];
     if (n < 1 || n > p.n_max) {
@@ -526,21 +557,25 @@ __global__ void hier_attend_kernel(Plan p, HierLevels hl) {
     const T* qg = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * p.d;
     for (int i = threadIdx.x; i < p.d; i += blockDim.x) qs[i] = to_f(qg[i]);
     for (int i = threadIdx.x; i < hl.mask_words; i += blockDim.x) bits[i] = 0u;
-    __syncthreads();
-    int off[kMaxLevels];
+    int off[kMaxLevels], soff[kMaxLevels];
     {
-        int o = 0;
+        int o = 0, so = 0;
         for (int l = 0; l < hl.levels; ++l) {
             off[l] = o;
+            soff[l] = so;
             o += (hl.umax[l] + 31) / 32;
+            so += hl.topk[l];
         }
     }
-    if (threadIdx.x == 0)
-        for (int l = 0; l < hl.levels; ++l)
-            for (int c = 0; c < hl.topk[l]; ++c) {
-                const int x = hl.sel[l][(size_t)pr * hl.topk[l] + c];
-                if (x >= 0) bits[off[l] + (x >> 5)] |= 1u << (x & 31);
-            }
+    for (int l = 0; l < hl.levels; ++l)
+        for (int c = threadIdx.x; c < hl.topk[l]; c += blockDim.x)
+            sels[soff[l] + c] = hl.sel[l][(size_t)pr * hl.topk[l] + c];
+    __syncthreads();
+    for (int l = 0; l < hl.levels; ++l)
+        for (int c = threadIdx.x; c < hl.topk[l]; c += blockDim.x) {
+            const int x = sels[soff[l] + c];
+            if (x >= 0) atomicOr(&bits[off[l] + (x >> 5)], 1u << (x & 31));
+        }
     __syncthreads();
     int U[kMaxLevels];
     hier_units(p, hl, n, U);
@@ -552,8 +587,13 @@ __global__ void hier_attend_kernel(Plan p, HierLevels hl) {
     float acc[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) acc[r] = 0.f;
-    auto visit = [&](const T* kbase, const T* vbase, int rows) {
-        attend_rows<T>(qs, kbase, vbase, rows, p.d, scale, m_run, l_run, acc);
+    int gi = 0;  // number of the next 32-row group, the same in every warp
+    // the warp's groups of `rows` rows at (kb, vb)
+    auto rows_of = [&](const T* kb, const T* vb, int rows) {
+        for (int r0 = 0; r0 < rows; r0 += 32, ++gi)
+            if (gi % nw == warp)
+                attend_rows<T>(qs, kb + (size_t)r0 * p.d, vb + (size_t)r0 * p.d,
+                               min(32, rows - r0), p.d, scale, m_run, l_run, acc);
     };
     for (int l = hl.levels - 1; l >= 0; --l) {
         int nkept;
@@ -563,16 +603,20 @@ __global__ void hier_attend_kernel(Plan p, HierLevels hl) {
                              : static_cast<const T*>(hl.k_sum[l]) + (size_t)pr * hl.umax[l] * ntok * p.d;
         const T* vs = l == 0 ? static_cast<const T*>(p.v_gist) + (size_t)pr * p.M_max * p.g * p.d
                              : static_cast<const T*>(hl.v_sum[l]) + (size_t)pr * hl.umax[l] * ntok * p.d;
-        for (int c = warp; c < nc; c += nw) {
-            const int x = hier_unit(hl, l, pr, U, p.J, nkept, c);
+        const int* up = l + 1 < hl.levels ? sels + soff[l + 1] : nullptr;
+        for (int c = 0; c < nc; ++c) {
+            int x;
+            if (l == hl.levels - 1) x = c;
+            else if (c < nkept * p.J) x = up[c / p.J] * p.J + c % p.J;
+            else x = U[l + 1] * p.J + (c - nkept * p.J);
             const bool kept = bits[off[l] + (x >> 5)] >> (x & 31) & 1u;
             if (!kept)
-                visit(ks + (size_t)x * ntok * p.d, vs + (size_t)x * ntok * p.d, ntok);
+                rows_of(ks + (size_t)x * ntok * p.d, vs + (size_t)x * ntok * p.d, ntok);
             else if (l == 0)
-                visit(kr + (size_t)x * p.C * p.d, vr + (size_t)x * p.C * p.d, p.C);
+                rows_of(kr + (size_t)x * p.C * p.d, vr + (size_t)x * p.C * p.d, p.C);
         }
     }
-    if (warp == nw - 1) visit(kr + (size_t)M * p.C * p.d, vr + (size_t)M * p.C * p.d, n - M * p.C);
+    rows_of(kr + (size_t)M * p.C * p.d, vr + (size_t)M * p.C * p.d, n - M * p.C);
     if (lane == 0) {
         wm[warp] = m_run;
         wl[warp] = l_run;

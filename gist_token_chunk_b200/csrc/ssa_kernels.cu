@@ -440,8 +440,15 @@ static cudaError_t launch_hier_t(const Plan& p, const HierLevels& hl, cudaStream
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int nw = 8;
+    int nsel = 0;
+    for (int l = 0; l < hl.levels; ++l) nsel += hl.topk[l];
     const size_t sm = (size_t)(p.d + 2 * nw + nw * p.d) * sizeof(float) +
-                      (size_t)hl.mask_words * sizeof(uint32_t);
+                      (size_t)hl.mask_words * sizeof(uint32_t) + (size_t)nsel * sizeof(int);
+    if (sm > 48 * 1024) {
+        e = cudaFuncSetAttribute(gen::hier_attend_kernel<T>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+    }
     gen::hier_attend_kernel<T><<<dim3(p.Hq, p.B), 32 * nw, sm, stream>>>(p, hl);
     return cudaGetLastError();
 }
