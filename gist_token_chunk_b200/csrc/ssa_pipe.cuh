@@ -1,5 +1,5 @@
 // ssa_pipe.cuh -- the two-kernel decode pipeline: single level, bf16,
-// d = 64, GQA groups of at most 8 query heads, at most 2048 chunks per
+// d = 64, GQA groups of at most 8 query heads, at most 8192 chunks per
 // sequence.
 //
 // "Simplified Sparse Attention via Gist Tokens": sec. 3.2 (each chunk is
@@ -15,11 +15,15 @@
 //                  workspace, and so does each chunk's score (the maximum over
 //                  its gist rows and the group's heads of q.k / sqrt(d));
 //   attend_kernel  the top-k of each (sequence, KV head) pair, run by the first
-//                  four warps of the block that owns the pair (the library's
-//                  deterministic block top-k over the pair's chunk scores,
-//                  published to the workspace and written to sel_idx); then
+//                  four warps of the block that owns the pair (a deterministic
+//                  top-k over the pair's chunk scores, or, for the App. A
+//                  reading, one per query head over its own scores and their
+//                  union; published to the workspace and written to sel_idx);
+//                  then
 //                  the unfolded context: the gist values of every chunk,
-//                  weighted by the kept logits and masked by the selection,
+//                  weighted by the kept logits and masked by the selection
+//                  (the selected chunks', or for the sec. 3.3 reading the
+//                  unselected ones),
 //                  and the raw K/V tiles of the selected chunks and of the
 //                  tail; one partial (m, l, o) per query head and (list, pair)
 //                  segment of a worker, combined into the output by the
