@@ -28,3 +28,66 @@ def test_reference_arm_prints_one_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["e2e"]["value"] == d["value"]
+
+
+# ------------------------------------------------ the bench's bytes models
+
+def _bench():
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _fixed(w, sel_entries):
+    """q, out, selection and lengths: the bytes every model adds per step."""
+    e = 2 if w.dtype == "bf16" else 4
+    return w.B * w.Hq * w.d * e + w.B * w.Hq * w.d * 4 + sel_entries * 4 + w.B * 4
+
+
+def test_bytes_models_match_the_oracles_context_sizes(orc):
+    """Every context row is read as a key and a value. The models add the
+    summary keys that are scored but not attended: the selected chunks' gists
+    (unselected-gist context), the unselected chunks' gists (selected-only
+    context), the kept units' summaries at every level (t levels). So
+    model = e d (2 |X| + those rows) + the fixed bytes, with |X| the oracle's
+    own context count."""
+    import numpy as np
+
+    sys.path.insert(0, ROOT)
+    from gist_token_chunk_b200.inputs import Workload, make_inputs, make_level_summaries
+
+    bench = _bench()
+    w = Workload("bytes", B=3, Hq=8, Hkv=2, d=16, n_max=640, C=16, g=4, topk=5,
+                 seq_lens=(640, 333, 40), dtype="fp32")
+    x = make_inputs(w, seed=3)
+    a = (x["q"], x["k_raw"], x["v_raw"], x["k_gist"], x["v_gist"], x["seq_lens"])
+    lens = [int(v) for v in x["seq_lens"]]
+    e = 4
+    for context in (0, 1):
+        for select in (0, 1):
+            r = orc.decode(*a, C=w.C, g=w.g, topk=w.topk, context=context, select=select)
+            sel = r["sel_idx"]
+            extra = 0
+            for b, n in enumerate(lens):
+                M = n // w.C
+                for j in range(w.Hkv):
+                    k = int((sel[b, j] >= 0).sum())
+                    extra += (k if context == 0 else M - k) * w.g
+            want = e * w.d * (2 * int(r["ctx"].sum()) + extra) + _fixed(w, sel.size)
+            if context == 0 and select == 0:
+                got = bench.algorithmic_bytes(w, lens)
+                assert got == want, (got, want)
+            got = bench.variant_bytes(w, lens, sel, context)
+            assert got == want, (context, select, got, want)
+    # t levels
+    J, g_sum, topks = 3, [2, 3], [4, 2, 1]
+    ks, vs = make_level_summaries(w, J, g_sum, seed=4)
+    r = orc.decode_hier(*a[:5], ks, vs, x["seq_lens"], C=w.C, g=w.g, J=J, topks=topks)
+    gl = [w.g] + g_sum
+    extra = sum(int((r["sels"][l] >= 0).sum()) * gl[l] for l in range(len(topks)))
+    want = e * w.d * (2 * int(r["ctx"].sum()) + extra) + _fixed(w, sum(s.size for s in r["sels"]))
+    got = bench.hier_bytes(w, lens, [np.asarray(s) for s in r["sels"]], J, g_sum, topks)
+    assert got == want, (got, want)
