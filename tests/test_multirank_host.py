@@ -52,7 +52,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of a process with OpenMP threads
     out = mgr.dict()
     mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
     assert out[0][0] == out[1][0] == 11.0
