@@ -16,13 +16,17 @@
  *   - chunk score s[b,j,m] = max over the query heads h of KV head j and the
  *     chunk's g gist tokens t of  q[b,h] . k_gist[b,j,m,t] / sqrt(d);
  *   - one selection per (sequence, KV head), shared by its query heads;
- *     ties go to the lower chunk index; NaN scores rank as -inf;
+ *     ties go to the lower chunk index; a NaN logit never wins a score
+ *     maximum, and NaN scores given to ssa_topk_chunks rank as -inf;
  *   - the attended context of (b, j) is: the gist K/V of every UNselected
  *     complete chunk, the raw K/V of every token of the selected chunks, and
  *     the raw K/V of the tail tokens M_b*C .. n_b-1 (selected chunks' own
  *     gists are not attended);
  *   - seq_lens[b] = n_b counts every cached raw token (the current one
  *     included); M_b = floor(n_b / C) chunks are complete.
+ * ssa_decode_variant offers the pages' other readings of the context and of
+ * the selection, and ssa_decode_hier the coarse-to-fine selection over more
+ * than two levels.
  *
  * Notation and layouts (row-major, contiguous, all device memory unless said):
  *   B batch, Hq query heads, Hkv KV heads, G = Hq/Hkv, query head h reads KV
@@ -57,18 +61,18 @@
  *     No C++ exception crosses this boundary.
  *   - topk > M_b selects every complete chunk; topk = 0 selects none.
  *
- * Workspace: the fused calls need device scratch of ssa_workspace_size()
- * bytes.  Pass ws = NULL, ws_bytes = 0 to let the library allocate it
- * stream-ordered (cudaMallocAsync) for that one call.  A caller-owned
- * workspace must be zeroed once with ssa_workspace_init() (or cudaMemset 0)
- * before its first use; every call leaves the state it used (control words,
- * score scratch and the scoring segments' candidate lists) zeroed again, so
- * it can be reused by later calls on the
- * same stream, for any sizes that fit, without re-initialising (when a call
- * lays the workspace out differently from the workspace's previous call, the
- * library zeroes the part it needs stream-ordered first).
- * After a call that reported SSA_ERR_DEVICE_TIMEOUT, initialise it again.
- * Two calls that share a workspace must not run concurrently.
+ * Workspace: the decode calls need device scratch of their
+ * ssa_workspace_size*() bytes.  Pass ws = NULL, ws_bytes = 0 to let the
+ * library allocate it stream-ordered (cudaMallocAsync) for that one call.  A
+ * caller-owned workspace must be zeroed once with ssa_workspace_init() (or
+ * cudaMemset 0) before its first use.  Every call leaves it reusable by later
+ * calls on the same stream, for any sizes that fit, without re-initialising:
+ * the two-kernel pipeline's words carry the launch's epoch, and the fused
+ * kernel clears the state it used (control words, score scratch, the scoring
+ * segments' candidate lists); when a call lays the workspace out differently
+ * from its previous call, the library zeroes the part it needs stream-ordered
+ * first.  After a call that reported SSA_ERR_DEVICE_TIMEOUT, initialise it
+ * again.  Two calls that share a workspace must not run concurrently.
  */
 #ifndef SSA_H_
 #define SSA_H_
