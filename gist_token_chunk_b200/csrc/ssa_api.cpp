@@ -519,7 +519,8 @@ ssa_status ssa_decode_hier(const ssa_shape* shape, const void* q, const void* k_
         if (topk[l] > 0 && !sel[l]) return fail(SSA_ERR_INVALID_ARG, "sel[%d] is NULL", l);
         hl.sel[l] = sel[l];
         if (l > 0) {
-            if (!k_sum[l - 1] || !v_sum[l - 1])
+            // a level with no unit at this capacity has an empty summary tensor
+            if (hl.umax[l] > 0 && (!k_sum[l - 1] || !v_sum[l - 1]))
                 return fail(SSA_ERR_INVALID_ARG, "k_sum[%d] or v_sum[%d] is NULL", l - 1, l - 1);
             hl.k_sum[l] = k_sum[l - 1];
             hl.v_sum[l] = v_sum[l - 1];

@@ -293,7 +293,8 @@ SSA_API ssa_status ssa_workspace_size_variant(const ssa_shape* shape, int32_t C,
  * and the raw tail.  levels = 1 is ssa_decode's step, levels = 2 is
  * ssa_decode_h2's.
  * k_sum, v_sum, g_sum (levels - 1 entries) and topk, sel (levels entries)
- * are HOST arrays; the tensors they point to are device memory.  1 <= levels
+ * are HOST arrays; the tensors they point to are device memory (a level
+ * with Umax(l) = 0 has no unit, and its k_sum, v_sum entries may be NULL).  1 <= levels
  * <= 8, J >= 1, 1 <= g_sum <= 1024, 0 <= topk <= 1024.  Runs on the
  * library's portable kernels.  Needs ssa_workspace_size_hier() bytes of
  * workspace (ws = NULL: allocated stream-ordered).
