@@ -236,17 +236,17 @@ SSA_API ssa_status ssa_decode_h2(const ssa_shape* shape, const void* q, const vo
  *   context SSA_CONTEXT_UNSELECTED_GISTS: gist K/V of the unselected complete
  *     chunks + raw K/V of the selected chunks + raw tail (ssa_decode);
  *   context SSA_CONTEXT_SELECTED_ONLY: gist K/V and raw K/V of the selected
- *     chunks + raw tail; unselected chunks contribute nothing (sec. 3.3,
- *     "each selected chunk's gist and raw tokens while excluding unselected
- *     chunks": |X| = k (C + g) + T);
+ *     chunks + raw tail; unselected chunks contribute nothing (sec. 3.3
+ *     read literally: a selected chunk brings its gists and its raw tokens,
+ *     the other chunks are left out; |X| = k (C + g) + T);
  *   select SSA_SELECT_GROUP_MAX: one top-k per KV head over the max of its
  *     group's query heads (ssa_decode);
  *   select SSA_SELECT_HEAD_UNION: every query head scores the chunks with its
  *     own query (max over the chunk's g gists of q_h.k / sqrt(d)) and keeps
  *     its own top-k (ties to the lower index); the KV head's selection is the
  *     union over its group, and all heads of the group attend over the
- *     context it defines (App. A, "each head selecting chunks independently
- *     before their union").
+ *     context it defines (App. A: the heads choose their chunks separately
+ *     and the group unfolds their union).
  * Out: out fp32 [B,Hq,d]; sel_idx int32 [B,Hkv,cap], the selection ascending
  * and -1 padded, cap = topk (group max) or G * topk (head union).
  * On a shape the two-kernel pipeline takes (see ssa_decode_path) both
@@ -274,8 +274,8 @@ SSA_API ssa_status ssa_workspace_size_variant(const ssa_shape* shape, int32_t C,
 
 /*
  * ssa_decode_hier -- coarse-to-fine selection over t = levels levels (sec.
- * 3.5, "additional hierarchy levels can be added as context grows"; App.
- * B.2, t = ceil(log_J M)), the two-level reading of ssa_decode_h2 applied
+ * 3.5: more levels of summaries as the context grows; App. B.2,
+ * t = ceil(log_J M)), the two-level reading of ssa_decode_h2 applied
  * level by level.  Level 1 is the chunks with their g gists (k_gist,
  * v_gist).  A level-l unit (l >= 2) groups J level-(l-1) units and has
  * g_sum[l-2] summary tokens in k_sum[l-2], v_sum[l-2], bf16/fp32 like the

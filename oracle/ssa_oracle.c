@@ -28,12 +28,12 @@
  *     of the selected chunks + tail;
  *   - seq_lens counts every cached raw token; all of them are visible.
  * Variants (oracle_decode_v):
- *   - context "selected only" (the sec. 3.3 wording "each selected chunk's
- *     gist and raw tokens while excluding unselected chunks"): gist K/V and
- *     raw K/V of the selected chunks + raw K/V of the tail; unselected
- *     chunks contribute nothing;
- *   - selection "per head + union" (App. A, "each head selecting chunks
- *     independently before their union"): every query head scores the
+ *   - context "selected only" (sec. 3.3 read literally: a selected chunk
+ *     brings both its gists and its raw tokens, and the other chunks are
+ *     left out): gist K/V and raw K/V of the selected chunks + raw K/V of
+ *     the tail; unselected chunks contribute nothing;
+ *   - selection "per head + union" (App. A: the heads choose their chunks
+ *     separately and the group unfolds their union): every query head scores the
  *     chunks with its own query only (max over the chunk's g gist tokens of
  *     q_h.k / sqrt(d)) and keeps its own top-k (ties to the lower index); the
  *     KV head's selection is the union of its group's selections, ascending,
@@ -530,8 +530,8 @@ int oracle_decode_h2(int B, int Hq, int Hkv, int d, int n_max, int C, int g, int
 
 /*
  * oracle_decode_hier: coarse-to-fine selection over `levels` = t levels
- * (sec. 3.5, "additional hierarchy levels can be added as context grows";
- * App. B.2, t = ceil(log_J M) levels), the two-level reading applied level by
+ * (sec. 3.5: more levels of summaries as the context grows; App. B.2,
+ * t = ceil(log_J M) levels), the two-level reading applied level by
  * level.  Level-1 units are the chunks (g gist tokens each).  A level-l unit
  * (l >= 2) groups J level-(l-1) units and has gs[l-2] summary tokens in
  * k_sum[l-2], v_sum[l-2] laid out [B,Hkv,Umax(l),gs[l-2],d] with Umax(l) =
