@@ -9,9 +9,9 @@
  *             softmax attention runs over the resulting hybrid context;
  *   sec. 3.5, App. B.2  gist-of-gist: meta-gists summarise J chunks and the
  *             selection runs coarse to fine;
- *   sec. 3.6  decoding touches only the selected keys plus O(n) bytes of
- *             metadata and splits the attention into partial passes that are
- *             combined afterwards.
+ *   sec. 3.6  a decode step reads the chosen keys and a per-chunk index
+ *             linear in the context, never the whole cache, and merges
+ *             split partial attentions at the end.
  * Where the pages leave a step open this library fixes it as follows:
  *   - chunk score s[b,j,m] = max over the query heads h of KV head j and the
  *     chunk's g gist tokens t of  q[b,h] . k_gist[b,j,m,t] / sqrt(d);
