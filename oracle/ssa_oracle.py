@@ -5,9 +5,10 @@ bench's CPU-baseline leg.  The product library never imports this module.
 
 The oracle follows "Simplified Sparse Attention via Gist Tokens", sec. 3.2
 (scoring against gist keys), sec. 3.3 (top-k, hybrid attention over the
-unfolded context) and sec. 3.5 / App. B.2 (two-level coarse-to-fine
-selection); the readings it takes where the pages are open are listed in the
-C file's header.
+unfolded context), sec. 3.5 / App. B.2 (coarse-to-fine selection) in
+``ssa_oracle.c``, and sec. 3.1 / 3.6 (prefill under the gist mask, its block
+mask) and App. A (adaptive top-k) in ``prefill_oracle.c``; the readings each
+takes where the pages are open are listed in the C files' headers.
 """
 from __future__ import annotations
 
@@ -20,6 +21,7 @@ import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "ssa_oracle.c")
+SOURCES = [SRC, os.path.join(HERE, "prefill_oracle.c")]
 
 
 def lib_path(mutant: int = 0, out_dir: Optional[str] = None) -> str:
@@ -31,10 +33,11 @@ def lib_path(mutant: int = 0, out_dir: Optional[str] = None) -> str:
 def build(mutant: int = 0, out_dir: Optional[str] = None, force: bool = False) -> str:
     """Compile the oracle (optionally with one planted mutant) with gcc."""
     out = lib_path(mutant, out_dir)
-    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(SRC):
+    if (not force and os.path.exists(out)
+            and os.path.getmtime(out) >= max(os.path.getmtime(f) for f in SOURCES)):
         return out
     tmp = out + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", f"-DORACLE_MUTANT={mutant}", SRC,
+    cmd = ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", f"-DORACLE_MUTANT={mutant}", *SOURCES,
            "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, out)
@@ -83,6 +86,14 @@ class Oracle:
         self.lib.oracle_decode_hier.restype = ctypes.c_int
         self.lib.oracle_decode_h2.restype = ctypes.c_int
         self.lib.oracle_mutant_id.restype = ctypes.c_int
+        self.lib.oracle_adaptive_topk.restype = ctypes.c_int64
+        self.lib.oracle_adaptive_topk.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_int]
+        self.lib.oracle_prefill.restype = ctypes.c_int
+        self.lib.oracle_prefill_blocks.restype = ctypes.c_int64
+        self.lib.oracle_prefill_blocks.argtypes = [
+            ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _I,
+            ctypes.c_int64, _I, ctypes.c_int64]
 
     @property
     def mutant(self) -> int:
@@ -206,6 +217,59 @@ class Oracle:
         return {"scores": [sc[:, :, :u] for sc, u in zip(scores, umax)],
                 "sels": [x[:, :, :int(k)] for x, k in zip(sel_arr, topks)],
                 "out": out, "lse": lse, "ctx": ctx, "bad_seq": rc}
+
+    def adaptive_topk(self, n_kv: int, L: int, G: int, J: int = 1) -> int:
+        """App. A budget: chunks each query head keeps at every level (J = 1:
+        SSA, J > 1: H-SSA with J chunks per meta-gist group)."""
+        k = int(self.lib.oracle_adaptive_topk(int(n_kv), int(L), int(G), int(J)))
+        if k < 0:
+            raise ValueError("oracle_adaptive_topk: bad arguments")
+        return k
+
+    def prefill(self, q_raw, q_gist, k_raw, k_gist, v_raw, v_gist, seq_lens, C: int,
+                g: int) -> dict:
+        """Prefill attention under the gist mask (sec. 3.1), dense, fp64.
+        Rows past each sequence's length are NaN in the result."""
+        q_raw, q_gist = _f32(q_raw), _f32(q_gist)
+        k_raw, k_gist, v_raw, v_gist = _f32(k_raw), _f32(k_gist), _f32(v_raw), _f32(v_gist)
+        lens = _i32(seq_lens)
+        B, Hq, n_max, d = q_raw.shape
+        Hkv = k_raw.shape[1]
+        M_max = n_max // C
+        assert q_gist.shape == (B, Hq, M_max, g, d), (q_gist.shape, (B, Hq, M_max, g, d))
+        assert k_gist.shape == v_gist.shape == (B, Hkv, M_max, g, d)
+        assert k_raw.shape == v_raw.shape == (B, Hkv, n_max, d)
+        o_raw = np.full((B, Hq, n_max, d), np.nan, np.float64)
+        o_gist = np.full((B, Hq, M_max, g, d), np.nan, np.float64)
+        rc = self.lib.oracle_prefill(
+            B, Hq, Hkv, d, n_max, C, g, _p(lens, _I), _p(q_raw, _F), _p(q_gist, _F),
+            _p(k_raw, _F), _p(k_gist, _F), _p(v_raw, _F), _p(v_gist, _F), _p(o_raw, _D),
+            _p(o_gist, _D))
+        if rc < 0:
+            raise ValueError("oracle_prefill: bad shape")
+        return {"o_raw": o_raw, "o_gist": o_gist, "bad_seq": rc}
+
+    def prefill_blocks(self, n: int, C: int, g: int, BM: int, BN: int) -> list:
+        """Block mask of one sequence (sec. 3.6) from the dense gist mask: a
+        list of ((kind, r0, rows), [entries]) in the order raw tiles, gist
+        tiles; entry = (block << 2) | (part << 1) | full, part 0 = gist
+        columns (listed first), 1 = raw columns."""
+        M = n // C
+        nt = -(-n // BM) + -(-(M * g) // BM)
+        cap = max(1, nt * (-(-n // BN) + -(-(M * g) // BN)))
+        tiles = np.zeros((max(nt, 1), 4), np.int32)
+        ents = np.zeros(cap, np.int32)
+        ne = int(self.lib.oracle_prefill_blocks(int(n), C, g, BM, BN, _p(tiles, _I), nt,
+                                                _p(ents, _I), cap))
+        if ne < 0:
+            raise ValueError("oracle_prefill_blocks: bad arguments")
+        res, off = [], 0
+        for i in range(nt):
+            kind, r0, rows, cnt = (int(x) for x in tiles[i])
+            res.append(((kind, r0, rows), [int(e) for e in ents[off:off + cnt]]))
+            off += cnt
+        assert off == ne
+        return res
 
 
 _default: Optional[Oracle] = None

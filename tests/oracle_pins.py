@@ -537,10 +537,248 @@ def pin_hier_reductions(orc):
                 assert upper["ctx"][b, j] == size, (t, b, j, upper["ctx"][b, j], size)
 
 
+# ------------------------------------------------- adaptive top-k (App. A) ---
+
+def pin_adaptive_topk_properties(orc):
+    """The properties App. A states for the budget (its formula is not
+    printed, so the exact value stays unpinned): a chunk is always chosen; the
+    group's union of raw tokens, G k L, tracks n_kv / L_eff (effective
+    compression L for SSA, L J for H-SSA); dividing by G keeps that union from
+    growing with the group size; more cache never lowers the budget."""
+    for L in (16, 64, 128):
+        for G in (1, 4, 8):
+            for J in (1, 4, 16):
+                l_eff = L * J
+                assert orc.adaptive_topk(0, L, G, J) == 1
+                assert orc.adaptive_topk(1, L, G, J) == 1
+                prev = 0
+                for e in range(8, 27, 2):
+                    n_kv = (1 << e) + 12345
+                    k = orc.adaptive_topk(n_kv, L, G, J)
+                    assert k >= 1 and k >= prev, (n_kv, L, G, J, k, prev)
+                    prev = k
+                    union = G * k * L
+                    target = n_kv / l_eff
+                    assert target < union <= target + G * L, (n_kv, L, G, J, k)
+    # the union budget is (nearly) independent of G at a fixed cache size
+    for G in (1, 2, 4, 8, 16):
+        k = orc.adaptive_topk(1 << 24, 64, G, 1)
+        assert abs(G * k - (1 << 24) // (64 * 64)) <= G, (G, k)
+
+
+# --------------------------------------- prefill under the gist mask (3.1) ---
+
+def _prefill_case(rng, B, Hq, Hkv, d, C, g, n_max, lens):
+    M_max = n_max // C
+    f = lambda *shape: rng.standard_normal(shape).astype(np.float32)
+    return {"q_raw": f(B, Hq, n_max, d), "q_gist": f(B, Hq, M_max, g, d),
+            "k_raw": f(B, Hkv, n_max, d), "k_gist": f(B, Hkv, M_max, g, d),
+            "v_raw": f(B, Hkv, n_max, d), "v_gist": f(B, Hkv, M_max, g, d),
+            "seq_lens": np.asarray(lens, np.int32)}
+
+
+def _prefill(orc, c, C, g):
+    return orc.prefill(c["q_raw"], c["q_gist"], c["k_raw"], c["k_gist"], c["v_raw"],
+                       c["v_gist"], c["seq_lens"], C, g)
+
+
+def pin_prefill_one_chunk_is_causal(orc):
+    """With at most one chunk the gist mask is plain causal attention over
+    the interleaved order (the chunk's raw tokens, then its gists): textbook
+    causal softmax from torch, fp64."""
+    B, Hq, Hkv, d, C, g = 3, 4, 2, 16, 16, 3
+    c = _prefill_case(np.random.default_rng(71), B, Hq, Hkv, d, C, g, C, [16, 11, 1])
+    res = _prefill(orc, c, C, g)
+    G = Hq // Hkv
+    for b, n in enumerate(c["seq_lens"]):
+        n = int(n)
+        ng = g if n == C else 0
+        for h in range(Hq):
+            j = h // G
+            q = np.concatenate([c["q_raw"][b, h, :n], c["q_gist"][b, h, 0, :ng]])
+            k = np.concatenate([c["k_raw"][b, j, :n], c["k_gist"][b, j, 0, :ng]])
+            v = np.concatenate([c["v_raw"][b, j, :n], c["v_gist"][b, j, 0, :ng]])
+            t = lambda x: torch.from_numpy(x.astype(np.float64))[None, None]
+            want = torch.nn.functional.scaled_dot_product_attention(
+                t(q), t(k), t(v), is_causal=True)[0, 0].numpy()
+            _close(res["o_raw"][b, h, :n], want[:n], 1e-12, f"raw rows b={b} h={h}")
+            if ng:
+                _close(res["o_gist"][b, h, 0, :ng], want[n:], 1e-12, f"gist rows b={b} h={h}")
+
+
+def _visible_sets(n, C, g):
+    """Interleaved positions each row sees, listed from the sentence of sec.
+    3.1 (its own chunk up to itself, every gist of the earlier chunks)."""
+    M = n // C
+    pos_raw = lambda i: (i // C) * (C + g) + i % C if i < M * C else M * (C + g) + i - M * C
+    pos_gist = lambda m, t: m * (C + g) + C + t
+    earlier_gists = lambda m: [pos_gist(mm, t) for mm in range(m) for t in range(g)]
+    raw_rows, gist_rows = [], []
+    for i in range(n):
+        m = i // C
+        own = [pos_raw(x) for x in range(m * C, i + 1)]
+        raw_rows.append((own, earlier_gists(m)))
+    for m in range(M):
+        for t in range(g):
+            own = [pos_raw(x) for x in range(m * C, m * C + C)] + [pos_gist(m, u) for u in range(t + 1)]
+            gist_rows.append((own, earlier_gists(m)))
+    return raw_rows, gist_rows, pos_raw, pos_gist
+
+
+def pin_prefill_visible_sets(orc):
+    """Zero keys make every visible key equally weighted, so each output row is
+    the mean of the value features over the row's visible set: the share of
+    gist keys, and the mean and mean square of their interleaved positions,
+    checked against the sets listed from the sentence of sec. 3.1."""
+    B, Hq, Hkv, d, C, g, n_max = 2, 2, 1, 8, 5, 2, 30
+    lens = [28, 13]
+    c = _prefill_case(np.random.default_rng(5), B, Hq, Hkv, d, C, g, n_max, lens)
+    c["k_raw"][:] = 0
+    c["k_gist"][:] = 0
+    c["v_raw"][:] = 0
+    c["v_gist"][:] = 0
+    for b, n in enumerate(lens):
+        raw_rows, gist_rows, pos_raw, pos_gist = _visible_sets(n, C, g)
+        scale = 1.0 / 64
+        for i in range(n):
+            c["v_raw"][b, 0, i, :3] = (0.0, pos_raw(i) * scale, (pos_raw(i) * scale) ** 2)
+        for m in range(n // C):
+            for t in range(g):
+                p = pos_gist(m, t) * scale
+                c["v_gist"][b, 0, m, t, :3] = (1.0, p, p * p)
+    res = _prefill(orc, c, C, g)
+    for b, n in enumerate(lens):
+        raw_rows, gist_rows, pos_raw, pos_gist = _visible_sets(n, C, g)
+        for kind, rows in (("raw", raw_rows), ("gist", gist_rows)):
+            for r, (own, gists) in enumerate(rows):
+                allp = np.asarray(own + gists, np.float64) / 64
+                n_gist = len(gists) + (sum(1 for x in own if x % (C + g) >= C
+                                           and x < (n // C) * (C + g)))
+                want = np.array([n_gist / len(allp), allp.mean(), (allp ** 2).mean()])
+                got = (res["o_raw"][b, :, r, :3] if kind == "raw"
+                       else res["o_gist"][b, :, r // g, r % g, :3])
+                for h in range(Hq):
+                    _close(got[h], want, 1e-12, f"{kind} row {r} b={b} h={h}")
+
+
+def pin_prefill_last_token_is_decode(orc):
+    """The last raw token of a sequence with a non-empty tail sees every gist
+    and the tail up to itself: the decode step's context with nothing
+    unfolded (k = 0), from the decode oracle."""
+    B, Hq, Hkv, d, C, g, n_max = 2, 4, 2, 16, 6, 2, 48
+    lens = [45, 20]
+    c = _prefill_case(np.random.default_rng(9), B, Hq, Hkv, d, C, g, n_max, lens)
+    res = _prefill(orc, c, C, g)
+    q_last = np.stack([c["q_raw"][b, :, n - 1] for b, n in enumerate(lens)])
+    dec = orc.decode(q_last, c["k_raw"], c["v_raw"], c["k_gist"], c["v_gist"], c["seq_lens"],
+                     C=C, g=g, topk=0)
+    for b, n in enumerate(lens):
+        _close(res["o_raw"][b, :, n - 1], dec["out"][b], 1e-12, f"b={b}")
+
+
+# ------------------------------------------- prefill block mask (sec. 3.6) ---
+
+def _entry(block, part, full):
+    return (block << 2) | (part << 1) | int(full)
+
+
+def pin_prefill_blocks_causal(orc):
+    """No complete chunk: the mask is causal over the raw tokens, so tile
+    [r0, r1) lists raw blocks 0 .. (r1 - 1) // BN, full when the block ends at
+    or before row r0's own column."""
+    for (n, C, BM, BN) in ((1, 8, 4, 4), (13, 16, 4, 4), (30, 64, 8, 4), (31, 32, 4, 8)):
+        plan = orc.prefill_blocks(n, C, 2, BM, BN)
+        want = []
+        for r0 in range(0, n, BM):
+            r1 = min(n, r0 + BM)
+            ents = [_entry(b, 1, b * BN + BN <= r0 + 1 and b * BN + BN <= n)
+                    for b in range(0, (r1 - 1) // BN + 1)]
+            want.append(((0, r0, r1 - r0), ents))
+        assert plan == want, (n, C, BM, BN, plan, want)
+
+
+def pin_prefill_blocks_counts(orc):
+    """Chunks of C >= BM rows: a raw tile of chunk m lists the gist blocks
+    covering [0, m g) (full when inside it) and the raw blocks of its own
+    chunk up to its last row; a gist tile lists the gist blocks up to its last
+    row (causal) and the raw blocks of the chunks its rows summarise (full
+    only when all its rows belong to one chunk)."""
+    for (n, C, g, BM, BN) in ((300, 128, 8, 64, 64), (1000, 64, 8, 16, 32), (517, 32, 3, 16, 16)):
+        M = n // C
+        ng = M * g
+        plan = orc.prefill_blocks(n, C, g, BM, BN)
+        want = []
+        for r0 in range(0, n, BM):
+            r1 = min(n, r0 + BM)
+            m = r0 // C
+            ents = [_entry(b, 0, b * BN + BN <= m * g) for b in range(-(-(m * g) // BN))]
+            ents += [_entry(b, 1, b * BN + BN <= r0 + 1)
+                     for b in range(m * C // BN, (r1 - 1) // BN + 1)]
+            want.append(((0, r0, r1 - r0), ents))
+        for r0 in range(0, ng, BM):
+            r1 = min(ng, r0 + BM)
+            m0, m1 = r0 // g, (r1 - 1) // g
+            ents = [_entry(b, 0, b * BN + BN <= min(r0 + 1, ng)) for b in range((r1 - 1) // BN + 1)]
+            ents += [_entry(b, 1, m0 == m1 and C % BN == 0)
+                     for b in range(m0 * C // BN, ((m1 + 1) * C - 1) // BN + 1)]
+            want.append(((1, r0, r1 - r0), ents))
+        assert plan == want, (n, C, g, BM, BN)
+
+
+def pin_prefill_block_sparse_matches_dense(orc):
+    """Attention evaluated only over the listed blocks, with the element mask
+    applied inside partial blocks and not inside full ones, gives the dense
+    masked result (the block mask keeps the defined attention)."""
+    B, Hq, Hkv, d, C, g, n_max = 2, 2, 1, 8, 12, 3, 96
+    lens = [95, 40]
+    BM, BN = 8, 8
+    c = _prefill_case(np.random.default_rng(13), B, Hq, Hkv, d, C, g, n_max, lens)
+    dense = _prefill(orc, c, C, g)
+    for b, n in enumerate(lens):
+        M = n // C
+        raw_rows, gist_rows, pos_raw, pos_gist = _visible_sets(n, C, g)
+        count = (M * g, n)  # columns of part 0 (gists) and part 1 (raw)
+        col_pos = (lambda r: pos_gist(r // g, r % g), pos_raw)
+        plan = orc.prefill_blocks(n, C, g, BM, BN)
+        for (kind, r0, rows), ents in plan:
+            for r in range(r0, r0 + rows):
+                own, gists = (raw_rows if kind == 0 else gist_rows)[r]
+                seen = set(own) | set(gists)
+                for h in range(Hq):
+                    q = (c["q_raw"][b, h, r] if kind == 0 else c["q_gist"][b, h, r // g, r % g])
+                    ks, vs = [], []
+                    for e in ents:
+                        blk, part, full = e >> 2, (e >> 1) & 1, e & 1
+                        for col in range(blk * BN, blk * BN + BN):
+                            exists = col < count[part]
+                            if not full and not (exists and col_pos[part](col) in seen):
+                                continue
+                            if part == 0:
+                                kv = ((c["k_gist"][b, 0, col // g, col % g],
+                                       c["v_gist"][b, 0, col // g, col % g]) if exists
+                                      else (np.zeros(d), np.full(d, 1e3)))
+                            else:
+                                kv = ((c["k_raw"][b, 0, col], c["v_raw"][b, 0, col]) if exists
+                                      else (np.zeros(d), np.full(d, 1e3)))
+                            ks.append(kv[0])
+                            vs.append(kv[1])
+                    K = np.asarray(ks, np.float64)
+                    V = np.asarray(vs, np.float64)
+                    lg = K @ np.asarray(q, np.float64) / math.sqrt(d)
+                    w = np.exp(lg - lg.max())
+                    out = (w[:, None] * V).sum(0) / w.sum()
+                    want = (dense["o_raw"][b, h, r] if kind == 0
+                            else dense["o_gist"][b, h, r // g, r % g])
+                    _close(out, want, 1e-10, f"b={b} kind={kind} row={r} h={h}")
+
+
 ALL_PINS = [
     pin_bruteforce_single, pin_given_selection, pin_ties, pin_dense_when_all_selected,
     pin_gists_when_none_selected, pin_single_token, pin_equal_keys_mean, pin_context_size,
     pin_parallel_query, pin_hand_example, pin_bruteforce_h2, pin_h2_reduces_to_single,
     pin_bad_length, pin_nan_gist_key, pin_variants_bruteforce, pin_selected_only_closed_forms,
     pin_union_reductions, pin_hier_bruteforce, pin_hier_reductions,
+    pin_adaptive_topk_properties, pin_prefill_one_chunk_is_causal, pin_prefill_visible_sets,
+    pin_prefill_last_token_is_decode, pin_prefill_blocks_causal, pin_prefill_blocks_counts,
+    pin_prefill_block_sparse_matches_dense,
 ]

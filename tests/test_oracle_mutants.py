@@ -8,13 +8,18 @@ The mutants live behind ``-DORACLE_MUTANT=<n>`` in ``oracle/ssa_oracle.c``:
 10 gist rows indexed token-major           11 selection not re-sorted by index
 12 per-head union keeps head 0 only        13 selected-only context drops the gists
 14 t levels: remainder units never candidates
+15 adaptive top-k without the +1           16 adaptive top-k ignores J (L_eff = L)
+17 prefill: earlier chunks' raw tokens seen 18 prefill: a gist hides its own chunk's gists
+19 prefill: gists placed before their chunk 20 prefill attention without the scale
+21 block mask: a block whose columns run past the end counted full
+(mutants 15-21 live in ``oracle/prefill_oracle.c``)
 """
 import pytest
 
 from oracle import ssa_oracle
 from oracle_pins import ALL_PINS
 
-MUTANTS = [1, 2, 3, 4, 5, 6, 7, 8, 10, 11, 12, 13, 14]
+MUTANTS = [1, 2, 3, 4, 5, 6, 7, 8, 10, 11, 12, 13, 14, 15, 16, 17, 18, 19, 20, 21]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS)
