@@ -250,10 +250,16 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# The files the decode kernels and their launches are compiled from (the
+# prefill is a translation unit of its own and changes none of them).
+DECODE_SOURCES = ("ssa_api.cpp", "ssa_device.cuh", "ssa_fused.cuh", "ssa_generic.cuh",
+                  "ssa_internal.h", "ssa_kernels.cu", "ssa_pipe.cuh")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gist_token_chunk_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(DECODE_SOURCES):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode())
             h.update(fh.read())
@@ -479,6 +485,122 @@ def run_reference(args):
     return 0
 
 
+# --------------------------------------------------------------- prefill ---
+
+# Prefill of one attention layer under the gist mask (Llama-3.2-1B heads).
+PREFILL = {"workload": "prefill_llama1b_32k", "B": 1, "Hq": 32, "Hkv": 8, "d": 64,
+           "n": 32768, "C": 128, "g": 8}
+
+
+def prefill_visible_pairs(n: int, C: int, g: int) -> int:
+    """(query, key) pairs the gist mask keeps for one sequence and head: raw
+    row i of chunk m sees m g gists and i - m C + 1 raw tokens; gist (m, t)
+    sees m g + t + 1 gists and the C raw tokens of its chunk."""
+    M = n // C
+    pairs = 0
+    for m in range(M + 1):
+        rows = min(C, n - m * C)
+        if rows <= 0:
+            break
+        pairs += rows * m * g + rows * (rows + 1) // 2
+    pairs += sum(M_ * g * g + g * (g + 1) // 2 + g * C for M_ in range(M))
+    return pairs
+
+
+def run_prefill(args):
+    """Times ssa_prefill (one layer, plan built once outside the timed
+    region) with CUDA events per step, L2 flushed between steps; prints one
+    JSON line.  The dense causal SDPA over the same interleaved length is
+    timed beside it for context."""
+    from gist_token_chunk_b200 import ssa
+
+    P = PREFILL
+    B, Hq, Hkv, d, n, C, g = (P[k] for k in ("B", "Hq", "Hkv", "d", "n", "C", "g"))
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    gen = torch.Generator(device=dev).manual_seed(args.seed)
+    M = n // C
+    f = lambda *sh: torch.randn(*sh, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    x = [f(B, Hq, n, d), f(B, Hq, M, g, d), f(B, Hkv, n, d), f(B, Hkv, M, g, d), f(B, Hkv, n, d),
+         f(B, Hkv, M, g, d)]
+    t0 = time.perf_counter()
+    tiles, entries = ssa.ssa_prefill_plan([n] * B, n, C, g)
+    plan_ms = (time.perf_counter() - t0) * 1e3
+    tiles_d, entries_d = tiles.to(dev), entries.to(dev)
+    o_raw = torch.empty((B, Hq, n, d), dtype=torch.float32, device=dev)
+    o_gist = torch.empty((B, Hq, M, g, d), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ssa.ssa_prefill(*x, C, g, tiles_d, entries_d, o_raw, o_gist, stream=stream)
+
+    def timed(fn, steps):
+        total = 0.0
+        for _ in range(steps):
+            flush.fill_(1)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            total += e0.elapsed_time(e1)
+        return total / steps
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ssa.ssa_prefill_get_status() == 0
+    clocks = ClockSampler(0)
+    with clocks:
+        ms = timed(step, args.steps)
+    T = B * (n + M * g)
+    pairs = B * Hq * prefill_visible_pairs(n, C, g)
+    flops = 4.0 * d * pairs                      # q.k and p.v per kept pair
+    blocks = int(entries.numel()) * Hq           # (tile, block) pairs run per head
+    exec_flops = blocks * SSA_BLOCK * SSA_BLOCK * (2.0 * d + 4.0 * d)  # p.v as a bf16 pair
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            peak, peak_kind = float(json.load(fh)["bf16_tflops"]), "measured"
+    except Exception:
+        peak, peak_kind = 1590.0, "fallback"
+    achieved = flops / (ms * 1e-3) / 1e12
+
+    # dense causal attention over the same interleaved length (context only)
+    qd = torch.randn(B, Hq, n + M * g, d, device=dev, dtype=torch.bfloat16)
+    kd = torch.randn(B, Hq, n + M * g, d, device=dev, dtype=torch.bfloat16)
+    vd = torch.randn(B, Hq, n + M * g, d, device=dev, dtype=torch.bfloat16)
+    sdpa = lambda: torch.nn.functional.scaled_dot_product_attention(qd, kd, vd, is_causal=True)
+    for _ in range(3):
+        sdpa()
+    dense_ms = timed(sdpa, max(3, min(args.steps, 20)))
+
+    line = {
+        "metric": "prefill tokens/s of one attention layer under the gist mask",
+        "value": T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": P["workload"], "B": B, "Hq": Hq, "Hkv": Hkv, "d": d, "n": n,
+                   "C": C, "g": g, "l2": "flushed between steps (256 MB write)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_kind": f"bf16 dense, burst, {peak_kind}",
+                     "flops": "4 d per kept (query, key) pair per head",
+                     "executed_tflops": exec_flops / (ms * 1e-3) / 1e12},
+        "plan": {"tiles": int(tiles.shape[0]), "entries": int(entries.numel()),
+                 "host_ms": plan_ms, "kept_pairs_per_head": pairs // (B * Hq),
+                 "block_pairs_per_head": int(entries.numel()) * SSA_BLOCK * SSA_BLOCK},
+        "dense_causal_sdpa_ms": dense_ms,
+        "clocks": clocks.summary(),
+        "gpu_launches": args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
+SSA_BLOCK = 64
+
+
 # ------------------------------------------------------------- GPU arm ---
 
 def main():
@@ -501,11 +623,15 @@ def main():
                     help="another context / selection reading (ssa_decode_variant)")
     ap.add_argument("--levels", default="",
                     help="coarse-to-fine over t levels (ssa_decode_hier): 'J:g2,..,gt:k1,..,kt'")
+    ap.add_argument("--prefill", action="store_true",
+                    help="time the block-sparse prefill of one layer instead (1 GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.prefill:
+        return run_prefill(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libssa.so")
-SOURCES = ["ssa_kernels.cu", "ssa_api.cpp"]
+SOURCES = ["ssa_kernels.cu", "ssa_api.cpp", "ssa_prefill.cu"]
 HEADERS = ["ssa_device.cuh", "ssa_fused.cuh", "ssa_generic.cuh", "ssa_internal.h", "ssa_pipe.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

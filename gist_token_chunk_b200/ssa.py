@@ -8,7 +8,9 @@ memory is plumbing) and maps status codes to exceptions.  Importing it raises
 The functions carry the C ABI's names (see ``include/ssa.h``):
 ``ssa_score_gists``, ``ssa_topk_chunks``, ``ssa_sparse_decode``, ``ssa_decode``,
 ``ssa_decode_h2``, ``ssa_workspace_size``, ``ssa_workspace_size_h2``,
-``ssa_workspace_init``, ``ssa_get_device_status``.
+``ssa_workspace_init``, ``ssa_get_device_status``, and for the prefill and the
+budget ``ssa_adaptive_topk``, ``ssa_prefill_plan_size``, ``ssa_prefill_plan``,
+``ssa_prefill``, ``ssa_prefill_get_status``.
 """
 from __future__ import annotations
 
@@ -47,6 +49,9 @@ SSA_CONTEXT_UNSELECTED_GISTS = 0
 SSA_CONTEXT_SELECTED_ONLY = 1
 SSA_SELECT_GROUP_MAX = 0
 SSA_SELECT_HEAD_UNION = 1
+SSA_PREFILL_BM = 64
+SSA_PREFILL_BN = 64
+SSA_PREFILL_TILE_INTS = 8
 
 
 class Shape(ctypes.Structure):
@@ -92,6 +97,18 @@ lib.ssa_status_string.restype = ctypes.c_char_p
 lib.ssa_last_error.argtypes = []
 lib.ssa_last_error.restype = ctypes.c_char_p
 lib.ssa_version.restype = _I
+_I64 = ctypes.c_int64
+lib.ssa_adaptive_topk.argtypes = [_I64, _I, _I, _I, ctypes.POINTER(_I)]
+lib.ssa_prefill_plan_size.argtypes = [_I, _P, _I, _I, _I, ctypes.POINTER(_I64),
+                                      ctypes.POINTER(_I64)]
+lib.ssa_prefill_plan.argtypes = [_I, _P, _I, _I, _I, _P, _I64, _P, _I64]
+lib.ssa_prefill.argtypes = [_SH, _P, _P, _P, _P, _P, _P, _I, _I, _P, _I64, _P, _I64, _P, _P, _P]
+lib.ssa_prefill_get_status.argtypes = [ctypes.POINTER(_I), _P]
+lib.ssa_prefill_last_error.argtypes = []
+lib.ssa_prefill_last_error.restype = ctypes.c_char_p
+for _f in ("ssa_adaptive_topk", "ssa_prefill_plan_size", "ssa_prefill_plan", "ssa_prefill",
+           "ssa_prefill_get_status"):
+    getattr(lib, _f).restype = _I
 for _f in ("ssa_score_gists", "ssa_topk_chunks", "ssa_sparse_decode", "ssa_decode",
            "ssa_decode_path", "ssa_decode_variant", "ssa_workspace_size_variant",
            "ssa_decode_hier", "ssa_workspace_size_hier", "ssa_decode_host",
@@ -102,16 +119,23 @@ for _f in ("ssa_score_gists", "ssa_topk_chunks", "ssa_sparse_decode", "ssa_decod
 
 
 class SSAError(RuntimeError):
-    def __init__(self, status: int, where: str):
+    def __init__(self, status: int, where: str, detail: Optional[str] = None):
         self.status = status
         msg = lib.ssa_status_string(status).decode()
-        detail = lib.ssa_last_error().decode()
+        if detail is None:
+            detail = lib.ssa_last_error().decode()
         super().__init__(f"{where}: {msg} ({status}){': ' + detail if detail else ''}")
 
 
 def _check(status: int, where: str) -> None:
     if status != SSA_OK:
         raise SSAError(status, where)
+
+
+def _check_pf(status: int, where: str) -> None:
+    """Status of a budget or prefill call (their detail text is kept apart)."""
+    if status != SSA_OK:
+        raise SSAError(status, where, lib.ssa_prefill_last_error().decode())
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -371,3 +395,70 @@ def ssa_set_debug_flags(flags: int) -> None:
 
 def ssa_set_tuning(max_blocks: int = 0, rows_per_score_item: int = 0) -> None:
     lib.ssa_set_tuning(int(max_blocks), int(rows_per_score_item))
+
+
+# ------------------------------------------------------- budget, prefill ---
+
+def ssa_adaptive_topk(n_kv: int, L: int, G: int, J: int = 1) -> int:
+    """App. A selection budget: floor(n_kv / (L J G L)) + 1 (see include/ssa.h)."""
+    k = _I(0)
+    _check_pf(lib.ssa_adaptive_topk(int(n_kv), int(L), int(G), int(J), ctypes.byref(k)),
+              "ssa_adaptive_topk")
+    return int(k.value)
+
+
+def _host_lens(seq_lens):
+    import numpy as np
+
+    if isinstance(seq_lens, torch.Tensor):
+        seq_lens = seq_lens.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+
+
+def ssa_prefill_plan_size(seq_lens, n_max: int, C: int, g: int):
+    lens = _host_lens(seq_lens)
+    nt, ne = ctypes.c_int64(0), ctypes.c_int64(0)
+    _check_pf(lib.ssa_prefill_plan_size(len(lens), lens.ctypes.data, int(n_max), int(C), int(g),
+                                        ctypes.byref(nt), ctypes.byref(ne)),
+              "ssa_prefill_plan_size")
+    return int(nt.value), int(ne.value)
+
+
+def ssa_prefill_plan(seq_lens, n_max: int, C: int, g: int):
+    """The block plan in host memory: (tiles int32 [n_tiles, 8], entries
+    int32 [n_entries]) as torch CPU tensors; copy them to the device once and
+    pass them to every layer's ssa_prefill."""
+    lens = _host_lens(seq_lens)
+    nt, ne = ssa_prefill_plan_size(lens, n_max, C, g)
+    tiles = torch.zeros((max(nt, 1), SSA_PREFILL_TILE_INTS), dtype=torch.int32)
+    entries = torch.zeros(max(ne, 1), dtype=torch.int32)
+    _check_pf(lib.ssa_prefill_plan(len(lens), lens.ctypes.data, int(n_max), int(C), int(g),
+                                   tiles.data_ptr(), nt, entries.data_ptr(), ne),
+              "ssa_prefill_plan")
+    return tiles[:nt], entries[:ne]
+
+
+def ssa_prefill(q_raw, q_gist, k_raw, k_gist, v_raw, v_gist, C: int, g: int, plan_tiles,
+                plan_entries, o_raw=None, o_gist=None, stream=None):
+    """Prefill attention under the gist mask over the plan's blocks; the plan
+    tensors live on the device.  Returns (o_raw, o_gist), fp32."""
+    B, Hq, n_max, d = q_raw.shape
+    shape = make_shape(B, Hq, k_raw.shape[1], d, n_max, _dtype_code(q_raw))
+    if o_raw is None:
+        o_raw = torch.zeros((B, Hq, n_max, d), dtype=torch.float32, device=q_raw.device)
+    if o_gist is None:
+        o_gist = torch.zeros(tuple(q_gist.shape), dtype=torch.float32, device=q_raw.device)
+    gp = (lambda t: _ptr(t) if t.numel() else None)
+    _check_pf(lib.ssa_prefill(ctypes.byref(shape), _ptr(q_raw), gp(q_gist), _ptr(k_raw),
+                              gp(k_gist), _ptr(v_raw), gp(v_gist), int(C), int(g),
+                              _ptr(plan_tiles), plan_tiles.shape[0], gp(plan_entries),
+                              plan_entries.numel(), _ptr(o_raw), gp(o_gist), _stream(stream)),
+              "ssa_prefill")
+    return o_raw, o_gist
+
+
+def ssa_prefill_get_status(stream=None) -> int:
+    code = _I(0)
+    _check_pf(lib.ssa_prefill_get_status(ctypes.byref(code), _stream(stream)),
+              "ssa_prefill_get_status")
+    return int(code.value)

@@ -26,7 +26,9 @@
  *     included); M_b = floor(n_b / C) chunks are complete.
  * ssa_decode_variant offers the pages' other readings of the context and of
  * the selection, and ssa_decode_hier the coarse-to-fine selection over more
- * than two levels.
+ * than two levels.  ssa_adaptive_topk gives App. A's selection budget, and
+ * ssa_prefill_plan / ssa_prefill the block-sparse prefill under the gist
+ * mask (sec. 3.1, 3.6).
  *
  * Notation and layouts (row-major, contiguous, all device memory unless said):
  *   B batch, Hq query heads, Hkv KV heads, G = Hq/Hkv, query head h reads KV
@@ -389,6 +391,119 @@ SSA_API const char* ssa_status_string(ssa_status status);
 /* Detail of the last error returned on this host thread ("" if none). */
 SSA_API const char* ssa_last_error(void);
 SSA_API int32_t ssa_version(void);
+
+/*
+ * ---------------------------------------------------------------- budget ---
+ * ssa_adaptive_topk -- per-level selection budget (App. A): the chunks each
+ * query head keeps, from the raw tokens in the cache n_kv, the chunk size L
+ * (= C), the group size G and, for H-SSA, the chunks per meta-gist group J
+ * (J = 1: single-level SSA).  With the effective compression L_eff = L * J:
+ *     *k = floor(n_kv / (L_eff * G * L)) + 1,
+ * so at least one chunk is kept, the group's union of unfolded raw tokens
+ * G * k * L stays just above n_kv / L_eff, and both H-SSA levels use the
+ * same k.  The pages name the inputs and the +1 but print no formula; this
+ * one is the plainest reading.  Host only, no CUDA call.  Errors: n_kv < 0,
+ * L, G or J < 1, k NULL -> SSA_ERR_INVALID_ARG; k above INT32_MAX ->
+ * SSA_ERR_UNSUPPORTED.
+ */
+SSA_API ssa_status ssa_adaptive_topk(int64_t n_kv, int32_t L, int32_t G, int32_t J, int32_t* k);
+
+/*
+ * --------------------------------------------------------------- prefill ---
+ * Prefill attention under the gist mask (sec. 3.1), run block-sparse over
+ * permuted key columns (sec. 3.6).
+ *
+ * The mask: sequence b interleaves each complete chunk m < M_b = n_b / C of C
+ * raw tokens with its g gist tokens (the gists follow the chunk and belong to
+ * it); the raw tokens after M_b C form chunk M_b, without gists.  A token sees
+ * an earlier-or-equal token of its own chunk, and every gist of an earlier
+ * chunk; never an earlier chunk's raw tokens.
+ *
+ * Layout: the permutation puts every gist column (chunk-major) before every
+ * raw column, which is how the decode cache already stores keys and values;
+ * queries and outputs use the same two arrays per tensor:
+ *   q_raw  [B,Hq,n_max,d]  bf16      q_gist [B,Hq,M_max,g,d]  bf16
+ *   k_raw, v_raw [B,Hkv,n_max,d]      k_gist, v_gist [B,Hkv,M_max,g,d]
+ *   o_raw  [B,Hq,n_max,d]  fp32      o_gist [B,Hq,M_max,g,d]  fp32
+ * With raw row i of chunk m = i / C and gist row r = m g + t, the visible
+ * columns of a row form one interval per part:
+ *   raw row i:   gist columns [0, m g),       raw columns [m C, i + 1);
+ *   gist row r:  gist columns [0, r + 1),     raw columns [m C, m C + C).
+ *
+ * The block plan (computed once per prefill on the host from the host copy of
+ * seq_lens, then copied to the device by the caller and shared by every layer's
+ * call): query tiles of SSA_PREFILL_BM consecutive rows of one part, key blocks of
+ * SSA_PREFILL_BN consecutive columns of one part.  A tile lists every block
+ * holding a visible pair, gist blocks first (ascending) then raw blocks; a
+ * block is full when every valid row of the tile sees all of its columns
+ * (the element mask is then skipped), else partial.  Per tile
+ * SSA_PREFILL_TILE_INTS int32:
+ *   [0] b  [1] part of the rows (0 raw, 1 gist)  [2] first row r0
+ *   [3] valid rows (1 .. BM)  [4] n_b  [5] first entry  [6] entries  [7] 0
+ * Tiles are ordered by decreasing entry count (ties: b, part, r0), so the
+ * longest tiles start first.  Entry = (block << 2) | (part << 1) | full, with
+ * part 0 = gist columns, 1 = raw columns and the block's first column
+ * block * SSA_PREFILL_BN.
+ */
+#define SSA_PREFILL_BM 64
+#define SSA_PREFILL_BN 64
+#define SSA_PREFILL_TILE_INTS 8
+
+/*
+ * ssa_prefill_plan_size -- tile and entry counts of the plan for these
+ * sizes.  seq_lens_host: B int32 in host memory.  Errors: B < 0, a NULL
+ * pointer, C < 1, g < 1, n_max < 0 or not a multiple of C, an n_b outside
+ * [0, n_max] -> SSA_ERR_INVALID_ARG; more than INT32_MAX entries ->
+ * SSA_ERR_UNSUPPORTED.
+ */
+SSA_API ssa_status ssa_prefill_plan_size(int32_t B, const int32_t* seq_lens_host, int32_t n_max,
+                                         int32_t C, int32_t g, int64_t* n_tiles,
+                                         int64_t* n_entries);
+
+/*
+ * ssa_prefill_plan -- writes the plan into caller-owned HOST arrays tiles
+ * [n_tiles * SSA_PREFILL_TILE_INTS] and entries [n_entries] (sizes from
+ * ssa_prefill_plan_size; caps smaller than those -> SSA_ERR_INVALID_ARG,
+ * with nothing written).  Same argument errors as ssa_prefill_plan_size.
+ */
+SSA_API ssa_status ssa_prefill_plan(int32_t B, const int32_t* seq_lens_host, int32_t n_max,
+                                    int32_t C, int32_t g, int32_t* tiles, int64_t tiles_cap,
+                                    int32_t* entries, int64_t entries_cap);
+
+/*
+ * ssa_prefill -- o = softmax(q k^T / sqrt(d) under the gist mask) v for every
+ * row of every sequence, each (tile, query head) one CUDA block that streams
+ * the tile's listed key blocks (tensor-core products, online softmax).
+ * plan_tiles and plan_entries are the plan in device memory.  Rows at or past
+ * n_b (raw) and M_b g (gist) of the outputs are not written.  bf16 inputs, d
+ * in {64, 128}; every array pointer 16-byte aligned.  Errors (nothing
+ * enqueued): NULL pointers (the gist arrays may be NULL when M_max g = 0),
+ * C < 1, g < 1, n_max not a multiple of C, Hq not a multiple of Hkv, n_tiles
+ * or n_entries < 0, misaligned pointers -> SSA_ERR_INVALID_ARG; fp32 or
+ * another d, more than INT32_MAX blocks -> SSA_ERR_UNSUPPORTED; launch
+ * failure -> SSA_ERR_CUDA.  A plan that does not fit these arrays (a tile or
+ * entry out of range) is caught on the device: the kernel skips that tile or
+ * block, records SSA_ERR_DEVICE_STATUS for ssa_prefill_get_status, and reads
+ * and writes nothing outside the arrays.
+ */
+SSA_API ssa_status ssa_prefill(const ssa_shape* shape, const void* q_raw, const void* q_gist,
+                               const void* k_raw, const void* k_gist, const void* v_raw,
+                               const void* v_gist, int32_t C, int32_t g,
+                               const int32_t* plan_tiles, int64_t n_tiles,
+                               const int32_t* plan_entries, int64_t n_entries, float* o_raw,
+                               float* o_gist, cudaStream_t stream);
+
+/*
+ * Synchronise `stream`, return in *host_code the prefill's device status word
+ * (SSA_OK or SSA_ERR_DEVICE_STATUS: the first plan error since the last read)
+ * and clear it.  The prefill kernels keep their own word; ssa_get_device_status
+ * does not see it.
+ */
+SSA_API ssa_status ssa_prefill_get_status(int32_t* host_code, cudaStream_t stream);
+
+/* Detail of the last error a budget or prefill call returned on this host
+ * thread ("" if none). */
+SSA_API const char* ssa_prefill_last_error(void);
 
 #ifdef __cplusplus
 }

@@ -106,6 +106,46 @@ static const float* row_of(const float* base, int64_t heads, int64_t h, int64_t 
     return base + (((b * heads + h) * rows + r) * (int64_t)d);
 }
 
+/* One output row: query (kq, iq) of head h, sequence b (n raw tokens), over
+ * every visible key, into o[0..d). */
+static void prefill_row(int Hq, int Hkv, int d, int64_t n_max, int C, int g, int b, int h,
+                        int64_t n, int kq, int64_t iq, const float* q_raw, const float* q_gist,
+                        const float* k_raw, const float* k_gist, const float* v_raw,
+                        const float* v_gist, double scale, double* o) {
+    const int G = Hq / Hkv, j = h / G;
+    const int64_t M = n / C, ng = M * g, T = n + ng, gr_max = (n_max / C) * g;
+    const float* q = kq ? row_of(q_gist, Hq, h, b, gr_max, iq, d)
+                        : row_of(q_raw, Hq, h, b, n_max, iq, d);
+    double* lg = (double*)malloc((size_t)T * sizeof(double));
+    double mx = -INFINITY;
+    for (int64_t ki = 0; ki < T; ++ki) {
+        const int kk = ki < n ? 0 : 1;
+        const int64_t ik = kk ? ki - n : ki;
+        lg[ki] = -INFINITY;
+        if (!visible(kq, iq, kk, ik, C, g, M)) continue;
+        const float* k = kk ? row_of(k_gist, Hkv, j, b, gr_max, ik, d)
+                            : row_of(k_raw, Hkv, j, b, n_max, ik, d);
+        double s = 0.0;
+        for (int c = 0; c < d; ++c) s += (double)q[c] * (double)k[c];
+        lg[ki] = s * scale;
+        if (lg[ki] > mx) mx = lg[ki];
+    }
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    double den = 0.0;
+    for (int64_t ki = 0; ki < T; ++ki) {
+        if (lg[ki] == -INFINITY) continue;
+        const int kk = ki < n ? 0 : 1;
+        const int64_t ik = kk ? ki - n : ki;
+        const float* v = kk ? row_of(v_gist, Hkv, j, b, gr_max, ik, d)
+                            : row_of(v_raw, Hkv, j, b, n_max, ik, d);
+        const double p = exp(lg[ki] - mx);
+        den += p;
+        for (int c = 0; c < d; ++c) o[c] += p * (double)v[c];
+    }
+    for (int c = 0; c < d; ++c) o[c] /= den;
+    free(lg);
+}
+
 /* Dense masked softmax attention of every row of every sequence: o_raw
  * [B,Hq,n_max,d] and o_gist [B,Hq,M_max,g,d] (fp64) for rows < n_b and
  * < M_b g; other rows are left untouched.  Returns -1 on bad shapes, else the
@@ -117,7 +157,6 @@ int oracle_prefill(int B, int Hq, int Hkv, int d, int n_max, int C, int g,
     if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || d < 1 || C < 1 || g < 1 || n_max < 0 ||
         n_max % C)
         return -1;
-    const int G = Hq / Hkv;
     const int64_t M_max = n_max / C, gr_max = M_max * g;
     const double scale = MUT(20) ? 1.0 : 1.0 / sqrt((double)d);
     int bad = 0;
@@ -131,45 +170,43 @@ int oracle_prefill(int B, int Hq, int Hkv, int d, int n_max, int C, int g,
 #pragma omp parallel for collapse(2) schedule(dynamic, 16)
         for (int h = 0; h < Hq; ++h) {
             for (int64_t qi = 0; qi < T; ++qi) {
-                const int j = h / G;
-                double* lg = (double*)malloc((size_t)T * sizeof(double));
                 const int kq = qi < n ? 0 : 1;
                 const int64_t iq = kq ? qi - n : qi;
-                const float* q = kq ? row_of(q_gist, Hq, h, b, gr_max, iq, d)
-                                    : row_of(q_raw, Hq, h, b, n_max, iq, d);
-                double mx = -INFINITY;
-                for (int64_t ki = 0; ki < T; ++ki) {
-                    const int kk = ki < n ? 0 : 1;
-                    const int64_t ik = kk ? ki - n : ki;
-                    lg[ki] = -INFINITY;
-                    if (!visible(kq, iq, kk, ik, C, g, M)) continue;
-                    const float* k = kk ? row_of(k_gist, Hkv, j, b, gr_max, ik, d)
-                                        : row_of(k_raw, Hkv, j, b, n_max, ik, d);
-                    double s = 0.0;
-                    for (int c = 0; c < d; ++c) s += (double)q[c] * (double)k[c];
-                    lg[ki] = s * scale;
-                    if (lg[ki] > mx) mx = lg[ki];
-                }
                 double* o = kq ? o_gist + (((int64_t)b * Hq + h) * gr_max + iq) * d
                                : o_raw + (((int64_t)b * Hq + h) * n_max + iq) * d;
-                for (int c = 0; c < d; ++c) o[c] = 0.0;
-                double den = 0.0;
-                for (int64_t ki = 0; ki < T; ++ki) {
-                    if (lg[ki] == -INFINITY) continue;
-                    const int kk = ki < n ? 0 : 1;
-                    const int64_t ik = kk ? ki - n : ki;
-                    const float* v = kk ? row_of(v_gist, Hkv, j, b, gr_max, ik, d)
-                                        : row_of(v_raw, Hkv, j, b, n_max, ik, d);
-                    const double p = exp(lg[ki] - mx);
-                    den += p;
-                    for (int c = 0; c < d; ++c) o[c] += p * (double)v[c];
-                }
-                for (int c = 0; c < d; ++c) o[c] /= den;
-                free(lg);
+                prefill_row(Hq, Hkv, d, n_max, C, g, b, h, n, kq, iq, q_raw, q_gist, k_raw,
+                            k_gist, v_raw, v_gist, scale, o);
             }
         }
     }
     return bad;
+}
+
+/* The same rows for a list of queries only: query i is sequence rows[4 i],
+ * head rows[4 i + 1], part rows[4 i + 2] (0 raw, 1 gist), row rows[4 i + 3];
+ * its output goes to out[i * d ..].  Returns -1 on bad shapes or a query
+ * outside the sequence, else 0. */
+int oracle_prefill_rows(int B, int Hq, int Hkv, int d, int n_max, int C, int g,
+                        const int32_t* seq_lens, const float* q_raw, const float* q_gist,
+                        const float* k_raw, const float* k_gist, const float* v_raw,
+                        const float* v_gist, int64_t n_rows, const int32_t* rows, double* out) {
+    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || d < 1 || C < 1 || g < 1 || n_max < 0 ||
+        n_max % C)
+        return -1;
+    for (int64_t i = 0; i < n_rows; ++i) {
+        const int b = rows[4 * i], h = rows[4 * i + 1], kq = rows[4 * i + 2];
+        const int64_t r = rows[4 * i + 3];
+        if (b < 0 || b >= B || h < 0 || h >= Hq || (kq != 0 && kq != 1) || r < 0) return -1;
+        const int64_t n = seq_lens[b];
+        if (n < 0 || n > n_max || r >= (kq ? (n / C) * g : n)) return -1;
+    }
+    const double scale = MUT(20) ? 1.0 : 1.0 / sqrt((double)d);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < n_rows; ++i)
+        prefill_row(Hq, Hkv, d, n_max, C, g, rows[4 * i], rows[4 * i + 1], seq_lens[rows[4 * i]],
+                    rows[4 * i + 2], rows[4 * i + 3], q_raw, q_gist, k_raw, k_gist, v_raw,
+                    v_gist, scale, out + i * d);
+    return 0;
 }
 
 /* ----------------------------------------------------------- block mask --- */

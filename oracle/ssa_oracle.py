@@ -90,6 +90,7 @@ class Oracle:
         self.lib.oracle_adaptive_topk.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                                   ctypes.c_int]
         self.lib.oracle_prefill.restype = ctypes.c_int
+        self.lib.oracle_prefill_rows.restype = ctypes.c_int
         self.lib.oracle_prefill_blocks.restype = ctypes.c_int64
         self.lib.oracle_prefill_blocks.argtypes = [
             ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _I,
@@ -248,6 +249,25 @@ class Oracle:
         if rc < 0:
             raise ValueError("oracle_prefill: bad shape")
         return {"o_raw": o_raw, "o_gist": o_gist, "bad_seq": rc}
+
+    def prefill_rows(self, q_raw, q_gist, k_raw, k_gist, v_raw, v_gist, seq_lens, C: int,
+                     g: int, rows) -> np.ndarray:
+        """The prefill output of the listed rows only: rows = [(b, h, part,
+        r), ...] with part 0 raw, 1 gist (r = m g + t); returns [len(rows), d]."""
+        q_raw, q_gist = _f32(q_raw), _f32(q_gist)
+        k_raw, k_gist, v_raw, v_gist = _f32(k_raw), _f32(k_gist), _f32(v_raw), _f32(v_gist)
+        lens = _i32(seq_lens)
+        B, Hq, n_max, d = q_raw.shape
+        Hkv = k_raw.shape[1]
+        rr = np.ascontiguousarray(np.asarray(rows, np.int32).reshape(-1, 4))
+        out = np.empty((len(rr), d), np.float64)
+        rc = self.lib.oracle_prefill_rows(
+            B, Hq, Hkv, d, n_max, C, g, _p(lens, _I), _p(q_raw, _F), _p(q_gist, _F),
+            _p(k_raw, _F), _p(k_gist, _F), _p(v_raw, _F), _p(v_gist, _F),
+            ctypes.c_int64(len(rr)), _p(rr, _I), _p(out, _D))
+        if rc < 0:
+            raise ValueError("oracle_prefill_rows: bad shape or row")
+        return out
 
     def prefill_blocks(self, n: int, C: int, g: int, BM: int, BN: int) -> list:
         """Block mask of one sequence (sec. 3.6) from the dense gist mask: a

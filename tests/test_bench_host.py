@@ -91,3 +91,22 @@ def test_bytes_models_match_the_oracles_context_sizes(orc):
     want = e * w.d * (2 * int(r["ctx"].sum()) + extra) + _fixed(w, sum(s.size for s in r["sels"]))
     got = bench.hier_bytes(w, lens, [np.asarray(s) for s in r["sels"]], J, g_sum, topks)
     assert got == want, (got, want)
+
+
+def test_prefill_pair_count_matches_the_mask():
+    """The bench's count of kept (query, key) pairs against a pair-by-pair
+    walk of the interleaved sequence under the sec. 3.1 mask."""
+    import bench
+
+    for n, C, g in ((300, 128, 8), (517, 32, 3), (64, 64, 2), (1, 8, 2), (129, 16, 5)):
+        M = n // C
+        pos = {}
+        for i in range(n):
+            m = i // C
+            pos[("r", i)] = (m * (C + g) + i % C if m < M else M * (C + g) + i - M * C, m, False)
+        for m in range(M):
+            for t in range(g):
+                pos[("g", m * g + t)] = (m * (C + g) + C + t, m, True)
+        want = sum(1 for pq, mq, _ in pos.values() for pk, mk, gk in pos.values()
+                   if pk <= pq and (mk == mq or (gk and mk < mq)))
+        assert bench.prefill_visible_pairs(n, C, g) == want, (n, C, g)
