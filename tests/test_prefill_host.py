@@ -150,3 +150,27 @@ def test_prefill_argument_checks_before_cuda():
     assert call(nt=0) == ssa.SSA_OK                          # nothing to do
     assert ssa.lib.ssa_prefill(None, buf, buf, buf, buf, buf, buf, 64, 8, tiles, 1, buf, 1, buf,
                                buf, None) == ssa.SSA_ERR_INVALID_ARG
+
+
+def test_header_intervals_are_the_mask():
+    """The per-row column intervals include/ssa.h states (and the kernel's
+    element mask evaluates) give exactly the visible sets listed from the
+    sentence of sec. 3.1, for every shape the GPU tests use."""
+    from oracle_pins import _visible_sets
+
+    def intervals(kind, r, C, g):
+        if kind == 0:
+            m = r // C
+            return (0, m * g), (m * C, r + 1)
+        m = r // g
+        return (0, r + 1), (m * C, m * C + C)
+
+    for n, C, g in ((1024, 128, 8), (777, 128, 8), (768, 16, 2), (1000, 100, 7), (450, 100, 7),
+                    (256, 64, 80), (100, 128, 8), (5, 128, 8), (2047, 32, 3), (3000, 64, 4)):
+        raw_rows, gist_rows, pos_raw, pos_gist = _visible_sets(n, C, g)
+        for kind, rows in ((0, raw_rows), (1, gist_rows)):
+            for r, (own, gists) in enumerate(rows):
+                (gl, gh), (rl, rh) = intervals(kind, r, C, g)
+                got = ({pos_gist(c // g, c % g) for c in range(gl, gh)}
+                       | {pos_raw(c) for c in range(rl, rh)})
+                assert got == set(own) | set(gists), (n, C, g, kind, r)
