@@ -481,7 +481,8 @@ SSA_API ssa_status ssa_prefill_plan(int32_t B, const int32_t* seq_lens_host, int
  * C < 1, g < 1, n_max not a multiple of C, Hq not a multiple of Hkv, n_tiles
  * or n_entries < 0, misaligned pointers -> SSA_ERR_INVALID_ARG; fp32 or
  * another d, more than INT32_MAX blocks -> SSA_ERR_UNSUPPORTED; launch
- * failure -> SSA_ERR_CUDA.  A plan that does not fit these arrays (a tile or
+ * failure -> SSA_ERR_CUDA.  n_tiles = 0 or B = 0 is SSA_OK with nothing
+ * enqueued (checked before the pointers).  A plan that does not fit these arrays (a tile or
  * entry out of range) is caught on the device: the kernel skips that tile or
  * block, records SSA_ERR_DEVICE_STATUS for ssa_prefill_get_status, and reads
  * and writes nothing outside the arrays.
