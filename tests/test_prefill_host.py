@@ -174,3 +174,22 @@ def test_header_intervals_are_the_mask():
                 got = ({pos_gist(c // g, c % g) for c in range(gl, gh)}
                        | {pos_raw(c) for c in range(rl, rh)})
                 assert got == set(own) | set(gists), (n, C, g, kind, r)
+
+
+def test_plan_random_sizes_match_oracle(orc):
+    """Seeded random (n, C, g): the library's plan equals the oracle's,
+    derived pair by pair from the dense mask (the kernel trusts the full
+    flags, so a wrong one would go unmasked)."""
+    rng = np.random.default_rng(2024)
+    done = 0
+    while done < 40:
+        C = int(rng.choice([1, 2, 3, 7, 16, 33, 64, 100, 128, 200, 256]))
+        g = int(rng.integers(1, 90))
+        n = int(rng.integers(0, 3000))
+        if n + (n // C) * g > 3000:
+            continue
+        n_max = -(-max(n, 1) // C) * C
+        tiles, entries = ssa.ssa_prefill_plan([n], n_max, C, g)
+        got = _by_sequence(tiles, entries).get(0, [])
+        assert [(t, e) for t, e, _ in got] == orc.prefill_blocks(n, C, g, BM, BN), (n, C, g)
+        done += 1
